@@ -1,0 +1,84 @@
+"""c4a / c128a compression of raw tokens into shared K=V entries, and the
+sliding-window copy of the raw tokens.
+
+TEST INFRASTRUCTURE (oracle).
+
+P1 §2.1: a c4a layer folds a group of raw tokens into one entry by a learned
+weighted sum with a position bias (ratio 1/4); a c128a layer folds 128 raw
+tokens into one entry. P1 §2.3: every layer also keeps the last 128 raw tokens
+uncompressed (bf16 or fp8). P1 §3.1.2: the compressor keeps a rolling state of
+the tokens of the group it has not finished.
+
+Readings adopted (the pages are garbled or silent on these points):
+  * a group is r = 4 (c4a) or r = 128 (c128a) consecutive raw tokens,
+    non-overlapping: group g holds tokens [g*r, (g+1)*r);
+  * the gate is one scalar logit a_t per raw token plus a learned bias
+    bias[t - g*r] for its place in the group; weights w_t are the softmax of
+    a_t + bias over the tokens of the group that exist so far;
+  * entry g = sum_t w_t * x_t, then RoPE at position g*r (the group's first
+    token) on the rope dims, then quantisation (fp8: per-entry absmax, see
+    codecs.quantize_entry) or bf16 rounding;
+  * a group that is not complete yet is stored too, normalised over the tokens
+    it has, and rewritten as more tokens arrive (ceil(N/r) stored entries);
+  * window token t = RoPE(x_t, t), stored bf16 (or quantised per token).
+
+The oracle works on a sequence's whole token history, so it has no rolling
+state: an append split into chunks must give exactly what one append gives.
+Arithmetic is fp64; the value handed to the quantiser is that fp64 value
+rounded once to fp32 (the "pre-quant" value).
+"""
+import numpy as np
+
+from . import codecs
+from .rope import rope_rotate
+
+
+def group_weights(gates, bias):
+    """Softmax over one group's tokens of gate + position bias (fp64).
+
+    gates: [n] logits of the group's present tokens (n <= r);
+    bias:  [r] position bias; token i of the group gets bias[i].
+    """
+    z = np.asarray(gates, dtype=np.float64) + np.asarray(bias, dtype=np.float64)[: len(gates)]
+    z = z - z.max()
+    u = np.exp(z)
+    return u / u.sum()
+
+
+def compress_prequant(x, gates, bias, ratio, n_tokens=None, theta=1e6, rope_dim=64,
+                      rope_offset=448):
+    """Pre-quantisation entries of one sequence, fp32 [ceil(N/r), D].
+
+    x: raw tokens [N, D] (any float dtype; bf16 inputs are passed as their
+    exact fp32 values); gates [N]; bias [r]. Only the first ``n_tokens`` tokens
+    are used (default all).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    gates = np.asarray(gates, dtype=np.float64)
+    n = x.shape[0] if n_tokens is None else int(n_tokens)
+    n_groups = -(-n // ratio)
+    out = np.zeros((n_groups, x.shape[1]), dtype=np.float64)
+    for g in range(n_groups):
+        lo, hi = g * ratio, min((g + 1) * ratio, n)
+        w = group_weights(gates[lo:hi], bias)
+        out[g] = w @ x[lo:hi]
+    if n_groups:
+        out = rope_rotate(out, np.arange(n_groups) * ratio, theta, rope_dim, rope_offset)
+    return out.astype(np.float32)
+
+
+def store_entries(prequant, dtype):
+    """What the cache holds for fp32 pre-quant entries.
+
+    dtype "fp8": (codes uint8 [G, D], scale fp32 [G]);
+    dtype "bf16": (bits uint16 [G, D], None).
+    """
+    if dtype == "fp8":
+        return codecs.quantize_entry(prequant)
+    return codecs.bf16_bits(prequant), None
+
+
+def window_tokens(x, positions, theta=1e6, rope_dim=64, rope_offset=448):
+    """Window copies: RoPE(x_t, t) in fp64, rounded to fp32 [n, D]."""
+    return rope_rotate(np.asarray(x, dtype=np.float64), np.asarray(positions),
+                       theta, rope_dim, rope_offset).astype(np.float32)
