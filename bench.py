@@ -1,0 +1,450 @@
+"""Benchmark of the decode step over a paged, compressed fp8 KV cache.
+
+Default workload (one GPU): c4a decode, batch 64, context lengths uniform on
+[4K, 64K], 64 query heads, shared KV dim 512 stored as fp8-e4m3 with one fp32
+scale per entry, 128-token bf16 window, physical pages randomly permuted.
+One step = the whole hot path for one new token per sequence:
+v4kv_slot_mapping -> v4kv_compress_append (1 token each) ->
+v4kv_decode_attention (all visible entries + window). Inputs are synthetic
+(seeded device draws) and resident in HBM; L2 is flushed between steps.
+
+    python bench.py [--gpus N --steps K --warmup W] [--config 1|2|3|4]
+    python bench.py --impl reference ...   # the CPU oracle on host cores
+
+Prints one JSON line (rank 0).
+"""
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "decode-attention tokens/s and achieved HBM GB/s (% of B200 peak), fp8 paged KV"
+D = 512
+W = 128
+HEADS = 64
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ workloads
+
+def decode_config(cfg):
+    r = synth.rng(synth.seed_for(cfg))
+    if cfg == 1:
+        lens = synth.lengths_uniform(r, 64, 4096, 65536, 4)
+        return dict(name="c4a decode, batch 64, context U[4K, 64K], 64 heads, fp8-e4m3 KV dim 512 "
+                         "+ fp32 per-entry scale, 128-token bf16 window, shuffled pages",
+                    lens=lens, ratio=4, r=r)
+    if cfg == 2:
+        lens = synth.lengths_loguniform(r, 32, 131072, 1_000_000)
+        return dict(name="c128a decode, batch 32, context log-uniform [128K, 1M], 64 heads, fp8-e4m3 "
+                         "KV dim 512 + fp32 per-entry scale, 128-token bf16 window, shuffled pages",
+                    lens=lens, ratio=128, r=r)
+    if cfg == 0:
+        return dict(name="tiny c4a decode, 1 sequence, context 1024, 8 heads", lens=np.array([1024]),
+                    ratio=4, r=r, heads=8)
+    raise ValueError(cfg)
+
+
+class DecodeStep:
+    """Device-resident caches and per-step inputs of one decode workload."""
+
+    def __init__(self, cfg, device, seed_offset=0):
+        from paged_compressed_kv_b200 import PagedPool, v4kv
+        c = decode_config(cfg)
+        self.v4kv = v4kv
+        self.name = c["name"]
+        self.lens = c["lens"].astype(np.int64)
+        self.ratio = c["ratio"]
+        self.H = c.get("heads", HEADS)
+        self.B = len(self.lens)
+        r = c["r"]
+        g = synth.device_generator(synth.seed_for(cfg) + 7919 * seed_offset, device)
+        spb = 256 // self.ratio
+        n_ent = [-(-int(L) // self.ratio) for L in self.lens]
+        nblk = [-(-n // spb) for n in n_ent]
+        P = int(sum(nblk))
+        perm = synth.permutation(r, P)
+        bt = np.full((self.B, max(nblk)), -1, dtype=np.int32)
+        k = 0
+        for b, nb in enumerate(nblk):
+            bt[b, :nb] = perm[k:k + nb]
+            k += nb
+        self.P = P
+        data = torch.empty(P, spb, D, dtype=torch.uint8, device=device)
+        synth.fill_fp8_codes(data, g)
+        scales = torch.empty(P, spb, dtype=torch.float32, device=device)
+        synth.fill_uniform(scales, g, 0.5 / 112, 1.5 / 112)
+        self.main = PagedPool(data=data, block_table=torch.from_numpy(bt).to(device), scales=scales)
+        # window: pages only for the blocks holding tokens [L - W, L)
+        wfirst = [max(0, int(L) - W) // 256 for L in self.lens]
+        wlast = [(int(L) - 1) // 256 for L in self.lens]
+        Pw = int(sum(l - f + 1 for f, l in zip(wfirst, wlast)))
+        wperm = synth.permutation(r, Pw)
+        wbt = np.full((self.B, max(wlast) + 1), -1, dtype=np.int32)
+        k = 0
+        for b in range(self.B):
+            for blk in range(wfirst[b], wlast[b] + 1):
+                wbt[b, blk] = wperm[k]
+                k += 1
+        wdata = torch.empty(Pw, 256, D, dtype=torch.bfloat16, device=device)
+        synth.fill_normal_bf16(wdata, g)
+        self.win = PagedPool(data=wdata, block_table=torch.from_numpy(wbt).to(device))
+        # per-step inputs: the new token at position L - 1, then decode at L
+        self.q = torch.randn(self.B, self.H, D, generator=g, device=device)
+        self.x = torch.randn(self.B, D, generator=g, device=device).to(torch.bfloat16)
+        self.gate = torch.randn(self.B, generator=g, device=device)
+        self.bias = torch.randn(self.ratio, generator=g, device=device) * 0.5
+        self.state_x = torch.randn(self.B, self.ratio, D, generator=g, device=device).to(torch.bfloat16)
+        self.state_g = torch.randn(self.B, self.ratio, generator=g, device=device)
+        self.seq_start = torch.from_numpy((self.lens - 1).astype(np.int32)).to(device)
+        self.n_new = torch.ones(self.B, dtype=torch.int32, device=device)
+        self.cu_seqlens = torch.arange(self.B + 1, dtype=torch.int32, device=device)
+        self.seq_lens = torch.from_numpy(self.lens.astype(np.int32)).to(device)
+        self.slots = torch.empty(2 * self.B + 1, dtype=torch.int64, device=device)
+        self.cu_e = torch.empty(self.B + 1, dtype=torch.int32, device=device)
+        self.out = torch.empty(self.B, self.H, D, dtype=torch.bfloat16, device=device)
+        self.max_len = int(self.lens.max())
+        ws = v4kv.v4kv_workspace_size(v4kv.V4KV_OP_DECODE, self.B, self.H, self.max_len, self.ratio,
+                                      W, 0, v4kv.V4KV_FP8_E4M3)
+        self.workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def launches_per_step(self):
+        # slot mapping 1, compressor 3 (entries, window, state), decode 2 (sweep, merge)
+        return 6
+
+    def append(self, stream=None):
+        v = self.v4kv
+        v.v4kv_slot_mapping(self.main.block_table, self.seq_start, self.n_new, self.ratio, self.P,
+                            self.slots, self.cu_e, dev_status=self.status, stream=stream)
+        v.v4kv_compress_append(self.x, self.gate, self.cu_seqlens, self.seq_start, self.bias,
+                               self.ratio, self.state_x, self.state_g, self.main, self.slots,
+                               self.cu_e, window=self.win, window_len=W, dev_status=self.status,
+                               stream=stream)
+
+    def decode(self, stream=None, q=None, out=None):
+        self.v4kv.v4kv_decode_attention(self.q if q is None else q, self.main, self.win,
+                                        self.seq_lens, self.max_len, self.ratio, W,
+                                        self.out if out is None else out, self.workspace,
+                                        dev_status=self.status, stream=stream)
+
+    def algorithmic_bytes(self):
+        """KV, scales, window, q, output and block-table bytes one decode call must touch."""
+        tot = 0
+        for L in self.lens:
+            L = int(L)
+            n_vis = max(0, L - W) // self.ratio
+            tot += n_vis * (D + 4) + min(L, W) * D * 2 + self.H * D * 4 + self.H * D * 2
+            tot += 4 * (-(-L // 256))
+        return tot
+
+    def h2d_bytes(self):
+        return (self.q.numel() * 4 + self.x.numel() * 2 + self.gate.numel() * 4 +
+                self.seq_start.numel() * 4 + self.n_new.numel() * 4 + self.seq_lens.numel() * 4)
+
+    def d2h_bytes(self):
+        return self.out.numel() * 2
+
+
+# ------------------------------------------------------------------ helpers
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def l2_flush(buf):
+    buf.add_(1)
+
+
+def cores_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(step, seconds=10.0, max_seqs=None):
+    """Time the CPU oracle on whole sequences of the workload (rank 0 only).
+
+    The caches are copied to the host once (outside the timed region); the
+    oracle then gathers each sample sequence's pages and runs the fp64
+    attention. Returns (sequences per second, sequences timed, seconds)."""
+    from oracle import attention
+    main = {"data": step.main.data.cpu().numpy(), "scales": step.main.scales.cpu().numpy(),
+            "dtype": "fp8"}
+    win = {"data": step.win.data.view(torch.int16).cpu().numpy().view(np.uint16), "scales": None,
+           "dtype": "bf16"}
+    bt = step.main.block_table.cpu().numpy()
+    wbt = step.win.block_table.cpu().numpy()
+    q = step.q.cpu().numpy().astype(np.float64)
+    order = np.random.default_rng(0).permutation(step.B)
+    done, t0 = 0, time.perf_counter()
+    for b in order:
+        m = dict(main, block_table_row=bt[b])
+        w = dict(win, block_table_row=wbt[b])
+        attention.decode_one(q[b], m, w, int(step.lens[b]), step.ratio, W, 1 / math.sqrt(D))
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_seqs and done >= max_seqs):
+            break
+    el = time.perf_counter() - t0
+    return done / el, done, el
+
+
+# ------------------------------------------------------------------ arms
+
+def run_ours(args, rank, world, device):
+    peak, peak_kind = load_peaks()
+    step = DecodeStep(args.config, device, seed_offset=rank)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    for _ in range(args.warmup):
+        step.append()
+        step.decode()
+        l2_flush(flush)
+    torch.cuda.synchronize()
+    if step.status.item() != 0:
+        raise RuntimeError(f"device status {step.status.item()}")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device.index) as clk:
+        for i in range(args.steps):
+            s0, s1, s2 = ev[i]
+            s0.record(stream)
+            step.append()
+            s1.record(stream)
+            step.decode()
+            s2.record(stream)
+            l2_flush(flush)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    dec_ms = [b.elapsed_time(c) for _, b, c in ev]
+    t_step = float(np.sum(step_ms)) / args.steps
+    t_dec = float(np.mean(dec_ms))
+    t_max = torch.tensor([t_step, t_dec], device=device, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(t_max, op=torch.distributed.ReduceOp.MAX)
+    t_step, t_dec = float(t_max[0]), float(t_max[1])
+
+    # end to end through the public API with host buffers (pinned), copies timed
+    q_h = step.q.cpu().pin_memory()
+    x_h = step.x.cpu().pin_memory()
+    g_h = step.gate.cpu().pin_memory()
+    ss_h = step.seq_start.cpu().pin_memory()
+    nn_h = step.n_new.cpu().pin_memory()
+    sl_h = step.seq_lens.cpu().pin_memory()
+    out_h = torch.empty(step.out.shape, dtype=torch.bfloat16).pin_memory()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for i in range(args.steps + args.warmup):
+        timed = i >= args.warmup
+        if timed:
+            e2e_ev[i - args.warmup][0].record(stream)
+        step.q.copy_(q_h, non_blocking=True)
+        step.x.copy_(x_h, non_blocking=True)
+        step.gate.copy_(g_h, non_blocking=True)
+        step.seq_start.copy_(ss_h, non_blocking=True)
+        step.n_new.copy_(nn_h, non_blocking=True)
+        step.seq_lens.copy_(sl_h, non_blocking=True)
+        step.append()
+        step.decode()
+        out_h.copy_(step.out, non_blocking=True)
+        if timed:
+            e2e_ev[i - args.warmup][1].record(stream)
+        l2_flush(flush)
+    torch.cuda.synchronize()
+    t_e2e = float(np.mean([a.elapsed_time(b) for a, b in e2e_ev]))
+    te = torch.tensor([t_e2e], device=device, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+    t_e2e = float(te[0])
+    if step.status.item() != 0:
+        raise RuntimeError(f"device status {step.status.item()}")
+
+    tokens = step.B * world
+    alg = step.algorithmic_bytes()
+    achieved = alg / (t_dec * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": tokens / (t_step * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": t_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": DTYPE,
+        "data": "synthetic (seeded device draws: fp8 codes, fp32 scales, bf16 window, fp32 q)",
+        "config": {"workload": step.name, "batch": step.B, "heads": step.H, "dim": D,
+                   "ratio": step.ratio, "window": W, "parallelism": f"replicas x{world}",
+                   "l2": "flushed between steps (256 MB write), inputs also exceed L2",
+                   "decode_ms": t_dec, "hbm_gbs": achieved},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "v4kv_decode_attention (sweep + merge)",
+                     "algorithmic_bytes": alg, "peak_source": peak_kind},
+        "e2e": {"value": tokens / (t_e2e * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": step.d2h_bytes()},
+        "gpu_launches": step.launches_per_step() * args.steps,
+    }
+    clocks = clk.summary()
+    if clocks is not None:
+        line["clocks"] = clocks
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, n, el = oracle_sample(step, seconds=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate * 1.0, "unit": "tokens/s", "cores": cores_used(),
+                                "kind": "oracle",
+                                "sample": f"{n} whole sequences of the same workload (fp64 numpy "
+                                          f"oracle, pages gathered on the host), {el:.1f} s"}
+    return line
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step times a bounded sample."""
+    if rank != 0:
+        return None
+    torch.set_grad_enabled(False)
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else None
+    if dev is None:
+        return {"impl": "reference", "unavailable": "needs the workload's caches on a CUDA device"}
+    step = DecodeStep(args.config, dev)
+    per = max(1, int(args.ref_seqs))
+    for _ in range(args.warmup):
+        oracle_sample(step, seconds=1e9, max_seqs=1)
+    rates = []
+    t_all = 0.0
+    for _ in range(args.steps):
+        rate, n, el = oracle_sample(step, seconds=1e9, max_seqs=per)
+        rates.append(rate)
+        t_all += el
+    value = float(np.mean(rates))
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * t_all / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded device draws)",
+        "config": {"workload": step.name, "batch": step.B, "heads": step.H, "dim": D,
+                   "ratio": step.ratio, "window": W, "parallelism": "cpu oracle, rank 0"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
+                         "sample": f"{per} whole sequences per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+DTYPE = "fp32"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seqs", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        line = run_ours(args, rank, world, device)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,114 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace v4kv {
+
+struct PoolArgs {
+  void* data;
+  float* scales;
+  const int32_t* block_table;
+  int num_pages;
+  int spb;  // slots per page
+  int dim;
+  int dtype;
+  int max_blocks;
+};
+
+struct RopeArgs {
+  double theta;
+  int rope_dim;
+  int rope_offset;
+};
+
+struct CompressArgs {
+  const uint16_t* x;
+  const float* gate;
+  const int32_t* cu_seqlens;
+  const int32_t* seq_start;
+  const float* pos_bias;
+  const uint16_t* state_x;
+  const float* state_gate;
+  uint16_t* state_x_out;  // same memory as state_x (updated in place)
+  float* state_gate_out;
+  const int64_t* slot_mapping;
+  const int32_t* cu_entries;
+  float* prequant_out;
+  int32_t* dev_status;
+  PoolArgs main;
+  PoolArgs window;
+  RopeArgs rope;
+  int batch;
+  int ratio;
+  int dim;
+  int window_len;
+};
+
+struct IndexArgs {
+  const float* q_idx;
+  const int32_t* seq_lens;
+  int32_t* topk_out;
+  float* score_out;
+  float* scores_ws;  // [batch, ws_stride] scratch
+  int32_t* dev_status;
+  PoolArgs cache;
+  int batch;
+  int ratio;
+  int window_len;
+  int k;
+  int max_len;        // host bound on seq_lens; longer sequences are clamped and flagged
+  int ws_stride;      // max visible entries (row stride of scores_ws)
+  int chunk;          // entries scored per block
+};
+
+struct DecodePlan {
+  int path;          // 0 = CUDA-core kernel, 1 = tensor-core kernel
+  int items_max;     // max attended items (entries + window) of one sequence
+  int split;         // items per split
+  int n_splits;      // splits per sequence
+  size_t ws_bytes;   // partial results
+};
+
+struct DecodeArgs {
+  const void* q;
+  const int32_t* seq_lens;
+  const int32_t* topk;
+  void* out;
+  float* part_o;  // [batch, n_splits, heads, dim]
+  float* part_ml; // [batch, n_splits, heads, 2]  (max in log2 units, sum)
+  int32_t* dev_status;
+  PoolArgs main;
+  PoolArgs window;
+  RopeArgs rope;
+  int q_dtype;
+  int batch;
+  int heads;
+  int dim;
+  int ratio;
+  int window_len;
+  int k;
+  float sm_scale;
+  int split;
+  int n_splits;
+  int max_len;  // host bound on seq_lens; longer sequences are clamped and flagged
+};
+
+cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, int batch,
+                                const int32_t* seq_start, const int32_t* n_new, int ratio, int spb,
+                                int num_pages, int32_t* cu_out, int64_t* slot_out, long long cap,
+                                int32_t* st, cudaStream_t stream);
+
+cudaError_t launch_compress_append(const CompressArgs& a, int max_groups, cudaStream_t stream);
+
+size_t index_workspace_bytes(int batch, int max_seq_len, int ratio, int window_len);
+cudaError_t launch_index_topk(IndexArgs a, int max_seq_len, cudaStream_t stream);
+
+DecodePlan plan_decode(int batch, int heads, int max_seq_len, int ratio, int window_len, int k,
+                       int main_dtype, int dim, int num_sms);
+cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream);
+
+}  // namespace v4kv

@@ -1,0 +1,93 @@
+"""CPU-side checks of the C-ABI library: it loads, exports every function the
+header declares, rejects bad arguments on the host before touching the
+device, and its host-only footprint formula matches the oracle's."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from oracle import footprint
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "v4kv.h")
+
+
+def declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(v4kv_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_hot_path_calls():
+    names = declared()
+    for n in ["v4kv_slot_mapping", "v4kv_compress_append", "v4kv_index_topk",
+              "v4kv_decode_attention", "v4kv_workspace_size", "v4kv_kv_footprint_bytes"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    from paged_compressed_kv_b200 import v4kv
+    lib = ctypes.CDLL(v4kv.LIB_PATH)
+    for name in declared():
+        assert hasattr(lib, name), name
+    assert set(declared()) <= set(v4kv.EXPORTED)
+
+
+def test_status_strings_and_version():
+    from paged_compressed_kv_b200 import v4kv
+    assert v4kv.v4kv_version() >= 1
+    assert v4kv.v4kv_status_string(0) == "ok"
+    assert "invalid" in v4kv.v4kv_status_string(1)
+
+
+def test_host_argument_checks_return_invalid_arg_without_a_device():
+    from paged_compressed_kv_b200 import v4kv
+    lib = v4kv._lib
+    fake = ctypes.c_void_p(0x10000)
+    # ratio 3 is not a divisor of the 256-token block
+    assert lib.v4kv_slot_mapping(fake, 4, 1, fake, fake, 3, 85, 10, None, fake, 10, None, None) == 1
+    # negative batch
+    assert lib.v4kv_slot_mapping(fake, 4, -1, fake, fake, 4, 64, 10, None, fake, 10, None, None) == 1
+    # decode: misaligned query pointer
+    pool = v4kv._Paged(0x10000, 0x20000, 4, 64, 512, 1, 0x30000, 4)
+    win = v4kv._Paged(0x40000, None, 4, 256, 512, 0, 0x50000, 4)
+    rope = v4kv._Rope(1e6, 64, 448)
+    st = lib.v4kv_decode_attention(0x10001, 2, 1, 8, ctypes.byref(pool), ctypes.byref(win), fake,
+                                   1024, 4, 128, None, 0, 0.04, rope, fake, fake, 1 << 20, None, None)
+    assert st == 1
+    # decode: heads beyond 128 are unsupported
+    st = lib.v4kv_decode_attention(fake, 2, 1, 129, ctypes.byref(pool), ctypes.byref(win), fake,
+                                   1024, 4, 128, None, 0, 0.04, rope, fake, fake, 1 << 20, None, None)
+    assert st == 2
+    # decode: a pool whose slots per page does not match the ratio
+    bad = v4kv._Paged(0x10000, 0x20000, 4, 2, 512, 1, 0x30000, 4)
+    st = lib.v4kv_decode_attention(fake, 2, 1, 8, ctypes.byref(bad), ctypes.byref(win), fake,
+                                   1024, 4, 128, None, 0, 0.04, rope, fake, fake, 1 << 20, None, None)
+    assert st == 1
+    # rope dims outside the vector
+    st = lib.v4kv_decode_attention(fake, 2, 1, 8, ctypes.byref(pool), ctypes.byref(win), fake,
+                                   1024, 4, 128, None, 0, 0.04, v4kv._Rope(1e6, 64, 480), fake, fake,
+                                   1 << 20, None, None)
+    assert st == 1
+    # index: k above 2048
+    st = lib.v4kv_index_topk(fake, ctypes.byref(pool), fake, 1, 1024, 4, 128, 4096, fake, None,
+                             fake, 1 << 20, None, None)
+    assert st == 1
+    # compress: ratio 8
+    st = lib.v4kv_compress_append(fake, fake, fake, fake, 1, 4, fake, 8, rope, fake, fake,
+                                  ctypes.byref(pool), fake, fake, None, 128, None, None, None)
+    assert st == 1
+
+
+@pytest.mark.parametrize("n", [0, 1, 1000, 131072, 1_000_000])
+def test_footprint_matches_oracle(n):
+    from paged_compressed_kv_b200 import v4kv
+    layers = [4] * 30 + [128] * 31
+    got = v4kv.v4kv_kv_footprint_bytes(n, layers, 512, 8, 4, 128, 8, 4, 128, 16)
+    want = footprint.kv_bytes(n, layers, 512, 1, 4, indexer_dim=128, indexer_elem_bytes=1,
+                              indexer_scale_bytes=4, window=128, window_elem_bytes=2)
+    assert got == want
+    # the page's bf16 configuration
+    got = v4kv.v4kv_kv_footprint_bytes(n, layers, 5120, 16)
+    assert got == footprint.kv_bytes(n, layers, 5120, 2)

@@ -1,0 +1,218 @@
+"""Parity of v4kv_slot_mapping and v4kv_compress_append (through the C ABI)
+with the oracle: slots bit-exact, pre-quant values within tolerance, fp8 bytes
+and scales bit-exact on the kernel's own pre-quant values, window copies,
+rolling state, and chunking invariance."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import codecs, compressor, paging
+
+pytestmark = pytest.mark.gpu
+
+D = 512
+
+
+class Appender:
+    """Runs appends of per-sequence chunks through the library."""
+
+    def __init__(self, seed, n_tokens, ratio, main_dtype="fp8", W=128, gates=None, dim=D,
+                 rope=True):
+        from paged_compressed_kv_b200 import PagedPool, Rope
+        self.r = synth.rng(seed)
+        self.n = [int(v) for v in n_tokens]
+        self.B, self.ratio, self.W, self.dim = len(n_tokens), ratio, W, dim
+        self.main_dtype = main_dtype
+        self.rope = Rope() if rope else Rope(rope_dim=0)
+        self.x = [synth.normal(self.r, (N, dim)) for N in self.n]
+        self.x = [codecs.bf16_round(v) for v in self.x]             # exact bf16 values
+        self.g = gates if gates is not None else [synth.normal(self.r, N) for N in self.n]
+        self.bias = synth.normal(self.r, ratio, 0.5)
+        spb = 256 // ratio
+        nblk = [-(-paging.entry_count(N, ratio) // spb) for N in self.n]
+        self.bt, self.P = paging.allocate_block_tables(nblk, synth.permutation(self.r, sum(nblk) + 2))
+        wblk = [-(-N // 256) for N in self.n]
+        self.wbt, self.Pw = paging.allocate_block_tables(wblk, synth.permutation(self.r, sum(wblk) + 1))
+        dev = torch.device("cuda")
+        if main_dtype == "fp8":
+            data = torch.zeros(self.P, spb, dim, dtype=torch.uint8, device=dev)
+            sc = torch.zeros(self.P, spb, dtype=torch.float32, device=dev)
+        else:
+            data = torch.zeros(self.P, spb, dim, dtype=torch.bfloat16, device=dev)
+            sc = None
+        self.main = PagedPool(data=data, block_table=torch.from_numpy(self.bt).to(dev), scales=sc)
+        self.win = PagedPool(data=torch.zeros(self.Pw, 256, dim, dtype=torch.bfloat16, device=dev),
+                             block_table=torch.from_numpy(self.wbt).to(dev))
+        self.state_x = torch.zeros(self.B, ratio, dim, dtype=torch.bfloat16, device=dev)
+        self.state_g = torch.zeros(self.B, ratio, dtype=torch.float32, device=dev)
+        self.done = [0] * self.B
+        self.prequant = [np.full((paging.entry_count(N, ratio), dim), np.nan, np.float32) for N in self.n]
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def append(self, sizes):
+        from paged_compressed_kv_b200 import v4kv
+        dev = torch.device("cuda")
+        sizes = [min(int(s), N - d) for s, N, d in zip(sizes, self.n, self.done)]
+        seq_start = np.array(self.done, dtype=np.int32)
+        n_new = np.array(sizes, dtype=np.int32)
+        cu = np.concatenate([[0], np.cumsum(n_new)]).astype(np.int32)
+        xs = np.concatenate([self.x[b][self.done[b]:self.done[b] + sizes[b]] for b in range(self.B)])
+        gs = np.concatenate([self.g[b][self.done[b]:self.done[b] + sizes[b]] for b in range(self.B)])
+        cap = int(n_new.sum()) // self.ratio + 2 * self.B
+        slots = torch.full((cap,), -7, dtype=torch.int64, device=dev)
+        cu_e = torch.zeros(self.B + 1, dtype=torch.int32, device=dev)
+        ss = torch.from_numpy(seq_start).to(dev)
+        nn = torch.from_numpy(n_new).to(dev)
+        v4kv.v4kv_slot_mapping(self.main.block_table, ss, nn, self.ratio, self.P, slots, cu_e,
+                               dev_status=self.status)
+        # slots must equal the oracle's slot mapping bit for bit
+        want, want_cu = paging.slot_mapping(self.bt, seq_start, n_new, self.ratio, 256 // self.ratio)
+        got_cu = cu_e.cpu().numpy()
+        assert np.array_equal(got_cu, want_cu)
+        assert np.array_equal(slots[: len(want)].cpu().numpy(), want)
+        pre = torch.full((max(1, len(want)), self.dim), np.nan, dtype=torch.float32, device=dev)
+        v4kv.v4kv_compress_append(
+            synth.bf16_tensor(xs).to(dev).reshape(-1, self.dim), torch.from_numpy(gs).to(dev),
+            torch.from_numpy(cu).to(dev), ss, torch.from_numpy(self.bias).to(dev), self.ratio,
+            self.state_x, self.state_g, self.main, slots, cu_e, window=self.win, window_len=self.W,
+            rope=self.rope, prequant_out=pre, dev_status=self.status)
+        pre = pre.cpu().numpy()
+        for b in range(self.B):
+            first, end = paging.touched_range(self.done[b], sizes[b], self.ratio)
+            self.prequant[b][first:end] = pre[want_cu[b]:want_cu[b + 1]]
+            self.done[b] += sizes[b]
+        assert int(self.status.item()) == 0
+
+    def entries(self, b):
+        """Stored entries of sequence b: (codes or bf16 bits [n, D], scales or None)."""
+        spb = 256 // self.ratio
+        n = paging.entry_count(self.n[b], self.ratio)
+        data = self.main.data
+        if self.main_dtype == "bf16":
+            data = data.view(torch.int16)
+        data = data.cpu().numpy()
+        sc = self.main.scales.cpu().numpy() if self.main.scales is not None else None
+        rows = np.stack([data[self.bt[b, j // spb], j % spb] for j in range(n)]) if n else data[:0, 0]
+        scs = np.array([sc[self.bt[b, j // spb], j % spb] for j in range(n)]) if sc is not None else None
+        return rows, scs
+
+    def window_values(self, b):
+        N = self.n[b]
+        w = self.win.data.view(torch.int16).cpu().numpy().view(np.uint16)
+        ts = range(max(0, N - self.W), N)
+        return np.stack([w[self.wbt[b, t // 256], t % 256] for t in ts]) if N else np.zeros((0, self.dim), np.uint16)
+
+
+def check_against_oracle(ap):
+    rope_dim = ap.rope.rope_dim
+    for b in range(ap.B):
+        N = ap.n[b]
+        ref = compressor.compress_prequant(ap.x[b], ap.g[b], ap.bias, ap.ratio, rope_dim=rope_dim)
+        got = ap.prequant[b]
+        assert not np.isnan(got).any()
+        amax = np.abs(ref).max(axis=1, keepdims=True)
+        assert np.all(np.abs(got - ref) <= 5e-5 * amax + 1e-30), f"seq {b}: pre-quant"
+        rows, scs = ap.entries(b)
+        if ap.main_dtype == "fp8":
+            codes, sc = codecs.quantize_entry(got)
+            assert np.array_equal(rows, codes), f"seq {b}: fp8 bytes"
+            assert np.array_equal(scs.view(np.uint32), sc.view(np.uint32)), f"seq {b}: scales"
+        else:
+            assert np.array_equal(rows.view(np.uint16), codecs.bf16_bits(got)), f"seq {b}: bf16"
+        # window: last W tokens RoPE'd at their own position, bf16
+        w0 = max(0, N - ap.W)
+        wref = codecs.bf16_round(compressor.window_tokens(ap.x[b][w0:], np.arange(w0, N), rope_dim=rope_dim))
+        wgot = codecs.bf16_to_f32(ap.window_values(b))
+        assert np.all(np.abs(wgot - wref) <= np.abs(wref) * 2.0**-7 + 1e-30), f"seq {b}: window"
+        # state: the unfinished group's raw tokens and gates
+        gs = (N // ap.ratio) * ap.ratio
+        st = ap.state_x[b, : N - gs].float().cpu().numpy()
+        assert np.array_equal(st, ap.x[b][gs:N]), f"seq {b}: state"
+
+
+@pytest.mark.parametrize("ratio", [4, 128])
+@pytest.mark.parametrize("main_dtype", ["fp8", "bf16"])
+def test_one_shot_append(ratio, main_dtype):
+    ap = Appender(400 + ratio, [1, 3, 4, 5, 127, 128, 129, 1024, 3000], ratio, main_dtype)
+    ap.append(ap.n)
+    check_against_oracle(ap)
+
+
+def test_tiny_c4a_workload():
+    # one sequence of 1024 raw tokens, bf16 entries: 256 entries
+    ap = Appender(synth.seed_for(0), [1024], 4, "bf16")
+    ap.append([1024])
+    check_against_oracle(ap)
+    assert ap.prequant[0].shape[0] == 256
+
+
+@pytest.mark.parametrize("ratio", [4, 128])
+def test_chunked_equals_one_shot_bitwise(ratio):
+    n = [5000, 2049, 777, 9000]
+    a = Appender(410, n, ratio)
+    a.append(n)
+    b = Appender(410, n, ratio)
+    r = synth.rng(411)
+    while any(d < N for d, N in zip(b.done, b.n)):
+        b.append([int(r.integers(1, 700)) for _ in n])
+    check_against_oracle(b)
+    for s in range(len(n)):
+        ra, sa = a.entries(s)
+        rb, sb = b.entries(s)
+        assert np.array_equal(ra, rb) and np.array_equal(sa, sb)
+        assert np.array_equal(a.prequant[s].view(np.uint32), b.prequant[s].view(np.uint32))
+
+
+def test_one_hot_gates_store_the_selected_token():
+    r = synth.rng(420)
+    n = [64, 130]
+    gates = []
+    for N in n:
+        g = np.full(N, -1e30, dtype=np.float32)
+        g[::4] = 0.0                       # the first token of every group
+        gates.append(g)
+    ap = Appender(421, n, 4, "bf16", gates=gates)
+    ap.append(n)
+    check_against_oracle(ap)
+    for b, N in enumerate(n):
+        rows, _ = ap.entries(b)
+        # entry g == window-style copy of token 4g (RoPE at 4g), as bf16
+        want = codecs.bf16_bits(compressor.window_tokens(ap.x[b][::4], np.arange(0, N, 4)))
+        d = np.abs(codecs.bf16_to_f32(rows) - codecs.bf16_to_f32(want))
+        assert np.all(d <= np.abs(codecs.bf16_to_f32(want)) * 2.0**-7 + 1e-30)
+
+
+@pytest.mark.parametrize("ratio", [4, 128])
+def test_full_size_random_chunks(ratio):
+    # 8 sequences x 32K raw tokens appended in random chunks of 1..4096
+    r = synth.rng(synth.seed_for(3) + ratio)
+    n = [32768] * 8
+    ap = Appender(synth.seed_for(3), n, ratio)
+    while any(d < N for d, N in zip(ap.done, ap.n)):
+        ap.append([int(r.integers(1, 4097)) for _ in n])
+    check_against_oracle(ap)
+
+
+def test_slot_mapping_flags_bad_pages_and_overflow():
+    from paged_compressed_kv_b200 import v4kv
+    dev = torch.device("cuda")
+    bt = torch.tensor([[0, 5, -1, 2]], dtype=torch.int32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    slots = torch.zeros(300, dtype=torch.int64, device=dev)
+    cu = torch.zeros(2, dtype=torch.int32, device=dev)
+    ss = torch.tensor([0], dtype=torch.int32, device=dev)
+    nn = torch.tensor([1000], dtype=torch.int32, device=dev)
+    v4kv.v4kv_slot_mapping(bt, ss, nn, 4, 3, slots, cu, dev_status=st)
+    torch.cuda.synchronize()
+    s = slots.cpu().numpy()
+    assert cu.cpu().tolist() == [0, 250]
+    assert np.array_equal(s[:64], np.arange(64))
+    assert np.all(s[64:192] == -1)              # page 5 >= num_pages, and a -1 block
+    assert np.array_equal(s[192:250], 2 * 64 + np.arange(58))
+    assert int(st.item()) & 1
+    st.zero_()
+    small = torch.zeros(10, dtype=torch.int64, device=dev)
+    v4kv.v4kv_slot_mapping(bt, ss, nn, 4, 3, small, None, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & 8

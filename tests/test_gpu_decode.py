@@ -1,0 +1,135 @@
+"""Parity of v4kv_decode_attention (through the C ABI) with the oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests.helpers import DecodeCase, assert_close_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def run_decode(case, topk=None, q_dtype=torch.float32, sm_scale=None, k=None):
+    from paged_compressed_kv_b200 import v4kv
+    dev = torch.device("cuda")
+    q = torch.from_numpy(case.q).to(dev)
+    if q_dtype == torch.bfloat16:
+        q = q.to(torch.bfloat16)
+    main, win = case.main.to_cuda(), case.win.to_cuda()
+    seq = torch.from_numpy(case.lens.astype(np.int32)).to(dev)
+    out = torch.empty(case.B, case.H, 512, dtype=torch.bfloat16, device=dev)
+    kk = 0 if topk is None else topk.shape[1]
+    ws = v4kv.v4kv_workspace_size(v4kv.V4KV_OP_DECODE, case.B, case.H, case.max_len, case.ratio,
+                                  case.W, kk, main.dtype_code)
+    workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    tk = None if topk is None else torch.from_numpy(topk.astype(np.int32)).to(dev)
+    v4kv.v4kv_decode_attention(q, main, win, seq, case.max_len, case.ratio, case.W, out, workspace,
+                               topk=tk, sm_scale=sm_scale, dev_status=status)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), int(status.item())
+
+
+def check_all(case, got, topk=None, seqs=None, q_round=None):
+    for b in (range(case.B) if seqs is None else seqs):
+        ref = case.oracle(b, None if topk is None else topk[b])
+        assert_close_bf16(got[b], ref, f"seq {b} L={case.lens[b]}")
+
+
+def test_tiny_c4a_bf16_identity_table():
+    # 1 sequence, 1024 raw tokens, 8 heads, bf16 entries, identity table
+    case = DecodeCase(synth.seed_for(0), [1024], 8, 4, main_dtype="bf16", permute=False)
+    got, st = run_decode(case)
+    assert st == 0
+    check_all(case, got)
+
+
+@pytest.mark.parametrize("heads", [1, 8, 16, 64])
+def test_c4a_fp8_shuffled(heads):
+    lens = [1, 2, 127, 128, 129, 255, 256, 257, 1023, 4096 + 3, 9000]
+    case = DecodeCase(101 + heads, lens, heads, 4)
+    got, st = run_decode(case)
+    assert st == 0
+    check_all(case, got)
+
+
+def test_c128a_fp8_shuffled():
+    lens = [131072 + 5, 200000, 128, 129, 1000, 300000]
+    case = DecodeCase(202, lens, 64, 128)
+    got, st = run_decode(case)
+    assert st == 0
+    check_all(case, got)
+
+
+def test_bf16_query():
+    case = DecodeCase(203, [5000, 7777], 64, 4)
+    got, st = run_decode(case, q_dtype=torch.bfloat16)
+    assert st == 0
+    # the oracle sees the same bf16-rounded query
+    case.q = torch.from_numpy(case.q).to(torch.bfloat16).float().numpy()
+    check_all(case, got)
+
+
+def test_topk_selection_with_padding_and_holes():
+    r = synth.rng(204)
+    lens = [6000, 3000, 200]
+    case = DecodeCase(204, lens, 64, 4)
+    k = 512
+    topk = np.full((3, k), -1, dtype=np.int64)
+    for b, L in enumerate(lens):
+        nv = max(0, L - 128) // 4
+        sel = r.permutation(nv)[: min(k, nv)]
+        topk[b, : len(sel)] = sel
+    topk[0, 7] = -1      # a hole in the middle
+    got, st = run_decode(case, topk=topk)
+    assert st == 0
+    check_all(case, got, topk=topk)
+
+
+def test_window_covers_context_is_full_attention():
+    # W >= L: no entry is visible, attention runs over all raw tokens
+    lens = [1, 17, 300, 1000]
+    case = DecodeCase(205, lens, 16, 4, window=1024)
+    got, st = run_decode(case)
+    assert st == 0
+    check_all(case, got)
+
+
+def test_page_permutation_invariance_bitwise():
+    lens = [5000, 12345, 700]
+    a = DecodeCase(206, lens, 64, 4, permute=False)
+    b = DecodeCase(206, lens, 64, 4, permute=True)
+    ga, _ = run_decode(a)
+    gb, _ = run_decode(b)
+    assert np.array_equal(ga, gb)
+
+
+def test_empty_sequence_gives_zeros():
+    case = DecodeCase(207, [0, 500], 8, 4)
+    got, st = run_decode(case)
+    assert st == 0
+    assert np.all(got[0] == 0)
+    check_all(case, got, seqs=[1])
+
+
+def test_bad_page_is_flagged_not_read():
+    case = DecodeCase(208, [3000], 8, 4)
+    case.main.bt[0, 2] = 10_000_000
+    _, st = run_decode(case)
+    assert st & 1
+
+
+def test_out_of_range_topk_index_is_flagged():
+    case = DecodeCase(209, [3000], 8, 4)
+    topk = np.array([[1, 2, 100000, -1]], dtype=np.int64)
+    _, st = run_decode(case, topk=topk)
+    assert st & 4
+
+
+def test_sm_scale_argument():
+    case = DecodeCase(210, [2000], 8, 4)
+    got, _ = run_decode(case, sm_scale=0.2)
+    ref = case.oracle(0, sm_scale=0.2)
+    assert_close_bf16(got[0], ref)

@@ -1,0 +1,80 @@
+"""Parity of v4kv_index_topk (through the C ABI) with the oracle: bit-exact
+indices and reported scores, forced ties, shortfall padding."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import codecs, paging
+from tests.helpers import lay_out, oracle_index
+
+pytestmark = pytest.mark.gpu
+
+
+def build(seed, lens, dup_groups=0, dim=128, ratio=4):
+    r = synth.rng(seed)
+    rows = []
+    for L in lens:
+        n = paging.entry_count(L, ratio)
+        x = synth.normal(r, (n, dim))
+        if dup_groups and n:
+            base = x[: dup_groups].copy()
+            x = base[r.integers(0, dup_groups, n)]
+        rows.append(codecs.quantize_entry(x))
+    pool = lay_out(rows, 256 // ratio, r, "fp8")
+    q = synth.normal(r, (len(lens), dim))
+    return pool, q
+
+
+def run(pool, q, lens, k, ratio=4, W=128):
+    from paged_compressed_kv_b200 import v4kv
+    dev = torch.device("cuda")
+    B = len(lens)
+    max_len = int(max(lens))
+    ws = v4kv.v4kv_workspace_size(v4kv.V4KV_OP_INDEX_TOPK, B, 1, max_len, ratio, W, k,
+                                  v4kv.V4KV_FP8_E4M3, pool.data.shape[2])
+    workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+    topk = torch.empty(B, k, dtype=torch.int32, device=dev)
+    score = torch.empty(B, k, dtype=torch.float32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    v4kv.v4kv_index_topk(torch.from_numpy(q).to(dev), pool.to_cuda(),
+                         torch.tensor(lens, dtype=torch.int32, device=dev), max_len, ratio, W, k,
+                         topk, workspace, score_out=score, dev_status=st)
+    torch.cuda.synchronize()
+    return topk.cpu().numpy(), score.cpu().numpy(), int(st.item())
+
+
+@pytest.mark.parametrize("k", [1, 16, 512, 2048])
+def test_topk_bit_exact(k):
+    lens = [0, 100, 128 + 4 * 300, 4096, 20000, 65536]
+    pool, q = build(300 + k, lens)
+    got, sc, st = run(pool, q, lens, k)
+    assert st == 0
+    for b, L in enumerate(lens):
+        sel, rs = oracle_index(q[b], pool, b, L, 4, 128, k)
+        assert np.array_equal(got[b], sel), f"seq {b}"
+        assert np.array_equal(sc[b].view(np.uint32), rs.view(np.uint32)), f"seq {b}"
+
+
+def test_forced_ties_lowest_index_wins():
+    lens = [8000, 3000]
+    pool, q = build(310, lens, dup_groups=7)
+    got, sc, st = run(pool, q, lens, 512)
+    assert st == 0
+    for b, L in enumerate(lens):
+        sel, rs = oracle_index(q[b], pool, b, L, 4, 128, 512)
+        assert np.array_equal(got[b], sel)
+
+
+def test_full_size_sampled():
+    # the mixed-stack indexer shape: 128 sequences, L ~ U[1K, 256K], k = 512;
+    # the oracle checks a sample of sequences
+    r = synth.rng(synth.seed_for(4))
+    lens = synth.lengths_uniform(r, 128, 1024, 262144, 4)
+    pool, q = build(311, lens.tolist())
+    got, sc, st = run(pool, q, lens.tolist(), 512)
+    assert st == 0
+    for b in [0, int(np.argmax(lens)), int(np.argmin(lens)), 77]:
+        sel, rs = oracle_index(q[b], pool, b, int(lens[b]), 4, 128, 512)
+        assert np.array_equal(got[b], sel)
+        assert np.array_equal(sc[b].view(np.uint32), rs.view(np.uint32))
