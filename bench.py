@@ -45,7 +45,14 @@ def load_peaks():
 
 # ------------------------------------------------------------------ workloads
 
-def decode_config(cfg):
+def decode_config(cfg, seqs=0):
+    c = _decode_config(cfg)
+    if seqs:
+        c["lens"] = c["lens"][:seqs]
+    return c
+
+
+def _decode_config(cfg):
     r = synth.rng(synth.seed_for(cfg))
     if cfg == 1:
         lens = synth.lengths_uniform(r, 64, 4096, 65536, 4)
@@ -66,9 +73,9 @@ def decode_config(cfg):
 class DecodeStep:
     """Device-resident caches and per-step inputs of one decode workload."""
 
-    def __init__(self, cfg, device, seed_offset=0):
+    def __init__(self, cfg, device, seed_offset=0, seqs=0):
         from paged_compressed_kv_b200 import PagedPool, v4kv
-        c = decode_config(cfg)
+        c = decode_config(cfg, seqs)
         self.v4kv = v4kv
         self.name = c["name"]
         self.lens = c["lens"].astype(np.int64)
@@ -264,7 +271,7 @@ def oracle_sample(step, seconds=10.0, max_seqs=None):
 
 def run_ours(args, rank, world, device):
     peak, peak_kind = load_peaks()
-    step = DecodeStep(args.config, device, seed_offset=rank)
+    step = DecodeStep(args.config, device, seed_offset=rank, seqs=args.seqs)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     for _ in range(args.warmup):
@@ -383,7 +390,7 @@ def run_reference(args, rank, world):
     dev = torch.device("cuda", 0) if torch.cuda.is_available() else None
     if dev is None:
         return {"impl": "reference", "unavailable": "needs the workload's caches on a CUDA device"}
-    step = DecodeStep(args.config, dev)
+    step = DecodeStep(args.config, dev, seqs=args.seqs)
     per = max(1, int(args.ref_seqs))
     for _ in range(args.warmup):
         oracle_sample(step, seconds=1e9, max_seqs=1)
@@ -420,6 +427,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seqs", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seqs", type=int, default=0,
+                    help="keep only the first n sequences (small cases for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -51,7 +51,9 @@ def lay_out(rows_per_seq, spb, r, dtype, first_block=None, extra_pages=3, max_bl
         f = 0 if first_block is None else min(first_block[b], nb)
         nblk.append((f, nb))
     total = sum(nb - f for f, nb in nblk) + extra_pages
-    perm = synth.permutation(r, total) if permute else np.arange(total)
+    perm = synth.permutation(r, total)      # drawn either way: same stream after
+    if not permute:
+        perm = np.arange(total)
     mb = max_blocks or max([nb for _, nb in nblk] + [1])
     bt = np.full((B, mb), -1, dtype=np.int32)
     vdt = rows_per_seq[0][0].dtype if rows_per_seq else np.uint8
