@@ -50,6 +50,7 @@ typedef int32_t v4kv_status;
 #define V4KV_DEV_BAD_SLOT 2  /* slot or logical block beyond its table     */
 #define V4KV_DEV_BAD_INDEX 4 /* top-k index outside the stored entries     */
 #define V4KV_DEV_OVERFLOW 8  /* output array too small for what is needed  */
+#define V4KV_DEV_TIMEOUT 16  /* a wait inside a kernel gave up (no progress) */
 
 typedef enum { V4KV_BF16 = 0, V4KV_FP8_E4M3 = 1, V4KV_FP32 = 2 } v4kv_dtype;
 
@@ -216,6 +217,41 @@ v4kv_status v4kv_decode_attention(const void* q, int32_t q_dtype, int32_t batch,
                                   int32_t window_len, const int32_t* topk, int32_t k,
                                   float sm_scale, v4kv_rope rope, void* out, void* workspace,
                                   size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * v4kv_decode_attention_noalloc -- v4kv_decode_attention for callers that
+ * cannot allocate device memory. The paper has no counterpart: this is a
+ * deployment convenience of this library.
+ *
+ * Some callers cannot call cudaMalloc (or any allocator) where they run
+ * decode attention -- for example code that runs inside another framework's
+ * memory pool, or a serving thread that must not synchronise or take an
+ * allocator lock per request -- so they cannot provide the workspace that
+ * v4kv_decode_attention needs. This entry point takes the same arguments
+ * without the workspace and uses a fixed scratch array of
+ * V4KV_NOALLOC_SCRATCH_BYTES that lives in the library's device memory image:
+ * every GPU that loads the library holds it until the process exits. It
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ *   - Sizes: returns V4KV_ERR_INVALID_ARG, launching nothing, when the
+ *     workspace v4kv_workspace_size(V4KV_OP_DECODE, ...) reports for these
+ *     arguments exceeds V4KV_NOALLOC_SCRATCH_BYTES.
+ *   - First call on a device: it looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) with that device current, once per device; make
+ *     that first call before any stream capture.
+ *   - Sharing: all calls on a device share the one scratch array, which keeps
+ *     the last call's contents; nothing in it needs to start at zero (a call
+ *     writes every partial result it reads). Calls that overlap on the GPU
+ *     (other streams, other host threads on the same device) race on the
+ *     scratch and must be serialised by the caller.
+ */
+#define V4KV_NOALLOC_SCRATCH_BYTES (32u << 20)
+v4kv_status v4kv_decode_attention_noalloc(const void* q, int32_t q_dtype, int32_t batch,
+                                          int32_t heads, const v4kv_paged* main_cache,
+                                          const v4kv_paged* window, const int32_t* seq_lens,
+                                          int32_t max_seq_len, int32_t ratio, int32_t window_len,
+                                          const int32_t* topk, int32_t k, float sm_scale,
+                                          v4kv_rope rope, void* out, int32_t* dev_status,
+                                          void* stream);
 
 #define V4KV_OP_INDEX_TOPK 1
 #define V4KV_OP_DECODE 2

@@ -33,7 +33,10 @@ V4KV_OP_DECODE = 2
 EXPORTED = [
     "v4kv_status_string", "v4kv_version", "v4kv_slot_mapping", "v4kv_compress_append",
     "v4kv_index_topk", "v4kv_decode_attention", "v4kv_workspace_size", "v4kv_kv_footprint_bytes",
+    "v4kv_decode_attention_noalloc",
 ]
+
+V4KV_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class V4KVError(RuntimeError):
@@ -79,6 +82,9 @@ def _load():
         "v4kv_decode_attention": (I32, [P, I32, I32, I32, ctypes.POINTER(_Paged),
                                         ctypes.POINTER(_Paged), P, I32, I32, I32, P, I32, F32,
                                         _Rope, P, P, SZ, P, P]),
+        "v4kv_decode_attention_noalloc": (I32, [P, I32, I32, I32, ctypes.POINTER(_Paged),
+                                                ctypes.POINTER(_Paged), P, I32, I32, I32, P, I32,
+                                                F32, _Rope, P, P, P]),
         "v4kv_workspace_size": (I32, [I32, I32, I32, I32, I32, I32, I32, I32, I32,
                                       ctypes.POINTER(SZ)]),
         "v4kv_kv_footprint_bytes": (ctypes.c_uint64, [ctypes.c_uint64, ctypes.POINTER(_Footprint)]),
@@ -242,6 +248,31 @@ def v4kv_decode_attention(q, main, window, seq_lens, max_seq_len, ratio, window_
         _ptr(topk), topk.shape[1] if topk is not None else 0, sm_scale, rope.c(), out.data_ptr(),
         workspace.data_ptr(), workspace.numel(), _ptr(dev_status), _stream(stream))
     _check("v4kv_decode_attention", st)
+
+
+def v4kv_decode_attention_noalloc(q, main, window, seq_lens, max_seq_len, ratio, window_len, out,
+                                  topk=None, sm_scale=None, rope=None, dev_status=None,
+                                  stream=None):
+    """v4kv_decode_attention without a workspace: for callers that cannot
+    allocate device memory. The library's fixed device scratch array
+    (V4KV_NOALLOC_SCRATCH_BYTES, shared by all calls on a device) holds the
+    partial results; sizes needing more scratch are rejected. Overlapping
+    calls on one device race on that scratch."""
+    _need(q, (torch.float32, torch.bfloat16), "q", ndim=3)
+    _need(seq_lens, (torch.int32,), "seq_lens")
+    _need(out, (torch.bfloat16,), "out", ndim=3)
+    if topk is not None:
+        _need(topk, (torch.int32,), "topk", ndim=2)
+    rope = rope or Rope()
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(q.shape[2])
+    mc, wc = main.c(), window.c()
+    st = _lib.v4kv_decode_attention_noalloc(
+        q.data_ptr(), V4KV_FP32 if q.dtype == torch.float32 else V4KV_BF16, q.shape[0], q.shape[1],
+        ctypes.byref(mc), ctypes.byref(wc), seq_lens.data_ptr(), max_seq_len, ratio, window_len,
+        _ptr(topk), topk.shape[1] if topk is not None else 0, sm_scale, rope.c(), out.data_ptr(),
+        _ptr(dev_status), _stream(stream))
+    _check("v4kv_decode_attention_noalloc", st)
 
 
 def v4kv_kv_footprint_bytes(n_tokens, layer_ratios, dim, entry_bits, entry_scale_bytes=0,
