@@ -267,7 +267,9 @@ v4kv_status v4kv_decode_attention(const void* q, int32_t q_dtype, int32_t batch,
   a.split = plan.split;
   a.n_splits = plan.n_splits;
   a.max_len = max_seq_len;
-  cudaError_t e = launch_decode_simt(a, (cudaStream_t)stream);
+  a.pad_sel = plan.path == 1;
+  cudaError_t e = plan.path == 1 ? launch_decode_tc(a, (cudaStream_t)stream)
+                                 : launch_decode_simt(a, (cudaStream_t)stream);
   if (e != cudaSuccess) return V4KV_ERR_CUDA;
   return to_status(launch_decode_merge(a, (cudaStream_t)stream));
 }

@@ -34,7 +34,7 @@ __device__ __forceinline__ SeqItems seq_items(const DecodeArgs& a, int b) {
   s.n_sel = a.topk ? a.k : s.n_vis;
   s.w0 = max(0, s.L - a.window_len);
   s.n_win = s.L - s.w0;
-  s.n_items = s.n_sel + s.n_win;
+  s.n_items = (a.pad_sel ? (s.n_sel + 127) / 128 * 128 : s.n_sel) + s.n_win;
   return s;
 }
 
@@ -251,15 +251,24 @@ DecodePlan plan_decode(int batch, int heads, int max_seq_len, int ratio, int win
   const int L = max(0, max_seq_len);
   const int n_vis = max(0, L - window_len) / ratio;
   const int n_sel = k > 0 ? k : n_vis;
-  p.items_max = n_sel + min(L, window_len);
-  p.path = 0;
-  // aim for about two waves of blocks over the SMs
-  const int head_groups = (heads + kSimtHeads - 1) / kSimtHeads;
-  long long target = (long long)num_sms * 4 / max(1, head_groups);
-  long long total = (long long)p.items_max * batch;
-  long long split = (total + target - 1) / max(1LL, target);
-  split = max(64LL, min(8192LL, ((split + 63) / 64) * 64));
-  p.split = (int)split;
+  const int n_win = min(L, window_len);
+  if (heads == 64) {
+    // tensor-core kernel: items in tiles of 128, entries padded to whole tiles,
+    // one 217 KB block per SM; 16 tiles per split
+    p.path = 1;
+    p.items_max = (n_sel + 127) / 128 * 128 + n_win;
+    p.split = 2048;
+  } else {
+    p.path = 0;
+    p.items_max = n_sel + n_win;
+    // aim for about four blocks per SM over all head groups
+    const int head_groups = (heads + kSimtHeads - 1) / kSimtHeads;
+    long long target = (long long)num_sms * 4 / max(1, head_groups);
+    long long total = (long long)p.items_max * batch;
+    long long split = (total + target - 1) / max(1LL, target);
+    split = max(64LL, min(8192LL, ((split + 63) / 64) * 64));
+    p.split = (int)split;
+  }
   p.n_splits = max(1, (p.items_max + p.split - 1) / p.split);
   p.ws_bytes = (size_t)batch * p.n_splits * heads * (size_t)(kDim + 2) * sizeof(float);
   return p;

@@ -1,0 +1,609 @@
+// Decode attention on the tcgen05 tensor cores for 64 query heads sharing one
+// K = V vector per item (P1 §2.1: shared K/V; §2.3: raw-token window).
+//
+// Per tile of 128 items (entries or window tokens) of one sequence:
+//   S^T[128 x 64] = V[128 x 512] . Q^T          (M = items, N = heads, K = dims)
+//   P' = 2^(S^T * c_j + log2 ks_j - m_h)        (CUDA cores, one thread per item)
+//   O^T[512 x 64] += V^T[512 x 128] . P'^T      (M = dims in 4 tiles of 128)
+// V sits once in shared memory as f16 in 128-byte-swizzled atoms; it is the
+// K-major A operand of the first product and the MN-major A operand of the
+// second. fp8 codes convert to f16 exactly; the entry's fp32 scale ks_j enters
+// the score multiplier c_j and, through log2 ks_j, the exponent, so P' is the
+// weight of the raw code vector. The normaliser is sum_j P'_hj / ks_j.
+// q is scaled per sequence by a power of two into f16 range. m_h is a
+// reference maximum per head, raised only when a score exceeds it by more
+// than 2^8 (P' <= 256), at which point O^T and the partial sums are rescaled.
+//
+// Warp roles (288 threads): warps 0-3 softmax (thread = tile row = TMEM lane),
+// warps 4-7 gather + convert (16-byte coalesced page loads), warp 8 allocates
+// tensor memory and one of its threads issues the MMAs. Each softmax thread
+// keeps its item rows' partial normalisers (one per head) in tensor memory.
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace v4kv {
+
+namespace {
+
+constexpr int kH = 64;          // heads (MMA N)
+constexpr int kD = 512;         // dims
+constexpr int kT = 128;         // items per tile (MMA M of the first product)
+constexpr int kThreads = 288;
+constexpr float kTau = 8.f;     // rescale when a score exceeds the reference by 2^8
+constexpr float kNone = -1e30f; // reference maximum before any item
+
+// shared memory map (bytes from a 1024-aligned base)
+constexpr uint32_t kVOff = 0;                    // 8 dim atoms x 128 rows x 128 B
+constexpr uint32_t kQOff = 131072;               // 8 dim atoms x 64 rows x 128 B
+constexpr uint32_t kPOff = 196608;               // 128 rows x 128 B (64 heads f16)
+constexpr uint32_t kMetaOff = 212992;            // [2][128] fp32 item scales
+constexpr uint32_t kMrefOff = kMetaOff + 1024;   // [64] reference max per head
+constexpr uint32_t kAlphaOff = kMrefOff + 256;   // [64] rescale factors
+constexpr uint32_t kRedOff = kAlphaOff + 256;    // [4][64] per-warp maxima
+constexpr uint32_t kBarOff = kRedOff + 1024;     // mbarriers
+constexpr uint32_t kMiscOff = kBarOff + 256;     // tmem address, flags
+constexpr uint32_t kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
+
+// TMEM columns: S double buffer [0, 128), O^T 4 x 64 at [128, 384), partial
+// normalisers of each lane (64 heads) at [384, 448)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kOCol = 128;
+constexpr uint32_t kLCol = 384;
+
+struct Bars {
+  uint64_t v_full[4];
+  uint64_t v_empty[4];
+  uint64_t s_full[2];
+  uint64_t p_full;
+  uint64_t pv_done;
+  uint64_t drain;
+};
+
+__device__ __forceinline__ int ordered(float f) {
+  int k = __float_as_int(f);
+  return k >= 0 ? k : (k ^ 0x7fffffff);
+}
+__device__ __forceinline__ float unordered(int k) {
+  return __int_as_float(k >= 0 ? k : (k ^ 0x7fffffff));
+}
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ bool named_and(int id, int n, bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred a, b;\n\t"
+      "setp.ne.u32 a, %1, 0;\n\t"
+      "bar.red.and.pred b, %2, %3, a;\n\t"
+      "selp.u32 %0, 1, 0, b;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)p), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ bool named_or(int id, int n, bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred a, b;\n\t"
+      "setp.ne.u32 a, %1, 0;\n\t"
+      "bar.red.or.pred b, %2, %3, a;\n\t"
+      "selp.u32 %0, 1, 0, b;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)p), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                   taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7])
+               : "memory");
+}
+
+struct Seq {
+  int L, n_sel, n_sel_pad, n_win, w0, n_items;
+};
+
+__device__ __forceinline__ Seq seq_of(const DecodeArgs& a, int b, int32_t* st) {
+  Seq s;
+  int L = a.seq_lens[b];
+  if (L > a.max_len) {
+    if (threadIdx.x == 0) flag(st, V4KV_DEV_OVERFLOW);
+    L = a.max_len;
+  }
+  s.L = max(0, L);
+  const int n_vis = max(0, s.L - a.window_len) / a.ratio;
+  s.n_sel = a.topk ? a.k : n_vis;
+  s.n_sel_pad = (s.n_sel + kT - 1) / kT * kT;
+  s.w0 = max(0, s.L - a.window_len);
+  s.n_win = s.L - s.w0;
+  s.n_items = s.n_sel_pad + s.n_win;
+  return s;
+}
+
+// address of item `it` and its scale (0 if the item is skipped)
+__device__ __forceinline__ const uint8_t* item_ptr(const DecodeArgs& a, int b, const Seq& s, int it,
+                                                   float* ks) {
+  *ks = 0.f;
+  if (it < s.n_sel_pad) {
+    if (it >= s.n_sel) return nullptr;
+    const long long j = a.topk ? (long long)a.topk[(size_t)b * a.k + it] : (long long)it;
+    if (j < 0) return nullptr;
+    if (j >= ((long long)s.L + a.ratio - 1) / a.ratio) {
+      flag(a.dev_status, V4KV_DEV_BAD_INDEX);
+      return nullptr;
+    }
+    const int p = page_of(a.main.block_table + (size_t)b * a.main.max_blocks, a.main.max_blocks, j,
+                          a.main.spb, a.main.num_pages, a.dev_status);
+    if (p < 0) return nullptr;
+    const long long slot = (long long)p * a.main.spb + j % a.main.spb;
+    const bool fp8 = a.main.dtype == V4KV_FP8_E4M3;
+    *ks = fp8 ? a.main.scales[slot] : 1.f;
+    return reinterpret_cast<const uint8_t*>(a.main.data) + slot * (fp8 ? kD : 2 * kD);
+  }
+  const int w = it - s.n_sel_pad;
+  if (w >= s.n_win) return nullptr;
+  const long long t = s.w0 + w;
+  const int p = page_of(a.window.block_table + (size_t)b * a.window.max_blocks, a.window.max_blocks,
+                        t, a.window.spb, a.window.num_pages, a.dev_status);
+  if (p < 0) return nullptr;
+  const long long slot = (long long)p * a.window.spb + t % a.window.spb;
+  const bool fp8 = a.window.dtype == V4KV_FP8_E4M3;
+  *ks = fp8 ? a.window.scales[slot] : 1.f;
+  return reinterpret_cast<const uint8_t*>(a.window.data) + slot * (fp8 ? kD : 2 * kD);
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const uint8_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
+// 16 fp8 codes -> 16 f16 values as two 16-byte halves
+__device__ __forceinline__ void fp8x16_to_f16(uint4 raw, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    o[2 * i] = h2u(e4m3x2_to_half2((uint16_t)(w[i] & 0xffffu)));
+    o[2 * i + 1] = h2u(e4m3x2_to_half2((uint16_t)(w[i] >> 16)));
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// 8 bf16 -> 8 f16 (round to nearest, saturating to the f16 range)
+__device__ __forceinline__ uint4 bf16x8_to_f16(uint4 raw) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float a = __uint_as_float(w[i] << 16), b = __uint_as_float(w[i] & 0xffff0000u);
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    o[i] = r;
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = tc::smem_u32(smem_raw);
+  const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
+  uint8_t* sm = smem_raw + pad;
+  const uint32_t sbase = raw_addr + pad;
+  Bars* bars = reinterpret_cast<Bars*>(sm + kBarOff);
+  float* meta = reinterpret_cast<float*>(sm + kMetaOff);
+  float* mref = reinterpret_cast<float*>(sm + kMrefOff);
+  float* alpha = reinterpret_cast<float*>(sm + kAlphaOff);
+  float* red = reinterpret_cast<float*>(sm + kRedOff);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kMiscOff + 4);
+  float* k0_slot = reinterpret_cast<float*>(sm + kMiscOff + 8);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.y, split = blockIdx.x;
+  const Seq s = seq_of(a, b, a.dev_status);
+  const int i0 = split * a.split;
+  if (i0 >= s.n_items) return;
+  const int i1 = min(s.n_items, i0 + a.split);
+  const int n_tiles = (i1 - i0 + kT - 1) / kT;
+
+  if (tid == 0) {
+    for (int c = 0; c < 4; ++c) {
+      tc::mbar_init(&bars->v_full[c], 128);
+      tc::mbar_init(&bars->v_empty[c], 1);
+    }
+    tc::mbar_init(&bars->s_full[0], 1);
+    tc::mbar_init(&bars->s_full[1], 1);
+    tc::mbar_init(&bars->p_full, 128);
+    tc::mbar_init(&bars->pv_done, 1);
+    tc::mbar_init(&bars->drain, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 8) tc::tmem_alloc(tmem_slot, kTmemCols);
+  if (tid < kH) mref[tid] = kNone;
+
+  // ---- q -> f16, scaled by 2^e so that max|q| * 2^e < 2^15 (warps 0-7)
+  if (warp < 8) {
+    const size_t qoff = (size_t)b * kH * kD;
+    float m = 0.f;
+    for (int u = tid; u < kH * kD / 8; u += 256) {
+      const size_t o = qoff + (size_t)u * 8;
+      if (a.q_dtype == V4KV_FP32) {
+        const float4 x0 = reinterpret_cast<const float4*>(a.q)[o / 4];
+        const float4 x1 = reinterpret_cast<const float4*>(a.q)[o / 4 + 1];
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(x0.x), fabsf(x0.y)), fmaxf(fabsf(x0.z), fabsf(x0.w))));
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(x1.x), fabsf(x1.y)), fmaxf(fabsf(x1.z), fabsf(x1.w))));
+      } else {
+        const uint4 r = reinterpret_cast<const uint4*>(a.q)[o / 8];
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xffff0000u))));
+      }
+    }
+    m = warp_max(m);
+    if (lane == 0) red[warp] = m;
+    named_sync(2, 256);
+    float amax = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) amax = fmaxf(amax, red[w]);
+    int e = 0;
+    if (amax > 0.f) {
+      int k;
+      frexpf(amax, &k);  // amax < 2^k
+      e = 15 - k;
+    }
+    const float qs = ldexpf(1.f, e);
+    if (tid == 0) *k0_slot = a.sm_scale * 1.4426950408889634f * ldexpf(1.f, -e);
+    for (int u = tid; u < kH * kD / 8; u += 256) {
+      const int h = u / (kD / 8), c8 = u % (kD / 8);  // 8-dim chunk c8 of head h
+      const size_t o = qoff + (size_t)h * kD + c8 * 8;
+      float x[8];
+      if (a.q_dtype == V4KV_FP32) {
+        const float4 x0 = reinterpret_cast<const float4*>(a.q)[o / 4];
+        const float4 x1 = reinterpret_cast<const float4*>(a.q)[o / 4 + 1];
+        x[0] = x0.x; x[1] = x0.y; x[2] = x0.z; x[3] = x0.w;
+        x[4] = x1.x; x[5] = x1.y; x[6] = x1.z; x[7] = x1.w;
+      } else {
+        const uint4 r = reinterpret_cast<const uint4*>(a.q)[o / 8];
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          x[2 * i] = __uint_as_float(w[i] << 16);
+          x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+      }
+      uint32_t hv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) hv[i] = h2u(__floats2half2_rn(x[2 * i] * qs, x[2 * i + 1] * qs));
+      *reinterpret_cast<uint4*>(sm + kQOff + (c8 >> 3) * 8192 + tc::sw128_off(h, c8 & 7)) =
+          make_uint4(hv[0], hv[1], hv[2], hv[3]);
+    }
+    tc::fence_proxy_async_smem();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ======================= MMA issuer
+    if (lane == 0) {
+      const uint32_t iq = tc::idesc_f16(128, kH, 0, 0);
+      const uint32_t ip = tc::idesc_f16(128, kH, 1, 1);
+      bool ok = true;
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        const uint32_t par = i & 1;
+        const uint32_t s_col = (uint32_t)(i & 1) * kH;
+        for (int c = 0; c < 4 && ok; ++c) {
+          ok = tc::mbar_wait(&bars->v_full[c], par, abort_flag);
+          if (!ok) break;
+          tc::tc_fence_after();
+          for (int kk = 8 * c; kk < 8 * c + 8; ++kk) {
+            const uint64_t ad = tc::sw128_desc(sbase + kVOff + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = tc::sw128_desc(sbase + kQOff + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+            tc::mma_f16(tmem + s_col, ad, bd, iq, kk > 0 ? 1u : 0u);
+          }
+        }
+        if (!ok) break;
+        tc::mma_commit(&bars->s_full[i & 1]);
+        ok = tc::mbar_wait(&bars->p_full, par, abort_flag);
+        if (!ok) break;
+        tc::tc_fence_after();
+        for (int mt = 0; mt < 4; ++mt) {
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t ad = tc::sw128_desc(sbase + kVOff + 2 * mt * 16384 + kk * 2048, 16384, 1024);
+            const uint64_t bd = tc::sw128_desc(sbase + kPOff + kk * 2048, 0, 1024);
+            tc::mma_f16(tmem + kOCol + kH * mt, ad, bd, ip, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc::mma_commit(&bars->v_empty[mt]);
+        }
+        tc::mma_commit(&bars->pv_done);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        flag(a.dev_status, V4KV_DEV_TIMEOUT);
+      }
+      // every MMA issued has completed once this barrier flips; this wait
+      // ignores the abort flag (tensor memory is freed after it)
+      volatile int never = 0;
+      tc::mma_commit(&bars->drain);
+      if (!tc::mbar_wait(&bars->drain, 0, &never)) flag(a.dev_status, V4KV_DEV_TIMEOUT);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ======================= gather + convert
+    const int cw = warp - 4;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int tile0 = i0 + i * kT;
+      const bool entries = tile0 < s.n_sel_pad;
+      const bool fp8 = (entries ? a.main.dtype : a.window.dtype) == V4KV_FP8_E4M3;
+      float* mt = meta + (i & 1) * kT;
+      if (fp8) {
+        // lane covers rows 32cw + 4r + lane/8 (r = 0..7), 16 bytes at 16*(lane%8)
+        // of each 128-byte dim chunk
+        const uint8_t* ptr[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int row = 32 * cw + 4 * r + (lane >> 3);
+          float ks;
+          ptr[r] = item_ptr(a, b, s, tile0 + row, &ks);
+          if ((lane & 7) == 0) mt[row] = ptr[r] ? ks : 0.f;
+        }
+        uint4 rawv[4][8];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int r = 0; r < 8; ++r)
+            rawv[c][r] = ptr[r] ? ldg_stream(ptr[r] + 128 * c + 16 * (lane & 7)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (i > 0 && !tc::mbar_wait(&bars->v_empty[c], (i - 1) & 1, abort_flag)) goto conv_abort;
+          const int part = lane & 7;                 // 16-dim piece within the chunk
+          const uint32_t atom = 2 * c + (part >> 2);
+          const uint32_t q = 2 * (part & 3);
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            const uint32_t row = 32 * cw + 4 * r + (lane >> 3);
+            uint4 lo, hi;
+            fp8x16_to_f16(rawv[c][r], lo, hi);
+            uint8_t* base = sm + kVOff + atom * 16384;
+            if (part & 4) {
+              *reinterpret_cast<uint4*>(base + tc::sw128_off(row, q + 1)) = hi;
+              *reinterpret_cast<uint4*>(base + tc::sw128_off(row, q)) = lo;
+            } else {
+              *reinterpret_cast<uint4*>(base + tc::sw128_off(row, q)) = lo;
+              *reinterpret_cast<uint4*>(base + tc::sw128_off(row, q + 1)) = hi;
+            }
+          }
+          tc::fence_proxy_async_smem();
+          tc::mbar_arrive(&bars->v_full[c]);
+        }
+      } else {
+        // bf16 rows: lane covers rows 32cw + 2r + lane/16 (r = 0..15), 16 bytes at
+        // 16*(lane%16) of each 256-byte dim chunk
+        const uint8_t* ptr[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const int row = 32 * cw + 2 * r + (lane >> 4);
+          float ks;
+          ptr[r] = item_ptr(a, b, s, tile0 + row, &ks);
+          if ((lane & 15) == 0) mt[row] = ptr[r] ? ks : 0.f;
+        }
+        for (int c = 0; c < 4; ++c) {
+          uint4 rawv[16];
+#pragma unroll
+          for (int r = 0; r < 16; ++r)
+            rawv[r] = ptr[r] ? ldg_stream(ptr[r] + 256 * c + 16 * (lane & 15)) : make_uint4(0, 0, 0, 0);
+          if (i > 0 && !tc::mbar_wait(&bars->v_empty[c], (i - 1) & 1, abort_flag)) goto conv_abort;
+          const int part = lane & 15;                // 8-dim piece within the chunk
+          const uint32_t atom = 2 * c + (part >> 3);
+#pragma unroll
+          for (int r = 0; r < 16; ++r) {
+            const uint32_t row = 32 * cw + 2 * r + (lane >> 4);
+            *reinterpret_cast<uint4*>(sm + kVOff + atom * 16384 + tc::sw128_off(row, part & 7)) =
+                bf16x8_to_f16(rawv[r]);
+          }
+          tc::fence_proxy_async_smem();
+          tc::mbar_arrive(&bars->v_full[c]);
+        }
+      }
+    }
+  conv_abort:;
+  } else {
+    // ======================= softmax (thread = tile row = TMEM lane)
+    const int row = tid;
+    const float k0 = *k0_slot;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+    {
+      uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+      for (int c = 0; c < 8; ++c) tmem_st8(lane_base + kLCol + 8 * c, z);
+      tc::tmem_wait_st();
+    }
+    bool ok = true;
+    for (int i = 0; i < n_tiles && ok; ++i) {
+      // S(i) complete implies PV(i-1) complete (the MMAs run in issue order),
+      // so waiting for pv_done(i-1) here costs nothing and frees P and O^T
+      ok = tc::mbar_wait(&bars->v_full[0], i & 1, abort_flag) &&
+           tc::mbar_wait(&bars->s_full[i & 1], (i >> 1) & 1, abort_flag) &&
+           (i == 0 || tc::mbar_wait(&bars->pv_done, (i - 1) & 1, abort_flag));
+      // the four softmax warps leave together (they meet at named barriers)
+      ok = named_and(1, 128, ok);
+      if (!ok) break;
+      tc::tc_fence_after();
+      const float ks = meta[(i & 1) * kT + row];
+      const bool valid = ks > 0.f;
+      const float cj = valid ? k0 * ks : 0.f;
+      const float lk = valid ? __log2f(ks) : -INFINITY;
+      const float inv_k = valid ? __frcp_rn(ks) : 0.f;
+      float u[kH];
+      {
+        uint32_t r32[32];
+        tc::tmem_ld32(lane_base + (uint32_t)(i & 1) * kH, r32);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 32; ++h) u[h] = fmaf(__uint_as_float(r32[h]), cj, lk);
+        tc::tmem_ld32(lane_base + (uint32_t)(i & 1) * kH + 32, r32);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 32; ++h) u[32 + h] = fmaf(__uint_as_float(r32[h]), cj, lk);
+      }
+      bool need = false;
+#pragma unroll
+      for (int h = 0; h < kH; ++h) need |= u[h] > mref[h] + kTau;
+      if (named_or(1, 128, need)) {
+        // raise the reference to the running maximum of every head
+#pragma unroll
+        for (int h = 0; h < kH; ++h) {
+          const int wm = __reduce_max_sync(0xffffffffu, ordered(u[h]));
+          if (lane == 0) red[warp * kH + h] = unordered(wm);
+        }
+        named_sync(1, 128);
+        if (row < kH) {
+          const float old = mref[row];
+          float nm = old;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) nm = fmaxf(nm, red[w * kH + row]);
+          alpha[row] = exp2f(old - nm);
+          mref[row] = nm;
+        }
+        named_sync(1, 128);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t lv[8];
+          tmem_ld8(lane_base + kLCol + 8 * c, lv);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 8; ++e) lv[e] = __float_as_uint(__uint_as_float(lv[e]) * alpha[8 * c + e]);
+          tmem_st8(lane_base + kLCol + 8 * c, lv);
+        }
+        tc::tmem_wait_st();
+        if (i > 0) {
+          // O^T rows of this lane (dims 128 mt + row) times alpha per head column
+#pragma unroll 1
+          for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+              uint32_t r32[32];
+              const uint32_t ta = lane_base + kOCol + kH * mt + 32 * half;
+              tc::tmem_ld32(ta, r32);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int h = 0; h < 32; ++h)
+                r32[h] = __float_as_uint(__uint_as_float(r32[h]) * alpha[32 * half + h]);
+              tc::tmem_st32(ta, r32);
+            }
+          }
+          tc::tmem_wait_st();
+        }
+      }
+      // P' row of this item: 64 heads in f16, MN-major swizzled, 8 heads per chunk
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t pk[4], lv[8];
+        tmem_ld8(lane_base + kLCol + 8 * c, lv);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int h = 8 * c + 2 * e;
+          const float p0 = exp2f(u[h] - mref[h]);
+          const float p1 = exp2f(u[h + 1] - mref[h + 1]);
+          lv[2 * e] = __float_as_uint(fmaf(p0, inv_k, __uint_as_float(lv[2 * e])));
+          lv[2 * e + 1] = __float_as_uint(fmaf(p1, inv_k, __uint_as_float(lv[2 * e + 1])));
+          pk[e] = h2u(__floats2half2_rn(p0, p1));
+        }
+        tmem_st8(lane_base + kLCol + 8 * c, lv);
+        *reinterpret_cast<uint4*>(sm + kPOff + tc::sw128_off(row, c)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      tc::tmem_wait_st();
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&bars->p_full);
+    }
+    if (ok) ok = tc::mbar_wait(&bars->pv_done, (n_tiles - 1) & 1, abort_flag);
+    ok = named_and(1, 128, ok);
+    if (!ok) {
+      *abort_flag = 1;
+      flag(a.dev_status, V4KV_DEV_TIMEOUT);
+    } else {
+      tc::tc_fence_after();
+      // O^T -> partial output (un-normalised, relative to the reference max)
+      const size_t prow = ((size_t)b * a.n_splits + split) * kH;
+#pragma unroll 1
+      for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          uint32_t r32[32];
+          tc::tmem_ld32(lane_base + kOCol + kH * mt + 32 * half, r32);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < 32; ++h)
+            a.part_o[(prow + 32 * half + h) * kD + 128 * mt + row] = __uint_as_float(r32[h]);
+        }
+      }
+      // partial sums of the normaliser: reduce over the 128 rows per head
+      float* lred = reinterpret_cast<float*>(sm + kVOff);
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t lv[8];
+        tmem_ld8(lane_base + kLCol + 8 * c, lv);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 8; ++e) lred[(8 * c + e) * 129 + row] = __uint_as_float(lv[e]);
+      }
+      named_sync(1, 128);
+      if (row < kH) {
+        float l = 0.f;
+        for (int r = 0; r < kT; ++r) l += lred[row * 129 + r];
+        a.part_ml[(prow + row) * 2] = mref[row];
+        a.part_ml[(prow + row) * 2 + 1] = l;
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc::tc_fence_after();
+    tc::tmem_free(tmem, kTmemCols);
+  }
+}
+
+size_t decode_tc_smem_bytes() { return kSmemBytes; }
+
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid(a.n_splits, a.batch);
+  decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace v4kv

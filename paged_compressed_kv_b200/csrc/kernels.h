@@ -94,6 +94,7 @@ struct DecodeArgs {
   int split;
   int n_splits;
   int max_len;  // host bound on seq_lens; longer sequences are clamped and flagged
+  int pad_sel;  // 1: entries are padded to a multiple of 128 items (tensor-core path)
 };
 
 cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, int batch,
@@ -110,5 +111,6 @@ DecodePlan plan_decode(int batch, int heads, int max_seq_len, int ratio, int win
                        int main_dtype, int dim, int num_sms);
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
 
 }  // namespace v4kv
