@@ -29,7 +29,7 @@ namespace {
 constexpr int kH = 64;          // heads (MMA N)
 constexpr int kD = 512;         // dims
 constexpr int kT = 128;         // items per tile (MMA M of the first product)
-constexpr int kThreads = 288;
+constexpr int kThreads = 320;
 constexpr float kTau = 8.f;     // rescale when a score exceeds the reference by 2^8
 constexpr float kNone = -1e30f; // reference maximum before any item
 
@@ -37,8 +37,9 @@ constexpr float kNone = -1e30f; // reference maximum before any item
 constexpr uint32_t kVOff = 0;                    // 8 dim atoms x 128 rows x 128 B
 constexpr uint32_t kQOff = 131072;               // 8 dim atoms x 64 rows x 128 B
 constexpr uint32_t kPOff = 196608;               // 128 rows x 128 B (64 heads f16)
-constexpr uint32_t kMetaOff = 212992;            // [2][128] fp32 item scales
-constexpr uint32_t kMrefOff = kMetaOff + 1024;   // [64] reference max per head
+constexpr uint32_t kMetaOff = 212992;            // [3][128] fp32 item scales (0 = skip)
+constexpr uint32_t kPtrOff = kMetaOff + 1536;    // [3][128] item row addresses
+constexpr uint32_t kMrefOff = kPtrOff + 3072;    // [64] reference max per head
 constexpr uint32_t kAlphaOff = kMrefOff + 256;   // [64] rescale factors
 constexpr uint32_t kRedOff = kAlphaOff + 256;    // [4][64] per-warp maxima
 constexpr uint32_t kBarOff = kRedOff + 1024;     // mbarriers
@@ -52,6 +53,8 @@ constexpr uint32_t kOCol = 128;
 constexpr uint32_t kLCol = 384;
 
 struct Bars {
+  uint64_t addr_ready[3];
+  uint64_t addr_free[3];
   uint64_t v_full[4];
   uint64_t v_empty[4];
   uint64_t s_full[2];
@@ -59,6 +62,13 @@ struct Bars {
   uint64_t pv_done;
   uint64_t drain;
 };
+
+// 2^x on the special-function unit (ftz: results below 2^-126 become 0)
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ int ordered(float f) {
   int k = __float_as_int(f);
@@ -132,36 +142,78 @@ __device__ __forceinline__ Seq seq_of(const DecodeArgs& a, int b, int32_t* st) {
   return s;
 }
 
-// address of item `it` and its scale (0 if the item is skipped)
+// Address of item `it` and its scale; nullptr (scale 0) if the item is
+// skipped. Problems are returned as V4KV_DEV_* bits in *err instead of being
+// flagged here, so that the loads of several items can overlap.
 __device__ __forceinline__ const uint8_t* item_ptr(const DecodeArgs& a, int b, const Seq& s, int it,
-                                                   float* ks) {
+                                                   float* ks, int* err) {
   *ks = 0.f;
+  long long j;
+  bool main_item;
   if (it < s.n_sel_pad) {
     if (it >= s.n_sel) return nullptr;
-    const long long j = a.topk ? (long long)a.topk[(size_t)b * a.k + it] : (long long)it;
+    j = a.topk ? (long long)a.topk[(size_t)b * a.k + it] : (long long)it;
     if (j < 0) return nullptr;
     if (j >= ((long long)s.L + a.ratio - 1) / a.ratio) {
-      flag(a.dev_status, V4KV_DEV_BAD_INDEX);
+      *err |= V4KV_DEV_BAD_INDEX;
       return nullptr;
     }
-    const int p = page_of(a.main.block_table + (size_t)b * a.main.max_blocks, a.main.max_blocks, j,
-                          a.main.spb, a.main.num_pages, a.dev_status);
-    if (p < 0) return nullptr;
-    const long long slot = (long long)p * a.main.spb + j % a.main.spb;
-    const bool fp8 = a.main.dtype == V4KV_FP8_E4M3;
-    *ks = fp8 ? a.main.scales[slot] : 1.f;
-    return reinterpret_cast<const uint8_t*>(a.main.data) + slot * (fp8 ? kD : 2 * kD);
+    main_item = true;
+  } else {
+    const int w = it - s.n_sel_pad;
+    if (w >= s.n_win) return nullptr;
+    j = s.w0 + w;
+    main_item = false;
   }
-  const int w = it - s.n_sel_pad;
-  if (w >= s.n_win) return nullptr;
-  const long long t = s.w0 + w;
-  const int p = page_of(a.window.block_table + (size_t)b * a.window.max_blocks, a.window.max_blocks,
-                        t, a.window.spb, a.window.num_pages, a.dev_status);
-  if (p < 0) return nullptr;
-  const long long slot = (long long)p * a.window.spb + t % a.window.spb;
-  const bool fp8 = a.window.dtype == V4KV_FP8_E4M3;
-  *ks = fp8 ? a.window.scales[slot] : 1.f;
-  return reinterpret_cast<const uint8_t*>(a.window.data) + slot * (fp8 ? kD : 2 * kD);
+  const int spb = main_item ? a.main.spb : a.window.spb;
+  const int max_blocks = main_item ? a.main.max_blocks : a.window.max_blocks;
+  const int num_pages = main_item ? a.main.num_pages : a.window.num_pages;
+  const int32_t* bt = main_item ? a.main.block_table : a.window.block_table;
+  const bool fp8 = (main_item ? a.main.dtype : a.window.dtype) == V4KV_FP8_E4M3;
+  const long long blk = j / spb;
+  if (blk >= max_blocks) {
+    *err |= V4KV_DEV_BAD_SLOT;
+    return nullptr;
+  }
+  const int p = bt[(size_t)b * max_blocks + blk];
+  if (p < 0 || p >= num_pages) {
+    *err |= V4KV_DEV_BAD_PAGE;
+    return nullptr;
+  }
+  const long long slot = (long long)p * spb + j % spb;
+  const float* scales = main_item ? a.main.scales : a.window.scales;
+  const void* data = main_item ? a.main.data : a.window.data;
+  *ks = fp8 ? scales[slot] : 1.f;
+  return reinterpret_cast<const uint8_t*>(data) + slot * (fp8 ? kD : 2 * kD);
+}
+
+__device__ __forceinline__ void prefetch_l2_line(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// Address warp: lane l resolves rows l, l+32, l+64, l+96 of the tile that
+// starts at item tile0 into the row-address and scale tables, then asks L2 for
+// the rows' cache lines so that the converters' loads find them there.
+__device__ __forceinline__ void resolve_tile(const DecodeArgs& a, int b, const Seq& s, int tile0,
+                                             int lane, const uint8_t** rp, float* ms) {
+  int err = 0;
+  const uint8_t* p[4];
+  float ks[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) p[r] = item_ptr(a, b, s, tile0 + lane + 32 * r, &ks[r], &err);
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    rp[lane + 32 * r] = p[r];
+    ms[lane + 32 * r] = p[r] ? ks[r] : 0.f;
+  }
+  const bool main_tile = tile0 < s.n_sel_pad;
+  const bool fp8 = (main_tile ? a.main.dtype : a.window.dtype) == V4KV_FP8_E4M3;
+  const int lines = fp8 ? kD / 128 : 2 * kD / 128;
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+    if (p[r])
+      for (int k = 0; k < lines; ++k) prefetch_l2_line(p[r] + 128 * k);
+  if (err) flag(a.dev_status, err);
 }
 
 __device__ __forceinline__ uint4 ldg_stream(const uint8_t* p) {
@@ -211,6 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   const uint32_t sbase = raw_addr + pad;
   Bars* bars = reinterpret_cast<Bars*>(sm + kBarOff);
   float* meta = reinterpret_cast<float*>(sm + kMetaOff);
+  const uint8_t** rowptr = reinterpret_cast<const uint8_t**>(sm + kPtrOff);
   float* mref = reinterpret_cast<float*>(sm + kMrefOff);
   float* alpha = reinterpret_cast<float*>(sm + kAlphaOff);
   float* red = reinterpret_cast<float*>(sm + kRedOff);
@@ -227,6 +280,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   const int n_tiles = (i1 - i0 + kT - 1) / kT;
 
   if (tid == 0) {
+    for (int k = 0; k < 3; ++k) {
+      tc::mbar_init(&bars->addr_ready[k], 32);
+      tc::mbar_init(&bars->addr_free[k], 256);
+    }
     for (int c = 0; c < 4; ++c) {
       tc::mbar_init(&bars->v_full[c], 128);
       tc::mbar_init(&bars->v_empty[c], 1);
@@ -306,7 +363,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == 9) {
+    // ======================= address resolution + L2 prefetch, two tiles ahead
+    for (int t = 0; t < n_tiles; ++t) {
+      const int buf = t % 3;
+      if (t >= 3 && !tc::mbar_wait(&bars->addr_free[buf], ((t - 3) / 3) & 1, abort_flag)) break;
+      resolve_tile(a, b, s, i0 + t * kT, lane, rowptr + buf * kT, meta + buf * kT);
+      __syncwarp();
+      tc::mbar_arrive(&bars->addr_ready[buf]);
+    }
+  } else if (warp == 8) {
     // ======================= MMA issuer
     if (lane == 0) {
       const uint32_t iq = tc::idesc_f16(128, kH, 0, 0);
@@ -353,29 +419,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
     __syncwarp();
   } else if (warp >= 4) {
     // ======================= gather + convert
+    // Warp cw owns rows [32 cw, 32 cw + 32) of every tile. Lane l resolves row
+    // 32 cw + l of the next tile while the current one is loaded and converted.
     const int cw = warp - 4;
     for (int i = 0; i < n_tiles; ++i) {
+      if (!tc::mbar_wait(&bars->addr_ready[i % 3], (i / 3) & 1, abort_flag)) goto conv_abort;
       const int tile0 = i0 + i * kT;
       const bool entries = tile0 < s.n_sel_pad;
       const bool fp8 = (entries ? a.main.dtype : a.window.dtype) == V4KV_FP8_E4M3;
-      float* mt = meta + (i & 1) * kT;
+      const uint8_t** rp = rowptr + (i % 3) * kT;
       if (fp8) {
         // lane covers rows 32cw + 4r + lane/8 (r = 0..7), 16 bytes at 16*(lane%8)
         // of each 128-byte dim chunk
-        const uint8_t* ptr[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          const int row = 32 * cw + 4 * r + (lane >> 3);
-          float ks;
-          ptr[r] = item_ptr(a, b, s, tile0 + row, &ks);
-          if ((lane & 7) == 0) mt[row] = ptr[r] ? ks : 0.f;
-        }
         uint4 rawv[4][8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int r = 0; r < 8; ++r) {
+          const uint8_t* p = rp[32 * cw + 4 * r + (lane >> 3)];
 #pragma unroll
-          for (int r = 0; r < 8; ++r)
-            rawv[c][r] = ptr[r] ? ldg_stream(ptr[r] + 128 * c + 16 * (lane & 7)) : make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < 4; ++c)
+            rawv[c][r] = p ? ldg_stream(p + 128 * c + 16 * (lane & 7)) : make_uint4(0, 0, 0, 0);
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           if (i > 0 && !tc::mbar_wait(&bars->v_empty[c], (i - 1) & 1, abort_flag)) goto conv_abort;
@@ -404,12 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
         // 16*(lane%16) of each 256-byte dim chunk
         const uint8_t* ptr[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          const int row = 32 * cw + 2 * r + (lane >> 4);
-          float ks;
-          ptr[r] = item_ptr(a, b, s, tile0 + row, &ks);
-          if ((lane & 15) == 0) mt[row] = ptr[r] ? ks : 0.f;
-        }
+        for (int r = 0; r < 16; ++r) ptr[r] = rp[32 * cw + 2 * r + (lane >> 4)];
         for (int c = 0; c < 4; ++c) {
           uint4 rawv[16];
 #pragma unroll
@@ -428,6 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
           tc::mbar_arrive(&bars->v_full[c]);
         }
       }
+      tc::mbar_arrive(&bars->addr_free[i % 3]);
     }
   conv_abort:;
   } else {
@@ -452,31 +511,56 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       ok = named_and(1, 128, ok);
       if (!ok) break;
       tc::tc_fence_after();
-      const float ks = meta[(i & 1) * kT + row];
+      const float ks = meta[(i % 3) * kT + row];
+      tc::mbar_arrive(&bars->addr_free[i % 3]);
       const bool valid = ks > 0.f;
       const float cj = valid ? k0 * ks : 0.f;
       const float lk = valid ? __log2f(ks) : -INFINITY;
       const float inv_k = valid ? __frcp_rn(ks) : 0.f;
-      float u[kH];
+      // u = score in log2 units including log2 ks; d = u - m_ref (in place)
+      float d[kH];
+      const uint32_t s_addr = lane_base + (uint32_t)(i & 1) * kH;
       {
         uint32_t r32[32];
-        tc::tmem_ld32(lane_base + (uint32_t)(i & 1) * kH, r32);
+        tc::tmem_ld32(s_addr, r32);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < 32; ++h) u[h] = fmaf(__uint_as_float(r32[h]), cj, lk);
-        tc::tmem_ld32(lane_base + (uint32_t)(i & 1) * kH + 32, r32);
+        for (int h = 0; h < 32; ++h) d[h] = fmaf(__uint_as_float(r32[h]), cj, lk);
+        tc::tmem_ld32(s_addr + 32, r32);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < 32; ++h) u[32 + h] = fmaf(__uint_as_float(r32[h]), cj, lk);
+        for (int h = 0; h < 32; ++h) d[32 + h] = fmaf(__uint_as_float(r32[h]), cj, lk);
       }
-      bool need = false;
+      float dmax = -INFINITY;
+      {
+        const float4* mr4 = reinterpret_cast<const float4*>(mref);
 #pragma unroll
-      for (int h = 0; h < kH; ++h) need |= u[h] > mref[h] + kTau;
-      if (named_or(1, 128, need)) {
-        // raise the reference to the running maximum of every head
+        for (int h4 = 0; h4 < kH / 4; ++h4) {
+          const float4 m4 = mr4[h4];
+          d[4 * h4] -= m4.x;
+          d[4 * h4 + 1] -= m4.y;
+          d[4 * h4 + 2] -= m4.z;
+          d[4 * h4 + 3] -= m4.w;
+          dmax = fmaxf(dmax, fmaxf(fmaxf(d[4 * h4], d[4 * h4 + 1]), fmaxf(d[4 * h4 + 2], d[4 * h4 + 3])));
+        }
+      }
+      if (named_or(1, 128, dmax > kTau)) {
+        // rare: raise the reference of every head to its running maximum.
+        // u is recomputed from S (still in tensor memory) to keep it exact.
+        {
+          uint32_t r32[32];
+          tc::tmem_ld32(s_addr, r32);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < 32; ++h) d[h] = fmaf(__uint_as_float(r32[h]), cj, lk);
+          tc::tmem_ld32(s_addr + 32, r32);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < 32; ++h) d[32 + h] = fmaf(__uint_as_float(r32[h]), cj, lk);
+        }
 #pragma unroll
         for (int h = 0; h < kH; ++h) {
-          const int wm = __reduce_max_sync(0xffffffffu, ordered(u[h]));
+          const int wm = __reduce_max_sync(0xffffffffu, ordered(d[h]));
           if (lane == 0) red[warp * kH + h] = unordered(wm);
         }
         named_sync(1, 128);
@@ -490,13 +574,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
         }
         named_sync(1, 128);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t lv[8];
-          tmem_ld8(lane_base + kLCol + 8 * c, lv);
+        for (int h = 0; h < kH; ++h) d[h] -= mref[h];
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          uint32_t lv[32];
+          tc::tmem_ld32(lane_base + kLCol + 32 * half, lv);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 8; ++e) lv[e] = __float_as_uint(__uint_as_float(lv[e]) * alpha[8 * c + e]);
-          tmem_st8(lane_base + kLCol + 8 * c, lv);
+          for (int e = 0; e < 32; ++e)
+            lv[e] = __float_as_uint(__uint_as_float(lv[e]) * alpha[32 * half + e]);
+          tc::tmem_st32(lane_base + kLCol + 32 * half, lv);
         }
         tc::tmem_wait_st();
         if (i > 0) {
@@ -518,24 +605,30 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
           tc::tmem_wait_st();
         }
       }
-      // P' row of this item: 64 heads in f16, MN-major swizzled, 8 heads per chunk
+      // P' row of this item: 64 heads in f16, MN-major swizzled, 8 heads per
+      // 16-byte chunk; the normaliser partial sums live in tensor memory
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t pk[4], lv[8];
-        tmem_ld8(lane_base + kLCol + 8 * c, lv);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t lv[32];
+        tc::tmem_ld32(lane_base + kLCol + 32 * half, lv);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int h = 8 * c + 2 * e;
-          const float p0 = exp2f(u[h] - mref[h]);
-          const float p1 = exp2f(u[h + 1] - mref[h + 1]);
-          lv[2 * e] = __float_as_uint(fmaf(p0, inv_k, __uint_as_float(lv[2 * e])));
-          lv[2 * e + 1] = __float_as_uint(fmaf(p1, inv_k, __uint_as_float(lv[2 * e + 1])));
-          pk[e] = h2u(__floats2half2_rn(p0, p1));
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int h = 32 * half + 8 * c + 2 * e;
+            const float p0 = fast_exp2(d[h]);
+            const float p1 = fast_exp2(d[h + 1]);
+            const int k = 8 * c + 2 * e;
+            lv[k] = __float_as_uint(fmaf(p0, inv_k, __uint_as_float(lv[k])));
+            lv[k + 1] = __float_as_uint(fmaf(p1, inv_k, __uint_as_float(lv[k + 1])));
+            pk[e] = h2u(__floats2half2_rn(p0, p1));
+          }
+          *reinterpret_cast<uint4*>(sm + kPOff + tc::sw128_off(row, 4 * half + c)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
-        tmem_st8(lane_base + kLCol + 8 * c, lv);
-        *reinterpret_cast<uint4*>(sm + kPOff + tc::sw128_off(row, c)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        tc::tmem_st32(lane_base + kLCol + 32 * half, lv);
       }
       tc::tmem_wait_st();
       tc::fence_proxy_async_smem();
