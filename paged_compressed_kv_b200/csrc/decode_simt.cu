@@ -253,22 +253,24 @@ DecodePlan plan_decode(int batch, int heads, int max_seq_len, int ratio, int win
   const int n_sel = k > 0 ? k : n_vis;
   const int n_win = min(L, window_len);
   if (heads == 64) {
-    // tensor-core kernel: items in tiles of 128, entries padded to whole tiles,
-    // one 217 KB block per SM; 16 tiles per split
+    // tensor-core kernel: a persistent grid of one block per SM over the tile
+    // list of all sequences (entries padded to whole tiles of 128 items)
     p.path = 1;
     p.items_max = (n_sel + 127) / 128 * 128 + n_win;
-    p.split = 2048;
-  } else {
-    p.path = 0;
-    p.items_max = n_sel + n_win;
-    // aim for about four blocks per SM over all head groups
-    const int head_groups = (heads + kSimtHeads - 1) / kSimtHeads;
-    long long target = (long long)num_sms * 4 / max(1, head_groups);
-    long long total = (long long)p.items_max * batch;
-    long long split = (total + target - 1) / max(1LL, target);
-    split = max(64LL, min(8192LL, ((split + 63) / 64) * 64));
-    p.split = (int)split;
+    p.split = 128;
+    p.n_splits = max(1, num_sms);
+    p.ws_bytes = decode_tc_workspace_bytes(batch, p.n_splits);
+    return p;
   }
+  p.path = 0;
+  p.items_max = n_sel + n_win;
+  // aim for about four blocks per SM over all head groups
+  const int head_groups = (heads + kSimtHeads - 1) / kSimtHeads;
+  const long long target = (long long)num_sms * 4 / max(1, head_groups);
+  const long long total = (long long)p.items_max * batch;
+  long long split = (total + target - 1) / max(1LL, target);
+  split = max(64LL, min(8192LL, ((split + 63) / 64) * 64));
+  p.split = (int)split;
   p.n_splits = max(1, (p.items_max + p.split - 1) / p.split);
   p.ws_bytes = (size_t)batch * p.n_splits * heads * (size_t)(kDim + 2) * sizeof(float);
   return p;

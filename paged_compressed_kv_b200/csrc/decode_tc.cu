@@ -14,10 +14,19 @@
 // reference maximum per head, raised only when a score exceeds it by more
 // than 2^8 (P' <= 256), at which point O^T and the partial sums are rescaled.
 //
-// Warp roles (288 threads): warps 0-3 softmax (thread = tile row = TMEM lane),
+// Warp roles (320 threads): warps 0-3 softmax (thread = tile row = TMEM lane),
 // warps 4-7 gather + convert (16-byte coalesced page loads), warp 8 allocates
-// tensor memory and one of its threads issues the MMAs. Each softmax thread
+// tensor memory and one of its threads issues the MMAs, warp 9 resolves the
+// rows of the tiles two ahead and prefetches them into L2. Each softmax thread
 // keeps its item rows' partial normalisers (one per head) in tensor memory.
+//
+// Schedule: the kernel is persistent. The tiles of all sequences form one
+// list (each sequence: its entries padded to whole tiles, then its window);
+// block c of G processes tiles [c*T/G, (c+1)*T/G), so every SM gets the same
+// number of tiles whatever the length mix. A block writes one partial result
+// (O, m, l) per sequence it touches into slot b + c, which is unique because
+// b + c increases strictly along the tile list; the merge kernel combines the
+// slots of each sequence.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -43,7 +52,8 @@ constexpr uint32_t kMrefOff = kPtrOff + 3072;    // [64] reference max per head
 constexpr uint32_t kAlphaOff = kMrefOff + 256;   // [64] rescale factors
 constexpr uint32_t kRedOff = kAlphaOff + 256;    // [4][64] per-warp maxima
 constexpr uint32_t kBarOff = kRedOff + 1024;     // mbarriers
-constexpr uint32_t kMiscOff = kBarOff + 256;     // tmem address, flags
+constexpr uint32_t kInfoOff = kBarOff + 256;     // [3] tile info words
+constexpr uint32_t kMiscOff = kInfoOff + 64;     // tmem address, flags, range
 constexpr uint32_t kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
 
 // TMEM columns: S double buffer [0, 128), O^T 4 x 64 at [128, 384), partial
@@ -60,8 +70,13 @@ struct Bars {
   uint64_t s_full[2];
   uint64_t p_full;
   uint64_t pv_done;
+  uint64_t q_ready;
   uint64_t drain;
 };
+
+// tile info word written by the address warp
+constexpr uint32_t kInfoFp8 = 1;    // rows are fp8 codes (else bf16)
+constexpr uint32_t kInfoFirst = 2;  // first tile of a segment (new sequence)
 
 // 2^x on the special-function unit (ftz: results below 2^-126 become 0)
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -104,21 +119,6 @@ __device__ __forceinline__ bool named_or(int id, int n, bool p) {
       : "r"((uint32_t)p), "r"(id), "r"(n)
       : "memory");
   return r != 0;
-}
-
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                 "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
-                   taddr),
-               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
-               "r"(r[7])
-               : "memory");
 }
 
 struct Seq {
@@ -253,6 +253,119 @@ __device__ __forceinline__ uint4 bf16x8_to_f16(uint4 raw) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+
+__device__ __forceinline__ int tiles_of(const Seq& s) {
+  return s.n_sel_pad / kT + (s.n_win + kT - 1) / kT;
+}
+
+// Walks the global tile list: sequence b, tile lt of nt in that sequence.
+struct Cursor {
+  int b, lt, nt;
+  Seq s;
+};
+
+__device__ __forceinline__ void cursor_set(Cursor& c, const DecodeArgs& a, int b, int lt) {
+  c.b = b;
+  c.lt = lt;
+  c.s = seq_of(a, b, nullptr);
+  c.nt = tiles_of(c.s);
+}
+
+__device__ __forceinline__ void cursor_next(Cursor& c, const DecodeArgs& a) {
+  ++c.lt;
+  while (c.lt >= c.nt && c.b + 1 < a.batch) {
+    ++c.b;
+    c.lt = 0;
+    c.s = seq_of(a, c.b, nullptr);
+    c.nt = tiles_of(c.s);
+  }
+}
+
+// q[b] -> f16 in shared memory, scaled by 2^e so that max|q| * 2^e < 2^15;
+// returns sm_scale * log2(e) * 2^-e. Run by `nthreads` threads (thread index
+// t) that meet at named barrier `bar`; `red` holds nthreads/32 floats.
+__device__ __forceinline__ float load_q(const DecodeArgs& a, int b, uint8_t* qsm, float* red, int t,
+                                        int nthreads, int bar) {
+  const size_t qoff = (size_t)b * kH * kD;
+  float m = 0.f;
+  for (int u = t; u < kH * kD / 8; u += nthreads) {
+    const size_t o = qoff + (size_t)u * 8;
+    if (a.q_dtype == V4KV_FP32) {
+      const float4 x0 = reinterpret_cast<const float4*>(a.q)[o / 4];
+      const float4 x1 = reinterpret_cast<const float4*>(a.q)[o / 4 + 1];
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(x0.x), fabsf(x0.y)), fmaxf(fabsf(x0.z), fabsf(x0.w))));
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(x1.x), fabsf(x1.y)), fmaxf(fabsf(x1.z), fabsf(x1.w))));
+    } else {
+      const uint4 r = reinterpret_cast<const uint4*>(a.q)[o / 8];
+      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xffff0000u))));
+    }
+  }
+  m = warp_max(m);
+  if ((t & 31) == 0) red[t >> 5] = m;
+  named_sync(bar, nthreads);
+  float amax = 0.f;
+  for (int w = 0; w < nthreads / 32; ++w) amax = fmaxf(amax, red[w]);
+  int e = 0;
+  if (amax > 0.f) {
+    int k;
+    frexpf(amax, &k);  // amax < 2^k
+    e = 15 - k;
+  }
+  const float qs = ldexpf(1.f, e);
+  for (int u = t; u < kH * kD / 8; u += nthreads) {
+    const int h = u / (kD / 8), c8 = u % (kD / 8);  // 8-dim chunk c8 of head h
+    const size_t o = qoff + (size_t)h * kD + c8 * 8;
+    float x[8];
+    if (a.q_dtype == V4KV_FP32) {
+      const float4 x0 = reinterpret_cast<const float4*>(a.q)[o / 4];
+      const float4 x1 = reinterpret_cast<const float4*>(a.q)[o / 4 + 1];
+      x[0] = x0.x; x[1] = x0.y; x[2] = x0.z; x[3] = x0.w;
+      x[4] = x1.x; x[5] = x1.y; x[6] = x1.z; x[7] = x1.w;
+    } else {
+      const uint4 r = reinterpret_cast<const uint4*>(a.q)[o / 8];
+      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+      }
+    }
+    uint32_t hv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) hv[i] = h2u(__floats2half2_rn(x[2 * i] * qs, x[2 * i + 1] * qs));
+    *reinterpret_cast<uint4*>(qsm + (c8 >> 3) * 8192 + tc::sw128_off(h, c8 & 7)) =
+        make_uint4(hv[0], hv[1], hv[2], hv[3]);
+  }
+  tc::fence_proxy_async_smem();
+  return a.sm_scale * 1.4426950408889634f * ldexpf(1.f, -e);
+}
+
+// Sum 64 per-lane values over the 32 lanes of a warp (reduce-scatter): lane l
+// ends with the sums of heads 2*rev and 2*rev+1 where the lane bits pick
+// halves (bit 4: 32 heads, bit 3: 16, ... bit 0: 2). Returns the head index.
+__device__ __forceinline__ int warp_reduce_scatter64(float* v, int lane, float* out2) {
+  int base = 0;
+#pragma unroll
+  for (int level = 0; level < 5; ++level) {
+    const int off = 16 >> level;   // shuffle distance
+    const int n = 32 >> level;     // values kept after this level
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int k = 0; k < n; ++k) {
+      const float mine = upper ? v[n + k] : v[k];
+      const float other = upper ? v[k] : v[n + k];
+      v[k] = mine + __shfl_xor_sync(0xffffffffu, other, off);
+    }
+    if (upper) base += n;
+  }
+  out2[0] = v[0];
+  out2[1] = v[1];
+  return base;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
@@ -264,20 +377,64 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   Bars* bars = reinterpret_cast<Bars*>(sm + kBarOff);
   float* meta = reinterpret_cast<float*>(sm + kMetaOff);
   const uint8_t** rowptr = reinterpret_cast<const uint8_t**>(sm + kPtrOff);
+  uint32_t* info = reinterpret_cast<uint32_t*>(sm + kInfoOff);
   float* mref = reinterpret_cast<float*>(sm + kMrefOff);
   float* alpha = reinterpret_cast<float*>(sm + kAlphaOff);
   float* red = reinterpret_cast<float*>(sm + kRedOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kMiscOff + 4);
   float* k0_slot = reinterpret_cast<float*>(sm + kMiscOff + 8);
+  int* range = reinterpret_cast<int*>(sm + kMiscOff + 16);  // x0, x1, b0, lt0
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int b = blockIdx.y, split = blockIdx.x;
-  const Seq s = seq_of(a, b, a.dev_status);
-  const int i0 = split * a.split;
-  if (i0 >= s.n_items) return;
-  const int i1 = min(s.n_items, i0 + a.split);
-  const int n_tiles = (i1 - i0 + kT - 1) / kT;
+  const int G = gridDim.x, cta = blockIdx.x;
+
+  // ---- this block's tile range: T = total tiles, [c*T/G, (c+1)*T/G)
+  if (warp == 0) {
+    long long T = 0;
+    for (int base = 0; base < a.batch; base += 32) {
+      const int bb = base + lane;
+      int t = bb < a.batch ? tiles_of(seq_of(a, bb, a.dev_status)) : 0;
+      T += __reduce_add_sync(0xffffffffu, t);
+    }
+    const int x0 = (int)((long long)cta * T / G), x1 = (int)((long long)(cta + 1) * T / G);
+    // first sequence of the range and the tile within it; block 0 also
+    // publishes the tile prefix sums for the merge
+    int b0 = a.batch, lt0 = 0;
+    long long run = 0;
+    for (int base = 0; base < a.batch; base += 32) {
+      const int bb = base + lane;
+      const int t = bb < a.batch ? tiles_of(seq_of(a, bb, nullptr)) : 0;
+      int incl = t;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const long long before = run + incl - t;  // tiles before sequence bb
+      if (cta == 0 && bb < a.batch) a.cum[bb] = (int32_t)before;
+      const bool mine = bb < a.batch && t > 0 && before <= x0 && x0 < before + t;
+      const unsigned hit = __ballot_sync(0xffffffffu, mine);
+      if (hit && b0 == a.batch) {
+        const int src = __ffs(hit) - 1;
+        b0 = __shfl_sync(0xffffffffu, bb, src);
+        lt0 = x0 - (int)__shfl_sync(0xffffffffu, before, src);
+      }
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (cta == 0 && lane == 0) a.cum[a.batch] = (int32_t)T;
+    if (lane == 0) {
+      range[0] = x0;
+      range[1] = (b0 < a.batch) ? x1 : x0;
+      range[2] = b0;
+      range[3] = lt0;
+    }
+  }
+  __syncthreads();
+  const int x0 = range[0], x1 = range[1];
+  if (x0 >= x1) return;
+  const int n_tiles = x1 - x0;
+  const int b0 = range[2], lt0 = range[3];
 
   if (tid == 0) {
     for (int k = 0; k < 3; ++k) {
@@ -292,71 +449,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
     tc::mbar_init(&bars->s_full[1], 1);
     tc::mbar_init(&bars->p_full, 128);
     tc::mbar_init(&bars->pv_done, 1);
+    tc::mbar_init(&bars->q_ready, 128);
     tc::mbar_init(&bars->drain, 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
   if (warp == 8) tc::tmem_alloc(tmem_slot, kTmemCols);
   if (tid < kH) mref[tid] = kNone;
-
-  // ---- q -> f16, scaled by 2^e so that max|q| * 2^e < 2^15 (warps 0-7)
   if (warp < 8) {
-    const size_t qoff = (size_t)b * kH * kD;
-    float m = 0.f;
-    for (int u = tid; u < kH * kD / 8; u += 256) {
-      const size_t o = qoff + (size_t)u * 8;
-      if (a.q_dtype == V4KV_FP32) {
-        const float4 x0 = reinterpret_cast<const float4*>(a.q)[o / 4];
-        const float4 x1 = reinterpret_cast<const float4*>(a.q)[o / 4 + 1];
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(x0.x), fabsf(x0.y)), fmaxf(fabsf(x0.z), fabsf(x0.w))));
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(x1.x), fabsf(x1.y)), fmaxf(fabsf(x1.z), fabsf(x1.w))));
-      } else {
-        const uint4 r = reinterpret_cast<const uint4*>(a.q)[o / 8];
-        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xffff0000u))));
-      }
-    }
-    m = warp_max(m);
-    if (lane == 0) red[warp] = m;
-    named_sync(2, 256);
-    float amax = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) amax = fmaxf(amax, red[w]);
-    int e = 0;
-    if (amax > 0.f) {
-      int k;
-      frexpf(amax, &k);  // amax < 2^k
-      e = 15 - k;
-    }
-    const float qs = ldexpf(1.f, e);
-    if (tid == 0) *k0_slot = a.sm_scale * 1.4426950408889634f * ldexpf(1.f, -e);
-    for (int u = tid; u < kH * kD / 8; u += 256) {
-      const int h = u / (kD / 8), c8 = u % (kD / 8);  // 8-dim chunk c8 of head h
-      const size_t o = qoff + (size_t)h * kD + c8 * 8;
-      float x[8];
-      if (a.q_dtype == V4KV_FP32) {
-        const float4 x0 = reinterpret_cast<const float4*>(a.q)[o / 4];
-        const float4 x1 = reinterpret_cast<const float4*>(a.q)[o / 4 + 1];
-        x[0] = x0.x; x[1] = x0.y; x[2] = x0.z; x[3] = x0.w;
-        x[4] = x1.x; x[5] = x1.y; x[6] = x1.z; x[7] = x1.w;
-      } else {
-        const uint4 r = reinterpret_cast<const uint4*>(a.q)[o / 8];
-        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          x[2 * i] = __uint_as_float(w[i] << 16);
-          x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-        }
-      }
-      uint32_t hv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) hv[i] = h2u(__floats2half2_rn(x[2 * i] * qs, x[2 * i + 1] * qs));
-      *reinterpret_cast<uint4*>(sm + kQOff + (c8 >> 3) * 8192 + tc::sw128_off(h, c8 & 7)) =
-          make_uint4(hv[0], hv[1], hv[2], hv[3]);
-    }
-    tc::fence_proxy_async_smem();
+    const float k0 = load_q(a, b0, sm + kQOff, red, tid, 256, 2);
+    if (tid == 0) *k0_slot = k0;
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -365,30 +467,62 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
 
   if (warp == 9) {
     // ======================= address resolution + L2 prefetch, two tiles ahead
+    Cursor cu;
+    cursor_set(cu, a, b0, lt0);
     for (int t = 0; t < n_tiles; ++t) {
       const int buf = t % 3;
       if (t >= 3 && !tc::mbar_wait(&bars->addr_free[buf], ((t - 3) / 3) & 1, abort_flag)) break;
-      resolve_tile(a, b, s, i0 + t * kT, lane, rowptr + buf * kT, meta + buf * kT);
+      if (t > 0 && cu.lt == 0 && a.q_dtype == V4KV_FP32) {
+        // a new sequence starts: pull its query into L2 as well
+        const uint8_t* qp = reinterpret_cast<const uint8_t*>(a.q) + (size_t)cu.b * kH * kD * 4;
+        for (int k = lane; k < kH * kD * 4 / 128; k += 32) prefetch_l2_line(qp + 128 * k);
+      }
+      const int tile0 = cu.lt * kT;
+      resolve_tile(a, cu.b, cu.s, tile0, lane, rowptr + buf * kT, meta + buf * kT);
+      if (lane == 0) {
+        const bool main_tile = tile0 < cu.s.n_sel_pad;
+        const bool fp8 = (main_tile ? a.main.dtype : a.window.dtype) == V4KV_FP8_E4M3;
+        info[buf] = (fp8 ? kInfoFp8 : 0u) | ((t == 0 || cu.lt == 0) ? kInfoFirst : 0u);
+      }
       __syncwarp();
       tc::mbar_arrive(&bars->addr_ready[buf]);
+      cursor_next(cu, a);
     }
   } else if (warp == 8) {
     // ======================= MMA issuer
     if (lane == 0) {
       const uint32_t iq = tc::idesc_f16(128, kH, 0, 0);
       const uint32_t ip = tc::idesc_f16(128, kH, 1, 1);
+      // descriptors at the operands' bases; a step adds its byte offset / 16
+      const uint64_t vk_desc = tc::sw128_desc(sbase + kVOff, 16, 1024);     // V, K-major
+      const uint64_t qk_desc = tc::sw128_desc(sbase + kQOff, 16, 1024);     // Q, K-major
+      const uint64_t vm_desc = tc::sw128_desc(sbase + kVOff, 16384, 1024);  // V^T, MN-major
+      const uint64_t p_desc = tc::sw128_desc(sbase + kPOff, 0, 1024);       // P^T, MN-major
       bool ok = true;
+      int seg = 0;
       for (int i = 0; i < n_tiles && ok; ++i) {
         const uint32_t par = i & 1;
         const uint32_t s_col = (uint32_t)(i & 1) * kH;
+        bool first = i == 0;
         for (int c = 0; c < 4 && ok; ++c) {
           ok = tc::mbar_wait(&bars->v_full[c], par, abort_flag);
           if (!ok) break;
+          if (c == 0) {
+            // the converters read this tile's info word before arriving
+            first = (info[i % 3] & kInfoFirst) != 0;
+            if (first && i > 0) {
+              ok = tc::mbar_wait(&bars->q_ready, (seg - 1) & 1, abort_flag);
+              if (!ok) break;
+            }
+            if (first) ++seg;
+          }
           tc::tc_fence_after();
-          for (int kk = 8 * c; kk < 8 * c + 8; ++kk) {
-            const uint64_t ad = tc::sw128_desc(sbase + kVOff + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = tc::sw128_desc(sbase + kQOff + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-            tc::mma_f16(tmem + s_col, ad, bd, iq, kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int k8 = 0; k8 < 8; ++k8) {
+            const int kk = 8 * c + k8;  // 16-dim step: atom kk/4, 32-byte column kk%4
+            tc::mma_f16(tmem + s_col, vk_desc + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
+                        qk_desc + (uint64_t)((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), iq,
+                        kk > 0 ? 1u : 0u);
           }
         }
         if (!ok) break;
@@ -396,12 +530,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
         ok = tc::mbar_wait(&bars->p_full, par, abort_flag);
         if (!ok) break;
         tc::tc_fence_after();
+#pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ad = tc::sw128_desc(sbase + kVOff + 2 * mt * 16384 + kk * 2048, 16384, 1024);
-            const uint64_t bd = tc::sw128_desc(sbase + kPOff + kk * 2048, 0, 1024);
-            tc::mma_f16(tmem + kOCol + kH * mt, ad, bd, ip, (i > 0 || kk > 0) ? 1u : 0u);
-          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc::mma_f16(tmem + kOCol + kH * mt, vm_desc + (uint64_t)((2 * mt * 16384 + kk * 2048) >> 4),
+                        p_desc + (uint64_t)((kk * 2048) >> 4), ip, (!first || kk > 0) ? 1u : 0u);
           tc::mma_commit(&bars->v_empty[mt]);
         }
         tc::mma_commit(&bars->pv_done);
@@ -419,14 +553,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
     __syncwarp();
   } else if (warp >= 4) {
     // ======================= gather + convert
-    // Warp cw owns rows [32 cw, 32 cw + 32) of every tile. Lane l resolves row
-    // 32 cw + l of the next tile while the current one is loaded and converted.
     const int cw = warp - 4;
     for (int i = 0; i < n_tiles; ++i) {
       if (!tc::mbar_wait(&bars->addr_ready[i % 3], (i / 3) & 1, abort_flag)) goto conv_abort;
-      const int tile0 = i0 + i * kT;
-      const bool entries = tile0 < s.n_sel_pad;
-      const bool fp8 = (entries ? a.main.dtype : a.window.dtype) == V4KV_FP8_E4M3;
+      const bool fp8 = (info[i % 3] & kInfoFp8) != 0;
       const uint8_t** rp = rowptr + (i % 3) * kT;
       if (fp8) {
         // lane covers rows 32cw + 4r + lane/8 (r = 0..7), 16 bytes at 16*(lane%8)
@@ -492,16 +622,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   } else {
     // ======================= softmax (thread = tile row = TMEM lane)
     const int row = tid;
-    const float k0 = *k0_slot;
+    float k0 = *k0_slot;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
     {
-      uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      uint32_t z[32];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) tmem_st8(lane_base + kLCol + 8 * c, z);
+      for (int e = 0; e < 32; ++e) z[e] = 0u;
+      tc::tmem_st32(lane_base + kLCol, z);
+      tc::tmem_st32(lane_base + kLCol + 32, z);
       tc::tmem_wait_st();
     }
+    Cursor cu;
+    cursor_set(cu, a, b0, lt0);
     bool ok = true;
+    bool seg_first = true;  // the current tile opens a segment
     for (int i = 0; i < n_tiles && ok; ++i) {
+      const bool seg_last = i == n_tiles - 1 || cu.lt == cu.nt - 1;
       // S(i) complete implies PV(i-1) complete (the MMAs run in issue order),
       // so waiting for pv_done(i-1) here costs nothing and frees P and O^T
       ok = tc::mbar_wait(&bars->v_full[0], i & 1, abort_flag) &&
@@ -586,7 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
           tc::tmem_st32(lane_base + kLCol + 32 * half, lv);
         }
         tc::tmem_wait_st();
-        if (i > 0) {
+        if (!seg_first) {
           // O^T rows of this lane (dims 128 mt + row) times alpha per head column
 #pragma unroll 1
           for (int mt = 0; mt < 4; ++mt) {
@@ -634,45 +770,76 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       tc::mbar_arrive(&bars->p_full);
+
+      if (seg_last) {
+        const int b_done = cu.b;
+        cursor_next(cu, a);
+        if (i + 1 < n_tiles) {
+          // QK(i) is complete (S(i) was read), so Q is free: load the next
+          // segment's query while PV(i) runs
+          k0 = load_q(a, cu.b, sm + kQOff, red, row, 128, 1);
+          tc::mbar_arrive(&bars->q_ready);
+        }
+        ok = tc::mbar_wait(&bars->pv_done, i & 1, abort_flag);
+        ok = named_and(1, 128, ok);
+        if (!ok) break;
+        tc::tc_fence_after();
+        // partial result of (sequence b_done, block cta) in slot b_done + cta:
+        // O^T un-normalised, relative to the reference maximum
+        const size_t prow = ((size_t)b_done + cta) * kH;
+#pragma unroll 1
+        for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            uint32_t r32[32];
+            tc::tmem_ld32(lane_base + kOCol + kH * mt + 32 * half, r32);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < 32; ++h)
+              a.part_o[(prow + 32 * half + h) * kD + 128 * mt + row] = __uint_as_float(r32[h]);
+          }
+        }
+        // normaliser: sum the 128 rows' partial sums per head
+        {
+          float v[kH];
+          uint32_t r32[32];
+          tc::tmem_ld32(lane_base + kLCol, r32);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r32[e]);
+          tc::tmem_ld32(lane_base + kLCol + 32, r32);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[32 + e] = __uint_as_float(r32[e]);
+          float two[2];
+          const int hb = warp_reduce_scatter64(v, lane, two);
+          named_sync(1, 128);  // red is free (no slow path in flight)
+          red[warp * kH + hb] = two[0];
+          red[warp * kH + hb + 1] = two[1];
+          named_sync(1, 128);
+          if (row < kH) {
+            const float l = red[row] + red[kH + row] + red[2 * kH + row] + red[3 * kH + row];
+            a.part_ml[(prow + row) * 2] = mref[row];
+            a.part_ml[(prow + row) * 2 + 1] = l;
+            mref[row] = kNone;
+          }
+          uint32_t z[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) z[e] = 0u;
+          tc::tmem_st32(lane_base + kLCol, z);
+          tc::tmem_st32(lane_base + kLCol + 32, z);
+          tc::tmem_wait_st();
+          named_sync(1, 128);
+        }
+        seg_first = true;
+      } else {
+        cursor_next(cu, a);
+        seg_first = false;
+      }
     }
-    if (ok) ok = tc::mbar_wait(&bars->pv_done, (n_tiles - 1) & 1, abort_flag);
-    ok = named_and(1, 128, ok);
     if (!ok) {
       *abort_flag = 1;
       flag(a.dev_status, V4KV_DEV_TIMEOUT);
-    } else {
-      tc::tc_fence_after();
-      // O^T -> partial output (un-normalised, relative to the reference max)
-      const size_t prow = ((size_t)b * a.n_splits + split) * kH;
-#pragma unroll 1
-      for (int mt = 0; mt < 4; ++mt) {
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          uint32_t r32[32];
-          tc::tmem_ld32(lane_base + kOCol + kH * mt + 32 * half, r32);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < 32; ++h)
-            a.part_o[(prow + 32 * half + h) * kD + 128 * mt + row] = __uint_as_float(r32[h]);
-        }
-      }
-      // partial sums of the normaliser: reduce over the 128 rows per head
-      float* lred = reinterpret_cast<float*>(sm + kVOff);
-#pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t lv[8];
-        tmem_ld8(lane_base + kLCol + 8 * c, lv);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 8; ++e) lred[(8 * c + e) * 129 + row] = __uint_as_float(lv[e]);
-      }
-      named_sync(1, 128);
-      if (row < kH) {
-        float l = 0.f;
-        for (int r = 0; r < kT; ++r) l += lred[row * 129 + r];
-        a.part_ml[(prow + row) * 2] = mref[row];
-        a.part_ml[(prow + row) * 2 + 1] = l;
-      }
     }
   }
 
@@ -684,7 +851,65 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   }
 }
 
-size_t decode_tc_smem_bytes() { return kSmemBytes; }
+// grid (heads, batch), 128 threads x 4 dims: merge the partial results of the
+// blocks whose tile ranges cover the sequence, normalise, inverse RoPE at
+// position L - 1, store bf16
+__global__ void __launch_bounds__(128) decode_tc_merge_kernel(DecodeArgs a) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int G = a.n_splits;
+  const long long T = a.cum[a.batch];
+  const int c0 = a.cum[b], c1 = a.cum[b + 1];
+  const int d0 = threadIdx.x * 4;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f}, L = 0.f;
+  if (c1 > c0) {
+    const int cf = (int)(((long long)(c0 + 1) * G + T - 1) / T) - 1;
+    const int cl = (int)(((long long)c1 * G + T - 1) / T) - 1;
+    float M = -INFINITY;
+    for (int c = cf; c <= cl; ++c) {
+      const long long s0 = (long long)c * T / G, s1 = (long long)(c + 1) * T / G;
+      if (s1 <= c0 || s0 >= c1 || s1 <= s0) continue;
+      M = fmaxf(M, a.part_ml[(((size_t)b + c) * kH + h) * 2]);
+    }
+    for (int c = cf; c <= cl; ++c) {
+      const long long s0 = (long long)c * T / G, s1 = (long long)(c + 1) * T / G;
+      if (s1 <= c0 || s0 >= c1 || s1 <= s0) continue;
+      const size_t row = ((size_t)b + c) * kH + h;
+      const float w = exp2f(a.part_ml[row * 2] - M);
+      L = fmaf(w, a.part_ml[row * 2 + 1], L);
+      const float4 o = *reinterpret_cast<const float4*>(a.part_o + row * kD + d0);
+      acc[0] = fmaf(w, o.x, acc[0]);
+      acc[1] = fmaf(w, o.y, acc[1]);
+      acc[2] = fmaf(w, o.z, acc[2]);
+      acc[3] = fmaf(w, o.w, acc[3]);
+    }
+  }
+  float o[4];
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) o[i] = acc[i] * inv;
+  int Lb = a.seq_lens[b];
+  Lb = min(Lb, a.max_len);
+  if (a.rope.rope_dim > 0 && Lb > 0) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int d = d0 + 2 * k;
+      if (d >= a.rope.rope_offset && d + 1 < a.rope.rope_offset + a.rope.rope_dim) {
+        float c, s;
+        rope_cs(a.rope.theta, a.rope.rope_dim, (d - a.rope.rope_offset) >> 1, (long long)Lb - 1, &c, &s);
+        rope_apply(o[2 * k], o[2 * k + 1], c, -s);
+      }
+    }
+  }
+  uint16_t* dst = reinterpret_cast<uint16_t*>(a.out) + ((size_t)b * kH + h) * kD + d0;
+  const uint32_t w0 = (uint32_t)float_to_bf16_bits(o[0]) | ((uint32_t)float_to_bf16_bits(o[1]) << 16);
+  const uint32_t w1 = (uint32_t)float_to_bf16_bits(o[2]) | ((uint32_t)float_to_bf16_bits(o[3]) << 16);
+  *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
+}
+
+size_t decode_tc_workspace_bytes(int batch, int num_sms) {
+  const size_t slots = (size_t)batch + num_sms;
+  return slots * kH * (size_t)(kD + 2) * sizeof(float) + ((size_t)batch + 1) * sizeof(int32_t) + 256;
+}
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   static bool attr_set = false;
@@ -694,8 +919,10 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid(a.n_splits, a.batch);
-  decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(a);
+  decode_tc_kernel<<<a.n_splits, kThreads, kSmemBytes, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_tc_merge_kernel<<<dim3(kH, a.batch), 128, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -68,7 +68,7 @@ struct DecodePlan {
   int path;          // 0 = CUDA-core kernel, 1 = tensor-core kernel
   int items_max;     // max attended items (entries + window) of one sequence
   int split;         // items per split
-  int n_splits;      // splits per sequence
+  int n_splits;      // splits per sequence (tensor-core path: blocks of the persistent grid)
   size_t ws_bytes;   // partial results
 };
 
@@ -95,6 +95,7 @@ struct DecodeArgs {
   int n_splits;
   int max_len;  // host bound on seq_lens; longer sequences are clamped and flagged
   int pad_sel;  // 1: entries are padded to a multiple of 128 items (tensor-core path)
+  int32_t* cum; // tensor-core path: [batch + 1] tile prefix sums (workspace)
 };
 
 cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, int batch,
@@ -111,6 +112,7 @@ DecodePlan plan_decode(int batch, int heads, int max_seq_len, int ratio, int win
                        int main_dtype, int dim, int num_sms);
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream);
-cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);  // sweep + merge
+size_t decode_tc_workspace_bytes(int batch, int num_sms);
 
 }  // namespace v4kv
