@@ -414,7 +414,236 @@ def run_reference(args, rank, world):
     }
 
 
-DTYPE = "fp32"
+# ------------------------------------------------------------------ other rows (--config 3, 4)
+
+class CompressStep:
+    """Compressor write path: 8 sequences x 32K raw bf16 tokens appended in
+    random chunks of 1..4096 (one chunk per sequence per call), ratio 4 or 128,
+    fp8 entries into shuffled pages, window copies of each chunk's last 128."""
+
+    def __init__(self, device, ratio, seqs=8, tokens=32768):
+        from paged_compressed_kv_b200 import PagedPool, v4kv
+        self.v4kv, self.ratio, self.B, self.N = v4kv, ratio, seqs, tokens
+        r = synth.rng(synth.seed_for(3) + ratio)
+        g = synth.device_generator(synth.seed_for(3) + ratio, device)
+        self.chunks = [synth.chunk_sizes(r, tokens) for _ in range(seqs)]
+        self.calls = max(len(c) for c in self.chunks)
+        spb = 256 // ratio
+        nblk = -(-(-(-tokens // ratio)) // spb)
+        P = nblk * seqs
+        perm = synth.permutation(r, P)
+        bt = perm.reshape(seqs, nblk).astype(np.int32)
+        self.P = P
+        self.main = PagedPool(data=torch.zeros(P, spb, D, dtype=torch.uint8, device=device),
+                              block_table=torch.from_numpy(bt).to(device),
+                              scales=torch.zeros(P, spb, dtype=torch.float32, device=device))
+        wblk = -(-tokens // 256)
+        wperm = synth.permutation(r, wblk * seqs).reshape(seqs, wblk).astype(np.int32)
+        self.win = PagedPool(data=torch.zeros(wblk * seqs, 256, D, dtype=torch.bfloat16, device=device),
+                             block_table=torch.from_numpy(wperm).to(device))
+        self.x = torch.empty(seqs * tokens, D, dtype=torch.bfloat16, device=device)
+        synth.fill_normal_bf16(self.x, g)
+        self.gate = torch.randn(seqs * tokens, generator=g, device=device)
+        self.bias = torch.randn(ratio, generator=g, device=device) * 0.5
+        self.state_x = torch.zeros(seqs, ratio, D, dtype=torch.bfloat16, device=device)
+        self.state_g = torch.zeros(seqs, ratio, dtype=torch.float32, device=device)
+        # per call: chunk rows gathered contiguously (inputs resident before timing)
+        self.call_inputs = []
+        done = [0] * seqs
+        for c in range(self.calls):
+            sizes = [self.chunks[b][c] if c < len(self.chunks[b]) else 0 for b in range(seqs)]
+            rows = torch.cat([torch.arange(b * tokens + done[b], b * tokens + done[b] + sizes[b],
+                                           device=device) for b in range(seqs)])
+            cu = torch.tensor(np.concatenate([[0], np.cumsum(sizes)]), dtype=torch.int32, device=device)
+            ss = torch.tensor(done, dtype=torch.int32, device=device)
+            nn = torch.tensor(sizes, dtype=torch.int32, device=device)
+            cap = int(sum(sizes)) // ratio + 2 * seqs
+            self.call_inputs.append(dict(x=self.x[rows].contiguous(), gate=self.gate[rows].contiguous(),
+                                         cu=cu, ss=ss, nn=nn, n=int(sum(sizes)),
+                                         slots=torch.empty(cap, dtype=torch.int64, device=device),
+                                         cue=torch.empty(seqs + 1, dtype=torch.int32, device=device)))
+            for b in range(seqs):
+                done[b] += sizes[b]
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def call(self, c):
+        v, ci = self.v4kv, self.call_inputs[c]
+        v.v4kv_slot_mapping(self.main.block_table, ci["ss"], ci["nn"], self.ratio, self.P, ci["slots"],
+                            ci["cue"], dev_status=self.status)
+        v.v4kv_compress_append(ci["x"], ci["gate"], ci["cu"], ci["ss"], self.bias, self.ratio,
+                               self.state_x, self.state_g, self.main, ci["slots"], ci["cue"],
+                               window=self.win, window_len=W, dev_status=self.status)
+
+    def algorithmic_bytes(self, c):
+        ci = self.call_inputs[c]
+        n = ci["n"]
+        sizes = ci["nn"].cpu().numpy()
+        starts = ci["ss"].cpu().numpy()
+        touched = sum((-(-(s0 + m) // self.ratio)) - s0 // self.ratio for s0, m in zip(starts, sizes) if m)
+        win = sum(min(int(m), W) for m in sizes)
+        return n * (D * 2 + 4) + touched * (D + 4) + win * D * 2 + self.B * self.ratio * (D * 2 + 4)
+
+
+def run_compress(args, device):
+    peak, _ = load_peaks()
+    out = {}
+    for ratio in (4, 128):
+        st = CompressStep(device, ratio)
+        for c in range(st.calls):  # warm-up pass (also fills the cache once)
+            st.call(c)
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(st.calls)]
+        for c in range(st.calls):
+            ev[c][0].record()
+            st.call(c)
+            ev[c][1].record()
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in ev)
+        byts = sum(st.algorithmic_bytes(c) for c in range(st.calls))
+        out[f"r{ratio}"] = {"calls": st.calls, "tokens": st.B * st.N, "ms": ms,
+                            "tokens_per_s": st.B * st.N / (ms * 1e-3),
+                            "gbs": byts / (ms * 1e-3) / 1e9, "frac": byts / (ms * 1e-3) / 1e9 / peak,
+                            "status": int(st.status.item())}
+    return {"config": "compressor write path, 8 x 32K raw bf16 tokens, random chunks 1..4096, fp8 "
+                      "entries, shuffled pages", "results": out}
+
+
+class MixedStep:
+    """61-layer mixed decode step: 30 c4a layers (indexer top-512 over fp8 keys
+    of dim 128, then attention over the selected entries + window) and 31 c128a
+    layers (attention over all visible entries + window); batch 128, context
+    U[1K, 256K], 64 heads, fp8 KV dim 512. Every layer has its own caches."""
+
+    def __init__(self, device, seqs=128, c4a_layers=30, c128a_layers=31, k=512):
+        from paged_compressed_kv_b200 import PagedPool, v4kv
+        self.v4kv, self.k = v4kv, k
+        r = synth.rng(synth.seed_for(4))
+        self.lens = synth.lengths_uniform(r, seqs, 1024, 262144, 4)
+        self.B = seqs
+        g = synth.device_generator(synth.seed_for(4), device)
+        self.max_len = int(self.lens.max())
+        self.seq_lens = torch.from_numpy(self.lens.astype(np.int32)).to(device)
+
+        def pool(ratio, dim, dtype_fp8=True):
+            spb = 256 // ratio
+            nblk = [-(-(-(-int(L) // ratio)) // spb) for L in self.lens]
+            P = int(sum(nblk))
+            perm = synth.permutation(r, P)
+            bt = np.full((seqs, max(nblk)), -1, dtype=np.int32)
+            kk = 0
+            for b, nb in enumerate(nblk):
+                bt[b, :nb] = perm[kk:kk + nb]
+                kk += nb
+            data = torch.empty(P, spb, dim, dtype=torch.uint8, device=device)
+            synth.fill_fp8_codes(data, g)
+            sc = torch.empty(P, spb, dtype=torch.float32, device=device)
+            synth.fill_uniform(sc, g, 0.5 / 112, 1.5 / 112)
+            return PagedPool(data=data, block_table=torch.from_numpy(bt).to(device), scales=sc)
+
+        def window():
+            wf = [max(0, int(L) - W) // 256 for L in self.lens]
+            wl = [(int(L) - 1) // 256 for L in self.lens]
+            Pw = int(sum(l - f + 1 for f, l in zip(wf, wl)))
+            wperm = synth.permutation(r, Pw)
+            wbt = np.full((seqs, max(wl) + 1), -1, dtype=np.int32)
+            kk = 0
+            for b in range(seqs):
+                for blk in range(wf[b], wl[b] + 1):
+                    wbt[b, blk] = wperm[kk]
+                    kk += 1
+            wd = torch.empty(Pw, 256, D, dtype=torch.bfloat16, device=device)
+            synth.fill_normal_bf16(wd, g)
+            return PagedPool(data=wd, block_table=torch.from_numpy(wbt).to(device))
+
+        self.c4a = []
+        for _ in range(c4a_layers):
+            self.c4a.append(dict(main=pool(4, D), idx=pool(4, 128), win=window(),
+                                 q=torch.randn(seqs, HEADS, D, generator=g, device=device),
+                                 qi=torch.randn(seqs, 128, generator=g, device=device)))
+        self.c128a = []
+        for _ in range(c128a_layers):
+            self.c128a.append(dict(main=pool(128, D), win=window(),
+                                   q=torch.randn(seqs, HEADS, D, generator=g, device=device)))
+        self.topk = torch.empty(seqs, k, dtype=torch.int32, device=device)
+        self.out = torch.empty(seqs, HEADS, D, dtype=torch.bfloat16, device=device)
+        v = v4kv
+        wsa = v.v4kv_workspace_size(v.V4KV_OP_DECODE, seqs, HEADS, self.max_len, 4, W, k, v.V4KV_FP8_E4M3)
+        wsb = v.v4kv_workspace_size(v.V4KV_OP_DECODE, seqs, HEADS, self.max_len, 128, W, 0, v.V4KV_FP8_E4M3)
+        wsi = v.v4kv_workspace_size(v.V4KV_OP_INDEX_TOPK, seqs, 1, self.max_len, 4, W, k, v.V4KV_FP8_E4M3, 128)
+        self.ws = torch.empty(max(wsa, wsb, wsi, 256), dtype=torch.uint8, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def index(self, l):
+        L = self.c4a[l]
+        self.v4kv.v4kv_index_topk(L["qi"], L["idx"], self.seq_lens, self.max_len, 4, W, self.k, self.topk,
+                                  self.ws, dev_status=self.status)
+
+    def attend_c4a(self, l):
+        L = self.c4a[l]
+        self.v4kv.v4kv_decode_attention(L["q"], L["main"], L["win"], self.seq_lens, self.max_len, 4, W,
+                                        self.out, self.ws, topk=self.topk, dev_status=self.status)
+
+    def attend_c128a(self, l):
+        L = self.c128a[l]
+        self.v4kv.v4kv_decode_attention(L["q"], L["main"], L["win"], self.seq_lens, self.max_len, 128, W,
+                                        self.out, self.ws, dev_status=self.status)
+
+    def bytes(self):
+        nv4 = np.maximum(0, self.lens - W) // 4
+        nv128 = np.maximum(0, self.lens - W) // 128
+        win = np.minimum(self.lens, W) * D * 2
+        qo = HEADS * D * 4 + HEADS * D * 2
+        idx = int(np.sum(nv4 * (128 + 4) + 128 * 4 + self.k * 4))
+        att4 = int(np.sum(np.minimum(nv4, self.k) * (D + 4) + win + qo))
+        att128 = int(np.sum(nv128 * (D + 4) + win + qo))
+        return idx, att4, att128
+
+
+def run_mixed(args, device):
+    peak, _ = load_peaks()
+    st = MixedStep(device)
+    nl4, nl128 = len(st.c4a), len(st.c128a)
+    ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(2)] for k in ("idx", "att4", "att128")}
+    tot = {"idx": 0.0, "att4": 0.0, "att128": 0.0}
+    for it in range(args.warmup + args.steps):
+        timed = it >= args.warmup
+        for l in range(nl4):
+            if timed:
+                ev["idx"][0].record()
+            st.index(l)
+            if timed:
+                ev["idx"][1].record()
+                ev["att4"][0].record()
+            st.attend_c4a(l)
+            if timed:
+                ev["att4"][1].record()
+                torch.cuda.synchronize()
+                tot["idx"] += ev["idx"][0].elapsed_time(ev["idx"][1])
+                tot["att4"] += ev["att4"][0].elapsed_time(ev["att4"][1])
+        for l in range(nl128):
+            if timed:
+                ev["att128"][0].record()
+            st.attend_c128a(l)
+            if timed:
+                ev["att128"][1].record()
+                torch.cuda.synchronize()
+                tot["att128"] += ev["att128"][0].elapsed_time(ev["att128"][1])
+    for k in tot:
+        tot[k] /= args.steps
+    idx_b, a4_b, a128_b = st.bytes()
+    step_ms = sum(tot.values())
+    res = {"step_ms": step_ms, "tokens_per_s": st.B / (step_ms * 1e-3),
+           "indexer": {"ms_per_layer": tot["idx"] / nl4, "gbs": idx_b / (tot["idx"] / nl4 * 1e-3) / 1e9},
+           "c4a_attention": {"ms_per_layer": tot["att4"] / nl4, "gbs": a4_b / (tot["att4"] / nl4 * 1e-3) / 1e9},
+           "c128a_attention": {"ms_per_layer": tot["att128"] / nl128, "gbs": a128_b / (tot["att128"] / nl128 * 1e-3) / 1e9},
+           "step_gbs": (nl4 * (idx_b + a4_b) + nl128 * a128_b) / (step_ms * 1e-3) / 1e9,
+           "status": int(st.status.item())}
+    res["step_frac"] = res["step_gbs"] / peak
+    return {"config": "61-layer mixed step (30 c4a with indexer top-512 + 31 c128a), batch 128, "
+                      "context U[1K, 256K], 64 heads, fp8 KV", "results": res}
+
+
+DTYPE = "f16"
 
 
 def main():
@@ -442,6 +671,10 @@ def main():
         return
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
+    if args.config in (3, 4) and world == 1:
+        print(json.dumps(run_compress(args, device) if args.config == 3 else run_mixed(args, device)),
+              flush=True)
+        return
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),

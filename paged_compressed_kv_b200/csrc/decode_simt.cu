@@ -258,7 +258,7 @@ DecodePlan plan_decode(int batch, int heads, int max_seq_len, int ratio, int win
     p.path = 1;
     p.items_max = (n_sel + 127) / 128 * 128 + n_win;
     p.split = 128;
-    p.n_splits = max(1, num_sms);
+    p.n_splits = max(1, min(num_sms, 160));  // the merge holds <= 160 weights per sequence
     p.ws_bytes = decode_tc_workspace_bytes(batch, p.n_splits);
     return p;
   }

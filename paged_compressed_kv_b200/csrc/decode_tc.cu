@@ -855,33 +855,51 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
 // blocks whose tile ranges cover the sequence, normalise, inverse RoPE at
 // position L - 1, store bf16
 __global__ void __launch_bounds__(128) decode_tc_merge_kernel(DecodeArgs a) {
+  __shared__ int slot_lo, slot_hi;      // blocks whose tile ranges meet the sequence
+  __shared__ float w_sh[160];           // their weights (max blocks per sequence: SMs)
+  __shared__ float l_sh;
   const int h = blockIdx.x, b = blockIdx.y;
-  const int G = a.n_splits;
-  const long long T = a.cum[a.batch];
-  const int c0 = a.cum[b], c1 = a.cum[b + 1];
   const int d0 = threadIdx.x * 4;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f}, L = 0.f;
-  if (c1 > c0) {
-    const int cf = (int)(((long long)(c0 + 1) * G + T - 1) / T) - 1;
-    const int cl = (int)(((long long)c1 * G + T - 1) / T) - 1;
+  if (threadIdx.x == 0) {
+    const int G = a.n_splits;
+    const long long T = a.cum[a.batch];
+    const int c0 = a.cum[b], c1 = a.cum[b + 1];
+    int lo = 0, hi = -1;
+    if (c1 > c0) {
+      lo = (int)(((long long)(c0 + 1) * G + T - 1) / T) - 1;
+      hi = (int)(((long long)c1 * G + T - 1) / T) - 1;
+      // skip blocks with empty ranges at either end (only when G > T)
+      while (lo <= hi && (long long)(lo + 1) * T / G <= (long long)lo * T / G) ++lo;
+    }
     float M = -INFINITY;
-    for (int c = cf; c <= cl; ++c) {
+    for (int c = lo; c <= hi; ++c) {
       const long long s0 = (long long)c * T / G, s1 = (long long)(c + 1) * T / G;
-      if (s1 <= c0 || s0 >= c1 || s1 <= s0) continue;
-      M = fmaxf(M, a.part_ml[(((size_t)b + c) * kH + h) * 2]);
+      w_sh[c - lo] = (s1 <= s0) ? -INFINITY : a.part_ml[(((size_t)b + c) * kH + h) * 2];
+      M = fmaxf(M, w_sh[c - lo]);
     }
-    for (int c = cf; c <= cl; ++c) {
-      const long long s0 = (long long)c * T / G, s1 = (long long)(c + 1) * T / G;
-      if (s1 <= c0 || s0 >= c1 || s1 <= s0) continue;
-      const size_t row = ((size_t)b + c) * kH + h;
-      const float w = exp2f(a.part_ml[row * 2] - M);
-      L = fmaf(w, a.part_ml[row * 2 + 1], L);
-      const float4 o = *reinterpret_cast<const float4*>(a.part_o + row * kD + d0);
-      acc[0] = fmaf(w, o.x, acc[0]);
-      acc[1] = fmaf(w, o.y, acc[1]);
-      acc[2] = fmaf(w, o.z, acc[2]);
-      acc[3] = fmaf(w, o.w, acc[3]);
+    float L = 0.f;
+    for (int c = lo; c <= hi; ++c) {
+      const float m = w_sh[c - lo];
+      const float w = m == -INFINITY ? 0.f : exp2f(m - M);
+      w_sh[c - lo] = w;
+      if (w > 0.f) L = fmaf(w, a.part_ml[(((size_t)b + c) * kH + h) * 2 + 1], L);
     }
+    slot_lo = lo;
+    slot_hi = hi;
+    l_sh = L;
+  }
+  __syncthreads();
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const float L = l_sh;
+  for (int c = slot_lo; c <= slot_hi; ++c) {
+    const float w = w_sh[c - slot_lo];
+    if (w == 0.f) continue;
+    const size_t row = ((size_t)b + c) * kH + h;
+    const float4 o = *reinterpret_cast<const float4*>(a.part_o + row * kD + d0);
+    acc[0] = fmaf(w, o.x, acc[0]);
+    acc[1] = fmaf(w, o.y, acc[1]);
+    acc[2] = fmaf(w, o.z, acc[2]);
+    acc[3] = fmaf(w, o.w, acc[3]);
   }
   float o[4];
   const float inv = L > 0.f ? 1.f / L : 0.f;

@@ -6,13 +6,18 @@
 // entry's fp32 scale. Ranking: score descending, index ascending, -0 == +0.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace v4kv {
 
 constexpr int kIdxMaxDim = 512;
 constexpr int kScoreThreads = 256;
+constexpr int kScoreChunk = 2048;   // entries per scoring block (8 per thread)
 constexpr int kSelectThreads = 1024;
 constexpr int kMaxK = 2048;
+constexpr int kBins = 4096;         // histogram of the top 12 bits of the ranking key
+constexpr int kBinShift = 20;
+constexpr int kCandCap = 1024;      // entries of the threshold bin sorted directly
 
 __host__ __device__ __forceinline__ int visible(int L, int W, int r) { return max(0, L - W) / r; }
 
@@ -40,44 +45,23 @@ __device__ void quantise_query(const float* q, int dim, float* q_f, float* red, 
   __syncthreads();
 }
 
-// grid (chunks, batch): each thread scores one entry at a time
-__global__ void __launch_bounds__(kScoreThreads) index_score_kernel(IndexArgs a) {
-  __shared__ __align__(16) float q_f[kIdxMaxDim];
-  __shared__ float red[32];
-  const int b = blockIdx.y;
-  const int L = seq_len_of(a, b);
-  const int n_vis = visible(L, a.window_len, a.ratio);
-  const int j0 = blockIdx.x * a.chunk;
-  if (j0 >= n_vis) return;
-  const int dim = a.cache.dim;
-  quantise_query(a.q_idx + (size_t)b * dim, dim, q_f, red, nullptr);
-  const int j1 = min(n_vis, j0 + a.chunk);
-  const int32_t* bt = a.cache.block_table + (size_t)b * a.cache.max_blocks;
-  const uint8_t* base = reinterpret_cast<const uint8_t*>(a.cache.data);
-  for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
-    const int p = page_of(bt, a.cache.max_blocks, j, a.cache.spb, a.cache.num_pages, a.dev_status);
-    float score = 0.f;
-    if (p >= 0) {
-      const long long slot = (long long)p * a.cache.spb + (j % a.cache.spb);
-      const uint8_t* key = base + slot * dim;
-      float acc = 0.f;
-      for (int d = 0; d < dim; d += 16) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(key + d);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 lo = __half22float2(e4m3x2_to_half2((uint16_t)(w[i] & 0xffff)));
-          const float2 hi = __half22float2(e4m3x2_to_half2((uint16_t)(w[i] >> 16)));
-          acc = fmaf(q_f[d + 4 * i + 0], lo.x, acc);
-          acc = fmaf(q_f[d + 4 * i + 1], lo.y, acc);
-          acc = fmaf(q_f[d + 4 * i + 2], hi.x, acc);
-          acc = fmaf(q_f[d + 4 * i + 3], hi.y, acc);
-        }
-      }
-      score = __fmul_rn(acc, a.cache.scales[slot]);
-    }
-    a.scores_ws[(size_t)b * a.ws_stride + j] = score;
-  }
+// acc = fl32(acc + q*k) for four consecutive dims, in ascending order; k4
+// holds four fp8 codes (lowest byte first), q01 / q23 the query's f16 pairs.
+// Both factors are exact in f16, so each step is the fp32 fused multiply-add
+// of the exact product.
+__device__ __forceinline__ float fma4_fp8(float acc, uint32_t k4, uint32_t q01, uint32_t q23) {
+  const __half2 k01 = e4m3x2_to_half2((uint16_t)(k4 & 0xffffu));
+  const __half2 k23 = e4m3x2_to_half2((uint16_t)(k4 >> 16));
+  const uint32_t a = *reinterpret_cast<const uint32_t*>(&k01);
+  const uint32_t c = *reinterpret_cast<const uint32_t*>(&k23);
+  asm("{\n\t.reg .f16 a0, a1, b0, b1, c0, c1, d0, d1;\n\t"
+      "mov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+      "mov.b32 {c0, c1}, %3;\n\tmov.b32 {d0, d1}, %4;\n\t"
+      "fma.rn.f32.f16 %0, a0, b0, %0;\n\tfma.rn.f32.f16 %0, a1, b1, %0;\n\t"
+      "fma.rn.f32.f16 %0, c0, d0, %0;\n\tfma.rn.f32.f16 %0, c1, d1, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(a), "r"(q01), "r"(c), "r"(q23));
+  return acc;
 }
 
 // order-preserving map of fp32 onto uint32 (larger float -> larger key)
@@ -86,6 +70,84 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   if (f == 0.f) u = 0u;  // -0 == +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+
+// grid (chunks of kScoreChunk entries, batch); 256 threads, each scoring two
+// entries at a time with all their row loads in flight. Also builds the
+// histogram of the top 12 key bits of every sequence (workspace hist[b][]).
+__global__ void __launch_bounds__(kScoreThreads) index_score_kernel(IndexArgs a) {
+  __shared__ __align__(16) uint32_t q16[kIdxMaxDim / 2];  // query codes as f16 pairs
+  __shared__ uint32_t hist[kBins];
+  __shared__ float red[32];
+  const int b = blockIdx.y;
+  const int L = seq_len_of(a, b);
+  const int n_vis = visible(L, a.window_len, a.ratio);
+  const int j0 = blockIdx.x * kScoreChunk;
+  if (j0 >= n_vis) return;
+  const int dim = a.cache.dim;
+  {
+    const float* q = a.q_idx + (size_t)b * dim;
+    float m = 0.f;
+    for (int d = threadIdx.x; d < dim; d += blockDim.x) m = fmaxf(m, fabsf(q[d]));
+    const float amax = block_reduce<true>(m, red);
+    const float scale = amax == 0.f ? 1.f : __fdiv_rn(amax, kE4m3Max);
+    for (int d = 2 * threadIdx.x; d < dim; d += 2 * blockDim.x) {
+      const uint16_t c2 = float2_to_e4m3x2(__fdiv_rn(q[d], scale), __fdiv_rn(q[d + 1], scale));
+      const __half2 h = e4m3x2_to_half2(c2);
+      q16[d / 2] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+  }
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
+  const int j1 = min(n_vis, j0 + kScoreChunk);
+  const int32_t* bt = a.cache.block_table + (size_t)b * a.cache.max_blocks;
+  const uint8_t* base = reinterpret_cast<const uint8_t*>(a.cache.data);
+  const int nq = dim / 16;  // 16-byte chunks per key
+  for (int jj = j0 + threadIdx.x; jj < j1; jj += 2 * blockDim.x) {
+    const int ja = jj, jb = jj + blockDim.x;
+    const bool hb = jb < j1;
+    const int pa = page_of(bt, a.cache.max_blocks, ja, a.cache.spb, a.cache.num_pages, a.dev_status);
+    const int pb = hb ? page_of(bt, a.cache.max_blocks, jb, a.cache.spb, a.cache.num_pages, a.dev_status) : -1;
+    const long long sa = pa < 0 ? -1 : (long long)pa * a.cache.spb + ja % a.cache.spb;
+    const long long sb = pb < 0 ? -1 : (long long)pb * a.cache.spb + jb % a.cache.spb;
+    float acc_a = 0.f, acc_b = 0.f;
+    for (int c0 = 0; c0 < nq; c0 += 8) {  // up to 128 dims per round, loads first
+      uint4 ra[8], rb[8];
+      const int nc = min(8, nq - c0);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        ra[c] = (c < nc && sa >= 0) ? *reinterpret_cast<const uint4*>(base + sa * dim + 16 * (c0 + c)) : make_uint4(0, 0, 0, 0);
+        rb[c] = (c < nc && sb >= 0) ? *reinterpret_cast<const uint4*>(base + sb * dim + 16 * (c0 + c)) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        if (c >= nc) break;
+        const uint4 qa = *reinterpret_cast<const uint4*>(&q16[8 * (c0 + c)]);
+        const uint4 qb = *reinterpret_cast<const uint4*>(&q16[8 * (c0 + c) + 4]);
+        acc_a = fma4_fp8(acc_a, ra[c].x, qa.x, qa.y);
+        acc_a = fma4_fp8(acc_a, ra[c].y, qa.z, qa.w);
+        acc_a = fma4_fp8(acc_a, ra[c].z, qb.x, qb.y);
+        acc_a = fma4_fp8(acc_a, ra[c].w, qb.z, qb.w);
+        acc_b = fma4_fp8(acc_b, rb[c].x, qa.x, qa.y);
+        acc_b = fma4_fp8(acc_b, rb[c].y, qa.z, qa.w);
+        acc_b = fma4_fp8(acc_b, rb[c].z, qb.x, qb.y);
+        acc_b = fma4_fp8(acc_b, rb[c].w, qb.z, qb.w);
+      }
+    }
+    const float score_a = sa >= 0 ? __fmul_rn(acc_a, a.cache.scales[sa]) : 0.f;
+    a.scores_ws[(size_t)b * a.ws_stride + ja] = score_a;
+    atomicAdd(&hist[score_key(score_a) >> kBinShift], 1u);
+    if (hb) {
+      const float score_b = sb >= 0 ? __fmul_rn(acc_b, a.cache.scales[sb]) : 0.f;
+      a.scores_ws[(size_t)b * a.ws_stride + jb] = score_b;
+      atomicAdd(&hist[score_key(score_b) >> kBinShift], 1u);
+    }
+  }
+  __syncthreads();
+  uint32_t* gh = a.hist_ws + (size_t)b * kBins;
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x)
+    if (hist[i]) atomicAdd(&gh[i], hist[i]);
+}
+
 
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* sh, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -113,15 +175,236 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
   return before;
 }
 
-// one block per sequence: radix select of the k-th largest key, collect, sort
+// ---- 128-byte keys (dim 128) on pages of a multiple of 64 entries.
+// Each group of 64 consecutive entries is 8 KB of one page, copied by one TMA
+// box with 128-byte swizzle: 16-byte chunk c of row r lands at chunk c ^ (r % 8),
+// so the eight threads of a quarter-warp, each reading chunk c of its own row,
+// hit eight different bank groups. Stages of 256 entries (four boxes) rotate
+// through a three-deep ring; every thread scores one entry of each stage with
+// the same ascending-d chain as the generic kernel.
+constexpr int kTmaBox = 64;                    // rows per box
+constexpr int kTmaBatch = 256;                 // entries per stage = threads
+constexpr int kTmaStages = 3;
+constexpr int kTmaChunk = 2048;                // entries per block
+constexpr int kTmaGroups = kTmaChunk / kTmaBox;
+constexpr uint32_t kStageBytes = kTmaBatch * 128;
+constexpr size_t kTmaSmem = 1024 + kTmaStages * kStageBytes + (kBins / 2) * 4 + 64 * 4 +
+                            kTmaGroups * 8 + 32 * 4 + kTmaStages * 8 + 16;
+
+__global__ void __launch_bounds__(kTmaBatch) index_score_tma_kernel(const __grid_constant__ CUtensorMap keys,
+                                                                    IndexArgs a) {
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* stages = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* hist2 = reinterpret_cast<uint32_t*>(stages + kTmaStages * kStageBytes);  // 16-bit pairs
+  uint32_t* q16 = hist2 + kBins / 2;
+  long long* row0 = reinterpret_cast<long long*>(q16 + 64);  // first slot of each group, -1 if bad
+  float* red = reinterpret_cast<float*>(row0 + kTmaGroups);
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + 32);
+  int* abort_sh = reinterpret_cast<int*>(full + kTmaStages);
+  const int b = blockIdx.y;
+  const int L = seq_len_of(a, b);
+  const int n_vis = visible(L, a.window_len, a.ratio);
+  const int j0 = blockIdx.x * kTmaChunk;
+  if (j0 >= n_vis) return;
+  const int t = threadIdx.x;
+  const int j1 = min(n_vis, j0 + kTmaChunk);
+  const int ngroups = (j1 - j0 + kTmaBox - 1) / kTmaBox;
+  const int nb = (j1 - j0 + kTmaBatch - 1) / kTmaBatch;
+  const int spb = a.cache.spb;
+  if (t < kTmaGroups) {
+    long long r = -1;
+    if (t < ngroups) {
+      const long long g0 = (long long)j0 + (long long)t * kTmaBox;  // first entry of the group
+      const long long blk = g0 / spb;
+      const int32_t* bt = a.cache.block_table + (size_t)b * a.cache.max_blocks;
+      const int p = blk < a.cache.max_blocks ? bt[blk] : -1;
+      if (p >= 0 && p < a.cache.num_pages) r = (long long)p * spb + g0 % spb;
+      else flag(a.dev_status, V4KV_DEV_BAD_PAGE);
+    }
+    row0[t] = r;
+  }
+  if (t == 0) {
+    for (int s = 0; s < kTmaStages; ++s) tc::mbar_init(&full[s], 1);
+    *abort_sh = 0;
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  const uint32_t stages_s = tc::smem_u32(stages);
+  auto issue = [&](int bi) {  // thread 0: the boxes of stage bi
+    const int s = bi % kTmaStages;
+    uint32_t bytes = 0;
+    for (int k = 0; k < kTmaBatch / kTmaBox; ++k) {
+      const int g = bi * (kTmaBatch / kTmaBox) + k;
+      if (g < ngroups && row0[g] >= 0) bytes += kTmaBox * 128;
+    }
+    tc::mbar_arrive_expect_tx(&full[s], bytes);
+    for (int k = 0; k < kTmaBatch / kTmaBox; ++k) {
+      const int g = bi * (kTmaBatch / kTmaBox) + k;
+      if (g < ngroups && row0[g] >= 0)
+        tc::tma_load_2d(stages_s + s * kStageBytes + k * kTmaBox * 128, &keys, 0, (int)row0[g], &full[s]);
+    }
+  };
+  int issued = 0;  // thread 0: stages issued so far
+  if (t == 0)
+    for (; issued < min(nb, kTmaStages); ++issued) issue(issued);
+  // query codes and histogram while the first boxes are in flight
+  {
+    const float* q = a.q_idx + (size_t)b * 128;
+    float m = 0.f;
+    if (t < 128) m = fabsf(q[t]);
+    const float amax = block_reduce<true>(m, red);
+    const float scale = amax == 0.f ? 1.f : __fdiv_rn(amax, kE4m3Max);
+    if (t < 64) {
+      const uint16_t c2 = float2_to_e4m3x2(__fdiv_rn(q[2 * t], scale), __fdiv_rn(q[2 * t + 1], scale));
+      const __half2 h = e4m3x2_to_half2(c2);
+      q16[t] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+  }
+  for (int i = t; i < kBins / 2; i += kTmaBatch) hist2[i] = 0u;
+  __syncthreads();
+  const int sw = (t & 7) * 16;  // swizzle of this thread's row (stage bases are 1024-aligned)
+  for (int bi = 0; bi < nb; ++bi) {
+    const int s = bi % kTmaStages;
+    const int e = bi * kTmaBatch + t;  // entry offset within the chunk
+    const int j = j0 + e;
+    const long long r = j < j1 ? row0[e / kTmaBox] : -1;
+    const long long slot = r >= 0 ? r + (e % kTmaBox) : -1;
+    const float ks = slot >= 0 ? a.cache.scales[slot] : 0.f;
+    if (!tc::mbar_wait(&full[s], (uint32_t)(bi / kTmaStages) & 1u, abort_sh)) {
+      flag(a.dev_status, V4KV_DEV_TIMEOUT);
+      *abort_sh = 1;
+    }
+    if (j < j1) {
+      float score = 0.f;
+      if (slot >= 0) {
+        const uint8_t* row = stages + s * kStageBytes + t * 128;
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 kv = *reinterpret_cast<const uint4*>(row + ((16 * c) ^ sw));
+          const uint4 qa = *reinterpret_cast<const uint4*>(&q16[8 * c]);
+          const uint4 qb = *reinterpret_cast<const uint4*>(&q16[8 * c + 4]);
+          acc = fma4_fp8(acc, kv.x, qa.x, qa.y);
+          acc = fma4_fp8(acc, kv.y, qa.z, qa.w);
+          acc = fma4_fp8(acc, kv.z, qb.x, qb.y);
+          acc = fma4_fp8(acc, kv.w, qb.z, qb.w);
+        }
+        score = __fmul_rn(acc, ks);
+      }
+      a.scores_ws[(size_t)b * a.ws_stride + j] = score;
+      const uint32_t bin = score_key(score) >> kBinShift;
+      atomicAdd(&hist2[bin >> 1], 1u << (16 * (bin & 1)));
+    }
+    __syncthreads();  // stage s is free again
+    if (t == 0 && issued < nb && !*abort_sh) issue(issued++);
+  }
+  if (*abort_sh && t == 0) {
+    // let copies still in flight land before the block's shared memory is released
+    for (int bi = max(0, issued - kTmaStages); bi < issued; ++bi)
+      tc::mbar_wait(&full[bi % kTmaStages], (uint32_t)(bi / kTmaStages) & 1u, nullptr);
+  }
+  uint32_t* gh = a.hist_ws + (size_t)b * kBins;
+  for (int i = t; i < kBins / 2; i += kTmaBatch) {
+    const uint32_t w = hist2[i];
+    if (w & 0xffffu) atomicAdd(&gh[2 * i], w & 0xffffu);
+    if (w >> 16) atomicAdd(&gh[2 * i + 1], w >> 16);
+  }
+}
+
+// Composite sort key: ranking key in the high word, bitwise-inverted index in
+// the low word, so that a descending sort gives (score desc, index asc).
+__device__ __forceinline__ unsigned long long comp_key(uint32_t key, int j) {
+  return ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)j);
+}
+
+// bitonic sort of v[0 .. n) (n a power of two) in descending order
+__device__ __forceinline__ void bitonic_desc(unsigned long long* v, int n) {
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int jx = i ^ stride;
+        if (jx > i) {
+          const bool desc = (i & size) == 0;
+          const unsigned long long x = v[i], y = v[jx];
+          if (desc ? (x < y) : (x > y)) {
+            v[i] = y;
+            v[jx] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Exact radix select, 8 bits per pass from the top: the keys above the k-th
+// largest in any order, then the ties at it by ascending index. Used when the
+// histogram's threshold bin holds more than kCandCap entries.
+__device__ void radix_select_exact(const float* sc, int n, int k, unsigned long long* sel,
+                                   uint32_t* hist, uint32_t* scan_sh, uint32_t* pick_sh,
+                                   uint32_t* n_sel_sh) {
+  uint32_t prefix = 0, mask = 0, remaining = (uint32_t)k;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+      const uint32_t key = score_key(sc[j]);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t cum = 0, digit = 0;
+      for (int d = 255; d >= 0; --d) {
+        if (cum + hist[d] >= remaining) {
+          digit = (uint32_t)d;
+          break;
+        }
+        cum += hist[d];
+      }
+      pick_sh[0] = digit;
+      pick_sh[1] = remaining - cum;
+    }
+    __syncthreads();
+    prefix |= pick_sh[0] << shift;
+    mask |= 255u << shift;
+    remaining = pick_sh[1];
+    __syncthreads();
+  }
+  const uint32_t T = prefix;
+  if (threadIdx.x == 0) *n_sel_sh = 0;
+  __syncthreads();
+  for (int j = threadIdx.x; j < n; j += blockDim.x) {
+    const uint32_t key = score_key(sc[j]);
+    if (key > T) sel[atomicAdd(n_sel_sh, 1u)] = comp_key(key, j);
+  }
+  __syncthreads();
+  uint32_t taken = 0;
+  const uint32_t base_pos = *n_sel_sh;
+  for (int j0 = 0; j0 < n && taken < remaining; j0 += blockDim.x) {
+    const int j = j0 + threadIdx.x;
+    const uint32_t is_tie = (j < n && score_key(sc[j]) == T) ? 1u : 0u;
+    uint32_t total;
+    const uint32_t before = block_exclusive_scan(is_tie, scan_sh, &total);
+    if (is_tie && taken + before < remaining) sel[base_pos + taken + before] = comp_key(T, j);
+    taken += total;
+  }
+  __syncthreads();
+}
+
+// One block per sequence. The histogram of the top 12 key bits (built while
+// scoring) gives the bin holding the k-th largest key; one pass keeps every
+// entry above that bin and collects the bin's own entries, which are sorted
+// to take the rest. The k results are then sorted (score desc, index asc).
 __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexArgs a) {
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[kBins];
   __shared__ uint32_t scan_sh[32];
   __shared__ unsigned long long sel[kMaxK];
+  __shared__ unsigned long long cand[kCandCap];
   __shared__ float red[32];
   __shared__ float q_f[kIdxMaxDim];
   __shared__ float qs_sh;
-  __shared__ uint32_t n_sel_sh;
+  __shared__ uint32_t n_sel_sh, n_cand_sh, bin_sh, above_sh;
   __shared__ uint32_t pick_sh[2];
 
   const int b = blockIdx.x;
@@ -134,85 +417,74 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexArgs 
   int kpow = 1;
   while (kpow < k) kpow <<= 1;
   for (int i = threadIdx.x; i < kpow; i += blockDim.x) sel[i] = 0ull;
-  if (threadIdx.x == 0) n_sel_sh = 0;
+  if (threadIdx.x == 0) {
+    n_sel_sh = 0;
+    n_cand_sh = 0;
+    bin_sh = 0xffffffffu;  // "not found" -> exact path
+    above_sh = 0;
+  }
   __syncthreads();
 
   if (n <= k) {
-    for (int j = threadIdx.x; j < n; j += blockDim.x)
-      sel[j] = ((unsigned long long)score_key(sc[j]) << 32) | (0xffffffffu - (uint32_t)j);
+    for (int j = threadIdx.x; j < n; j += blockDim.x) sel[j] = comp_key(score_key(sc[j]), j);
     __syncthreads();
   } else {
-    // radix select, 8 bits per pass from the top: find key T, the k-th largest
-    uint32_t prefix = 0, mask = 0, remaining = (uint32_t)k;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-      __syncthreads();
-      for (int j = threadIdx.x; j < n; j += blockDim.x) {
-        const uint32_t key = score_key(sc[j]);
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-      }
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        uint32_t cum = 0, digit = 0;
-        for (int d = 255; d >= 0; --d) {
-          if (cum + hist[d] >= remaining) {
-            digit = (uint32_t)d;
-            break;
-          }
-          cum += hist[d];
-        }
-        pick_sh[0] = digit;
-        pick_sh[1] = remaining - cum;
-      }
-      __syncthreads();
-      prefix |= pick_sh[0] << shift;
-      mask |= 255u << shift;
-      remaining = pick_sh[1];
-      __syncthreads();
+    // threshold bin: count(bins above) < k <= count(bins at or above)
+    const uint32_t* gh = a.hist_ws + (size_t)b * kBins;
+    uint32_t local = 0, cnt[kBins / kSelectThreads];
+#pragma unroll
+    for (int i = 0; i < kBins / kSelectThreads; ++i) {
+      cnt[i] = gh[kBins - 1 - (threadIdx.x * (kBins / kSelectThreads) + i)];  // descending bins
+      local += cnt[i];
     }
-    const uint32_t T = prefix;
-    // strictly greater keys: any order (sorted below)
+    uint32_t total;
+    const uint32_t before = block_exclusive_scan(local, scan_sh, &total);
+    if (before < (uint32_t)k && (uint32_t)k <= before + local) {
+      uint32_t run = before;
+#pragma unroll
+      for (int i = 0; i < kBins / kSelectThreads; ++i) {
+        if (run + cnt[i] >= (uint32_t)k) {
+          bin_sh = kBins - 1 - (threadIdx.x * (kBins / kSelectThreads) + i);
+          above_sh = run;
+          break;
+        }
+        run += cnt[i];
+      }
+    }
+    __syncthreads();
+    const uint32_t tb = bin_sh, above = above_sh;
     for (int j = threadIdx.x; j < n; j += blockDim.x) {
       const uint32_t key = score_key(sc[j]);
-      if (key > T) {
-        const uint32_t pos = atomicAdd(&n_sel_sh, 1u);
-        sel[pos] = ((unsigned long long)key << 32) | (0xffffffffu - (uint32_t)j);
+      const uint32_t bin = key >> kBinShift;
+      if (tb == 0xffffffffu) break;
+      if (bin > tb) {
+        const uint32_t p = atomicAdd(&n_sel_sh, 1u);
+        if (p < (uint32_t)k) sel[p] = comp_key(key, j);
+      } else if (bin == tb) {
+        const uint32_t p = atomicAdd(&n_cand_sh, 1u);
+        if (p < (uint32_t)kCandCap) cand[p] = comp_key(key, j);
       }
     }
     __syncthreads();
-    // ties at T: the `remaining` lowest indices, found in ascending index order
-    uint32_t taken = 0;
-    const uint32_t base_pos = n_sel_sh;
-    for (int j0 = 0; j0 < n && taken < remaining; j0 += blockDim.x) {
-      const int j = j0 + threadIdx.x;
-      const uint32_t is_tie = (j < n && score_key(sc[j]) == T) ? 1u : 0u;
-      uint32_t total;
-      const uint32_t before = block_exclusive_scan(is_tie, scan_sh, &total);
-      if (is_tie && taken + before < remaining)
-        sel[base_pos + taken + before] = ((unsigned long long)T << 32) | (0xffffffffu - (uint32_t)j);
-      taken += total;
-    }
-    __syncthreads();
-  }
-
-  // bitonic sort of sel[0 .. kpow) descending (score desc, then index asc)
-  for (int size = 2; size <= kpow; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < kpow; i += blockDim.x) {
-        const int jx = i ^ stride;
-        if (jx > i) {
-          const bool desc = (i & size) == 0;
-          const unsigned long long x = sel[i], y = sel[jx];
-          if (desc ? (x < y) : (x > y)) {
-            sel[i] = y;
-            sel[jx] = x;
-          }
-        }
-      }
+    const uint32_t nc = n_cand_sh;
+    if (tb == 0xffffffffu || nc > (uint32_t)kCandCap || n_sel_sh != above) {
+      // too many entries share the threshold bin: exact radix path
+      for (int i = threadIdx.x; i < kpow; i += blockDim.x) sel[i] = 0ull;
+      __syncthreads();
+      radix_select_exact(sc, n, k, sel, hist, scan_sh, pick_sh, &n_sel_sh);
+    } else {
+      int cpow = 1;
+      while (cpow < (int)nc) cpow <<= 1;
+      for (int i = nc + threadIdx.x; i < cpow; i += blockDim.x) cand[i] = 0ull;
+      __syncthreads();
+      bitonic_desc(cand, cpow);
+      const int need = k - (int)above;
+      for (int i = threadIdx.x; i < need; i += blockDim.x) sel[above + i] = cand[i];
       __syncthreads();
     }
   }
+
+  bitonic_desc(sel, kpow);
   const int valid = min(n, k);
   for (int i = threadIdx.x; i < k; i += blockDim.x) {
     int32_t idx = -1;
@@ -226,21 +498,40 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexArgs 
   }
 }
 
+static size_t score_stride(int nv) { return ((size_t)max(nv, 1) + 63) / 64 * 64; }
+
 size_t index_workspace_bytes(int batch, int max_seq_len, int ratio, int window_len) {
   const int nv = visible(max_seq_len, window_len, ratio);
-  const size_t stride = ((size_t)max(nv, 1) + 63) / 64 * 64;
-  return (size_t)batch * stride * sizeof(float);
+  return (size_t)batch * score_stride(nv) * sizeof(float) + (size_t)batch * kBins * sizeof(uint32_t);
 }
 
 cudaError_t launch_index_topk(IndexArgs a, int max_seq_len, cudaStream_t stream) {
   const int nv = visible(max_seq_len, a.window_len, a.ratio);
   a.max_len = max_seq_len;
-  a.ws_stride = (int)(((size_t)max(nv, 1) + 63) / 64 * 64);
-  a.chunk = 4096;
-  if (nv > 0) {
-    dim3 grid((nv + a.chunk - 1) / a.chunk, a.batch);
+  a.ws_stride = (int)score_stride(nv);
+  a.chunk = kScoreChunk;
+  a.hist_ws = reinterpret_cast<uint32_t*>(a.scores_ws + (size_t)a.batch * a.ws_stride);
+  cudaError_t e = cudaMemsetAsync(a.hist_ws, 0, (size_t)a.batch * kBins * sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return e;
+  // 128-byte keys on pages of whole 64-entry groups go through TMA boxes
+  const bool tma = a.cache.dim == 128 && a.cache.spb % kTmaBox == 0 &&
+                   (reinterpret_cast<uintptr_t>(a.cache.data) & 15) == 0 &&
+                   (long long)a.cache.num_pages * a.cache.spb <= 0x7fffffffLL;
+  if (nv > 0 && tma) {
+    CUtensorMap keys;
+    e = encode_rows_u8(&keys, a.cache.data, (uint64_t)a.cache.num_pages * a.cache.spb, 128, kTmaBox);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(index_score_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kTmaSmem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((nv + kTmaChunk - 1) / kTmaChunk, a.batch);
+    index_score_tma_kernel<<<grid, kTmaBatch, kTmaSmem, stream>>>(keys, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  } else if (nv > 0) {
+    dim3 grid((nv + kScoreChunk - 1) / kScoreChunk, a.batch);
     index_score_kernel<<<grid, kScoreThreads, 0, stream>>>(a);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   index_select_kernel<<<a.batch, kSelectThreads, 0, stream>>>(a);

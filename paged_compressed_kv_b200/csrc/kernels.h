@@ -1,6 +1,7 @@
 // Internal launch interface between the C ABI (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -53,6 +54,7 @@ struct IndexArgs {
   int32_t* topk_out;
   float* score_out;
   float* scores_ws;  // [batch, ws_stride] scratch
+  uint32_t* hist_ws; // [batch, 4096] histogram of the top 12 bits of the ranking key
   int32_t* dev_status;
   PoolArgs cache;
   int batch;
@@ -114,5 +116,10 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);  // sweep + merge
 size_t decode_tc_workspace_bytes(int batch, int num_sms);
+
+// Tensor map over `rows` rows of `row_bytes` bytes (uint8, 2-D, 128-byte
+// swizzle), boxes of `row_bytes` x `box_rows`. base must be 16-byte aligned.
+cudaError_t encode_rows_u8(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes,
+                           uint32_t box_rows);
 
 }  // namespace v4kv

@@ -67,15 +67,27 @@ __device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, 
 }
 
 // Wait until the phase with the given parity has completed. Returns false if
-// it did not complete within kWaitCycles or if *abort became non-zero.
+// it did not complete within kWaitCycles or if *abort (when given) became non-zero.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_test(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_test_sleep(bar, parity, 100000u)) return true;
-    if (*abort) return false;
+    if (abort && *abort) return false;
     if (clock64() - t0 > kWaitCycles) return false;
   }
+}
+
+// ------------------------------------------------------------------ TMA
+// 2-D tiled tensor copy global -> shared of one box at coordinates (x, y),
+// completing `bytes` of transaction count on the mbarrier (no multicast).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // ------------------------------------------------------------------ fences

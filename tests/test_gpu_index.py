@@ -78,3 +78,37 @@ def test_full_size_sampled():
         sel, rs = oracle_index(q[b], pool, b, int(lens[b]), 4, 128, 512)
         assert np.array_equal(got[b], sel)
         assert np.array_equal(sc[b].view(np.uint32), rs.view(np.uint32))
+
+
+@pytest.mark.parametrize("dim", [64, 256])
+def test_other_key_widths(dim):
+    # keys that are not 128 bytes take the generic scoring kernel
+    lens = [300, 128 + 4 * 1000 + 3, 30000]
+    pool, q = build(320 + dim, lens, dim=dim)
+    got, sc, st = run(pool, q, lens, 512)
+    assert st == 0
+    for b, L in enumerate(lens):
+        sel, rs = oracle_index(q[b], pool, b, L, 4, 128, 512)
+        assert np.array_equal(got[b], sel), f"seq {b}"
+        assert np.array_equal(sc[b].view(np.uint32), rs.view(np.uint32)), f"seq {b}"
+
+
+def test_bad_page_is_flagged_and_scored_zero():
+    # a block-table entry past the pool: the kernel flags it and scores the
+    # block's entries 0, the same as an oracle pool whose block is all-zero codes
+    from paged_compressed_kv_b200 import v4kv
+    from tests.helpers import NpPool
+    lens = [128 + 4 * 5000, 9000]
+    pool, q = build(330, lens)
+    P, spb, D = pool.data.shape
+    zero = NpPool(np.concatenate([pool.data, np.zeros((1, spb, D), np.uint8)]),
+                  np.concatenate([pool.scales, np.ones((1, spb), np.float32)]),
+                  pool.bt.copy(), "fp8")
+    zero.bt[0, 3] = P
+    pool.bt[0, 3] = P  # past the end of the device pool
+    got, sc, st = run(pool, q, lens, 512)
+    assert st & v4kv.V4KV_DEV_BAD_PAGE
+    for b, L in enumerate(lens):
+        sel, rs = oracle_index(q[b], zero, b, L, 4, 128, 512)
+        assert np.array_equal(got[b], sel), f"seq {b}"
+        assert np.array_equal(sc[b].view(np.uint32), rs.view(np.uint32)), f"seq {b}"
