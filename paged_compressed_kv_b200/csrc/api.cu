@@ -251,13 +251,7 @@ v4kv_status v4kv_decode_attention(const void* q, int32_t q_dtype, int32_t batch,
   a.topk = topk;
   a.out = out;
   a.part_o = static_cast<float*>(workspace);
-  if (plan.path == 1) {
-    const size_t slots = (size_t)batch + plan.n_splits;
-    a.part_ml = a.part_o + slots * heads * 512;
-    a.cum = reinterpret_cast<int32_t*>(a.part_ml + slots * heads * 2);
-  } else {
-    a.part_ml = a.part_o + (size_t)batch * plan.n_splits * heads * 512;
-  }
+  a.part_ml = a.part_o + (size_t)batch * plan.n_splits * heads * 512;
   a.dev_status = dev_status;
   a.main = to_args(main_cache);
   a.window = to_args(window);
@@ -274,7 +268,10 @@ v4kv_status v4kv_decode_attention(const void* q, int32_t q_dtype, int32_t batch,
   a.n_splits = plan.n_splits;
   a.max_len = max_seq_len;
   a.pad_sel = plan.path == 1;
-  if (plan.path == 1) return to_status(launch_decode_tc(a, (cudaStream_t)stream));
+  if (plan.path == 1) {
+    decode_tc_layout(a, workspace);
+    return to_status(launch_decode_tc(a, (cudaStream_t)stream));
+  }
   cudaError_t e = launch_decode_simt(a, (cudaStream_t)stream);
   if (e != cudaSuccess) return V4KV_ERR_CUDA;
   return to_status(launch_decode_merge(a, (cudaStream_t)stream));

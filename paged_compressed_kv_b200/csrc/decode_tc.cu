@@ -281,66 +281,15 @@ __device__ __forceinline__ void cursor_next(Cursor& c, const DecodeArgs& a) {
   }
 }
 
-// q[b] -> f16 in shared memory, scaled by 2^e so that max|q| * 2^e < 2^15;
-// returns sm_scale * log2(e) * 2^-e. Run by `nthreads` threads (thread index
-// t) that meet at named barrier `bar`; `red` holds nthreads/32 floats.
-__device__ __forceinline__ float load_q(const DecodeArgs& a, int b, uint8_t* qsm, float* red, int t,
-                                        int nthreads, int bar) {
-  const size_t qoff = (size_t)b * kH * kD;
-  float m = 0.f;
-  for (int u = t; u < kH * kD / 8; u += nthreads) {
-    const size_t o = qoff + (size_t)u * 8;
-    if (a.q_dtype == V4KV_FP32) {
-      const float4 x0 = reinterpret_cast<const float4*>(a.q)[o / 4];
-      const float4 x1 = reinterpret_cast<const float4*>(a.q)[o / 4 + 1];
-      m = fmaxf(m, fmaxf(fmaxf(fabsf(x0.x), fabsf(x0.y)), fmaxf(fabsf(x0.z), fabsf(x0.w))));
-      m = fmaxf(m, fmaxf(fmaxf(fabsf(x1.x), fabsf(x1.y)), fmaxf(fabsf(x1.z), fabsf(x1.w))));
-    } else {
-      const uint4 r = reinterpret_cast<const uint4*>(a.q)[o / 8];
-      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+constexpr uint32_t kQBytes = kH * kD * 2;  // one query image (f16)
+
+// Start the bulk copy of sequence b's query image into shared memory; the
+// copy completes phase by transaction count on `bar`.
+__device__ __forceinline__ void issue_q(const DecodeArgs& a, int b, uint32_t qdst, uint64_t* bar) {
+  tc::mbar_arrive_expect_tx(bar, kQBytes);
+  const uint8_t* src = a.qh + (size_t)b * kQBytes;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xffff0000u))));
-    }
-  }
-  m = warp_max(m);
-  if ((t & 31) == 0) red[t >> 5] = m;
-  named_sync(bar, nthreads);
-  float amax = 0.f;
-  for (int w = 0; w < nthreads / 32; ++w) amax = fmaxf(amax, red[w]);
-  int e = 0;
-  if (amax > 0.f) {
-    int k;
-    frexpf(amax, &k);  // amax < 2^k
-    e = 15 - k;
-  }
-  const float qs = ldexpf(1.f, e);
-  for (int u = t; u < kH * kD / 8; u += nthreads) {
-    const int h = u / (kD / 8), c8 = u % (kD / 8);  // 8-dim chunk c8 of head h
-    const size_t o = qoff + (size_t)h * kD + c8 * 8;
-    float x[8];
-    if (a.q_dtype == V4KV_FP32) {
-      const float4 x0 = reinterpret_cast<const float4*>(a.q)[o / 4];
-      const float4 x1 = reinterpret_cast<const float4*>(a.q)[o / 4 + 1];
-      x[0] = x0.x; x[1] = x0.y; x[2] = x0.z; x[3] = x0.w;
-      x[4] = x1.x; x[5] = x1.y; x[6] = x1.z; x[7] = x1.w;
-    } else {
-      const uint4 r = reinterpret_cast<const uint4*>(a.q)[o / 8];
-      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        x[2 * i] = __uint_as_float(w[i] << 16);
-        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-      }
-    }
-    uint32_t hv[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) hv[i] = h2u(__floats2half2_rn(x[2 * i] * qs, x[2 * i + 1] * qs));
-    *reinterpret_cast<uint4*>(qsm + (c8 >> 3) * 8192 + tc::sw128_off(h, c8 & 7)) =
-        make_uint4(hv[0], hv[1], hv[2], hv[3]);
-  }
-  tc::fence_proxy_async_smem();
-  return a.sm_scale * 1.4426950408889634f * ldexpf(1.f, -e);
+  for (int k = 0; k < 4; ++k) tc::bulk_load(qdst + k * (kQBytes / 4), src + k * (kQBytes / 4), kQBytes / 4, bar);
 }
 
 // Sum 64 per-lane values over the 32 lanes of a warp (reduce-scatter): lane l
@@ -383,59 +332,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   float* red = reinterpret_cast<float*>(sm + kRedOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kMiscOff + 4);
-  float* k0_slot = reinterpret_cast<float*>(sm + kMiscOff + 8);
   int* range = reinterpret_cast<int*>(sm + kMiscOff + 16);  // x0, x1, b0, lt0
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
 
-  // ---- this block's tile range: T = total tiles, [c*T/G, (c+1)*T/G)
-  if (warp == 0) {
-    long long T = 0;
-    for (int base = 0; base < a.batch; base += 32) {
-      const int bb = base + lane;
-      int t = bb < a.batch ? tiles_of(seq_of(a, bb, a.dev_status)) : 0;
-      T += __reduce_add_sync(0xffffffffu, t);
-    }
-    const int x0 = (int)((long long)cta * T / G), x1 = (int)((long long)(cta + 1) * T / G);
-    // first sequence of the range and the tile within it; block 0 also
-    // publishes the tile prefix sums for the merge
-    int b0 = a.batch, lt0 = 0;
-    long long run = 0;
-    for (int base = 0; base < a.batch; base += 32) {
-      const int bb = base + lane;
-      const int t = bb < a.batch ? tiles_of(seq_of(a, bb, nullptr)) : 0;
-      int incl = t;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const long long before = run + incl - t;  // tiles before sequence bb
-      if (cta == 0 && bb < a.batch) a.cum[bb] = (int32_t)before;
-      const bool mine = bb < a.batch && t > 0 && before <= x0 && x0 < before + t;
-      const unsigned hit = __ballot_sync(0xffffffffu, mine);
-      if (hit && b0 == a.batch) {
-        const int src = __ffs(hit) - 1;
-        b0 = __shfl_sync(0xffffffffu, bb, src);
-        lt0 = x0 - (int)__shfl_sync(0xffffffffu, before, src);
-      }
-      run += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (cta == 0 && lane == 0) a.cum[a.batch] = (int32_t)T;
-    if (lane == 0) {
-      range[0] = x0;
-      range[1] = (b0 < a.batch) ? x1 : x0;
-      range[2] = b0;
-      range[3] = lt0;
-    }
-  }
-  __syncthreads();
-  const int x0 = range[0], x1 = range[1];
-  if (x0 >= x1) return;
-  const int n_tiles = x1 - x0;
-  const int b0 = range[2], lt0 = range[3];
-
+  // barriers and tensor memory first: this overlaps the query-preparation
+  // kernel still running ahead of this one
   if (tid == 0) {
     for (int k = 0; k < 3; ++k) {
       tc::mbar_init(&bars->addr_ready[k], 32);
@@ -449,21 +352,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
     tc::mbar_init(&bars->s_full[1], 1);
     tc::mbar_init(&bars->p_full, 128);
     tc::mbar_init(&bars->pv_done, 1);
-    tc::mbar_init(&bars->q_ready, 128);
+    tc::mbar_init(&bars->q_ready, 1);
     tc::mbar_init(&bars->drain, 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
   if (warp == 8) tc::tmem_alloc(tmem_slot, kTmemCols);
   if (tid < kH) mref[tid] = kNone;
-  if (warp < 8) {
-    const float k0 = load_q(a, b0, sm + kQOff, red, tid, 256, 2);
-    if (tid == 0) *k0_slot = k0;
+  tc::pdl_wait();  // the tile prefix sums and query images are complete from here on
+  tc::pdl_launch_dependents();
+
+  // ---- this block's tile range: T = total tiles, [c*T/G, (c+1)*T/G); the
+  // first sequence b0 is the number of sequences whose tiles end at or before x0
+  if (warp == 0) {
+    const long long T = a.cum[a.batch];
+    const int x0 = (int)((long long)cta * T / G), x1 = (int)((long long)(cta + 1) * T / G);
+    int cnt = 0;
+#pragma unroll 4
+    for (int bb = lane; bb < a.batch; bb += 32) cnt += a.cum[bb + 1] <= x0 ? 1 : 0;
+    const int b0 = __reduce_add_sync(0xffffffffu, cnt);
+    if (lane == 0) {
+      range[0] = x0;
+      range[1] = (b0 < a.batch) ? x1 : x0;
+      range[2] = b0;
+      range[3] = b0 < a.batch ? x0 - a.cum[b0] : 0;
+      if (b0 < a.batch && x0 < x1) issue_q(a, b0, sbase + kQOff, &bars->q_ready);
+    }
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
+  const int x0 = range[0], x1 = range[1];
+  const int n_tiles = x1 - x0;
+  const int b0 = range[2], lt0 = range[3];
   const uint32_t tmem = *tmem_slot;
+  if (x0 >= x1) {
+    // nothing to do: release tensor memory and leave
+    if (warp == 8) tc::tmem_free(tmem, kTmemCols);
+    return;
+  }
 
   if (warp == 9) {
     // ======================= address resolution + L2 prefetch, two tiles ahead
@@ -472,10 +399,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
     for (int t = 0; t < n_tiles; ++t) {
       const int buf = t % 3;
       if (t >= 3 && !tc::mbar_wait(&bars->addr_free[buf], ((t - 3) / 3) & 1, abort_flag)) break;
-      if (t > 0 && cu.lt == 0 && a.q_dtype == V4KV_FP32) {
-        // a new sequence starts: pull its query into L2 as well
-        const uint8_t* qp = reinterpret_cast<const uint8_t*>(a.q) + (size_t)cu.b * kH * kD * 4;
-        for (int k = lane; k < kH * kD * 4 / 128; k += 32) prefetch_l2_line(qp + 128 * k);
+      if (t > 0 && cu.lt == 0) {
+        // a new sequence starts: pull its query image into L2 as well
+        const uint8_t* qp = a.qh + (size_t)cu.b * kQBytes;
+        for (int k = lane; k < (int)kQBytes / 128; k += 32) prefetch_l2_line(qp + 128 * k);
       }
       const int tile0 = cu.lt * kT;
       resolve_tile(a, cu.b, cu.s, tile0, lane, rowptr + buf * kT, meta + buf * kT);
@@ -510,11 +437,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
           if (c == 0) {
             // the converters read this tile's info word before arriving
             first = (info[i % 3] & kInfoFirst) != 0;
-            if (first && i > 0) {
-              ok = tc::mbar_wait(&bars->q_ready, (seg - 1) & 1, abort_flag);
+            if (first) {
+              // the segment's query image has landed in shared memory
+              ok = tc::mbar_wait(&bars->q_ready, seg & 1, abort_flag);
               if (!ok) break;
+              ++seg;
             }
-            if (first) ++seg;
           }
           tc::tc_fence_after();
 #pragma unroll
@@ -622,7 +550,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   } else {
     // ======================= softmax (thread = tile row = TMEM lane)
     const int row = tid;
-    float k0 = *k0_slot;
+    float k0 = a.qk0[b0];
+    int q_issued = 1;  // query copies started by this thread (row 0 only)
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
     {
       uint32_t z[32];
@@ -775,10 +704,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
         const int b_done = cu.b;
         cursor_next(cu, a);
         if (i + 1 < n_tiles) {
-          // QK(i) is complete (S(i) was read), so Q is free: load the next
-          // segment's query while PV(i) runs
-          k0 = load_q(a, cu.b, sm + kQOff, red, row, 128, 1);
-          tc::mbar_arrive(&bars->q_ready);
+          // QK(i) is complete (S(i) was read), so Q is free: copy the next
+          // segment's query image while PV(i) runs
+          k0 = a.qk0[cu.b];
+          if (row == 0) {
+            issue_q(a, cu.b, sbase + kQOff, &bars->q_ready);
+            ++q_issued;
+          }
         }
         ok = tc::mbar_wait(&bars->pv_done, i & 1, abort_flag);
         ok = named_and(1, 128, ok);
@@ -841,6 +773,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       *abort_flag = 1;
       flag(a.dev_status, V4KV_DEV_TIMEOUT);
     }
+    if (row == 0) {
+      // the last query copy has landed before shared memory is released
+      // (normally long since; after an abort it may still be in flight)
+      volatile int never = 0;
+      if (!tc::mbar_wait(&bars->q_ready, (q_issued - 1) & 1, &never)) flag(a.dev_status, V4KV_DEV_TIMEOUT);
+    }
   }
 
   tc::tc_fence_before();
@@ -858,6 +796,7 @@ __global__ void __launch_bounds__(128) decode_tc_merge_kernel(DecodeArgs a) {
   __shared__ int slot_lo, slot_hi;      // blocks whose tile ranges meet the sequence
   __shared__ float w_sh[160];           // their weights (max blocks per sequence: SMs)
   __shared__ float l_sh;
+  tc::pdl_wait();  // the sweep's partial results are complete from here on
   const int h = blockIdx.x, b = blockIdx.y;
   const int d0 = threadIdx.x * 4;
   if (threadIdx.x == 0) {
@@ -924,24 +863,147 @@ __global__ void __launch_bounds__(128) decode_tc_merge_kernel(DecodeArgs a) {
   *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
 }
 
+// grid (batch + 1), 256 threads. Block b < batch writes sequence b's query as
+// the shared-memory image of the first product's B operand: f16, scaled by
+// 2^e so that max|q| * 2^e < 2^15, eight 64-dim atoms of 64 head rows x 128 B
+// in the 128-byte swizzle, so that one linear copy puts it in place; and
+// qk0[b] = sm_scale * log2(e) * 2^-e. Block `batch` writes the tile prefix
+// sums cum[0..batch].
+__global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
+  tc::pdl_launch_dependents();
+  const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  __shared__ float red[8];
+  __shared__ int wsum[8];
+  if (b == a.batch) {
+    int carry = 0;
+    for (int base = 0; base < a.batch; base += 256) {
+      const int bb = base + t;
+      int n = 0;
+      if (bb < a.batch) {
+        if (a.seq_lens[bb] > a.max_len) flag(a.dev_status, V4KV_DEV_OVERFLOW);
+        n = tiles_of(seq_of(a, bb, nullptr));
+      }
+      int incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (lane == 31) wsum[warp] = incl;
+      __syncthreads();
+      int before = carry;
+      for (int w = 0; w < warp; ++w) before += wsum[w];
+      if (bb < a.batch) a.cum[bb] = before + incl - n;
+      int total = 0;
+      for (int w = 0; w < 8; ++w) total += wsum[w];
+      carry += total;
+      __syncthreads();
+    }
+    if (t == 0) a.cum[a.batch] = carry;
+    return;
+  }
+  // thread t holds 8-dim chunks u = t + 256 k (k < 16) of the 64 x 64 chunks
+  float x[16][8];
+  const size_t qoff = (size_t)b * kH * kD;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const size_t o = qoff + (size_t)(t + 256 * k) * 8;
+    if (a.q_dtype == V4KV_FP32) {
+      const float4 x0 = reinterpret_cast<const float4*>(a.q)[o / 4];
+      const float4 x1 = reinterpret_cast<const float4*>(a.q)[o / 4 + 1];
+      x[k][0] = x0.x; x[k][1] = x0.y; x[k][2] = x0.z; x[k][3] = x0.w;
+      x[k][4] = x1.x; x[k][5] = x1.y; x[k][6] = x1.z; x[k][7] = x1.w;
+    } else {
+      const uint4 r = reinterpret_cast<const uint4*>(a.q)[o / 8];
+      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        x[k][2 * i] = __uint_as_float(w[i] << 16);
+        x[k][2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+      }
+    }
+  }
+  float m = 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[k][i]));
+  m = warp_max(m);
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  float amax = 0.f;
+  for (int w = 0; w < 8; ++w) amax = fmaxf(amax, red[w]);
+  int e = 0;
+  if (amax > 0.f) {
+    int k;
+    frexpf(amax, &k);  // amax < 2^k
+    e = 15 - k;
+  }
+  const float qs = ldexpf(1.f, e);
+  uint8_t* img = a.qh + (size_t)b * kQBytes;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int u = t + 256 * k;
+    const int h = u / (kD / 8), c8 = u % (kD / 8);  // 8-dim chunk c8 of head h
+    uint32_t hv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) hv[i] = h2u(__floats2half2_rn(x[k][2 * i] * qs, x[k][2 * i + 1] * qs));
+    *reinterpret_cast<uint4*>(img + (c8 >> 3) * 8192 + tc::sw128_off(h, c8 & 7)) =
+        make_uint4(hv[0], hv[1], hv[2], hv[3]);
+  }
+  if (t == 0) a.qk0[b] = a.sm_scale * 1.4426950408889634f * ldexpf(1.f, -e);
+}
+
+// workspace of the tensor-core path: query images, their multipliers, partial
+// results (o, m, l) per slot, tile prefix sums
 size_t decode_tc_workspace_bytes(int batch, int num_sms) {
   const size_t slots = (size_t)batch + num_sms;
-  return slots * kH * (size_t)(kD + 2) * sizeof(float) + ((size_t)batch + 1) * sizeof(int32_t) + 256;
+  const size_t qk0 = ((size_t)batch * sizeof(float) + 255) / 256 * 256;
+  return (size_t)batch * kQBytes + qk0 + slots * kH * (size_t)(kD + 2) * sizeof(float) +
+         ((size_t)batch + 1) * sizeof(int32_t) + 256;
+}
+
+void decode_tc_layout(DecodeArgs& a, void* workspace) {
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  const size_t slots = (size_t)a.batch + a.n_splits;
+  a.qh = w;
+  w += (size_t)a.batch * kQBytes;
+  a.qk0 = reinterpret_cast<float*>(w);
+  w += ((size_t)a.batch * sizeof(float) + 255) / 256 * 256;
+  a.part_o = reinterpret_cast<float*>(w);
+  a.part_ml = a.part_o + slots * kH * kD;
+  a.cum = reinterpret_cast<int32_t*>(a.part_ml + slots * kH * 2);
+}
+
+// launch with programmatic stream serialization: the kernel may start while
+// the previous one in the stream finishes; it waits (griddepcontrol.wait)
+// before it reads that kernel's results
+template <typename... Args>
+static cudaError_t launch_pdl(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  decode_tc_kernel<<<a.n_splits, kThreads, kSmemBytes, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  decode_tc_merge_kernel<<<dim3(kH, a.batch), 128, 0, stream>>>(a);
-  return cudaGetLastError();
+  decode_tc_prep_kernel<<<a.batch + 1, 256, 0, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(decode_tc_kernel, dim3(a.n_splits), dim3(kThreads), kSmemBytes, stream, a);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(decode_tc_merge_kernel, dim3(kH, a.batch), dim3(128), 0, stream, a);
 }
 
 }  // namespace v4kv

@@ -98,6 +98,8 @@ struct DecodeArgs {
   int max_len;  // host bound on seq_lens; longer sequences are clamped and flagged
   int pad_sel;  // 1: entries are padded to a multiple of 128 items (tensor-core path)
   int32_t* cum; // tensor-core path: [batch + 1] tile prefix sums (workspace)
+  uint8_t* qh;  // tensor-core path: [batch] query images, 64 KB each (workspace)
+  float* qk0;   // tensor-core path: [batch] score multipliers of the query images
 };
 
 cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, int batch,
@@ -116,6 +118,7 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);  // sweep + merge
 size_t decode_tc_workspace_bytes(int batch, int num_sms);
+void decode_tc_layout(DecodeArgs& a, void* workspace);  // needs batch, n_splits
 
 // Tensor map over `rows` rows of `row_bytes` bytes (uint8, 2-D, 128-byte
 // swizzle), boxes of `row_bytes` x `box_rows`. base must be 16-byte aligned.
