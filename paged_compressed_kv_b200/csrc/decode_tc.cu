@@ -258,6 +258,32 @@ __device__ __forceinline__ int tiles_of(const Seq& s) {
   return s.n_sel_pad / kT + (s.n_win + kT - 1) / kT;
 }
 
+// Estimated cost of a sequence's tiles in the sweep (units of a quarter of an
+// fp8 tile): fp8 tiles 4, bf16 tiles 8 (twice the bytes and a slower
+// conversion), and 4 for opening a segment (query copy, epilogue).
+constexpr int kCostFp8 = 4, kCostBf16 = 8, kCostSeg = 4;
+
+__device__ __forceinline__ long long seq_cost(const DecodeArgs& a, const Seq& s) {
+  const int nm = s.n_sel_pad / kT, nw = (s.n_win + kT - 1) / kT;
+  if (nm + nw == 0) return 0;
+  const int cm = a.main.dtype == V4KV_FP8_E4M3 ? kCostFp8 : kCostBf16;
+  const int cw = a.window.dtype == V4KV_FP8_E4M3 ? kCostFp8 : kCostBf16;
+  return kCostSeg + (long long)nm * cm + (long long)nw * cw;
+}
+
+// tile of sequence s at which `off` cost units (from the sequence's start)
+// fall, clamped to the sequence's tiles
+__device__ __forceinline__ int tile_at_cost(const DecodeArgs& a, const Seq& s, long long off) {
+  const int nm = s.n_sel_pad / kT, nw = (s.n_win + kT - 1) / kT;
+  const int cm = a.main.dtype == V4KV_FP8_E4M3 ? kCostFp8 : kCostBf16;
+  const int cw = a.window.dtype == V4KV_FP8_E4M3 ? kCostFp8 : kCostBf16;
+  off -= kCostSeg;
+  if (off <= 0) return 0;
+  if (off < (long long)nm * cm) return (int)(off / cm);
+  const long long k = nm + (off - (long long)nm * cm) / cw;
+  return (int)min(k, (long long)(nm + nw - 1));
+}
+
 // Walks the global tile list: sequence b, tile lt of nt in that sequence.
 struct Cursor {
   int b, lt, nt;
@@ -335,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   int* range = reinterpret_cast<int*>(sm + kMiscOff + 16);  // x0, x1, b0, lt0
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int G = gridDim.x, cta = blockIdx.x;
+  const int cta = blockIdx.x;
 
   // barriers and tensor memory first: this overlaps the query-preparation
   // kernel still running ahead of this one
@@ -362,22 +388,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   tc::pdl_wait();  // the tile prefix sums and query images are complete from here on
   tc::pdl_launch_dependents();
 
-  // ---- this block's tile range: T = total tiles, [c*T/G, (c+1)*T/G); the
-  // first sequence b0 is the number of sequences whose tiles end at or before x0
-  if (warp == 0) {
-    const long long T = a.cum[a.batch];
-    const int x0 = (int)((long long)cta * T / G), x1 = (int)((long long)(cta + 1) * T / G);
-    int cnt = 0;
-#pragma unroll 4
-    for (int bb = lane; bb < a.batch; bb += 32) cnt += a.cum[bb + 1] <= x0 ? 1 : 0;
-    const int b0 = __reduce_add_sync(0xffffffffu, cnt);
-    if (lane == 0) {
-      range[0] = x0;
-      range[1] = (b0 < a.batch) ? x1 : x0;
-      range[2] = b0;
-      range[3] = b0 < a.batch ? x0 - a.cum[b0] : 0;
-      if (b0 < a.batch && x0 < x1) issue_q(a, b0, sbase + kQOff, &bars->q_ready);
-    }
+  // ---- this block's tile range [x0, x1) and the sequence of its first tile
+  // (the prep kernel balanced the ranges by estimated cost)
+  if (tid == 0) {
+    const int x0 = a.cta_x0[cta], x1 = a.cta_x0[cta + 1];
+    const int b0 = x0 < x1 ? a.cta_b0[cta] : a.batch;
+    range[0] = x0;
+    range[1] = (b0 < a.batch) ? x1 : x0;
+    range[2] = b0;
+    range[3] = b0 < a.batch ? x0 - a.cum[b0] : 0;
+    if (b0 < a.batch && x0 < x1) issue_q(a, b0, sbase + kQOff, &bars->q_ready);
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -800,20 +820,28 @@ __global__ void __launch_bounds__(128) decode_tc_merge_kernel(DecodeArgs a) {
   const int h = blockIdx.x, b = blockIdx.y;
   const int d0 = threadIdx.x * 4;
   if (threadIdx.x == 0) {
+    // blocks c whose ranges [x0[c], x0[c+1]) meet the sequence's tiles [c0, c1)
     const int G = a.n_splits;
-    const long long T = a.cum[a.batch];
     const int c0 = a.cum[b], c1 = a.cum[b + 1];
     int lo = 0, hi = -1;
     if (c1 > c0) {
-      lo = (int)(((long long)(c0 + 1) * G + T - 1) / T) - 1;
-      hi = (int)(((long long)c1 * G + T - 1) / T) - 1;
-      // skip blocks with empty ranges at either end (only when G > T)
-      while (lo <= hi && (long long)(lo + 1) * T / G <= (long long)lo * T / G) ++lo;
+      int l = 0, r = G;  // first c with x0[c+1] > c0
+      while (l < r) {
+        const int m = (l + r) >> 1;
+        if (a.cta_x0[m + 1] > c0) r = m; else l = m + 1;
+      }
+      lo = l;
+      l = lo; r = G;     // first c with x0[c] >= c1
+      while (l < r) {
+        const int m = (l + r) >> 1;
+        if (a.cta_x0[m] >= c1) r = m; else l = m + 1;
+      }
+      hi = l - 1;
     }
     float M = -INFINITY;
     for (int c = lo; c <= hi; ++c) {
-      const long long s0 = (long long)c * T / G, s1 = (long long)(c + 1) * T / G;
-      w_sh[c - lo] = (s1 <= s0) ? -INFINITY : a.part_ml[(((size_t)b + c) * kH + h) * 2];
+      const bool empty = a.cta_x0[c + 1] <= a.cta_x0[c];
+      w_sh[c - lo] = empty ? -INFINITY : a.part_ml[(((size_t)b + c) * kH + h) * 2];
       M = fmaxf(M, w_sh[c - lo]);
     }
     float L = 0.f;
@@ -875,31 +903,64 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
   __shared__ float red[8];
   __shared__ int wsum[8];
   if (b == a.batch) {
+    // tiles and estimated cost per sequence, their prefix sums, then each
+    // block's range: block c starts at the tile where the cost prefix reaches
+    // c/G of the total
+    __shared__ long long csum[8];
     int carry = 0;
+    long long ccarry = 0;
     for (int base = 0; base < a.batch; base += 256) {
       const int bb = base + t;
       int n = 0;
+      long long cost = 0;
       if (bb < a.batch) {
         if (a.seq_lens[bb] > a.max_len) flag(a.dev_status, V4KV_DEV_OVERFLOW);
-        n = tiles_of(seq_of(a, bb, nullptr));
+        const Seq sq = seq_of(a, bb, nullptr);
+        n = tiles_of(sq);
+        cost = seq_cost(a, sq);
       }
       int incl = n;
+      long long cincl = cost;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+        const long long cy = __shfl_up_sync(0xffffffffu, cincl, o);
+        if (lane >= o) { incl += y; cincl += cy; }
       }
-      if (lane == 31) wsum[warp] = incl;
+      if (lane == 31) { wsum[warp] = incl; csum[warp] = cincl; }
       __syncthreads();
       int before = carry;
-      for (int w = 0; w < warp; ++w) before += wsum[w];
-      if (bb < a.batch) a.cum[bb] = before + incl - n;
-      int total = 0;
-      for (int w = 0; w < 8; ++w) total += wsum[w];
-      carry += total;
+      long long cbefore = ccarry;
+      for (int w = 0; w < warp; ++w) { before += wsum[w]; cbefore += csum[w]; }
+      if (bb < a.batch) {
+        a.cum[bb] = before + incl - n;
+        a.costcum[bb] = cbefore + cincl - cost;
+      }
+      for (int w = 0; w < 8; ++w) { carry += wsum[w]; ccarry += csum[w]; }
       __syncthreads();
     }
-    if (t == 0) a.cum[a.batch] = carry;
+    if (t == 0) {
+      a.cum[a.batch] = carry;
+      a.costcum[a.batch] = ccarry;
+    }
+    __syncthreads();  // the prefix sums are visible to the whole block
+    const int G = a.n_splits;
+    for (int c = t; c <= G; c += 256) {
+      int x0 = carry, b0 = a.batch;
+      if (c < G && ccarry > 0) {
+        const long long target = (long long)c * ccarry / G;
+        int l = 0, r = a.batch - 1;  // last sequence whose cost prefix is <= target
+        while (l < r) {
+          const int m = (l + r + 1) >> 1;
+          if (a.costcum[m] <= target) l = m; else r = m - 1;
+        }
+        b0 = l;
+        const Seq sq = seq_of(a, b0, nullptr);
+        x0 = a.cum[b0] + tile_at_cost(a, sq, target - a.costcum[b0]);
+      }
+      a.cta_x0[c] = x0;
+      if (c < G) a.cta_b0[c] = b0;
+    }
     return;
   }
   // thread t holds 8-dim chunks u = t + 256 k (k < 16) of the 64 x 64 chunks
@@ -960,7 +1021,8 @@ size_t decode_tc_workspace_bytes(int batch, int num_sms) {
   const size_t slots = (size_t)batch + num_sms;
   const size_t qk0 = ((size_t)batch * sizeof(float) + 255) / 256 * 256;
   return (size_t)batch * kQBytes + qk0 + slots * kH * (size_t)(kD + 2) * sizeof(float) +
-         ((size_t)batch + 1) * sizeof(int32_t) + 256;
+         ((size_t)batch + 1) * sizeof(int32_t) + 256 + ((size_t)batch + 1) * sizeof(long long) +
+         (2 * (size_t)num_sms + 1) * sizeof(int32_t) + 256;
 }
 
 void decode_tc_layout(DecodeArgs& a, void* workspace) {
@@ -973,6 +1035,11 @@ void decode_tc_layout(DecodeArgs& a, void* workspace) {
   a.part_o = reinterpret_cast<float*>(w);
   a.part_ml = a.part_o + slots * kH * kD;
   a.cum = reinterpret_cast<int32_t*>(a.part_ml + slots * kH * 2);
+  uint8_t* c = reinterpret_cast<uint8_t*>(a.cum + a.batch + 1);
+  c = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(c) + 255) & ~uintptr_t(255));
+  a.costcum = reinterpret_cast<long long*>(c);
+  a.cta_x0 = reinterpret_cast<int32_t*>(a.costcum + a.batch + 1);
+  a.cta_b0 = a.cta_x0 + a.n_splits + 1;
 }
 
 // launch with programmatic stream serialization: the kernel may start while

@@ -100,6 +100,9 @@ struct DecodeArgs {
   int32_t* cum; // tensor-core path: [batch + 1] tile prefix sums (workspace)
   uint8_t* qh;  // tensor-core path: [batch] query images, 64 KB each (workspace)
   float* qk0;   // tensor-core path: [batch] score multipliers of the query images
+  long long* costcum;  // tensor-core path: [batch + 1] cost prefix sums (workspace)
+  int32_t* cta_x0;     // tensor-core path: [n_splits + 1] first tile of each block's range
+  int32_t* cta_b0;     // tensor-core path: [n_splits] sequence of that first tile
 };
 
 cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, int batch,
