@@ -373,7 +373,7 @@ def run_ours(args, rank, world, device):
                    "l2": "flushed between steps (256 MB write), inputs also exceed L2",
                    "decode_ms": t_dec, "hbm_gbs": achieved},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": SWEEP_TRAFFIC.get(args.config) if not args.seqs else None,
                      "kernel": "v4kv_decode_attention (query prep + sweep + merge)",
                      "algorithmic_bytes": alg, "peak_source": peak_kind},
         "e2e": {"value": rate_e2e, "unit": "tokens/s",
@@ -611,7 +611,13 @@ class MixedStep:
 
 def run_mixed(args, device):
     peak, _ = load_peaks()
-    st = MixedStep(device)
+    kw = {}
+    if args.seqs:
+        kw["seqs"] = args.seqs
+    if args.layers:
+        kw["c4a_layers"] = min(30, args.layers)
+        kw["c128a_layers"] = min(31, args.layers)
+    st = MixedStep(device, **kw)
     nl4, nl128 = len(st.c4a), len(st.c128a)
     ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(2)] for k in ("idx", "att4", "att128")}
     tot = {"idx": 0.0, "att4": 0.0, "att128": 0.0}
@@ -649,11 +655,17 @@ def run_mixed(args, device):
            "step_gbs": (nl4 * (idx_b + a4_b) + nl128 * a128_b) / (step_ms * 1e-3) / 1e9,
            "status": int(st.status.item())}
     res["step_frac"] = res["step_gbs"] / peak
-    return {"config": "61-layer mixed step (30 c4a with indexer top-512 + 31 c128a), batch 128, "
-                      "context U[1K, 256K], 64 heads, fp8 KV", "results": res}
+    name = (f"{nl4 + nl128}-layer mixed step ({nl4} c4a with indexer top-512 + {nl128} c128a), "
+            f"batch {st.B}, context U[1K, 256K], 64 heads, fp8 KV")
+    return {"config": name, "results": res}
 
 
 DTYPE = "f16"
+
+# DRAM bytes (read + write) of one sweep launch, from an ncu capture of the same
+# build on 32 sequences of the workload, scaled by the entries processed (see
+# profiles/decode_tc_c4a_b64.md); None where no capture of the current kernel exists
+SWEEP_TRAFFIC = {1: 301.8e6}
 
 
 def main():
@@ -666,6 +678,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seqs", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="config 4: c4a and c128a layers each (small cases for profiler captures)")
     ap.add_argument("--seqs", type=int, default=0,
                     help="keep only the first n sequences (small cases for profiler captures)")
     args = ap.parse_args()
