@@ -78,10 +78,12 @@ bool rope_ok(const v4kv_rope& r, int dim) {
 }
 
 RopeArgs to_rope(const v4kv_rope& r) {
-  RopeArgs a;
+  RopeArgs a{};
   a.theta = r.theta;
   a.rope_dim = r.rope_dim;
   a.rope_offset = r.rope_offset;
+  for (int i = 0; i < kRopeTable && 2 * i < r.rope_dim; ++i)
+    a.freq[i] = std::pow(r.theta, -2.0 * (double)i / (double)r.rope_dim);
   return a;
 }
 
@@ -165,7 +167,7 @@ v4kv_status v4kv_compress_append(const void* x, const float* gate, const int32_t
   // every sequence touches at most ceil(n/r) + 1 groups
   const long long max_groups = (long long)total_tokens / ratio + 2LL * batch;
   if (max_groups > 0x7fffffffLL) return V4KV_ERR_INVALID_ARG;
-  return to_status(launch_compress_append(a, (int)max_groups, (cudaStream_t)stream));
+  return to_status(launch_compress_append(a, (int)max_groups, total_tokens, (cudaStream_t)stream));
 }
 
 v4kv_status v4kv_index_topk(const float* q_idx, const v4kv_paged* idx_cache,

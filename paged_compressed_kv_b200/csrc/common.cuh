@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include "../../include/v4kv.h"
+#include "kernels.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "v4kv kernels are written for sm_100a (B200) only"
@@ -51,10 +52,14 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
 
 // ---------------------------------------------------------------- RoPE
 // cos / sin of pos * theta^(-2i/rope_dim), formed in fp64 and rounded to fp32.
-__device__ __forceinline__ void rope_cs(double theta, int rope_dim, int i, long long pos,
-                                        float* c, float* s) {
-  double freq = pow(theta, -2.0 * (double)i / (double)rope_dim);
-  double ang = (double)pos * freq;
+// cos and sin of pair i's angle at position pos: pos * theta^(-2i/rope_dim)
+// in fp64 (the host precomputes the first kRopeTable frequencies), rounded to
+// fp32
+__device__ __forceinline__ void rope_cs(const RopeArgs& rp, int i, long long pos, float* c,
+                                        float* s) {
+  const double freq =
+      i < kRopeTable ? rp.freq[i] : pow(rp.theta, -2.0 * (double)i / (double)rp.rope_dim);
+  const double ang = (double)pos * freq;
   double sd, cd;
   sincos(ang, &sd, &cd);
   *c = (float)cd;

@@ -44,7 +44,7 @@ __device__ __forceinline__ void rope8(Vec8& x, int d0, const RopeArgs& rp, long 
     int d = d0 + 2 * k;
     if (d >= rp.rope_offset && d + 1 < rp.rope_offset + rp.rope_dim) {
       float c, s;
-      rope_cs(rp.theta, rp.rope_dim, (d - rp.rope_offset) >> 1, pos, &c, &s);
+      rope_cs(rp, (d - rp.rope_offset) >> 1, pos, &c, &s);
       if (inverse) s = -s;
       rope_apply(x.v[2 * k], x.v[2 * k + 1], c, s);
     }
@@ -94,13 +94,29 @@ __device__ __forceinline__ int find_seq(const int32_t* cu, int batch, int i) {
 }
 
 // one block per touched group
+constexpr int kCuSmem = 1024;  // sequences whose prefix sums fit in shared memory
+
+// largest b with cu[b] <= i, from a shared-memory copy of cu[0..batch] when it fits
+__device__ __forceinline__ int find_seq_cached(const int32_t* cu, int batch, int i, int* cu_sh) {
+  if (batch + 1 > kCuSmem) return find_seq(cu, batch, i);
+  for (int k = threadIdx.x; k <= batch; k += blockDim.x) cu_sh[k] = cu[k];
+  __syncthreads();
+  int lo = 0, hi = batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cu_sh[mid] <= i) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 __global__ void compress_entries_kernel(CompressArgs a) {
   __shared__ float w[kMaxRatio];
   __shared__ float red[32];
+  __shared__ int cu_sh[kCuSmem];
   const int i = blockIdx.x;
   const int total = a.cu_entries[a.batch];
   if (i >= total) return;
-  const int b = find_seq(a.cu_entries, a.batch, i);
+  const int b = find_seq_cached(a.cu_entries, a.batch, i, cu_sh);
   const int r = a.ratio;
   const int s = a.seq_start[b];
   const int n = a.cu_seqlens[b + 1] - a.cu_seqlens[b];
@@ -170,16 +186,20 @@ __global__ void compress_entries_kernel(CompressArgs a) {
   store_entry(a.main, slot, d0, active, e, red);
 }
 
-// one block per window token written: tokens [max(s, end - W), end)
+// one block per input token; the last W tokens of each sequence's new ones
+// ([max(s, end - W), end)) are written to the window
 __global__ void compress_window_kernel(CompressArgs a) {
   __shared__ float red[32];
-  const int b = blockIdx.y;
+  __shared__ int cu_sh[kCuSmem];
+  const int g = blockIdx.x;
+  if (g >= a.cu_seqlens[a.batch]) return;
+  const int b = find_seq_cached(a.cu_seqlens, a.batch, g, cu_sh);
   const int s = a.seq_start[b];
   const int n = a.cu_seqlens[b + 1] - a.cu_seqlens[b];
   const int end = s + n;
   const int first = max(s, end - a.window_len);
-  const int t = first + blockIdx.x;
-  if (t >= end) return;
+  const int t = s + (g - a.cu_seqlens[b]);
+  if (t < first || t >= end) return;
   const int dim = a.dim;
   const int d0 = threadIdx.x * 8;
   const bool active = d0 < dim;
@@ -228,14 +248,14 @@ __global__ void compress_state_kernel(CompressArgs a) {
   }
 }
 
-cudaError_t launch_compress_append(const CompressArgs& a, int max_groups, cudaStream_t stream) {
+cudaError_t launch_compress_append(const CompressArgs& a, int max_groups, int total_tokens,
+                                   cudaStream_t stream) {
   const int threads = ((a.dim / 8 + 31) / 32) * 32;
   if (max_groups > 0) compress_entries_kernel<<<max_groups, threads, 0, stream>>>(a);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  if (a.window.data && a.window_len > 0) {
-    dim3 grid(a.window_len, a.batch);
-    compress_window_kernel<<<grid, threads, 0, stream>>>(a);
+  if (a.window.data && a.window_len > 0 && total_tokens > 0) {
+    compress_window_kernel<<<total_tokens, threads, 0, stream>>>(a);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }

@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
       const int d = d0 + 2 * k;
       if (d >= a.rope.rope_offset && d + 1 < a.rope.rope_offset + a.rope.rope_dim) {
         float c, s;
-        rope_cs(a.rope.theta, a.rope.rope_dim, (d - a.rope.rope_offset) >> 1, (long long)si.L - 1, &c, &s);
+        rope_cs(a.rope, (d - a.rope.rope_offset) >> 1, (long long)si.L - 1, &c, &s);
         rope_apply(o[2 * k], o[2 * k + 1], c, -s);
       }
     }

@@ -308,6 +308,7 @@ __device__ __forceinline__ void cursor_next(Cursor& c, const DecodeArgs& a) {
 }
 
 constexpr uint32_t kQBytes = kH * kD * 2;  // one query image (f16)
+constexpr int kMaxSplits = 160;            // sweep blocks at most (the plan caps the grid)
 
 // Start the bulk copy of sequence b's query image into shared memory; the
 // copy completes phase by transaction count on `bar`.
@@ -814,46 +815,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
 // position L - 1, store bf16
 __global__ void __launch_bounds__(128) decode_tc_merge_kernel(DecodeArgs a) {
   __shared__ int slot_lo, slot_hi;      // blocks whose tile ranges meet the sequence
-  __shared__ float w_sh[160];           // their weights (max blocks per sequence: SMs)
+  __shared__ float w_sh[kMaxSplits];    // their weights (at most every block)
   __shared__ float l_sh;
   tc::pdl_wait();  // the sweep's partial results are complete from here on
   const int h = blockIdx.x, b = blockIdx.y;
   const int d0 = threadIdx.x * 4;
-  if (threadIdx.x == 0) {
-    // blocks c whose ranges [x0[c], x0[c+1]) meet the sequence's tiles [c0, c1)
-    const int G = a.n_splits;
-    const int c0 = a.cum[b], c1 = a.cum[b + 1];
-    int lo = 0, hi = -1;
-    if (c1 > c0) {
-      int l = 0, r = G;  // first c with x0[c+1] > c0
-      while (l < r) {
-        const int m = (l + r) >> 1;
-        if (a.cta_x0[m + 1] > c0) r = m; else l = m + 1;
-      }
-      lo = l;
-      l = lo; r = G;     // first c with x0[c] >= c1
-      while (l < r) {
-        const int m = (l + r) >> 1;
-        if (a.cta_x0[m] >= c1) r = m; else l = m + 1;
-      }
-      hi = l - 1;
-    }
+  if (threadIdx.x < 32) {
+    // the blocks that met the sequence (an empty range writes no partial)
+    const int lane = threadIdx.x;
+    const int2 sl = a.seq_slots[b];
+    const int lo = sl.x, hi = sl.y;
     float M = -INFINITY;
-    for (int c = lo; c <= hi; ++c) {
+    for (int c = lo + lane; c <= hi; c += 32) {
       const bool empty = a.cta_x0[c + 1] <= a.cta_x0[c];
-      w_sh[c - lo] = empty ? -INFINITY : a.part_ml[(((size_t)b + c) * kH + h) * 2];
-      M = fmaxf(M, w_sh[c - lo]);
+      const float m = empty ? -INFINITY : a.part_ml[(((size_t)b + c) * kH + h) * 2];
+      w_sh[c - lo] = m;
+      M = fmaxf(M, m);
     }
+    M = warp_max(M);
     float L = 0.f;
-    for (int c = lo; c <= hi; ++c) {
+    for (int c = lo + lane; c <= hi; c += 32) {
       const float m = w_sh[c - lo];
       const float w = m == -INFINITY ? 0.f : exp2f(m - M);
       w_sh[c - lo] = w;
       if (w > 0.f) L = fmaf(w, a.part_ml[(((size_t)b + c) * kH + h) * 2 + 1], L);
     }
-    slot_lo = lo;
-    slot_hi = hi;
-    l_sh = L;
+    L = warp_sum(L);
+    if (lane == 0) {
+      slot_lo = lo;
+      slot_hi = hi;
+      l_sh = L;
+    }
   }
   __syncthreads();
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -880,7 +872,7 @@ __global__ void __launch_bounds__(128) decode_tc_merge_kernel(DecodeArgs a) {
       const int d = d0 + 2 * k;
       if (d >= a.rope.rope_offset && d + 1 < a.rope.rope_offset + a.rope.rope_dim) {
         float c, s;
-        rope_cs(a.rope.theta, a.rope.rope_dim, (d - a.rope.rope_offset) >> 1, (long long)Lb - 1, &c, &s);
+        rope_cs(a.rope, (d - a.rope.rope_offset) >> 1, (long long)Lb - 1, &c, &s);
         rope_apply(o[2 * k], o[2 * k + 1], c, -s);
       }
     }
@@ -907,6 +899,7 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
     // block's range: block c starts at the tile where the cost prefix reaches
     // c/G of the total
     __shared__ long long csum[8];
+    __shared__ int x0_sh[kMaxSplits + 1];
     int carry = 0;
     long long ccarry = 0;
     for (int base = 0; base < a.batch; base += 256) {
@@ -960,6 +953,28 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
       }
       a.cta_x0[c] = x0;
       if (c < G) a.cta_b0[c] = b0;
+      x0_sh[c] = x0;
+    }
+    __syncthreads();
+    // blocks whose ranges [x0[c], x0[c+1]) meet each sequence's tiles [c0, c1)
+    for (int bb = t; bb < a.batch; bb += 256) {
+      const int c0 = a.cum[bb], c1 = a.cum[bb + 1];
+      int lo = 0, hi = -1;
+      if (c1 > c0) {
+        int l = 0, r = G;  // first c with x0[c+1] > c0
+        while (l < r) {
+          const int m = (l + r) >> 1;
+          if (x0_sh[m + 1] > c0) r = m; else l = m + 1;
+        }
+        lo = l;
+        l = lo; r = G;     // first c with x0[c] >= c1
+        while (l < r) {
+          const int m = (l + r) >> 1;
+          if (x0_sh[m] >= c1) r = m; else l = m + 1;
+        }
+        hi = l - 1;
+      }
+      a.seq_slots[bb] = make_int2(lo, hi);
     }
     return;
   }
@@ -1022,7 +1037,7 @@ size_t decode_tc_workspace_bytes(int batch, int num_sms) {
   const size_t qk0 = ((size_t)batch * sizeof(float) + 255) / 256 * 256;
   return (size_t)batch * kQBytes + qk0 + slots * kH * (size_t)(kD + 2) * sizeof(float) +
          ((size_t)batch + 1) * sizeof(int32_t) + 256 + ((size_t)batch + 1) * sizeof(long long) +
-         (2 * (size_t)num_sms + 1) * sizeof(int32_t) + 256;
+         (2 * (size_t)num_sms + 1) * sizeof(int32_t) + 256 + (size_t)batch * sizeof(int2) + 256;
 }
 
 void decode_tc_layout(DecodeArgs& a, void* workspace) {
@@ -1040,6 +1055,9 @@ void decode_tc_layout(DecodeArgs& a, void* workspace) {
   a.costcum = reinterpret_cast<long long*>(c);
   a.cta_x0 = reinterpret_cast<int32_t*>(a.costcum + a.batch + 1);
   a.cta_b0 = a.cta_x0 + a.n_splits + 1;
+  uint8_t* q = reinterpret_cast<uint8_t*>(a.cta_b0 + a.n_splits);
+  q = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(q) + 255) & ~uintptr_t(255));
+  a.seq_slots = reinterpret_cast<int2*>(q);
 }
 
 // launch with programmatic stream serialization: the kernel may start while

@@ -19,10 +19,13 @@ struct PoolArgs {
   int max_blocks;
 };
 
+constexpr int kRopeTable = 32;  // pairs whose frequency the host precomputes
+
 struct RopeArgs {
   double theta;
   int rope_dim;
   int rope_offset;
+  double freq[kRopeTable];  // theta^(-2i / rope_dim), i < min(rope_dim / 2, kRopeTable)
 };
 
 struct CompressArgs {
@@ -103,6 +106,7 @@ struct DecodeArgs {
   long long* costcum;  // tensor-core path: [batch + 1] cost prefix sums (workspace)
   int32_t* cta_x0;     // tensor-core path: [n_splits + 1] first tile of each block's range
   int32_t* cta_b0;     // tensor-core path: [n_splits] sequence of that first tile
+  int2* seq_slots;     // tensor-core path: [batch] first and last block meeting the sequence
 };
 
 cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, int batch,
@@ -110,7 +114,8 @@ cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, int batch,
                                 int num_pages, int32_t* cu_out, int64_t* slot_out, long long cap,
                                 int32_t* st, cudaStream_t stream);
 
-cudaError_t launch_compress_append(const CompressArgs& a, int max_groups, cudaStream_t stream);
+cudaError_t launch_compress_append(const CompressArgs& a, int max_groups, int total_tokens,
+                                   cudaStream_t stream);
 
 size_t index_workspace_bytes(int batch, int max_seq_len, int ratio, int window_len);
 cudaError_t launch_index_topk(IndexArgs a, int max_seq_len, cudaStream_t stream);
