@@ -14,11 +14,13 @@
 // reference maximum per head, raised only when a score exceeds it by more
 // than 2^8 (P' <= 256), at which point O^T and the partial sums are rescaled.
 //
-// Warp roles (320 threads): warps 0-3 softmax (thread = tile row = TMEM lane),
-// warps 4-7 gather + convert (16-byte coalesced page loads), warp 8 allocates
-// tensor memory and one of its threads issues the MMAs, warp 9 resolves the
-// rows of the tiles two ahead and prefetches them into L2. Each softmax thread
-// keeps its item rows' partial normalisers (one per head) in tensor memory.
+// Warp roles (320 threads): warps 0-7 are workers. Each runs the softmax of
+// one tile row (its TMEM lane) for 32 of the 64 heads, then gathers and
+// converts 16 rows of the next tile (16-byte coalesced page loads) as the
+// second product releases each V chunk. Warp 8 allocates tensor memory and
+// one of its threads issues the MMAs; warp 9 resolves the rows of the tiles
+// up to kRing - 1 ahead and prefetches them into L2. The partial normalisers of each row
+// (one per head) live in tensor memory.
 //
 // Schedule: the kernel is persistent. The tiles of all sequences form one
 // list (each sequence: its entries padded to whole tiles, then its window);
@@ -46,15 +48,17 @@ constexpr float kNone = -1e30f; // reference maximum before any item
 constexpr uint32_t kVOff = 0;                    // 8 dim atoms x 128 rows x 128 B
 constexpr uint32_t kQOff = 131072;               // 8 dim atoms x 64 rows x 128 B
 constexpr uint32_t kPOff = 196608;               // 128 rows x 128 B (64 heads f16)
-constexpr uint32_t kMetaOff = 212992;            // [3][128] fp32 item scales (0 = skip)
-constexpr uint32_t kPtrOff = kMetaOff + 1536;    // [3][128] item row addresses
-constexpr uint32_t kMrefOff = kPtrOff + 3072;    // [64] reference max per head
+constexpr int kRing = 6;        // tiles of row addresses the address warp keeps ready
+constexpr uint32_t kMetaOff = 212992;                 // [kRing][128] fp32 item scales (0 = skip)
+constexpr uint32_t kPtrOff = kMetaOff + kRing * 512;  // [kRing][128] item row addresses
+constexpr uint32_t kMrefOff = kPtrOff + kRing * 1024;  // [64] reference max per head
 constexpr uint32_t kAlphaOff = kMrefOff + 256;   // [64] rescale factors
-constexpr uint32_t kRedOff = kAlphaOff + 256;    // [4][64] per-warp maxima
+constexpr uint32_t kRedOff = kAlphaOff + 256;    // [8][32] per-warp reductions
 constexpr uint32_t kBarOff = kRedOff + 1024;     // mbarriers
-constexpr uint32_t kInfoOff = kBarOff + 256;     // [3] tile info words
+constexpr uint32_t kInfoOff = kBarOff + 256;     // [kRing] tile info words
 constexpr uint32_t kMiscOff = kInfoOff + 64;     // tmem address, flags, range
 constexpr uint32_t kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 // TMEM columns: S double buffer [0, 128), O^T 4 x 64 at [128, 384), partial
 // normalisers of each lane (64 heads) at [384, 448)
@@ -63,8 +67,8 @@ constexpr uint32_t kOCol = 128;
 constexpr uint32_t kLCol = 384;
 
 struct Bars {
-  uint64_t addr_ready[3];
-  uint64_t addr_free[3];
+  uint64_t addr_ready[kRing];
+  uint64_t addr_free[kRing];
   uint64_t v_full[4];
   uint64_t v_empty[4];
   uint64_t s_full[2];
@@ -73,6 +77,7 @@ struct Bars {
   uint64_t q_ready;
   uint64_t drain;
 };
+static_assert(sizeof(Bars) <= 256, "barrier area");
 
 // tile info word written by the address warp
 constexpr uint32_t kInfoFp8 = 1;    // rows are fp8 codes (else bf16)
@@ -85,11 +90,11 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-__device__ __forceinline__ int ordered(float f) {
+__device__ __forceinline__ int ordered_key(float f) {
   int k = __float_as_int(f);
   return k >= 0 ? k : (k ^ 0x7fffffff);
 }
-__device__ __forceinline__ float unordered(int k) {
+__device__ __forceinline__ float from_ordered_key(int k) {
   return __int_as_float(k >= 0 ? k : (k ^ 0x7fffffff));
 }
 
@@ -319,15 +324,15 @@ __device__ __forceinline__ void issue_q(const DecodeArgs& a, int b, uint32_t qds
   for (int k = 0; k < 4; ++k) tc::bulk_load(qdst + k * (kQBytes / 4), src + k * (kQBytes / 4), kQBytes / 4, bar);
 }
 
-// Sum 64 per-lane values over the 32 lanes of a warp (reduce-scatter): lane l
-// ends with the sums of heads 2*rev and 2*rev+1 where the lane bits pick
-// halves (bit 4: 32 heads, bit 3: 16, ... bit 0: 2). Returns the head index.
-__device__ __forceinline__ int warp_reduce_scatter64(float* v, int lane, float* out2) {
+// Sum 32 per-lane values over the 32 lanes of a warp (reduce-scatter): lane l
+// ends with the sum of value `rev` where the lane bits pick halves (bit 4: 16
+// values, bit 3: 8, ... bit 0: 1). Returns that value's index.
+__device__ __forceinline__ int warp_reduce_scatter32(float* v, int lane, float* out1) {
   int base = 0;
 #pragma unroll
   for (int level = 0; level < 5; ++level) {
     const int off = 16 >> level;   // shuffle distance
-    const int n = 32 >> level;     // values kept after this level
+    const int n = 16 >> level;     // values kept after this level
     const bool upper = (lane & off) != 0;
 #pragma unroll
     for (int k = 0; k < n; ++k) {
@@ -337,8 +342,7 @@ __device__ __forceinline__ int warp_reduce_scatter64(float* v, int lane, float* 
     }
     if (upper) base += n;
   }
-  out2[0] = v[0];
-  out2[1] = v[1];
+  out1[0] = v[0];
   return base;
 }
 
@@ -367,17 +371,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   // barriers and tensor memory first: this overlaps the query-preparation
   // kernel still running ahead of this one
   if (tid == 0) {
-    for (int k = 0; k < 3; ++k) {
+    for (int k = 0; k < kRing; ++k) {
       tc::mbar_init(&bars->addr_ready[k], 32);
       tc::mbar_init(&bars->addr_free[k], 256);
     }
     for (int c = 0; c < 4; ++c) {
-      tc::mbar_init(&bars->v_full[c], 128);
+      tc::mbar_init(&bars->v_full[c], 256);
       tc::mbar_init(&bars->v_empty[c], 1);
     }
     tc::mbar_init(&bars->s_full[0], 1);
     tc::mbar_init(&bars->s_full[1], 1);
-    tc::mbar_init(&bars->p_full, 128);
+    tc::mbar_init(&bars->p_full, 256);
     tc::mbar_init(&bars->pv_done, 1);
     tc::mbar_init(&bars->q_ready, 1);
     tc::mbar_init(&bars->drain, 1);
@@ -414,12 +418,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   }
 
   if (warp == 9) {
-    // ======================= address resolution + L2 prefetch, two tiles ahead
+    // ======================= address resolution + L2 prefetch, up to kRing - 1 tiles ahead
     Cursor cu;
     cursor_set(cu, a, b0, lt0);
     for (int t = 0; t < n_tiles; ++t) {
-      const int buf = t % 3;
-      if (t >= 3 && !tc::mbar_wait(&bars->addr_free[buf], ((t - 3) / 3) & 1, abort_flag)) break;
+      const int buf = t % kRing;
+      if (t >= kRing && !tc::mbar_wait(&bars->addr_free[buf], ((t - kRing) / kRing) & 1, abort_flag)) break;
       if (t > 0 && cu.lt == 0) {
         // a new sequence starts: pull its query image into L2 as well
         const uint8_t* qp = a.qh + (size_t)cu.b * kQBytes;
@@ -457,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
           if (!ok) break;
           if (c == 0) {
             // the converters read this tile's info word before arriving
-            first = (info[i % 3] & kInfoFirst) != 0;
+            first = (info[i % kRing] & kInfoFirst) != 0;
             if (first) {
               // the segment's query image has landed in shared memory
               ok = tc::mbar_wait(&bars->q_ready, seg & 1, abort_flag);
@@ -500,128 +504,161 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       if (!tc::mbar_wait(&bars->drain, 0, &never)) flag(a.dev_status, V4KV_DEV_TIMEOUT);
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    // ======================= gather + convert
-    const int cw = warp - 4;
-    for (int i = 0; i < n_tiles; ++i) {
-      if (!tc::mbar_wait(&bars->addr_ready[i % 3], (i / 3) & 1, abort_flag)) goto conv_abort;
-      const bool fp8 = (info[i % 3] & kInfoFp8) != 0;
-      const uint8_t** rp = rowptr + (i % 3) * kT;
+  } else {
+    // ======================= workers (warps 0-7): softmax and gather + convert
+    // Softmax: thread (warp w, lane l) owns tile row j = 32 (w % 4) + l (its
+    // TMEM lane) and heads 32 hh .. 32 hh + 31 (hh = w / 4); its partial
+    // normalisers live in tensor memory (columns kLCol + 32 hh ..). Conversion: warp w writes rows 16w ..
+    // 16w + 15 of every V chunk. Per tile: softmax(i), then the conversion of
+    // tile i + 1 as the second product of tile i frees each V chunk; the codes
+    // of tile i + 1 are loaded before softmax(i).
+    const int hh = warp >> 2;
+    const int row = 32 * (warp & 3) + lane;   // tile row = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    uint4 rawv[4][4];
+    const uint32_t l_addr = lane_base + kLCol + 32 * hh;
+    {
+      uint32_t z[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) z[e] = 0u;
+      tc::tmem_st32(l_addr, z);
+      tc::tmem_wait_st();
+    }
+    float k0 = a.qk0[b0];
+    int q_issued = 1;  // query copies started by this thread (tid 0 only)
+    bool ok = true;
+
+    // fp8 rows: lane covers rows 16w + 4r + lane/8 (r = 0..3), 16 bytes at
+    // 16*(lane%8) of each 128-byte dim chunk
+    auto load_fp8 = [&](int t) {
+      const uint8_t** rp = rowptr + (t % kRing) * kT;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const uint8_t* p = rp[16 * warp + 4 * r + (lane >> 3)];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          rawv[c][r] = p ? ldg_stream(p + 128 * c + 16 * (lane & 7)) : make_uint4(0, 0, 0, 0);
+      }
+    };
+    // convert tile t into the V buffer; chunk c waits for the second product of
+    // tile t - 1 to release it (v_empty)
+    auto convert = [&](int t, bool fp8) -> bool {
       if (fp8) {
-        // lane covers rows 32cw + 4r + lane/8 (r = 0..7), 16 bytes at 16*(lane%8)
-        // of each 128-byte dim chunk
-        uint4 rawv[4][8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          const uint8_t* p = rp[32 * cw + 4 * r + (lane >> 3)];
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            rawv[c][r] = p ? ldg_stream(p + 128 * c + 16 * (lane & 7)) : make_uint4(0, 0, 0, 0);
-        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          if (i > 0 && !tc::mbar_wait(&bars->v_empty[c], (i - 1) & 1, abort_flag)) goto conv_abort;
+          if (t > 0 && !tc::mbar_wait(&bars->v_empty[c], (t - 1) & 1, abort_flag)) return false;
           const int part = lane & 7;                 // 16-dim piece within the chunk
           const uint32_t atom = 2 * c + (part >> 2);
           const uint32_t q = 2 * (part & 3);
 #pragma unroll
-          for (int r = 0; r < 8; ++r) {
-            const uint32_t row = 32 * cw + 4 * r + (lane >> 3);
+          for (int r = 0; r < 4; ++r) {
+            const uint32_t vr = 16 * warp + 4 * r + (lane >> 3);
             uint4 lo, hi;
             fp8x16_to_f16(rawv[c][r], lo, hi);
             uint8_t* base = sm + kVOff + atom * 16384;
             if (part & 4) {
-              *reinterpret_cast<uint4*>(base + tc::sw128_off(row, q + 1)) = hi;
-              *reinterpret_cast<uint4*>(base + tc::sw128_off(row, q)) = lo;
+              *reinterpret_cast<uint4*>(base + tc::sw128_off(vr, q + 1)) = hi;
+              *reinterpret_cast<uint4*>(base + tc::sw128_off(vr, q)) = lo;
             } else {
-              *reinterpret_cast<uint4*>(base + tc::sw128_off(row, q)) = lo;
-              *reinterpret_cast<uint4*>(base + tc::sw128_off(row, q + 1)) = hi;
+              *reinterpret_cast<uint4*>(base + tc::sw128_off(vr, q)) = lo;
+              *reinterpret_cast<uint4*>(base + tc::sw128_off(vr, q + 1)) = hi;
             }
           }
           tc::fence_proxy_async_smem();
           tc::mbar_arrive(&bars->v_full[c]);
         }
       } else {
-        // bf16 rows: lane covers rows 32cw + 2r + lane/16 (r = 0..15), 16 bytes at
-        // 16*(lane%16) of each 256-byte dim chunk
-        const uint8_t* ptr[16];
+        // bf16 rows: lane covers rows 16w + 2r + lane/16 (r = 0..7), 16 bytes at
+        // 16*(lane%16) of each 256-byte dim chunk; chunk c + 1 is loaded while
+        // chunk c is converted (the two buffers reuse the code registers)
+        const uint8_t** rp = rowptr + (t % kRing) * kT;
+#define V4KV_RB(k, r) rawv[2 * (k) + ((r) >> 2)][(r) & 3]
 #pragma unroll
-        for (int r = 0; r < 16; ++r) ptr[r] = rp[32 * cw + 2 * r + (lane >> 4)];
+        for (int r = 0; r < 8; ++r) {
+          const uint8_t* p = rp[16 * warp + 2 * r + (lane >> 4)];
+          V4KV_RB(0, r) = p ? ldg_stream(p + 16 * (lane & 15)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint4 rawv[16];
+          if (c + 1 < 4) {
 #pragma unroll
-          for (int r = 0; r < 16; ++r)
-            rawv[r] = ptr[r] ? ldg_stream(ptr[r] + 256 * c + 16 * (lane & 15)) : make_uint4(0, 0, 0, 0);
-          if (i > 0 && !tc::mbar_wait(&bars->v_empty[c], (i - 1) & 1, abort_flag)) goto conv_abort;
+            for (int r = 0; r < 8; ++r) {
+              const uint8_t* p = rp[16 * warp + 2 * r + (lane >> 4)];
+              V4KV_RB((c + 1) & 1, r) = p ? ldg_stream(p + 256 * (c + 1) + 16 * (lane & 15)) : make_uint4(0, 0, 0, 0);
+            }
+          }
+          if (t > 0 && !tc::mbar_wait(&bars->v_empty[c], (t - 1) & 1, abort_flag)) return false;
           const int part = lane & 15;                // 8-dim piece within the chunk
           const uint32_t atom = 2 * c + (part >> 3);
 #pragma unroll
-          for (int r = 0; r < 16; ++r) {
-            const uint32_t row = 32 * cw + 2 * r + (lane >> 4);
-            *reinterpret_cast<uint4*>(sm + kVOff + atom * 16384 + tc::sw128_off(row, part & 7)) =
-                bf16x8_to_f16(rawv[r]);
+          for (int r = 0; r < 8; ++r) {
+            const uint32_t vr = 16 * warp + 2 * r + (lane >> 4);
+            *reinterpret_cast<uint4*>(sm + kVOff + atom * 16384 + tc::sw128_off(vr, part & 7)) =
+                bf16x8_to_f16(V4KV_RB(c & 1, r));
           }
           tc::fence_proxy_async_smem();
           tc::mbar_arrive(&bars->v_full[c]);
         }
+#undef V4KV_RB
       }
-      tc::mbar_arrive(&bars->addr_free[i % 3]);
-    }
-  conv_abort:;
-  } else {
-    // ======================= softmax (thread = tile row = TMEM lane)
-    const int row = tid;
-    float k0 = a.qk0[b0];
-    int q_issued = 1;  // query copies started by this thread (row 0 only)
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+      return true;
+    };
+
+    // tile 0
     {
-      uint32_t z[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) z[e] = 0u;
-      tc::tmem_st32(lane_base + kLCol, z);
-      tc::tmem_st32(lane_base + kLCol + 32, z);
-      tc::tmem_wait_st();
+      ok = tc::mbar_wait(&bars->addr_ready[0], 0, abort_flag);
+      const bool fp8 = ok && (info[0] & kInfoFp8) != 0;
+      if (ok && fp8) load_fp8(0);
+      if (ok) ok = convert(0, fp8);
     }
     Cursor cu;
     cursor_set(cu, a, b0, lt0);
-    bool ok = true;
     bool seg_first = true;  // the current tile opens a segment
     for (int i = 0; i < n_tiles && ok; ++i) {
       const bool seg_last = i == n_tiles - 1 || cu.lt == cu.nt - 1;
+      // the next tile's codes (fp8) fly while tile i's softmax and PV run
+      bool nxt_fp8 = false;
+      if (i + 1 < n_tiles) {
+        ok = tc::mbar_wait(&bars->addr_ready[(i + 1) % kRing], ((i + 1) / kRing) & 1, abort_flag);
+        nxt_fp8 = ok && (info[(i + 1) % kRing] & kInfoFp8) != 0;
+        if (nxt_fp8) load_fp8(i + 1);
+      }
       // S(i) complete implies PV(i-1) complete (the MMAs run in issue order),
       // so waiting for pv_done(i-1) here costs nothing and frees P and O^T
-      ok = tc::mbar_wait(&bars->v_full[0], i & 1, abort_flag) &&
-           tc::mbar_wait(&bars->s_full[i & 1], (i >> 1) & 1, abort_flag) &&
+      ok = ok && tc::mbar_wait(&bars->s_full[i & 1], (i >> 1) & 1, abort_flag) &&
            (i == 0 || tc::mbar_wait(&bars->pv_done, (i - 1) & 1, abort_flag));
-      // the four softmax warps leave together (they meet at named barriers)
-      ok = named_and(1, 128, ok);
+      // the eight worker warps leave together (they meet at named barriers)
+      ok = named_and(1, 256, ok);
       if (!ok) break;
       tc::tc_fence_after();
-      const float ks = meta[(i % 3) * kT + row];
-      tc::mbar_arrive(&bars->addr_free[i % 3]);
+      const float ks = meta[(i % kRing) * kT + row];
       const bool valid = ks > 0.f;
       const float cj = valid ? k0 * ks : 0.f;
       const float lk = valid ? __log2f(ks) : -INFINITY;
       const float inv_k = valid ? __frcp_rn(ks) : 0.f;
       // u = score in log2 units including log2 ks; d = u - m_ref (in place)
-      float d[kH];
-      const uint32_t s_addr = lane_base + (uint32_t)(i & 1) * kH;
+      float d[32];
+      const uint32_t s_addr = lane_base + (uint32_t)(i & 1) * kH + 32 * hh;
       {
         uint32_t r32[32];
         tc::tmem_ld32(s_addr, r32);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int h = 0; h < 32; ++h) d[h] = fmaf(__uint_as_float(r32[h]), cj, lk);
-        tc::tmem_ld32(s_addr + 32, r32);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int h = 0; h < 32; ++h) d[32 + h] = fmaf(__uint_as_float(r32[h]), cj, lk);
+      }
+      if (seg_last && i + 1 < n_tiles && tid == 0) {
+        // QK(i) is complete (S(i) was read), so Q is free: copy the next
+        // segment's query image while the rest of this tile runs
+        Cursor nx = cu;
+        cursor_next(nx, a);
+        issue_q(a, nx.b, sbase + kQOff, &bars->q_ready);
+        ++q_issued;
       }
       float dmax = -INFINITY;
       {
-        const float4* mr4 = reinterpret_cast<const float4*>(mref);
+        const float4* mr4 = reinterpret_cast<const float4*>(mref + 32 * hh);
 #pragma unroll
-        for (int h4 = 0; h4 < kH / 4; ++h4) {
+        for (int h4 = 0; h4 < 8; ++h4) {
           const float4 m4 = mr4[h4];
           d[4 * h4] -= m4.x;
           d[4 * h4 + 1] -= m4.y;
@@ -630,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
           dmax = fmaxf(dmax, fmaxf(fmaxf(d[4 * h4], d[4 * h4 + 1]), fmaxf(d[4 * h4 + 2], d[4 * h4 + 3])));
         }
       }
-      if (named_or(1, 128, dmax > kTau)) {
+      if (named_or(1, 256, dmax > kTau)) {
         // rare: raise the reference of every head to its running maximum.
         // u is recomputed from S (still in tensor memory) to keep it exact.
         {
@@ -639,43 +676,41 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
           tc::tmem_wait_ld();
 #pragma unroll
           for (int h = 0; h < 32; ++h) d[h] = fmaf(__uint_as_float(r32[h]), cj, lk);
-          tc::tmem_ld32(s_addr + 32, r32);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < 32; ++h) d[32 + h] = fmaf(__uint_as_float(r32[h]), cj, lk);
         }
 #pragma unroll
-        for (int h = 0; h < kH; ++h) {
-          const int wm = __reduce_max_sync(0xffffffffu, ordered(d[h]));
-          if (lane == 0) red[warp * kH + h] = unordered(wm);
+        for (int h = 0; h < 32; ++h) {
+          const int wm = __reduce_max_sync(0xffffffffu, ordered_key(d[h]));
+          if (lane == 0) red[warp * 32 + h] = from_ordered_key(wm);
         }
-        named_sync(1, 128);
-        if (row < kH) {
-          const float old = mref[row];
+        named_sync(1, 256);
+        if (tid < kH) {
+          const int half = tid >> 5, hx = tid & 31;
+          const float old = mref[tid];
           float nm = old;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) nm = fmaxf(nm, red[w * kH + row]);
-          alpha[row] = exp2f(old - nm);
-          mref[row] = nm;
+          for (int w = 0; w < 4; ++w) nm = fmaxf(nm, red[(4 * half + w) * 32 + hx]);
+          alpha[tid] = exp2f(old - nm);
+          mref[tid] = nm;
         }
-        named_sync(1, 128);
+        named_sync(1, 256);
 #pragma unroll
-        for (int h = 0; h < kH; ++h) d[h] -= mref[h];
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
+        for (int h = 0; h < 32; ++h) d[h] -= mref[32 * hh + h];
+        {
           uint32_t lv[32];
-          tc::tmem_ld32(lane_base + kLCol + 32 * half, lv);
+          tc::tmem_ld32(l_addr, lv);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            lv[e] = __float_as_uint(__uint_as_float(lv[e]) * alpha[32 * half + e]);
-          tc::tmem_st32(lane_base + kLCol + 32 * half, lv);
+          for (int h = 0; h < 32; ++h)
+            lv[h] = __float_as_uint(__uint_as_float(lv[h]) * alpha[32 * hh + h]);
+          tc::tmem_st32(l_addr, lv);
+          tc::tmem_wait_st();
         }
-        tc::tmem_wait_st();
         if (!seg_first) {
-          // O^T rows of this lane (dims 128 mt + row) times alpha per head column
+          // O^T rows of this lane (dims 128 mt + row, mt = 2hh, 2hh + 1) times
+          // alpha per head column
 #pragma unroll 1
-          for (int mt = 0; mt < 4; ++mt) {
+          for (int m2 = 0; m2 < 2; ++m2) {
+            const int mt = 2 * hh + m2;
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
               uint32_t r32[32];
@@ -691,57 +726,53 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
           tc::tmem_wait_st();
         }
       }
-      // P' row of this item: 64 heads in f16, MN-major swizzled, 8 heads per
-      // 16-byte chunk; the normaliser partial sums live in tensor memory
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      // P' row of this item: heads 32 hh .. 32 hh + 31 in f16, 8 heads per
+      // 16-byte chunk (chunks 4 hh .. 4 hh + 3 of the MN-major swizzled row)
+      {
         uint32_t lv[32];
-        tc::tmem_ld32(lane_base + kLCol + 32 * half, lv);
+        tc::tmem_ld32(l_addr, lv);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int h = 32 * half + 8 * c + 2 * e;
+            const int h = 8 * c + 2 * e;
             const float p0 = fast_exp2(d[h]);
             const float p1 = fast_exp2(d[h + 1]);
-            const int k = 8 * c + 2 * e;
-            lv[k] = __float_as_uint(fmaf(p0, inv_k, __uint_as_float(lv[k])));
-            lv[k + 1] = __float_as_uint(fmaf(p1, inv_k, __uint_as_float(lv[k + 1])));
+            lv[h] = __float_as_uint(fmaf(p0, inv_k, __uint_as_float(lv[h])));
+            lv[h + 1] = __float_as_uint(fmaf(p1, inv_k, __uint_as_float(lv[h + 1])));
             pk[e] = h2u(__floats2half2_rn(p0, p1));
           }
-          *reinterpret_cast<uint4*>(sm + kPOff + tc::sw128_off(row, 4 * half + c)) =
+          *reinterpret_cast<uint4*>(sm + kPOff + tc::sw128_off(row, 4 * hh + c)) =
               make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
-        tc::tmem_st32(lane_base + kLCol + 32 * half, lv);
+        tc::tmem_st32(l_addr, lv);
+        tc::tmem_wait_st();
       }
-      tc::tmem_wait_st();
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       tc::mbar_arrive(&bars->p_full);
+      tc::mbar_arrive(&bars->addr_free[i % kRing]);
+      // convert tile i + 1 as PV(i) frees the V chunks (before the epilogue,
+      // so that QK(i + 1) overlaps it; PV(i + 1) cannot start before the
+      // epilogue has read O^T, since it needs this tile loop's next P')
+      if (i + 1 < n_tiles && !(ok = convert(i + 1, nxt_fp8))) break;
 
       if (seg_last) {
         const int b_done = cu.b;
         cursor_next(cu, a);
-        if (i + 1 < n_tiles) {
-          // QK(i) is complete (S(i) was read), so Q is free: copy the next
-          // segment's query image while PV(i) runs
-          k0 = a.qk0[cu.b];
-          if (row == 0) {
-            issue_q(a, cu.b, sbase + kQOff, &bars->q_ready);
-            ++q_issued;
-          }
-        }
+        if (i + 1 < n_tiles) k0 = a.qk0[cu.b];
         ok = tc::mbar_wait(&bars->pv_done, i & 1, abort_flag);
-        ok = named_and(1, 128, ok);
+        ok = named_and(1, 256, ok);
         if (!ok) break;
         tc::tc_fence_after();
         // partial result of (sequence b_done, block cta) in slot b_done + cta:
         // O^T un-normalised, relative to the reference maximum
         const size_t prow = ((size_t)b_done + cta) * kH;
 #pragma unroll 1
-        for (int mt = 0; mt < 4; ++mt) {
+        for (int m2 = 0; m2 < 2; ++m2) {
+          const int mt = 2 * hh + m2;
 #pragma unroll 1
           for (int half = 0; half < 2; ++half) {
             uint32_t r32[32];
@@ -754,35 +785,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
         }
         // normaliser: sum the 128 rows' partial sums per head
         {
-          float v[kH];
-          uint32_t r32[32];
-          tc::tmem_ld32(lane_base + kLCol, r32);
-          tc::tmem_wait_ld();
+          float lsum[32];
+          {
+            uint32_t lv[32];
+            tc::tmem_ld32(l_addr, lv);
+            tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r32[e]);
-          tc::tmem_ld32(lane_base + kLCol + 32, r32);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[32 + e] = __uint_as_float(r32[e]);
-          float two[2];
-          const int hb = warp_reduce_scatter64(v, lane, two);
-          named_sync(1, 128);  // red is free (no slow path in flight)
-          red[warp * kH + hb] = two[0];
-          red[warp * kH + hb + 1] = two[1];
-          named_sync(1, 128);
-          if (row < kH) {
-            const float l = red[row] + red[kH + row] + red[2 * kH + row] + red[3 * kH + row];
-            a.part_ml[(prow + row) * 2] = mref[row];
-            a.part_ml[(prow + row) * 2 + 1] = l;
-            mref[row] = kNone;
+            for (int e = 0; e < 32; ++e) lsum[e] = __uint_as_float(lv[e]);
           }
-          uint32_t z[32];
+          float two[1];
+          const int hb = warp_reduce_scatter32(lsum, lane, two);
+          named_sync(1, 256);  // red is free (no slow path in flight)
+          red[warp * 32 + hb] = two[0];
+          named_sync(1, 256);
+          if (tid < kH) {
+            const int half = tid >> 5, hx = tid & 31;
+            const float l = red[(4 * half) * 32 + hx] + red[(4 * half + 1) * 32 + hx] +
+                            red[(4 * half + 2) * 32 + hx] + red[(4 * half + 3) * 32 + hx];
+            a.part_ml[(prow + tid) * 2] = mref[tid];
+            a.part_ml[(prow + tid) * 2 + 1] = l;
+            mref[tid] = kNone;
+          }
+          {
+            uint32_t z[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) z[e] = 0u;
-          tc::tmem_st32(lane_base + kLCol, z);
-          tc::tmem_st32(lane_base + kLCol + 32, z);
-          tc::tmem_wait_st();
-          named_sync(1, 128);
+            for (int e = 0; e < 32; ++e) z[e] = 0u;
+            tc::tmem_st32(l_addr, z);
+            tc::tmem_wait_st();
+          }
+          named_sync(1, 256);
         }
         seg_first = true;
       } else {
@@ -794,7 +825,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       *abort_flag = 1;
       flag(a.dev_status, V4KV_DEV_TIMEOUT);
     }
-    if (row == 0) {
+    if (tid == 0) {
       // the last query copy has landed before shared memory is released
       // (normally long since; after an abort it may still be in flight)
       volatile int never = 0;
