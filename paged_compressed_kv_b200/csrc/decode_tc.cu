@@ -147,72 +147,82 @@ __device__ __forceinline__ Seq seq_of(const DecodeArgs& a, int b, int32_t* st) {
   return s;
 }
 
-// Address of item `it` and its scale; nullptr (scale 0) if the item is
-// skipped. Problems are returned as V4KV_DEV_* bits in *err instead of being
-// flagged here, so that the loads of several items can overlap.
-__device__ __forceinline__ const uint8_t* item_ptr(const DecodeArgs& a, int b, const Seq& s, int it,
-                                                   float* ks, int* err) {
-  *ks = 0.f;
-  long long j;
-  bool main_item;
-  if (it < s.n_sel_pad) {
-    if (it >= s.n_sel) return nullptr;
-    j = a.topk ? (long long)a.topk[(size_t)b * a.k + it] : (long long)it;
-    if (j < 0) return nullptr;
-    if (j >= ((long long)s.L + a.ratio - 1) / a.ratio) {
-      *err |= V4KV_DEV_BAD_INDEX;
-      return nullptr;
-    }
-    main_item = true;
-  } else {
-    const int w = it - s.n_sel_pad;
-    if (w >= s.n_win) return nullptr;
-    j = s.w0 + w;
-    main_item = false;
-  }
-  const int spb = main_item ? a.main.spb : a.window.spb;
-  const int max_blocks = main_item ? a.main.max_blocks : a.window.max_blocks;
-  const int num_pages = main_item ? a.main.num_pages : a.window.num_pages;
-  const int32_t* bt = main_item ? a.main.block_table : a.window.block_table;
-  const bool fp8 = (main_item ? a.main.dtype : a.window.dtype) == V4KV_FP8_E4M3;
-  const long long blk = j / spb;
-  if (blk >= max_blocks) {
-    *err |= V4KV_DEV_BAD_SLOT;
-    return nullptr;
-  }
-  const int p = bt[(size_t)b * max_blocks + blk];
-  if (p < 0 || p >= num_pages) {
-    *err |= V4KV_DEV_BAD_PAGE;
-    return nullptr;
-  }
-  const long long slot = (long long)p * spb + j % spb;
-  const float* scales = main_item ? a.main.scales : a.window.scales;
-  const void* data = main_item ? a.main.data : a.window.data;
-  *ks = fp8 ? scales[slot] : 1.f;
-  return reinterpret_cast<const uint8_t*>(data) + slot * (fp8 ? kD : 2 * kD);
-}
-
 __device__ __forceinline__ void prefetch_l2_line(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // Address warp: lane l resolves rows l, l+32, l+64, l+96 of the tile that
-// starts at item tile0 into the row-address and scale tables, then asks L2 for
-// the rows' cache lines so that the converters' loads find them there.
+// starts at item tile0 into the row-address and scale tables (nullptr / 0 for
+// a skipped item), then asks L2 for the rows' cache lines so that the workers'
+// loads find them there. The loads go in phases (top-k indices, block-table
+// entries, scales), each phase's four loads independent of one another, so a
+// tile costs three memory latencies rather than twelve. Problems are flagged
+// as V4KV_DEV_* bits.
 __device__ __forceinline__ void resolve_tile(const DecodeArgs& a, int b, const Seq& s, int tile0,
                                              int lane, const uint8_t** rp, float* ms) {
+  const bool main_tile = tile0 < s.n_sel_pad;  // a tile is all entries or all window
+  const int spb = main_tile ? a.main.spb : a.window.spb;
+  const int max_blocks = main_tile ? a.main.max_blocks : a.window.max_blocks;
+  const int num_pages = main_tile ? a.main.num_pages : a.window.num_pages;
+  const int32_t* bt = (main_tile ? a.main.block_table : a.window.block_table) + (size_t)b * max_blocks;
+  const bool fp8 = (main_tile ? a.main.dtype : a.window.dtype) == V4KV_FP8_E4M3;
+  const float* scales = main_tile ? a.main.scales : a.window.scales;
+  const uint8_t* data = reinterpret_cast<const uint8_t*>(main_tile ? a.main.data : a.window.data);
+  const long long n_stored = ((long long)s.L + a.ratio - 1) / a.ratio;
   int err = 0;
+  // phase 1: item indices (top-k entries are read from the selection)
+  long long j[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int it = tile0 + lane + 32 * r;
+    j[r] = -1;
+    if (main_tile) {
+      if (it < s.n_sel) j[r] = a.topk ? (long long)a.topk[(size_t)b * a.k + it] : (long long)it;
+    } else {
+      const int w = it - s.n_sel_pad;
+      if (w < s.n_win) j[r] = s.w0 + w;
+    }
+  }
+  // phase 2: block-table entries
+  int pg[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    pg[r] = -1;
+    if (j[r] < 0) continue;
+    if (main_tile && j[r] >= n_stored) {
+      err |= V4KV_DEV_BAD_INDEX;
+      j[r] = -1;
+      continue;
+    }
+    const long long blk = j[r] / spb;
+    if (blk >= max_blocks) {
+      err |= V4KV_DEV_BAD_SLOT;
+      j[r] = -1;
+      continue;
+    }
+    pg[r] = bt[blk];
+  }
+  // phase 3: slots, scales, row addresses
   const uint8_t* p[4];
   float ks[4];
 #pragma unroll
-  for (int r = 0; r < 4; ++r) p[r] = item_ptr(a, b, s, tile0 + lane + 32 * r, &ks[r], &err);
+  for (int r = 0; r < 4; ++r) {
+    p[r] = nullptr;
+    ks[r] = 0.f;
+    if (j[r] < 0) continue;
+    if (pg[r] < 0 || pg[r] >= num_pages) {
+      err |= V4KV_DEV_BAD_PAGE;
+      continue;
+    }
+    const long long slot = (long long)pg[r] * spb + j[r] % spb;
+    ks[r] = fp8 ? scales[slot] : 1.f;
+    p[r] = data + slot * (fp8 ? kD : 2 * kD);
+  }
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     rp[lane + 32 * r] = p[r];
-    ms[lane + 32 * r] = p[r] ? ks[r] : 0.f;
+    ms[lane + 32 * r] = ks[r];
   }
-  const bool main_tile = tile0 < s.n_sel_pad;
-  const bool fp8 = (main_tile ? a.main.dtype : a.window.dtype) == V4KV_FP8_E4M3;
   const int lines = fp8 ? kD / 128 : 2 * kD / 128;
 #pragma unroll
   for (int r = 0; r < 4; ++r)
@@ -727,33 +737,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
         }
       }
       // P' row of this item: heads 32 hh .. 32 hh + 31 in f16, 8 heads per
-      // 16-byte chunk (chunks 4 hh .. 4 hh + 3 of the MN-major swizzled row)
-      {
-        uint32_t lv[32];
-        tc::tmem_ld32(l_addr, lv);
-        tc::tmem_wait_ld();
+      // 16-byte chunk (chunks 4 hh .. 4 hh + 3 of the MN-major swizzled row);
+      // d keeps the fp32 weights for the normaliser update after the arrive
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[4];
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int h = 8 * c + 2 * e;
-            const float p0 = fast_exp2(d[h]);
-            const float p1 = fast_exp2(d[h + 1]);
-            lv[h] = __float_as_uint(fmaf(p0, inv_k, __uint_as_float(lv[h])));
-            lv[h + 1] = __float_as_uint(fmaf(p1, inv_k, __uint_as_float(lv[h + 1])));
-            pk[e] = h2u(__floats2half2_rn(p0, p1));
-          }
-          *reinterpret_cast<uint4*>(sm + kPOff + tc::sw128_off(row, 4 * hh + c)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        for (int e = 0; e < 4; ++e) {
+          const int h = 8 * c + 2 * e;
+          d[h] = fast_exp2(d[h]);
+          d[h + 1] = fast_exp2(d[h + 1]);
+          pk[e] = h2u(__floats2half2_rn(d[h], d[h + 1]));
         }
-        tc::tmem_st32(l_addr, lv);
-        tc::tmem_wait_st();
+        *reinterpret_cast<uint4*>(sm + kPOff + tc::sw128_off(row, 4 * hh + c)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       tc::mbar_arrive(&bars->p_full);
       tc::mbar_arrive(&bars->addr_free[i % kRing]);
+      {
+        uint32_t lv[32];
+        tc::tmem_ld32(l_addr, lv);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 32; ++h) lv[h] = __float_as_uint(fmaf(d[h], inv_k, __uint_as_float(lv[h])));
+        tc::tmem_st32(l_addr, lv);
+        tc::tmem_wait_st();
+      }
       // convert tile i + 1 as PV(i) frees the V chunks (before the epilogue,
       // so that QK(i + 1) overlaps it; PV(i + 1) cannot start before the
       // epilogue has read O^T, since it needs this tile loop's next P')
