@@ -14,13 +14,13 @@
 // reference maximum per head, raised only when a score exceeds it by more
 // than 2^8 (P' <= 256), at which point O^T and the partial sums are rescaled.
 //
-// Warp roles (320 threads): warps 0-7 are workers. Each runs the softmax of
+// Warp roles (352 threads): warps 0-7 are workers. Each runs the softmax of
 // one tile row (its TMEM lane) for 32 of the 64 heads, then gathers and
 // converts 16 rows of the next tile (16-byte coalesced page loads) as the
 // second product releases each V chunk. Warp 8 allocates tensor memory and
-// one of its threads issues the MMAs; warp 9 resolves the rows of the tiles
-// up to kRing - 1 ahead and prefetches them into L2. The partial normalisers of each row
-// (one per head) live in tensor memory.
+// one of its threads issues the MMAs; warps 9 and 10 resolve the rows of the
+// even and odd tiles up to kRing - 1 ahead and prefetch them into L2. The
+// partial normalisers of each row (one per head) live in tensor memory.
 //
 // Schedule: the kernel is persistent. The tiles of all sequences form one
 // list (each sequence: its entries padded to whole tiles, then its window);
@@ -40,7 +40,7 @@ namespace {
 constexpr int kH = 64;          // heads (MMA N)
 constexpr int kD = 512;         // dims
 constexpr int kT = 128;         // items per tile (MMA M of the first product)
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr float kTau = 8.f;     // rescale when a score exceeds the reference by 2^8
 constexpr float kNone = -1e30f; // reference maximum before any item
 
@@ -427,11 +427,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
     return;
   }
 
-  if (warp == 9) {
+  if (warp >= 9) {
     // ======================= address resolution + L2 prefetch, up to kRing - 1 tiles ahead
+    // (warp 9 the even tiles, warp 10 the odd ones)
+    const int aw = warp - 9;
     Cursor cu;
     cursor_set(cu, a, b0, lt0);
-    for (int t = 0; t < n_tiles; ++t) {
+    if (aw) cursor_next(cu, a);
+    for (int t = aw; t < n_tiles; t += 2) {
       const int buf = t % kRing;
       if (t >= kRing && !tc::mbar_wait(&bars->addr_free[buf], ((t - kRing) / kRing) & 1, abort_flag)) break;
       if (t > 0 && cu.lt == 0) {
@@ -448,6 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       }
       __syncwarp();
       tc::mbar_arrive(&bars->addr_ready[buf]);
+      cursor_next(cu, a);
       cursor_next(cu, a);
     }
   } else if (warp == 8) {
@@ -467,14 +471,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
         const uint32_t s_col = (uint32_t)(i & 1) * kH;
         bool first = i == 0;
         for (int c = 0; c < 4 && ok; ++c) {
-          ok = tc::mbar_wait(&bars->v_full[c], par, abort_flag);
+          ok = tc::mbar_wait_spin(&bars->v_full[c], par, abort_flag);
           if (!ok) break;
           if (c == 0) {
             // the converters read this tile's info word before arriving
             first = (info[i % kRing] & kInfoFirst) != 0;
             if (first) {
               // the segment's query image has landed in shared memory
-              ok = tc::mbar_wait(&bars->q_ready, seg & 1, abort_flag);
+              ok = tc::mbar_wait_spin(&bars->q_ready, seg & 1, abort_flag);
               if (!ok) break;
               ++seg;
             }
@@ -490,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
         }
         if (!ok) break;
         tc::mma_commit(&bars->s_full[i & 1]);
-        ok = tc::mbar_wait(&bars->p_full, par, abort_flag);
+        ok = tc::mbar_wait_spin(&bars->p_full, par, abort_flag);
         if (!ok) break;
         tc::tc_fence_after();
 #pragma unroll
@@ -635,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       }
       // S(i) complete implies PV(i-1) complete (the MMAs run in issue order),
       // so waiting for pv_done(i-1) here costs nothing and frees P and O^T
-      ok = ok && tc::mbar_wait(&bars->s_full[i & 1], (i >> 1) & 1, abort_flag) &&
+      ok = ok && tc::mbar_wait_spin(&bars->s_full[i & 1], (i >> 1) & 1, abort_flag, 32) &&
            (i == 0 || tc::mbar_wait(&bars->pv_done, (i - 1) & 1, abort_flag));
       // the eight worker warps leave together (they meet at named barriers)
       ok = named_and(1, 256, ok);

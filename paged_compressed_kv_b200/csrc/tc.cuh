@@ -78,6 +78,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait for latency-critical waiters: polls without letting the hardware
+// suspend the thread (a suspended thread can wake well after the phase flips),
+// backing off `backoff_ns` between polls. Same limits as mbar_wait.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               uint32_t backoff_ns = 0) {
+  if (mbar_poll(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_poll(bar, parity)) return true;
+    if (abort && *abort) return false;
+    if (clock64() - t0 > kWaitCycles) return false;
+    if (backoff_ns) __nanosleep(backoff_ns);
+  }
+}
+
 // ------------------------------------------------------------------ TMA
 // 2-D tiled tensor copy global -> shared of one box at coordinates (x, y),
 // completing `bytes` of transaction count on the mbarrier (no multicast).
