@@ -318,24 +318,17 @@ __device__ __forceinline__ unsigned long long comp_key(uint32_t key, int j) {
 }
 
 // bitonic sort of v[0 .. n) (n a power of two) in descending order
-__device__ __forceinline__ void bitonic_desc(unsigned long long* v, int n) {
-  for (int size = 2; size <= n; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int jx = i ^ stride;
-        if (jx > i) {
-          const bool desc = (i & size) == 0;
-          const unsigned long long x = v[i], y = v[jx];
-          if (desc ? (x < y) : (x > y)) {
-            v[i] = y;
-            v[jx] = x;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
+// number of the n keys v[] (distinct) larger than `mine`; every thread reads
+// the same v[j] at a time (shared-memory broadcast)
+__device__ __forceinline__ int rank_of(unsigned long long mine, const unsigned long long* v, int n) {
+  int r = 0;
+  int j = 0;
+  for (; j + 4 <= n; j += 4)
+    r += (v[j] > mine) + (v[j + 1] > mine) + (v[j + 2] > mine) + (v[j + 3] > mine);
+  for (; j < n; ++j) r += v[j] > mine;
+  return r;
 }
+
 
 // Exact radix select, 8 bits per pass from the top: the keys above the k-th
 // largest in any order, then the ties at it by ascending index. Used when the
@@ -453,16 +446,38 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexArgs 
     }
     __syncthreads();
     const uint32_t tb = bin_sh, above = above_sh;
-    for (int j = threadIdx.x; j < n; j += blockDim.x) {
-      const uint32_t key = score_key(sc[j]);
-      const uint32_t bin = key >> kBinShift;
-      if (tb == 0xffffffffu) break;
-      if (bin > tb) {
-        const uint32_t p = atomicAdd(&n_sel_sh, 1u);
-        if (p < (uint32_t)k) sel[p] = comp_key(key, j);
-      } else if (bin == tb) {
-        const uint32_t p = atomicAdd(&n_cand_sh, 1u);
-        if (p < (uint32_t)kCandCap) cand[p] = comp_key(key, j);
+    if (tb != 0xffffffffu) {
+      // four scores per 16-byte load, four loads in flight per thread (the
+      // score rows are 256-byte aligned; entries past n are skipped)
+      auto take = [&](float f, int j) {
+        if (j >= n) return;
+        const uint32_t key = score_key(f);
+        const uint32_t bin = key >> kBinShift;
+        if (bin > tb) {
+          const uint32_t p = atomicAdd(&n_sel_sh, 1u);
+          if (p < (uint32_t)k) sel[p] = comp_key(key, j);
+        } else if (bin == tb) {
+          const uint32_t p = atomicAdd(&n_cand_sh, 1u);
+          if (p < (uint32_t)kCandCap) cand[p] = comp_key(key, j);
+        }
+      };
+      const float4* sc4 = reinterpret_cast<const float4*>(sc);
+      const int n4 = (n + 3) / 4;
+      for (int q0 = threadIdx.x; q0 < n4; q0 += 4 * blockDim.x) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int q = q0 + u * blockDim.x;
+          v[u] = q < n4 ? sc4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = 4 * (q0 + u * blockDim.x);
+          take(v[u].x, j);
+          take(v[u].y, j + 1);
+          take(v[u].z, j + 2);
+          take(v[u].w, j + 3);
+        }
       }
     }
     __syncthreads();
@@ -473,28 +488,30 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexArgs 
       __syncthreads();
       radix_select_exact(sc, n, k, sel, hist, scan_sh, pick_sh, &n_sel_sh);
     } else {
-      int cpow = 1;
-      while (cpow < (int)nc) cpow <<= 1;
-      for (int i = nc + threadIdx.x; i < cpow; i += blockDim.x) cand[i] = 0ull;
-      __syncthreads();
-      bitonic_desc(cand, cpow);
+      // the threshold bin's best k - above candidates: a candidate's rank is
+      // the number of candidates with a larger key (keys are distinct)
       const int need = k - (int)above;
-      for (int i = threadIdx.x; i < need; i += blockDim.x) sel[above + i] = cand[i];
+      for (int c = threadIdx.x; c < (int)nc; c += blockDim.x) {
+        const unsigned long long mine = cand[c];
+        const int r = rank_of(mine, cand, (int)nc);
+        if (r < need) sel[above + r] = mine;
+      }
       __syncthreads();
     }
   }
 
-  bitonic_desc(sel, kpow);
+  // output position of each selected key = its rank among the selected keys
   const int valid = min(n, k);
-  for (int i = threadIdx.x; i < k; i += blockDim.x) {
-    int32_t idx = -1;
-    float s = 0.f;
-    if (i < valid) {
-      idx = (int32_t)(0xffffffffu - (uint32_t)(sel[i] & 0xffffffffull));
-      s = __fmul_rn(sc[idx], qs_sh);
-    }
-    a.topk_out[(size_t)b * k + i] = idx;
-    if (a.score_out) a.score_out[(size_t)b * k + i] = s;
+  for (int i = threadIdx.x; i < valid; i += blockDim.x) {
+    const unsigned long long mine = sel[i];
+    const int r = rank_of(mine, sel, valid);
+    const int32_t idx = (int32_t)(0xffffffffu - (uint32_t)(mine & 0xffffffffull));
+    a.topk_out[(size_t)b * k + r] = idx;
+    if (a.score_out) a.score_out[(size_t)b * k + r] = __fmul_rn(sc[idx], qs_sh);
+  }
+  for (int i = valid + threadIdx.x; i < k; i += blockDim.x) {
+    a.topk_out[(size_t)b * k + i] = -1;
+    if (a.score_out) a.score_out[(size_t)b * k + i] = 0.f;
   }
 }
 
