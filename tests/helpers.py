@@ -100,12 +100,20 @@ class DecodeCase:
     """A decode batch: caches on host and device, q, lengths."""
 
     def __init__(self, seed, lens, heads, ratio, main_dtype="fp8", window=128, win_dtype="bf16",
-                 permute=True, q_std=1.0, entry_std=0.5, max_blocks_extra=0):
+                 permute=True, q_std=1.0, entry_std=0.5, max_blocks_extra=0, entry_values=None):
+        """entry_values(b, n) -> [n, 512] float values of sequence b's stored
+        entries (quantised or rounded like the random ones); default random."""
         r = synth.rng(seed)
         self.lens = np.asarray(lens, dtype=np.int64)
         self.B, self.H, self.ratio, self.W = len(lens), heads, ratio, window
         spb = 256 // ratio
-        ents = [entry_rows(r, paging.entry_count(L, ratio), main_dtype, entry_std) for L in lens]
+        if entry_values is None:
+            ents = [entry_rows(r, paging.entry_count(L, ratio), main_dtype, entry_std) for L in lens]
+        else:
+            ents = []
+            for b, L in enumerate(lens):
+                x = np.asarray(entry_values(b, paging.entry_count(L, ratio)), dtype=np.float64)
+                ents.append(codecs.quantize_entry(x) if main_dtype == "fp8" else (codecs.bf16_bits(x), None))
         self.main = lay_out(ents, spb, r, main_dtype, permute=permute,
                             max_blocks=max([-(-paging.entry_count(L, ratio) // spb) for L in lens] + [1]) + max_blocks_extra)
         wins = [window_rows(r, int(L), window, win_dtype) for L in lens]

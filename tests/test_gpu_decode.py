@@ -38,9 +38,11 @@ def check_all(case, got, topk=None, seqs=None, q_round=None):
         assert_close_bf16(got[b], ref, f"seq {b} L={case.lens[b]}")
 
 
-def test_tiny_c4a_bf16_identity_table():
-    # 1 sequence, 1024 raw tokens, 8 heads, bf16 entries, identity table
-    case = DecodeCase(synth.seed_for(0), [1024], 8, 4, main_dtype="bf16", permute=False)
+@pytest.mark.parametrize("heads", [8, 64])
+def test_tiny_c4a_bf16_identity_table(heads):
+    # 1 sequence, 1024 raw tokens, bf16 entries, identity table (64 heads: the
+    # tensor-core path's bf16 entry tiles)
+    case = DecodeCase(synth.seed_for(0), [1024], heads, 4, main_dtype="bf16", permute=False)
     got, st = run_decode(case)
     assert st == 0
     check_all(case, got)
@@ -88,10 +90,11 @@ def test_topk_selection_with_padding_and_holes():
     check_all(case, got, topk=topk)
 
 
-def test_window_covers_context_is_full_attention():
+@pytest.mark.parametrize("heads", [16, 64])
+def test_window_covers_context_is_full_attention(heads):
     # W >= L: no entry is visible, attention runs over all raw tokens
     lens = [1, 17, 300, 1000]
-    case = DecodeCase(205, lens, 16, 4, window=1024)
+    case = DecodeCase(205, lens, heads, 4, window=1024)
     got, st = run_decode(case)
     assert st == 0
     check_all(case, got)
@@ -106,30 +109,75 @@ def test_page_permutation_invariance_bitwise():
     assert np.array_equal(ga, gb)
 
 
-def test_empty_sequence_gives_zeros():
-    case = DecodeCase(207, [0, 500], 8, 4)
+@pytest.mark.parametrize("heads", [8, 64])
+def test_empty_sequence_gives_zeros(heads):
+    case = DecodeCase(207, [0, 500, 0], heads, 4)
     got, st = run_decode(case)
     assert st == 0
-    assert np.all(got[0] == 0)
+    assert np.all(got[0] == 0) and np.all(got[2] == 0)
     check_all(case, got, seqs=[1])
 
 
-def test_bad_page_is_flagged_not_read():
-    case = DecodeCase(208, [3000], 8, 4)
+@pytest.mark.parametrize("heads", [8, 64])
+def test_bad_page_is_flagged_not_read(heads):
+    case = DecodeCase(208, [3000], heads, 4)
     case.main.bt[0, 2] = 10_000_000
     _, st = run_decode(case)
     assert st & 1
 
 
-def test_out_of_range_topk_index_is_flagged():
-    case = DecodeCase(209, [3000], 8, 4)
+@pytest.mark.parametrize("heads", [8, 64])
+def test_out_of_range_topk_index_is_flagged(heads):
+    case = DecodeCase(209, [3000], heads, 4)
     topk = np.array([[1, 2, 100000, -1]], dtype=np.int64)
     _, st = run_decode(case, topk=topk)
     assert st & 4
 
 
-def test_sm_scale_argument():
-    case = DecodeCase(210, [2000], 8, 4)
+@pytest.mark.parametrize("heads", [8, 64])
+def test_sm_scale_argument(heads):
+    case = DecodeCase(210, [2000], heads, 4)
     got, _ = run_decode(case, sm_scale=0.2)
     ref = case.oracle(0, sm_scale=0.2)
     assert_close_bf16(got[0], ref)
+
+
+@pytest.mark.parametrize("heads", [8, 64])
+def test_rising_scores_raise_the_reference(heads):
+    # entries increasingly aligned with the query: the scores climb by about
+    # 60 nats over the sequence, so the running reference maximum is raised
+    # (and the partial output rescaled) many times along the way
+    lens = [128 + 4 * 2500, 128 + 4 * 700]
+    r = synth.rng(211)
+    base = synth.normal(r, (len(lens), 512))
+
+    def values(b, n):
+        u = base[b] / np.linalg.norm(base[b])
+        c = 60.0 * np.arange(n) / max(n - 1, 1)  # score of entry j is about c_j
+        noise = synth.normal(r, (n, 512), 0.05)
+        return (c[:, None] * math.sqrt(512) / np.linalg.norm(base[b])) * (u[None, :] + noise)
+
+    case = DecodeCase(211, lens, heads, 4, entry_values=values)
+    for b in range(len(lens)):
+        case.q[b, :, :] = base[b]
+    got, st = run_decode(case)
+    assert st == 0
+    check_all(case, got)
+
+
+def test_many_short_sequences_per_block():
+    # 300 sequences of 1 to 3 tiles: every sweep block opens several segments
+    r = synth.rng(212)
+    lens = r.integers(1, 700, 300).tolist()
+    case = DecodeCase(212, lens, 64, 4)
+    got, st = run_decode(case)
+    assert st == 0
+    check_all(case, got, seqs=list(range(0, 300, 7)))
+
+
+@pytest.mark.parametrize("heads", [8, 64])
+def test_fp8_window(heads):
+    case = DecodeCase(213, [3000, 100], heads, 4, win_dtype="fp8")
+    got, st = run_decode(case)
+    assert st == 0
+    check_all(case, got)
