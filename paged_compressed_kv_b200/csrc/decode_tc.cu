@@ -856,77 +856,82 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   }
 }
 
-// grid (heads, batch), 128 threads x 4 dims: merge the partial results of the
-// blocks whose tile ranges cover the sequence, normalise, inverse RoPE at
-// position L - 1, store bf16
-__global__ void __launch_bounds__(128) decode_tc_merge_kernel(DecodeArgs a) {
-  __shared__ int slot_lo, slot_hi;      // blocks whose tile ranges meet the sequence
-  __shared__ float w_sh[kMaxSplits];    // their weights (at most every block)
-  __shared__ float l_sh;
+// grid (heads / 8, batch), 256 threads: warp w merges head 8 * blockIdx.x + w
+// of sequence b over the blocks whose tile ranges met it (lane l: dims 16l ..
+// 16l + 15), normalises, applies the inverse RoPE at position L - 1 (cos/sin
+// from the prep kernel's table) and stores bf16.
+__global__ void __launch_bounds__(256) decode_tc_merge_kernel(DecodeArgs a) {
+  __shared__ float w_sh[8][kMaxSplits];  // per warp: the blocks' weights
   tc::pdl_wait();  // the sweep's partial results are complete from here on
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int d0 = threadIdx.x * 4;
-  if (threadIdx.x < 32) {
-    // the blocks that met the sequence (an empty range writes no partial)
-    const int lane = threadIdx.x;
-    const int2 sl = a.seq_slots[b];
-    const int lo = sl.x, hi = sl.y;
-    float M = -INFINITY;
-    for (int c = lo + lane; c <= hi; c += 32) {
-      const bool empty = a.cta_x0[c + 1] <= a.cta_x0[c];
-      const float m = empty ? -INFINITY : a.part_ml[(((size_t)b + c) * kH + h) * 2];
-      w_sh[c - lo] = m;
-      M = fmaxf(M, m);
-    }
-    M = warp_max(M);
-    float L = 0.f;
-    for (int c = lo + lane; c <= hi; c += 32) {
-      const float m = w_sh[c - lo];
-      const float w = m == -INFINITY ? 0.f : exp2f(m - M);
-      w_sh[c - lo] = w;
-      if (w > 0.f) L = fmaf(w, a.part_ml[(((size_t)b + c) * kH + h) * 2 + 1], L);
-    }
-    L = warp_sum(L);
-    if (lane == 0) {
-      slot_lo = lo;
-      slot_hi = hi;
-      l_sh = L;
-    }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = 8 * blockIdx.x + warp, b = blockIdx.y;
+  const int2 sl = a.seq_slots[b];
+  const int lo = sl.x, hi = sl.y;
+  float M = -INFINITY;
+  for (int c = lo + lane; c <= hi; c += 32) {
+    const bool empty = a.cta_x0[c + 1] <= a.cta_x0[c];
+    const float m = empty ? -INFINITY : a.part_ml[(((size_t)b + c) * kH + h) * 2];
+    w_sh[warp][c - lo] = m;
+    M = fmaxf(M, m);
   }
-  __syncthreads();
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  const float L = l_sh;
-  for (int c = slot_lo; c <= slot_hi; ++c) {
-    const float w = w_sh[c - slot_lo];
+  M = warp_max(M);
+  float L = 0.f;
+  for (int c = lo + lane; c <= hi; c += 32) {
+    const float m = w_sh[warp][c - lo];
+    const float w = m == -INFINITY ? 0.f : exp2f(m - M);
+    w_sh[warp][c - lo] = w;
+    if (w > 0.f) L = fmaf(w, a.part_ml[(((size_t)b + c) * kH + h) * 2 + 1], L);
+  }
+  L = warp_sum(L);
+  __syncwarp();
+  const int d0 = 16 * lane;
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+  for (int c = lo; c <= hi; ++c) {
+    const float w = w_sh[warp][c - lo];
     if (w == 0.f) continue;
-    const size_t row = ((size_t)b + c) * kH + h;
-    const float4 o = *reinterpret_cast<const float4*>(a.part_o + row * kD + d0);
-    acc[0] = fmaf(w, o.x, acc[0]);
-    acc[1] = fmaf(w, o.y, acc[1]);
-    acc[2] = fmaf(w, o.z, acc[2]);
-    acc[3] = fmaf(w, o.w, acc[3]);
+    const float4* o4 = reinterpret_cast<const float4*>(a.part_o + (((size_t)b + c) * kH + h) * kD + d0);
+    float4 v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] = o4[q];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc[4 * q] = fmaf(w, v[q].x, acc[4 * q]);
+      acc[4 * q + 1] = fmaf(w, v[q].y, acc[4 * q + 1]);
+      acc[4 * q + 2] = fmaf(w, v[q].z, acc[4 * q + 2]);
+      acc[4 * q + 3] = fmaf(w, v[q].w, acc[4 * q + 3]);
+    }
   }
-  float o[4];
   const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) o[i] = acc[i] * inv;
-  int Lb = a.seq_lens[b];
-  Lb = min(Lb, a.max_len);
+  for (int e = 0; e < 16; ++e) acc[e] *= inv;
+  const int Lb = min(a.seq_lens[b], a.max_len);
   if (a.rope.rope_dim > 0 && Lb > 0) {
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < 8; ++k) {
       const int d = d0 + 2 * k;
       if (d >= a.rope.rope_offset && d + 1 < a.rope.rope_offset + a.rope.rope_dim) {
+        const int i = (d - a.rope.rope_offset) >> 1;
         float c, s;
-        rope_cs(a.rope, (d - a.rope.rope_offset) >> 1, (long long)Lb - 1, &c, &s);
-        rope_apply(o[2 * k], o[2 * k + 1], c, -s);
+        if (i < kRopeTable) {
+          const float2 cs = a.rope_tab[(size_t)b * kRopeTable + i];
+          c = cs.x;
+          s = cs.y;
+        } else {
+          rope_cs(a.rope, i, (long long)Lb - 1, &c, &s);
+        }
+        rope_apply(acc[2 * k], acc[2 * k + 1], c, -s);
       }
     }
   }
-  uint16_t* dst = reinterpret_cast<uint16_t*>(a.out) + ((size_t)b * kH + h) * kD + d0;
-  const uint32_t w0 = (uint32_t)float_to_bf16_bits(o[0]) | ((uint32_t)float_to_bf16_bits(o[1]) << 16);
-  const uint32_t w1 = (uint32_t)float_to_bf16_bits(o[2]) | ((uint32_t)float_to_bf16_bits(o[3]) << 16);
-  *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
+  uint32_t wv[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    wv[k] = (uint32_t)float_to_bf16_bits(acc[2 * k]) | ((uint32_t)float_to_bf16_bits(acc[2 * k + 1]) << 16);
+  uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.out) + ((size_t)b * kH + h) * kD + d0);
+  dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+  dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
 }
 
 // grid (batch + 1), 256 threads. Block b < batch writes sequence b's query as
@@ -1074,6 +1079,13 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
         make_uint4(hv[0], hv[1], hv[2], hv[3]);
   }
   if (t == 0) a.qk0[b] = a.sm_scale * 1.4426950408889634f * ldexpf(1.f, -e);
+  // cos/sin of the inverse RoPE at the query position, for the merge
+  if (t < kRopeTable && 2 * t < a.rope.rope_dim) {
+    const int Lb = min(a.seq_lens[b], a.max_len);
+    float c = 1.f, s = 0.f;
+    if (Lb > 0) rope_cs(a.rope, t, (long long)Lb - 1, &c, &s);
+    a.rope_tab[(size_t)b * kRopeTable + t] = make_float2(c, s);
+  }
 }
 
 // workspace of the tensor-core path: query images, their multipliers, partial
@@ -1083,7 +1095,8 @@ size_t decode_tc_workspace_bytes(int batch, int num_sms) {
   const size_t qk0 = ((size_t)batch * sizeof(float) + 255) / 256 * 256;
   return (size_t)batch * kQBytes + qk0 + slots * kH * (size_t)(kD + 2) * sizeof(float) +
          ((size_t)batch + 1) * sizeof(int32_t) + 256 + ((size_t)batch + 1) * sizeof(long long) +
-         (2 * (size_t)num_sms + 1) * sizeof(int32_t) + 256 + (size_t)batch * sizeof(int2) + 256;
+         (2 * (size_t)num_sms + 1) * sizeof(int32_t) + 256 + (size_t)batch * sizeof(int2) + 256 +
+         (size_t)batch * kRopeTable * sizeof(float2) + 256;
 }
 
 void decode_tc_layout(DecodeArgs& a, void* workspace) {
@@ -1104,6 +1117,9 @@ void decode_tc_layout(DecodeArgs& a, void* workspace) {
   uint8_t* q = reinterpret_cast<uint8_t*>(a.cta_b0 + a.n_splits);
   q = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(q) + 255) & ~uintptr_t(255));
   a.seq_slots = reinterpret_cast<int2*>(q);
+  uint8_t* r = reinterpret_cast<uint8_t*>(a.seq_slots + a.batch);
+  r = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(r) + 255) & ~uintptr_t(255));
+  a.rope_tab = reinterpret_cast<float2*>(r);
 }
 
 // launch with programmatic stream serialization: the kernel may start while
@@ -1134,7 +1150,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   e = launch_pdl(decode_tc_kernel, dim3(a.n_splits), dim3(kThreads), kSmemBytes, stream, a);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_tc_merge_kernel, dim3(kH, a.batch), dim3(128), 0, stream, a);
+  return launch_pdl(decode_tc_merge_kernel, dim3(kH / 8, a.batch), dim3(256), 0, stream, a);
 }
 
 }  // namespace v4kv

@@ -107,6 +107,7 @@ struct DecodeArgs {
   int32_t* cta_x0;     // tensor-core path: [n_splits + 1] first tile of each block's range
   int32_t* cta_b0;     // tensor-core path: [n_splits] sequence of that first tile
   int2* seq_slots;     // tensor-core path: [batch] first and last block meeting the sequence
+  float2* rope_tab;    // tensor-core path: [batch][kRopeTable] (cos, sin) at position L - 1
 };
 
 cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, int batch,
