@@ -135,9 +135,9 @@ class DecodeStep:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
     def launches_per_step(self):
-        # slot mapping 1, compressor 3 (entries, window, state), decode 3 for 64 heads
-        # (query prep, sweep, merge) or 2 otherwise (sweep, merge)
-        return 7 if self.H == 64 else 6
+        # slot mapping 1, compressor 1 (entries, window rows and state in one
+        # launch), decode 3 for 64 heads (query prep, sweep, merge) or 2 otherwise
+        return 5 if self.H == 64 else 4
 
     def append(self, stream=None):
         v = self.v4kv
@@ -502,20 +502,47 @@ def run_compress(args, device):
         for c in range(st.calls):  # warm-up pass (also fills the cache once)
             st.call(c)
         torch.cuda.synchronize()
+        # eager: each call timed on its own, Python enqueue included
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(st.calls)]
         for c in range(st.calls):
             ev[c][0].record()
             st.call(c)
             ev[c][1].record()
         torch.cuda.synchronize()
-        ms = sum(a.elapsed_time(b) for a, b in ev)
+        ms_eager = sum(a.elapsed_time(b) for a, b in ev)
+        # the same calls captured once into a CUDA graph and replayed
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                for c in range(st.calls):
+                    st.call(c)
+        torch.cuda.synchronize()
+        for _ in range(3):
+            graph.replay()
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        reps, ms_g = 5, []
+        for _ in range(reps):
+            flush.fill_(1)  # inputs of one pass (~300 MB) exceed L2 anyway
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ms_g.append(e0.elapsed_time(e1))
+        del graph
+        ms = float(np.median(ms_g))
         byts = sum(st.algorithmic_bytes(c) for c in range(st.calls))
         out[f"r{ratio}"] = {"calls": st.calls, "tokens": st.B * st.N, "ms": ms,
                             "tokens_per_s": st.B * st.N / (ms * 1e-3),
                             "gbs": byts / (ms * 1e-3) / 1e9, "frac": byts / (ms * 1e-3) / 1e9 / peak,
+                            "ms_eager": ms_eager,
+                            "gbs_eager": byts / (ms_eager * 1e-3) / 1e9,
                             "status": int(st.status.item())}
     return {"config": "compressor write path, 8 x 32K raw bf16 tokens, random chunks 1..4096, fp8 "
-                      "entries, shuffled pages", "results": out}
+                      "entries, shuffled pages; ms = one CUDA-graph replay of all calls (median of 5), "
+                      "ms_eager = the calls launched one by one from Python", "results": out}
 
 
 class MixedStep:
@@ -619,36 +646,49 @@ def run_mixed(args, device):
         kw["c128a_layers"] = min(31, args.layers)
     st = MixedStep(device, **kw)
     nl4, nl128 = len(st.c4a), len(st.c128a)
-    ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(2)] for k in ("idx", "att4", "att128")}
-    tot = {"idx": 0.0, "att4": 0.0, "att128": 0.0}
-    for it in range(args.warmup + args.steps):
-        timed = it >= args.warmup
+
+    def whole_step():
         for l in range(nl4):
-            if timed:
-                ev["idx"][0].record()
             st.index(l)
-            if timed:
-                ev["idx"][1].record()
-                ev["att4"][0].record()
             st.attend_c4a(l)
-            if timed:
-                ev["att4"][1].record()
-                torch.cuda.synchronize()
-                tot["idx"] += ev["idx"][0].elapsed_time(ev["idx"][1])
-                tot["att4"] += ev["att4"][0].elapsed_time(ev["att4"][1])
         for l in range(nl128):
-            if timed:
-                ev["att128"][0].record()
             st.attend_c128a(l)
-            if timed:
-                ev["att128"][1].record()
-                torch.cuda.synchronize()
-                tot["att128"] += ev["att128"][0].elapsed_time(ev["att128"][1])
-    for k in tot:
-        tot[k] /= args.steps
+
+    parts = {"step": whole_step,
+             "idx": lambda: [st.index(l) for l in range(nl4)],
+             "att4": lambda: [st.attend_c4a(l) for l in range(nl4)],
+             "att128": lambda: [st.attend_c128a(l) for l in range(nl128)]}
+    for _ in range(args.warmup):
+        whole_step()
+    torch.cuda.synchronize()
+    # each part is captured once into a CUDA graph and replayed, so the times
+    # are the device's, without the Python enqueue of ~150 calls per step
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graphs = {}
+    with torch.cuda.stream(side):
+        for name, fn in parts.items():
+            graphs[name] = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graphs[name], stream=side):
+                fn()
+    torch.cuda.synchronize()
+    tot = {}
+    for name, gr in graphs.items():
+        gr.replay()
+        gr.replay()
+        ms = []
+        for _ in range(args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            gr.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        tot[name] = float(np.median(ms))
+    graphs.clear()
     idx_b, a4_b, a128_b = st.bytes()
-    step_ms = sum(tot.values())
-    res = {"step_ms": step_ms, "tokens_per_s": st.B / (step_ms * 1e-3),
+    step_ms = tot["step"]
+    res = {"step_ms": step_ms, "parts_ms_sum": tot["idx"] + tot["att4"] + tot["att128"], "tokens_per_s": st.B / (step_ms * 1e-3),
            "indexer": {"ms_per_layer": tot["idx"] / nl4, "gbs": idx_b / (tot["idx"] / nl4 * 1e-3) / 1e9},
            "c4a_attention": {"ms_per_layer": tot["att4"] / nl4, "gbs": a4_b / (tot["att4"] / nl4 * 1e-3) / 1e9},
            "c128a_attention": {"ms_per_layer": tot["att128"] / nl128, "gbs": a128_b / (tot["att128"] / nl128 * 1e-3) / 1e9},
@@ -656,7 +696,8 @@ def run_mixed(args, device):
            "status": int(st.status.item())}
     res["step_frac"] = res["step_gbs"] / peak
     name = (f"{nl4 + nl128}-layer mixed step ({nl4} c4a with indexer top-512 + {nl128} c128a), "
-            f"batch {st.B}, context U[1K, 256K], 64 heads, fp8 KV")
+            f"batch {st.B}, context U[1K, 256K], 64 heads, fp8 KV; CUDA-graph replays, median of "
+            f"{args.steps}")
     return {"config": name, "results": res}
 
 

@@ -122,4 +122,23 @@ __device__ __forceinline__ int page_of(const int32_t* bt_row, int max_blocks, lo
   return p;
 }
 
+// launch with programmatic stream serialization: the kernel may start while
+// the previous one in the stream finishes; it waits (griddepcontrol.wait)
+// before it reads that kernel's results
+template <typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 }  // namespace v4kv

@@ -2,265 +2,379 @@
 // raw-token window copy, and the rolling state of the unfinished group.
 // (P1 §2.1 c4a / c128a compression, §2.3 window, §3.1.2 compressor state,
 //  §3.2.1 compressor + RoPE + cache-insert fusion.)
+//
+// One launch does all three. Its first blocks copy window rows (one warp per
+// token). The rest build entries:
+//   ratio <= 32: one warp per group, eight groups per block;
+//   larger ratios: one block per group, each warp summing a run of rows,
+//                  the eight partial sums added in warp order.
+// Every row is an 8-dim chunk per lane (chunk c = lane + 32k), so a lane
+// always touches the same columns of every row it reads or writes.
+//
+// The state of sequence b (its unfinished group's rows and gates) is
+// rewritten by the warp or block that builds b's first entry of the call,
+// after it has consumed the old state. That group is the only reader of the
+// old state, so no other block can observe a half-written state.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace v4kv {
+namespace {
 
 constexpr int kMaxRatio = 128;
+constexpr int kWarps = 8;       // warps per block
+constexpr int kCuSmem = 1024;   // sequences whose entry prefix sums fit in shared memory
 
-struct Vec8 {
-  float v[8];
-};
-
-// 8 consecutive bf16 elements (16 bytes) -> fp32
-__device__ __forceinline__ Vec8 load_bf16x8(const uint16_t* p) {
-  uint4 raw = *reinterpret_cast<const uint4*>(p);
-  Vec8 r;
-  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+__device__ __forceinline__ void unpack_bf16x8(uint4 q, float (&v)[8]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    r.v[2 * i] = __uint_as_float(w[i] << 16);
-    r.v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
   }
-  return r;
 }
 
-__device__ __forceinline__ void store_bf16x8(uint16_t* p, const Vec8& x) {
-  uint32_t w[4];
+template <int KC>
+__device__ __forceinline__ void load_row(const uint16_t* row, int lane, int nch, uint4 (&q)[KC]) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-    w[i] = (uint32_t)float_to_bf16_bits(x.v[2 * i]) |
-           ((uint32_t)float_to_bf16_bits(x.v[2 * i + 1]) << 16);
-  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  for (int k = 0; k < KC; ++k) {
+    const int c = lane + 32 * k;
+    q[k] = c < nch ? __ldcs(reinterpret_cast<const uint4*>(row + 8 * c)) : make_uint4(0, 0, 0, 0);
+  }
 }
 
-// rotate the pairs of this thread's 8 dims [d0, d0+8) that fall in the rope range
-__device__ __forceinline__ void rope8(Vec8& x, int d0, const RopeArgs& rp, long long pos,
-                                      bool inverse) {
+// rotate the rope pairs among this lane's dims at position `pos`. Pair p's
+// (cos, sin) is evaluated once per warp, by lane p % 32, and fetched with
+// shuffles, so every lane must call this.
+template <int KC>
+__device__ __forceinline__ void rope_warp(float (&e)[KC][8], int lane, int nch, const RopeArgs& rp,
+                                          long long pos) {
   if (rp.rope_dim == 0) return;
+  const int npairs = rp.rope_dim >> 1;
+  for (int base = 0; base < npairs; base += 32) {
+    float c = 1.f, s = 0.f;
+    if (base + lane < npairs) rope_cs(rp, base + lane, pos, &c, &s);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    int d = d0 + 2 * k;
-    if (d >= rp.rope_offset && d + 1 < rp.rope_offset + rp.rope_dim) {
-      float c, s;
-      rope_cs(rp, (d - rp.rope_offset) >> 1, pos, &c, &s);
-      if (inverse) s = -s;
-      rope_apply(x.v[2 * k], x.v[2 * k + 1], c, s);
+    for (int k = 0; k < KC; ++k) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int d = 8 * (lane + 32 * k) + 2 * j;
+        const int p = (d - rp.rope_offset) >> 1;
+        const float cc = __shfl_sync(0xffffffffu, c, p & 31);
+        const float ss = __shfl_sync(0xffffffffu, s, p & 31);
+        if (lane + 32 * k < nch && d >= rp.rope_offset && p >= base && p < base + 32 && p < npairs)
+          rope_apply(e[k][2 * j], e[k][2 * j + 1], cc, ss);
+      }
     }
   }
 }
 
-// quantise (fp8) or round (bf16) one vector spread over the block, 8 dims per
-// thread, and store it in `slot` of the pool. `active` marks threads owning dims.
-__device__ __forceinline__ void store_entry(const PoolArgs& pool, long long slot, int d0,
-                                            bool active, Vec8 e, float* red) {
+// quantise (fp8: absmax over the warp's whole vector) or round (bf16) one
+// vector held by a warp, and store it in `slot` of the pool
+template <int KC>
+__device__ __forceinline__ void store_entry_warp(const PoolArgs& pool, long long slot, int lane,
+                                                 int nch, const float (&e)[KC][8]) {
   if (pool.dtype == V4KV_FP8_E4M3) {
     float m = 0.f;
-    if (active)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(e.v[i]));
-    float amax = block_reduce<true>(m, red);
-    float scale = amax == 0.f ? 1.f : __fdiv_rn(amax, kE4m3Max);
-    if (active) {
-      uint16_t c[4];
+    for (int k = 0; k < KC; ++k)
+      if (lane + 32 * k < nch)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(e[k][i]));
+    const float amax = warp_max(m);
+    const float scale = amax == 0.f ? 1.f : __fdiv_rn(amax, kE4m3Max);
+    uint8_t* base = reinterpret_cast<uint8_t*>(pool.data) + slot * pool.dim;
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      const int c = lane + 32 * k;
+      if (c >= nch) continue;
+      uint16_t q[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        c[i] = float2_to_e4m3x2(__fdiv_rn(e.v[2 * i], scale), __fdiv_rn(e.v[2 * i + 1], scale));
-      uint2 w = make_uint2((uint32_t)c[0] | ((uint32_t)c[1] << 16),
-                           (uint32_t)c[2] | ((uint32_t)c[3] << 16));
-      uint8_t* dst = reinterpret_cast<uint8_t*>(pool.data) + slot * pool.dim + d0;
-      *reinterpret_cast<uint2*>(dst) = w;
+        q[i] = float2_to_e4m3x2(__fdiv_rn(e[k][2 * i], scale), __fdiv_rn(e[k][2 * i + 1], scale));
+      *reinterpret_cast<uint2*>(base + 8 * c) =
+          make_uint2((uint32_t)q[0] | ((uint32_t)q[1] << 16), (uint32_t)q[2] | ((uint32_t)q[3] << 16));
     }
-    if (threadIdx.x == 0) pool.scales[slot] = scale;
+    if (lane == 0) pool.scales[slot] = scale;
   } else {
-    if (active) {
-      uint16_t* dst = reinterpret_cast<uint16_t*>(pool.data) + slot * pool.dim + d0;
-      store_bf16x8(dst, e);
+    uint16_t* base = reinterpret_cast<uint16_t*>(pool.data) + slot * pool.dim;
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      const int c = lane + 32 * k;
+      if (c >= nch) continue;
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        w[i] = (uint32_t)float_to_bf16_bits(e[k][2 * i]) |
+               ((uint32_t)float_to_bf16_bits(e[k][2 * i + 1]) << 16);
+      *reinterpret_cast<uint4*>(base + 8 * c) = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
 }
 
-__device__ __forceinline__ int find_seq(const int32_t* cu, int batch, int i) {
-  int lo = 0, hi = batch - 1;  // largest b with cu[b] <= i
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (cu[mid] <= i)
-      lo = mid;
-    else
-      hi = mid - 1;
-  }
-  return lo;
-}
-
-// one block per touched group
-constexpr int kCuSmem = 1024;  // sequences whose prefix sums fit in shared memory
-
-// largest b with cu[b] <= i, from a shared-memory copy of cu[0..batch] when it fits
-__device__ __forceinline__ int find_seq_cached(const int32_t* cu, int batch, int i, int* cu_sh) {
-  if (batch + 1 > kCuSmem) return find_seq(cu, batch, i);
-  for (int k = threadIdx.x; k <= batch; k += blockDim.x) cu_sh[k] = cu[k];
-  __syncthreads();
-  int lo = 0, hi = batch - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (cu_sh[mid] <= i) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
-__global__ void compress_entries_kernel(CompressArgs a) {
-  __shared__ float w[kMaxRatio];
-  __shared__ float red[32];
-  __shared__ int cu_sh[kCuSmem];
-  const int i = blockIdx.x;
-  const int total = a.cu_entries[a.batch];
-  if (i >= total) return;
-  const int b = find_seq_cached(a.cu_entries, a.batch, i, cu_sh);
-  const int r = a.ratio;
+// one window row: token first + u of sequence b, RoPE'd at its own position
+template <int KC>
+__device__ __forceinline__ void window_row(const CompressArgs& a, int b, int u, int lane, int nch) {
   const int s = a.seq_start[b];
   const int n = a.cu_seqlens[b + 1] - a.cu_seqlens[b];
   const int end = s + n;
-  const int g = s / r + (i - a.cu_entries[b]);
-  const int t0 = g * r;
-  const int t1 = min(t0 + r, end);
-  const int np = t1 - t0;
-  const int dim = a.dim;
-  const int d0 = threadIdx.x * 8;
-  const bool active = d0 < dim;
-
-  auto gate_of = [&](int t) -> float {
-    return t < s ? a.state_gate[(size_t)b * r + (t - t0)] : a.gate[a.cu_seqlens[b] + (t - s)];
-  };
-  auto row_of = [&](int t) -> const uint16_t* {
-    return t < s ? a.state_x + ((size_t)b * r + (t - t0)) * dim
-                 : a.x + (size_t)(a.cu_seqlens[b] + (t - s)) * dim;
-  };
-
-  // softmax over the group's present tokens of gate + position bias
-  float m = -INFINITY;
-  for (int t = threadIdx.x; t < np; t += blockDim.x) {
-    float z = gate_of(t0 + t) + a.pos_bias[t];
-    w[t] = z;
-    m = fmaxf(m, z);
-  }
-  m = block_reduce<true>(m, red);
-  for (int t = threadIdx.x; t < np; t += blockDim.x) w[t] = expf(w[t] - m);
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float sum = 0.f;
-    for (int t = 0; t < np; ++t) sum += w[t];
-    red[0] = sum;
-  }
-  __syncthreads();
-  const float sum = red[0];
-  __syncthreads();
-  for (int t = threadIdx.x; t < np; t += blockDim.x) w[t] = __fdiv_rn(w[t], sum);
-  __syncthreads();
-
-  // weighted sum in ascending token order
-  Vec8 e;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) e.v[k] = 0.f;
-  if (active) {
-    for (int t = 0; t < np; ++t) {
-      Vec8 x = load_bf16x8(row_of(t0 + t) + d0);
-      const float wt = w[t];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) e.v[k] = fmaf(wt, x.v[k], e.v[k]);
-    }
-    rope8(e, d0, a.rope, (long long)t0, false);
-    if (a.prequant_out) {
-      float* po = a.prequant_out + (size_t)i * dim + d0;
-      *reinterpret_cast<float4*>(po) = make_float4(e.v[0], e.v[1], e.v[2], e.v[3]);
-      *reinterpret_cast<float4*>(po + 4) = make_float4(e.v[4], e.v[5], e.v[6], e.v[7]);
-    }
-  }
-  long long slot = a.slot_mapping[i];
-  const long long cap = (long long)a.main.num_pages * a.main.spb;
-  if (slot < 0) return;  // unmapped page (already flagged by the slot mapping)
-  if (slot >= cap) {
-    if (threadIdx.x == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
-    return;
-  }
-  store_entry(a.main, slot, d0, active, e, red);
-}
-
-// one block per input token; the last W tokens of each sequence's new ones
-// ([max(s, end - W), end)) are written to the window
-__global__ void compress_window_kernel(CompressArgs a) {
-  __shared__ float red[32];
-  __shared__ int cu_sh[kCuSmem];
-  const int g = blockIdx.x;
-  if (g >= a.cu_seqlens[a.batch]) return;
-  const int b = find_seq_cached(a.cu_seqlens, a.batch, g, cu_sh);
-  const int s = a.seq_start[b];
-  const int n = a.cu_seqlens[b + 1] - a.cu_seqlens[b];
-  const int end = s + n;
-  const int first = max(s, end - a.window_len);
-  const int t = s + (g - a.cu_seqlens[b]);
-  if (t < first || t >= end) return;
-  const int dim = a.dim;
-  const int d0 = threadIdx.x * 8;
-  const bool active = d0 < dim;
+  const int t = max(s, end - a.window_len) + u;
+  if (t >= end) return;
   const int32_t* row = a.window.block_table + (size_t)b * a.window.max_blocks;
   const int blk = t / kLogicalBlock;
   if (blk >= a.window.max_blocks) {
-    if (threadIdx.x == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
+    if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
     return;
   }
   const int p = row[blk];
   if (p < 0) return;  // no page for this block: nothing to keep
   if (p >= a.window.num_pages) {
-    if (threadIdx.x == 0) flag(a.dev_status, V4KV_DEV_BAD_PAGE);
+    if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_PAGE);
     return;
   }
-  Vec8 x;
+  uint4 q[KC];
+  load_row<KC>(a.x + (size_t)(a.cu_seqlens[b] + (t - s)) * a.dim, lane, nch, q);
+  float e[KC][8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) x.v[k] = 0.f;
-  if (active) {
-    x = load_bf16x8(a.x + (size_t)(a.cu_seqlens[b] + (t - s)) * dim + d0);
-    rope8(x, d0, a.rope, (long long)t, false);
-  }
-  const long long slot = (long long)p * kLogicalBlock + (t % kLogicalBlock);
-  store_entry(a.window, slot, d0, active, x, red);
+  for (int k = 0; k < KC; ++k) unpack_bf16x8(q[k], e[k]);
+  rope_warp<KC>(e, lane, nch, a.rope, (long long)t);
+  store_entry_warp<KC>(a.window, (long long)p * kLogicalBlock + (t % kLogicalBlock), lane, nch, e);
 }
 
-// after the entries kernel: keep tokens [floor(end/r)*r, end) as state rows
-__global__ void compress_state_kernel(CompressArgs a) {
-  const int b = blockIdx.x;
+// the group's softmax weights over its np present tokens (gate + position
+// bias), written to w[0..np) by one warp
+template <int NQ>
+__device__ __forceinline__ void group_weights(const CompressArgs& a, int b, int s, int t0, int np,
+                                              int lane, float* w) {
   const int r = a.ratio;
-  const int s = a.seq_start[b];
-  const int n = a.cu_seqlens[b + 1] - a.cu_seqlens[b];
-  if (n <= 0) return;
-  const int end = s + n;
-  const int gs = (end / r) * r;
-  const int rows = end - gs;
-  const int chunks = a.dim / 8;
-  for (int q = threadIdx.x; q < rows * chunks; q += blockDim.x) {
-    const int i = q / chunks, c = q % chunks;
-    const int t = gs + i;
-    if (t < s) continue;  // already in the state from an earlier call
-    const uint16_t* src = a.x + (size_t)(a.cu_seqlens[b] + (t - s)) * a.dim + c * 8;
-    uint16_t* dst = a.state_x_out + ((size_t)b * r + i) * a.dim + c * 8;
-    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
-    if (c == 0) a.state_gate_out[(size_t)b * r + i] = a.gate[a.cu_seqlens[b] + (t - s)];
+  float z[NQ];
+  float m = -INFINITY;
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int t = lane + 32 * q;
+    z[q] = -INFINITY;
+    if (t < np) {
+      const int tt = t0 + t;
+      const float g = tt < s ? a.state_gate[(size_t)b * r + t] : a.gate[a.cu_seqlens[b] + (tt - s)];
+      z[q] = g + a.pos_bias[t];
+      m = fmaxf(m, z[q]);
+    }
+  }
+  m = warp_max(m);
+  float part = 0.f;
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    z[q] = lane + 32 * q < np ? expf(z[q] - m) : 0.f;
+    part += z[q];
+  }
+  const float sum = warp_sum(part);
+#pragma unroll
+  for (int q = 0; q < NQ; ++q)
+    if (lane + 32 * q < np) w[lane + 32 * q] = __fdiv_rn(z[q], sum);
+  __syncwarp();
+}
+
+// acc += sum over rows [lo, hi) of the group (ascending) of w[t] * row t
+template <int KC, int RB>
+__device__ __forceinline__ void weighted_rows(const CompressArgs& a, int b, int s, int t0, int lo,
+                                              int hi, const float* w, int lane, int nch,
+                                              float (&acc)[KC][8]) {
+  const int r = a.ratio;
+  for (int t = lo; t < hi; t += RB) {
+    uint4 q[RB][KC];
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+      const int tt = t0 + t + j;
+      if (t + j < hi) {
+        const uint16_t* row = tt < s ? a.state_x + ((size_t)b * r + (t + j)) * a.dim
+                                     : a.x + (size_t)(a.cu_seqlens[b] + (tt - s)) * a.dim;
+        load_row<KC>(row, lane, nch, q[j]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+      if (t + j >= hi) break;
+      const float wt = w[t + j];
+#pragma unroll
+      for (int k = 0; k < KC; ++k) {
+        float v[8];
+        unpack_bf16x8(q[j][k], v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wt, v[e], acc[k][e]);
+      }
+    }
   }
 }
+
+// RoPE at the group's first position, optional pre-quantisation copy, and
+// the store into the entry's slot
+template <int KC>
+__device__ __forceinline__ void finish_entry(const CompressArgs& a, int i, int t0, int lane, int nch,
+                                             float (&e)[KC][8]) {
+  rope_warp<KC>(e, lane, nch, a.rope, (long long)t0);
+  if (a.prequant_out) {
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      const int c = lane + 32 * k;
+      if (c >= nch) continue;
+      float* po = a.prequant_out + (size_t)i * a.dim + 8 * c;
+      *reinterpret_cast<float4*>(po) = make_float4(e[k][0], e[k][1], e[k][2], e[k][3]);
+      *reinterpret_cast<float4*>(po + 4) = make_float4(e[k][4], e[k][5], e[k][6], e[k][7]);
+    }
+  }
+  const long long slot = a.slot_mapping[i];
+  const long long cap = (long long)a.main.num_pages * a.main.spb;
+  if (slot < 0) return;  // unmapped page (already flagged by the slot mapping)
+  if (slot >= cap) {
+    if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
+    return;
+  }
+  store_entry_warp<KC>(a.main, slot, lane, nch, e);
+}
+
+// state rows [lo, hi) of sequence b after this call: tokens gs + i of the
+// unfinished group that arrived in this call (earlier ones are already there)
+template <int KC, int RB>
+__device__ __forceinline__ void copy_state(const CompressArgs& a, int b, int s, int end, int lo,
+                                           int hi, int lane, int nch) {
+  const int r = a.ratio;
+  const int gs = (end / r) * r;
+  lo = max(lo, s - gs);
+  hi = min(hi, end - gs);
+  for (int i = lo; i < hi; i += RB) {
+    uint4 q[RB][KC];
+#pragma unroll
+    for (int j = 0; j < RB; ++j)
+      if (i + j < hi) load_row<KC>(a.x + (size_t)(a.cu_seqlens[b] + (gs + i + j - s)) * a.dim, lane, nch, q[j]);
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+      if (i + j >= hi) break;
+      uint16_t* dst = a.state_x_out + ((size_t)b * r + (i + j)) * a.dim;
+#pragma unroll
+      for (int k = 0; k < KC; ++k)
+        if (lane + 32 * k < nch) *reinterpret_cast<uint4*>(dst + 8 * (lane + 32 * k)) = q[j][k];
+    }
+  }
+  for (int i = lo + lane; i < hi; i += 32)
+    a.state_gate_out[(size_t)b * r + i] = a.gate[a.cu_seqlens[b] + (gs + i - s)];
+}
+
+// largest b with cu[b] <= i
+__device__ __forceinline__ int seq_of(const int32_t* cu, int batch, int i) {
+  int lo = 0, hi = batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cu[mid] <= i) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// KC: 8-dim chunks per lane (dim <= 256 * KC). kBlockGroup: one block per
+// group (ratio > 32) instead of one warp per group.
+template <int KC, bool kBlockGroup>
+__global__ void __launch_bounds__(kWarps * 32) compress_append_kernel(CompressArgs a,
+                                                                     int window_blocks,
+                                                                     int window_blocks_per_seq) {
+  constexpr int kRB = (KC <= 2 && kBlockGroup) ? 8 : 4;  // rows in flight per warp
+  constexpr int kNQ = kBlockGroup ? kMaxRatio / 32 : 1;  // gates per lane
+  __shared__ float w_sh[kWarps][kNQ * 32];
+  __shared__ float part[kBlockGroup ? kWarps : 1][kBlockGroup ? KC * 256 : 1];
+  __shared__ int cu_sh[kCuSmem];
+  tc::pdl_wait();  // the slot mapping (and whatever produced x) is complete from here on
+  tc::pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nch = a.dim >> 3;
+  if ((int)blockIdx.x < window_blocks) {
+    window_row<KC>(a, blockIdx.x / window_blocks_per_seq,
+                   (blockIdx.x % window_blocks_per_seq) * kWarps + warp, lane, nch);
+    return;
+  }
+  const int eb = blockIdx.x - window_blocks;
+  const bool cached = a.batch + 1 <= kCuSmem;
+  if (cached) {
+    for (int k = threadIdx.x; k <= a.batch; k += blockDim.x) cu_sh[k] = a.cu_entries[k];
+    __syncthreads();
+  }
+  const int32_t* cu = cached ? cu_sh : a.cu_entries;
+  const int total = cu[a.batch];
+  const int i = kBlockGroup ? eb : eb * kWarps + warp;
+  if (i >= total) return;  // uniform over the warp (and over the block for block groups)
+  const int b = seq_of(cu, a.batch, i);
+  const int r = a.ratio;
+  const int s = a.seq_start[b];
+  const int end = s + (a.cu_seqlens[b + 1] - a.cu_seqlens[b]);
+  const int t0 = (s / r + (i - cu[b])) * r;
+  const int np = min(t0 + r, end) - t0;
+  const bool first_of_seq = i == cu[b];
+
+  float* w = w_sh[warp];
+  group_weights<kNQ>(a, b, s, t0, np, lane, w);
+  float acc[KC][8];
+#pragma unroll
+  for (int k = 0; k < KC; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
+
+  if constexpr (!kBlockGroup) {
+    weighted_rows<KC, kRB>(a, b, s, t0, 0, np, w, lane, nch, acc);
+    finish_entry<KC>(a, i, t0, lane, nch, acc);
+    // this warp consumed every old state row and gate it read (the sums and
+    // the softmax reductions depend on them), so the state may be rewritten
+    if (first_of_seq) copy_state<KC, kRB>(a, b, s, end, 0, r, lane, nch);
+  } else {
+    const int rpw = (r + kWarps - 1) / kWarps;
+    weighted_rows<KC, kRB>(a, b, s, t0, min(np, warp * rpw), min(np, (warp + 1) * rpw), w, lane, nch,
+                           acc);
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      float* p = &part[warp][8 * (lane + 32 * k)];
+      *reinterpret_cast<float4*>(p) = make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]);
+      *reinterpret_cast<float4*>(p + 4) = make_float4(acc[k][4], acc[k][5], acc[k][6], acc[k][7]);
+    }
+    __syncthreads();  // partial sums in place; every read of the old state is done
+    if (warp == 0) {
+#pragma unroll
+      for (int k = 0; k < KC; ++k) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[k][e] = part[0][8 * (lane + 32 * k) + e];
+        for (int ww = 1; ww < kWarps; ++ww)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[k][e] += part[ww][8 * (lane + 32 * k) + e];
+      }
+      finish_entry<KC>(a, i, t0, lane, nch, acc);
+    }
+    if (first_of_seq) copy_state<KC, kRB>(a, b, s, end, warp * rpw, (warp + 1) * rpw, lane, nch);
+  }
+}
+
+template <int KC>
+cudaError_t launch_kc(const CompressArgs& a, int max_groups, int window_blocks, int per_seq,
+                      cudaStream_t stream) {
+  const bool block_group = a.ratio > 32;
+  const int entry_blocks = block_group ? max_groups : (max_groups + kWarps - 1) / kWarps;
+  const dim3 grid(window_blocks + entry_blocks), block(kWarps * 32);
+  if (block_group)
+    return launch_pdl(compress_append_kernel<KC, true>, grid, block, 0, stream, a, window_blocks, per_seq);
+  return launch_pdl(compress_append_kernel<KC, false>, grid, block, 0, stream, a, window_blocks, per_seq);
+}
+
+}  // namespace
 
 cudaError_t launch_compress_append(const CompressArgs& a, int max_groups, int total_tokens,
                                    cudaStream_t stream) {
-  const int threads = ((a.dim / 8 + 31) / 32) * 32;
-  if (max_groups > 0) compress_entries_kernel<<<max_groups, threads, 0, stream>>>(a);
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-  if (a.window.data && a.window_len > 0 && total_tokens > 0) {
-    compress_window_kernel<<<total_tokens, threads, 0, stream>>>(a);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
-  }
-  compress_state_kernel<<<a.batch, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  if (a.ratio > kMaxRatio) return cudaErrorInvalidValue;
+  // window rows: per sequence the last min(n, W) new tokens, W <= total new tokens
+  int per_seq = 0;
+  if (a.window.data && a.window_len > 0 && total_tokens > 0)
+    per_seq = (min(a.window_len, total_tokens) + kWarps - 1) / kWarps;
+  const long long wb = (long long)per_seq * a.batch;
+  if (wb + max_groups > 0x7fffffffLL) return cudaErrorInvalidValue;
+  if (wb + max_groups == 0) return cudaSuccess;
+  const int kc = (a.dim + 255) / 256;
+  if (kc <= 1) return launch_kc<1>(a, max_groups, (int)wb, per_seq, stream);
+  if (kc <= 2) return launch_kc<2>(a, max_groups, (int)wb, per_seq, stream);
+  return launch_kc<4>(a, max_groups, (int)wb, per_seq, stream);
 }
 
 }  // namespace v4kv

@@ -1122,25 +1122,6 @@ void decode_tc_layout(DecodeArgs& a, void* workspace) {
   a.rope_tab = reinterpret_cast<float2*>(r);
 }
 
-// launch with programmatic stream serialization: the kernel may start while
-// the previous one in the stream finishes; it waits (griddepcontrol.wait)
-// before it reads that kernel's results
-template <typename... Args>
-static cudaError_t launch_pdl(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem,
-                              cudaStream_t stream, Args... args) {
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, args...);
-}
-
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);

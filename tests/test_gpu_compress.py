@@ -18,13 +18,14 @@ class Appender:
     """Runs appends of per-sequence chunks through the library."""
 
     def __init__(self, seed, n_tokens, ratio, main_dtype="fp8", W=128, gates=None, dim=D,
-                 rope=True):
+                 rope=True, win_dtype="bf16"):
         from paged_compressed_kv_b200 import PagedPool, Rope
         self.r = synth.rng(seed)
         self.n = [int(v) for v in n_tokens]
         self.B, self.ratio, self.W, self.dim = len(n_tokens), ratio, W, dim
-        self.main_dtype = main_dtype
-        self.rope = Rope() if rope else Rope(rope_dim=0)
+        self.main_dtype, self.win_dtype = main_dtype, win_dtype
+        # the last 64 dims carry RoPE (dims 448..511 at the model width)
+        self.rope = Rope(rope_offset=dim - 64) if rope else Rope(rope_dim=0)
         self.x = [synth.normal(self.r, (N, dim)) for N in self.n]
         self.x = [codecs.bf16_round(v) for v in self.x]             # exact bf16 values
         self.g = gates if gates is not None else [synth.normal(self.r, N) for N in self.n]
@@ -42,8 +43,13 @@ class Appender:
             data = torch.zeros(self.P, spb, dim, dtype=torch.bfloat16, device=dev)
             sc = None
         self.main = PagedPool(data=data, block_table=torch.from_numpy(self.bt).to(dev), scales=sc)
-        self.win = PagedPool(data=torch.zeros(self.Pw, 256, dim, dtype=torch.bfloat16, device=dev),
-                             block_table=torch.from_numpy(self.wbt).to(dev))
+        if win_dtype == "fp8":
+            self.win = PagedPool(data=torch.zeros(self.Pw, 256, dim, dtype=torch.uint8, device=dev),
+                                 block_table=torch.from_numpy(self.wbt).to(dev),
+                                 scales=torch.zeros(self.Pw, 256, dtype=torch.float32, device=dev))
+        else:
+            self.win = PagedPool(data=torch.zeros(self.Pw, 256, dim, dtype=torch.bfloat16, device=dev),
+                                 block_table=torch.from_numpy(self.wbt).to(dev))
         self.state_x = torch.zeros(self.B, ratio, dim, dtype=torch.bfloat16, device=dev)
         self.state_g = torch.zeros(self.B, ratio, dtype=torch.float32, device=dev)
         self.done = [0] * self.B
@@ -98,17 +104,27 @@ class Appender:
         return rows, scs
 
     def window_values(self, b):
+        """Stored window rows of sequence b as fp32 (bf16 values, or fp8 codes x scale)."""
         N = self.n[b]
+        ts = list(range(max(0, N - self.W), N))
+        if not ts:
+            return np.zeros((0, self.dim), np.float32)
+        pages = [self.wbt[b, t // 256] for t in ts]
+        if self.win_dtype == "fp8":
+            codes = self.win.data.cpu().numpy()
+            sc = self.win.scales.cpu().numpy()
+            return np.stack([codecs.dequantize_entry(codes[p, t % 256][None], sc[p, t % 256])[0]
+                             for p, t in zip(pages, ts)])
         w = self.win.data.view(torch.int16).cpu().numpy().view(np.uint16)
-        ts = range(max(0, N - self.W), N)
-        return np.stack([w[self.wbt[b, t // 256], t % 256] for t in ts]) if N else np.zeros((0, self.dim), np.uint16)
+        return codecs.bf16_to_f32(np.stack([w[p, t % 256] for p, t in zip(pages, ts)]))
 
 
 def check_against_oracle(ap):
     rope_dim = ap.rope.rope_dim
     for b in range(ap.B):
         N = ap.n[b]
-        ref = compressor.compress_prequant(ap.x[b], ap.g[b], ap.bias, ap.ratio, rope_dim=rope_dim)
+        ref = compressor.compress_prequant(ap.x[b], ap.g[b], ap.bias, ap.ratio, rope_dim=rope_dim,
+                                           rope_offset=ap.rope.rope_offset)
         got = ap.prequant[b]
         assert not np.isnan(got).any()
         amax = np.abs(ref).max(axis=1, keepdims=True)
@@ -120,11 +136,25 @@ def check_against_oracle(ap):
             assert np.array_equal(scs.view(np.uint32), sc.view(np.uint32)), f"seq {b}: scales"
         else:
             assert np.array_equal(rows.view(np.uint16), codecs.bf16_bits(got)), f"seq {b}: bf16"
-        # window: last W tokens RoPE'd at their own position, bf16
+        # window: last W tokens RoPE'd at their own position, bf16 or fp8
         w0 = max(0, N - ap.W)
-        wref = codecs.bf16_round(compressor.window_tokens(ap.x[b][w0:], np.arange(w0, N), rope_dim=rope_dim))
-        wgot = codecs.bf16_to_f32(ap.window_values(b))
-        assert np.all(np.abs(wgot - wref) <= np.abs(wref) * 2.0**-7 + 1e-30), f"seq {b}: window"
+        wtok = compressor.window_tokens(ap.x[b][w0:], np.arange(w0, N), rope_dim=rope_dim,
+                                        rope_offset=ap.rope.rope_offset)
+        wgot = ap.window_values(b)
+        if ap.win_dtype == "fp8":
+            # e4m3: 3 mantissa bits (relative step 2^-3, so rounding error <= 2^-4),
+            # subnormal spacing 2^-9 of the scale unit amax / 448
+            amax = np.abs(wtok).max(axis=1, keepdims=True)
+            bound = np.abs(wtok) * 2.0**-4 * 1.001 + amax / 448 * 2.0**-9 + 1e-30
+            assert np.all(np.abs(wgot - wtok) <= bound), f"seq {b}: fp8 window"
+        else:
+            # bf16 rounding of the result, plus the fp32 rotation's own error: a*c - b*s
+            # in fp32 is off by up to about 3 * 2^-24 * (|a| + |b|), which a near-total
+            # cancellation turns into a large relative error
+            wref = codecs.bf16_round(wtok)
+            xmax = np.abs(ap.x[b][w0:]).max(axis=1, keepdims=True) if N else 0.0
+            bound = np.abs(wref) * 2.0**-7 + xmax * 2.0**-20 + 1e-30
+            assert np.all(np.abs(wgot - wref) <= bound), f"seq {b}: window"
         # state: the unfinished group's raw tokens and gates
         gs = (N // ap.ratio) * ap.ratio
         st = ap.state_x[b, : N - gs].float().cpu().numpy()
@@ -191,6 +221,38 @@ def test_full_size_random_chunks(ratio):
     ap = Appender(synth.seed_for(3), n, ratio)
     while any(d < N for d, N in zip(ap.done, ap.n)):
         ap.append([int(r.integers(1, 4097)) for _ in n])
+    check_against_oracle(ap)
+
+
+@pytest.mark.parametrize("ratio", [4, 128])
+@pytest.mark.parametrize("dim", [128, 200, 1024])
+def test_other_widths(ratio, dim):
+    # one, ragged and four 256-dim spans per lane; two appends so the second
+    # reads back the rolling state
+    n = [1, 300, 1000, 129]
+    ap = Appender(430 + dim + ratio, n, ratio, dim=dim)
+    ap.append([v // 2 + 1 for v in n])
+    ap.append(n)
+    check_against_oracle(ap)
+
+
+def test_fp8_window():
+    n = [5, 128, 700, 2000]
+    ap = Appender(440, n, 4, win_dtype="fp8")
+    ap.append([v // 3 + 1 for v in n])
+    ap.append(n)
+    check_against_oracle(ap)
+
+
+@pytest.mark.parametrize("ratio", [4, 128])
+def test_more_sequences_than_cached_prefix_sums(ratio):
+    # 1100 sequences (entry prefix sums do not fit the kernel's shared copy),
+    # several with no new tokens in a call
+    r = synth.rng(450 + ratio)
+    n = [int(v) for v in r.integers(0, 300, 1100)]
+    ap = Appender(451 + ratio, n, ratio)
+    ap.append([int(v) for v in r.integers(0, 150, 1100)])
+    ap.append(n)
     check_against_oracle(ap)
 
 
