@@ -706,7 +706,7 @@ DTYPE = "f16"
 # DRAM bytes (read + write) of one sweep launch, from an ncu capture of the same
 # build on 32 sequences of the workload, scaled by the entries processed (see
 # profiles/decode_tc_c4a_b64.md); None where no capture of the current kernel exists
-SWEEP_TRAFFIC = {1: 301.4e6}
+SWEEP_TRAFFIC = {}
 
 
 def main():

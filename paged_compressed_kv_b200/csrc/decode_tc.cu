@@ -324,6 +324,7 @@ __device__ __forceinline__ void cursor_next(Cursor& c, const DecodeArgs& a) {
 
 constexpr uint32_t kQBytes = kH * kD * 2;  // one query image (f16)
 constexpr int kMaxSplits = 160;            // sweep blocks at most (the plan caps the grid)
+constexpr int kPrepCache = 2048;           // batches whose prefix sums the prep keeps in shared memory
 
 // Start the bulk copy of sequence b's query image into shared memory; the
 // copy completes phase by transaction count on `bar`.
@@ -456,67 +457,78 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
     }
   } else if (warp == 8) {
     // ======================= MMA issuer
-    if (lane == 0) {
-      const uint32_t iq = tc::idesc_f16(128, kH, 0, 0);
-      const uint32_t ip = tc::idesc_f16(128, kH, 1, 1);
-      // descriptors at the operands' bases; a step adds its byte offset / 16
-      const uint64_t vk_desc = tc::sw128_desc(sbase + kVOff, 16, 1024);     // V, K-major
-      const uint64_t qk_desc = tc::sw128_desc(sbase + kQOff, 16, 1024);     // Q, K-major
-      const uint64_t vm_desc = tc::sw128_desc(sbase + kVOff, 16384, 1024);  // V^T, MN-major
-      const uint64_t p_desc = tc::sw128_desc(sbase + kPOff, 0, 1024);       // P^T, MN-major
-      bool ok = true;
-      int seg = 0;
-      for (int i = 0; i < n_tiles && ok; ++i) {
-        const uint32_t par = i & 1;
-        const uint32_t s_col = (uint32_t)(i & 1) * kH;
-        bool first = i == 0;
-        for (int c = 0; c < 4 && ok; ++c) {
-          ok = tc::mbar_wait_spin(&bars->v_full[c], par, abort_flag);
-          if (!ok) break;
-          if (c == 0) {
-            // the converters read this tile's info word before arriving
-            first = (info[i % kRing] & kInfoFirst) != 0;
-            if (first) {
-              // the segment's query image has landed in shared memory
-              ok = tc::mbar_wait_spin(&bars->q_ready, seg & 1, abort_flag);
-              if (!ok) break;
-              ++seg;
-            }
+    // The whole warp runs the loop, so descriptors, addresses and wait results
+    // stay warp-uniform; one lane, elected once, issues every MMA and commit
+    // (a commit tracks the MMAs of the thread that issues it).
+    const bool leader = tc::elect_one();
+    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+    const uint32_t iq = tc::idesc_f16(128, kH, 0, 0);
+    const uint32_t ip = tc::idesc_f16(128, kH, 1, 1);
+    // descriptors at the operands' bases; a step adds its byte offset / 16
+    const uint64_t vk_desc = tc::sw128_desc(sbase + kVOff, 16, 1024);     // V, K-major
+    const uint64_t qk_desc = tc::sw128_desc(sbase + kQOff, 16, 1024);     // Q, K-major
+    const uint64_t vm_desc = tc::sw128_desc(sbase + kVOff, 16384, 1024);  // V^T, MN-major
+    const uint64_t p_desc = tc::sw128_desc(sbase + kPOff, 0, 1024);       // P^T, MN-major
+    bool ok = true;
+    int seg = 0;
+    for (int i = 0; i < n_tiles && ok; ++i) {
+      const uint32_t par = i & 1;
+      const uint32_t s_col = (uint32_t)(i & 1) * kH;
+      bool first = i == 0;
+      for (int c = 0; c < 4 && ok; ++c) {
+        ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->v_full[c], par, abort_flag));
+        if (!ok) break;
+        if (c == 0) {
+          // the converters read this tile's info word before arriving
+          first = (info[i % kRing] & kInfoFirst) != 0;
+          if (first) {
+            // the segment's query image has landed in shared memory
+            ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->q_ready, seg & 1, abort_flag));
+            if (!ok) break;
+            ++seg;
           }
-          tc::tc_fence_after();
+        }
+        tc::tc_fence_after();
+        if (leader) {
 #pragma unroll
           for (int k8 = 0; k8 < 8; ++k8) {
             const int kk = 8 * c + k8;  // 16-dim step: atom kk/4, 32-byte column kk%4
-            tc::mma_f16(tmem + s_col, vk_desc + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
+            tc::mma_f16(tm + s_col, vk_desc + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
                         qk_desc + (uint64_t)((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), iq,
                         kk > 0 ? 1u : 0u);
           }
         }
-        if (!ok) break;
-        tc::mma_commit(&bars->s_full[i & 1]);
-        ok = tc::mbar_wait_spin(&bars->p_full, par, abort_flag);
-        if (!ok) break;
-        tc::tc_fence_after();
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (leader) tc::mma_commit(&bars->s_full[i & 1]);
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->p_full, par, abort_flag));
+      if (!ok) break;
+      tc::tc_fence_after();
+      if (leader) {
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            tc::mma_f16(tmem + kOCol + kH * mt, vm_desc + (uint64_t)((2 * mt * 16384 + kk * 2048) >> 4),
+            tc::mma_f16(tm + kOCol + kH * mt, vm_desc + (uint64_t)((2 * mt * 16384 + kk * 2048) >> 4),
                         p_desc + (uint64_t)((kk * 2048) >> 4), ip, (!first || kk > 0) ? 1u : 0u);
           tc::mma_commit(&bars->v_empty[mt]);
         }
         tc::mma_commit(&bars->pv_done);
       }
-      if (!ok) {
-        *abort_flag = 1;
-        flag(a.dev_status, V4KV_DEV_TIMEOUT);
-      }
-      // every MMA issued has completed once this barrier flips; this wait
-      // ignores the abort flag (tensor memory is freed after it)
-      volatile int never = 0;
-      tc::mma_commit(&bars->drain);
-      if (!tc::mbar_wait(&bars->drain, 0, &never)) flag(a.dev_status, V4KV_DEV_TIMEOUT);
+      __syncwarp();
     }
+    if (!ok && leader) {
+      *abort_flag = 1;
+      flag(a.dev_status, V4KV_DEV_TIMEOUT);
+    }
+    // every MMA issued has completed once this barrier flips; this wait
+    // ignores the abort flag (tensor memory is freed after it)
+    if (leader) tc::mma_commit(&bars->drain);
+    __syncwarp();
+    volatile int never = 0;
+    if (!tc::mbar_wait(&bars->drain, 0, &never) && leader) flag(a.dev_status, V4KV_DEV_TIMEOUT);
     __syncwarp();
   } else {
     // ======================= workers (warps 0-7): softmax and gather + convert
@@ -951,6 +963,11 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
     // c/G of the total
     __shared__ long long csum[8];
     __shared__ int x0_sh[kMaxSplits + 1];
+    // the prefix sums also go to shared memory (when they fit) for the
+    // binary searches below, which would otherwise chain global loads
+    __shared__ int cum_sh[kPrepCache + 1];
+    __shared__ long long ccum_sh[kPrepCache + 1];
+    const bool cached = a.batch <= kPrepCache;
     int carry = 0;
     long long ccarry = 0;
     for (int base = 0; base < a.batch; base += 256) {
@@ -979,6 +996,10 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
       if (bb < a.batch) {
         a.cum[bb] = before + incl - n;
         a.costcum[bb] = cbefore + cincl - cost;
+        if (cached) {
+          cum_sh[bb] = before + incl - n;
+          ccum_sh[bb] = cbefore + cincl - cost;
+        }
       }
       for (int w = 0; w < 8; ++w) { carry += wsum[w]; ccarry += csum[w]; }
       __syncthreads();
@@ -986,8 +1007,14 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
     if (t == 0) {
       a.cum[a.batch] = carry;
       a.costcum[a.batch] = ccarry;
+      if (cached) {
+        cum_sh[a.batch] = carry;
+        ccum_sh[a.batch] = ccarry;
+      }
     }
     __syncthreads();  // the prefix sums are visible to the whole block
+    const int* cum = cached ? cum_sh : a.cum;
+    const long long* costcum = cached ? ccum_sh : a.costcum;
     const int G = a.n_splits;
     for (int c = t; c <= G; c += 256) {
       int x0 = carry, b0 = a.batch;
@@ -996,11 +1023,11 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
         int l = 0, r = a.batch - 1;  // last sequence whose cost prefix is <= target
         while (l < r) {
           const int m = (l + r + 1) >> 1;
-          if (a.costcum[m] <= target) l = m; else r = m - 1;
+          if (costcum[m] <= target) l = m; else r = m - 1;
         }
         b0 = l;
         const Seq sq = seq_of(a, b0, nullptr);
-        x0 = a.cum[b0] + tile_at_cost(a, sq, target - a.costcum[b0]);
+        x0 = cum[b0] + tile_at_cost(a, sq, target - costcum[b0]);
       }
       a.cta_x0[c] = x0;
       if (c < G) a.cta_b0[c] = b0;
@@ -1009,7 +1036,7 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
     __syncthreads();
     // blocks whose ranges [x0[c], x0[c+1]) meet each sequence's tiles [c0, c1)
     for (int bb = t; bb < a.batch; bb += 256) {
-      const int c0 = a.cum[bb], c1 = a.cum[bb + 1];
+      const int c0 = cum[bb], c1 = cum[bb + 1];
       int lo = 0, hi = -1;
       if (c1 > c0) {
         int l = 0, r = G;  // first c with x0[c+1] > c0

@@ -194,6 +194,18 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64
       : "memory");
 }
 
+// one lane of a converged warp (the same lane on every call while the warp
+// stays converged): the lane that issues single-thread tcgen05 instructions
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // the mbarrier gets one arrival once every MMA issued so far by this thread
 // has completed
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
