@@ -704,9 +704,10 @@ def run_mixed(args, device):
 DTYPE = "f16"
 
 # DRAM bytes (read + write) of one sweep launch, from an ncu capture of the same
-# build on 32 sequences of the workload, scaled by the entries processed (see
-# profiles/decode_tc_c4a_b64.md); None where no capture of the current kernel exists
-SWEEP_TRAFFIC = {}
+# build on the first 32 sequences of the workload (149.8 MB for 150.9 MB of
+# algorithmic bytes), scaled by the algorithmic bytes of the full workload; None
+# where no capture of the current kernel exists
+SWEEP_TRAFFIC = {1: 300.7e6}
 
 
 def main():
