@@ -8,7 +8,12 @@ v4kv_slot_mapping -> v4kv_compress_append (1 token each) ->
 v4kv_decode_attention (all visible entries + window). Inputs are synthetic
 (seeded device draws) and resident in HBM; L2 is flushed between steps.
 
-    python bench.py [--gpus N --steps K --warmup W] [--config 1|2|3|4]
+    python bench.py [--gpus N --steps K --warmup W] [--workload NAME]
+
+Workloads: c4a-b64 (default, above); c128a-b32 (c128a decode, batch 32,
+context log-uniform [128K, 1M]); tiny-c4a (1 sequence of 1024 tokens, 8 heads);
+compressor (the compressor write path alone); mixed-61 (a 61-layer mixed decode
+step with the indexer).
     python bench.py --impl reference ...   # the CPU oracle on host cores
 
 Prints one JSON line (rank 0).
@@ -45,37 +50,37 @@ def load_peaks():
 
 # ------------------------------------------------------------------ workloads
 
-def decode_config(cfg, seqs=0):
-    c = _decode_config(cfg)
+def decode_workload(name, seqs=0):
+    c = _decode_workload(name)
     if seqs:
         c["lens"] = c["lens"][:seqs]
     return c
 
 
-def _decode_config(cfg):
-    r = synth.rng(synth.seed_for(cfg))
-    if cfg == 1:
+def _decode_workload(name):
+    r = synth.rng(synth.seed_for(name))
+    if name == "c4a-b64":
         lens = synth.lengths_uniform(r, 64, 4096, 65536, 4)
         return dict(name="c4a decode, batch 64, context U[4K, 64K], 64 heads, fp8-e4m3 KV dim 512 "
                          "+ fp32 per-entry scale, 128-token bf16 window, shuffled pages",
                     lens=lens, ratio=4, r=r)
-    if cfg == 2:
+    if name == "c128a-b32":
         lens = synth.lengths_loguniform(r, 32, 131072, 1_000_000)
         return dict(name="c128a decode, batch 32, context log-uniform [128K, 1M], 64 heads, fp8-e4m3 "
                          "KV dim 512 + fp32 per-entry scale, 128-token bf16 window, shuffled pages",
                     lens=lens, ratio=128, r=r)
-    if cfg == 0:
+    if name == "tiny-c4a":
         return dict(name="tiny c4a decode, 1 sequence, context 1024, 8 heads", lens=np.array([1024]),
                     ratio=4, r=r, heads=8)
-    raise ValueError(cfg)
+    raise ValueError(name)
 
 
 class DecodeStep:
     """Device-resident caches and per-step inputs of one decode workload."""
 
-    def __init__(self, cfg, device, seed_offset=0, seqs=0):
+    def __init__(self, workload, device, seed_offset=0, seqs=0):
         from paged_compressed_kv_b200 import PagedPool, v4kv
-        c = decode_config(cfg, seqs)
+        c = decode_workload(workload, seqs)
         self.v4kv = v4kv
         self.name = c["name"]
         self.lens = c["lens"].astype(np.int64)
@@ -83,7 +88,7 @@ class DecodeStep:
         self.H = c.get("heads", HEADS)
         self.B = len(self.lens)
         r = c["r"]
-        g = synth.device_generator(synth.seed_for(cfg) + 7919 * seed_offset, device)
+        g = synth.device_generator(synth.seed_for(workload) + 7919 * seed_offset, device)
         spb = 256 // self.ratio
         n_ent = [-(-int(L) // self.ratio) for L in self.lens]
         nblk = [-(-n // spb) for n in n_ent]
@@ -287,7 +292,7 @@ def oracle_sample(step, seconds=10.0, max_seqs=None):
 
 def run_ours(args, rank, world, device):
     peak, peak_kind = load_peaks()
-    step = DecodeStep(args.config, device, seed_offset=rank, seqs=args.seqs)
+    step = DecodeStep(args.workload, device, seed_offset=rank, seqs=args.seqs)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     for _ in range(args.warmup):
@@ -373,7 +378,7 @@ def run_ours(args, rank, world, device):
                    "l2": "flushed between steps (256 MB write), inputs also exceed L2",
                    "decode_ms": t_dec, "hbm_gbs": achieved},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": SWEEP_TRAFFIC.get(args.config) if not args.seqs else None,
+                     "frac": achieved / peak, "traffic": SWEEP_TRAFFIC.get(args.workload) if not args.seqs else None,
                      "kernel": "v4kv_decode_attention (query prep + sweep + merge)",
                      "algorithmic_bytes": alg, "peak_source": peak_kind},
         "e2e": {"value": rate_e2e, "unit": "tokens/s",
@@ -400,7 +405,7 @@ def run_reference(args, rank, world):
     dev = torch.device("cuda", 0) if torch.cuda.is_available() else None
     if dev is None:
         return {"impl": "reference", "unavailable": "needs the workload's caches on a CUDA device"}
-    step = DecodeStep(args.config, dev, seqs=args.seqs)
+    step = DecodeStep(args.workload, dev, seqs=args.seqs)
     per = max(1, int(args.ref_seqs))
     for _ in range(args.warmup):
         oracle_sample(step, seconds=1e9, max_seqs=1)
@@ -424,7 +429,7 @@ def run_reference(args, rank, world):
     }
 
 
-# ------------------------------------------------------------------ other rows (--config 3, 4)
+# ------------------------------------------------------------------ other rows (compressor, mixed-61)
 
 class CompressStep:
     """Compressor write path: 8 sequences x 32K raw bf16 tokens appended in
@@ -434,8 +439,8 @@ class CompressStep:
     def __init__(self, device, ratio, seqs=8, tokens=32768):
         from paged_compressed_kv_b200 import PagedPool, v4kv
         self.v4kv, self.ratio, self.B, self.N = v4kv, ratio, seqs, tokens
-        r = synth.rng(synth.seed_for(3) + ratio)
-        g = synth.device_generator(synth.seed_for(3) + ratio, device)
+        r = synth.rng(synth.seed_for("compressor") + ratio)
+        g = synth.device_generator(synth.seed_for("compressor") + ratio, device)
         self.chunks = [synth.chunk_sizes(r, tokens) for _ in range(seqs)]
         self.calls = max(len(c) for c in self.chunks)
         spb = 256 // ratio
@@ -554,10 +559,10 @@ class MixedStep:
     def __init__(self, device, seqs=128, c4a_layers=30, c128a_layers=31, k=512):
         from paged_compressed_kv_b200 import PagedPool, v4kv
         self.v4kv, self.k = v4kv, k
-        r = synth.rng(synth.seed_for(4))
+        r = synth.rng(synth.seed_for("mixed-61"))
         self.lens = synth.lengths_uniform(r, seqs, 1024, 262144, 4)
         self.B = seqs
-        g = synth.device_generator(synth.seed_for(4), device)
+        g = synth.device_generator(synth.seed_for("mixed-61"), device)
         self.max_len = int(self.lens.max())
         self.seq_lens = torch.from_numpy(self.lens.astype(np.int32)).to(device)
 
@@ -707,7 +712,7 @@ DTYPE = "f16"
 # build on the first 32 sequences of the workload (149.8 MB for 150.9 MB of
 # algorithmic bytes), scaled by the algorithmic bytes of the full workload; None
 # where no capture of the current kernel exists
-SWEEP_TRAFFIC = {1: 300.7e6}
+SWEEP_TRAFFIC = {"c4a-b64": 300.7e6}
 
 
 def main():
@@ -715,13 +720,14 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--workload", default="c4a-b64",
+                    choices=["c4a-b64", "c128a-b32", "tiny-c4a", "compressor", "mixed-61"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seqs", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0,
-                    help="config 4: c4a and c128a layers each (small cases for profiler captures)")
+                    help="mixed-61: c4a and c128a layers each (small cases for profiler captures)")
     ap.add_argument("--seqs", type=int, default=0,
                     help="keep only the first n sequences (small cases for profiler captures)")
     args = ap.parse_args()
@@ -737,8 +743,8 @@ def main():
         return
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    if args.config in (3, 4) and world == 1:
-        print(json.dumps(run_compress(args, device) if args.config == 3 else run_mixed(args, device)),
+    if args.workload in ("compressor", "mixed-61") and world == 1:
+        print(json.dumps(run_compress(args, device) if args.workload == "compressor" else run_mixed(args, device)),
               flush=True)
         return
     if world > 1:

@@ -17,9 +17,12 @@ import torch
 
 SEED_BASE = 20260000
 
+# one seed per named workload (fixed numbers, so stored inputs never change)
+WORKLOAD_SEEDS = {"tiny-c4a": 0, "c4a-b64": 1, "c128a-b32": 2, "compressor": 3, "mixed-61": 4}
 
-def seed_for(config_id):
-    return SEED_BASE + int(config_id)
+
+def seed_for(workload):
+    return SEED_BASE + WORKLOAD_SEEDS[workload]
 
 
 def rng(seed):
