@@ -953,6 +953,7 @@ __global__ void __launch_bounds__(256) decode_tc_merge_kernel(DecodeArgs a) {
 // qk0[b] = sm_scale * log2(e) * 2^-e. Block `batch` writes the tile prefix
 // sums cum[0..batch].
 __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
+  tc::pdl_wait();  // q and the lengths (written by earlier work in the stream) are complete
   tc::pdl_launch_dependents();
   const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   __shared__ float red[8];
@@ -1153,8 +1154,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  decode_tc_prep_kernel<<<a.batch + 1, 256, 0, stream>>>(a);
-  e = cudaGetLastError();
+  e = launch_pdl(decode_tc_prep_kernel, dim3(a.batch + 1), dim3(256), 0, stream, a);
   if (e != cudaSuccess) return e;
   e = launch_pdl(decode_tc_kernel, dim3(a.n_splits), dim3(kThreads), kSmemBytes, stream, a);
   if (e != cudaSuccess) return e;

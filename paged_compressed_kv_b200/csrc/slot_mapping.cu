@@ -2,6 +2,7 @@
 // (P1 §3.1.1: one 256-token logical block per page of each cache kind).
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace v4kv {
 
@@ -24,6 +25,8 @@ __global__ void slot_mapping_kernel(const int32_t* __restrict__ bt, int max_bloc
                                     int num_pages, int32_t* __restrict__ cu_out,
                                     int64_t* __restrict__ slot_out, long long cap,
                                     int32_t* __restrict__ st) {
+  tc::pdl_wait();  // the lengths and block tables (earlier work in the stream) are complete
+  tc::pdl_launch_dependents();
   const int b = blockIdx.x;
   long long part = 0;
   for (int i = threadIdx.x; i < b; i += blockDim.x) {
@@ -69,9 +72,8 @@ cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, int batch,
                                 const int32_t* seq_start, const int32_t* n_new, int ratio, int spb,
                                 int num_pages, int32_t* cu_out, int64_t* slot_out, long long cap,
                                 int32_t* st, cudaStream_t stream) {
-  slot_mapping_kernel<<<batch, 256, 0, stream>>>(bt, max_blocks, batch, seq_start, n_new, ratio,
-                                                 spb, num_pages, cu_out, slot_out, cap, st);
-  return cudaGetLastError();
+  return launch_pdl(slot_mapping_kernel, dim3(batch), dim3(256), 0, stream, bt, max_blocks, batch,
+                    seq_start, n_new, ratio, spb, num_pages, cu_out, slot_out, cap, st);
 }
 
 }  // namespace v4kv
