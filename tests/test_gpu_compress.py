@@ -55,8 +55,10 @@ class Appender:
         self.done = [0] * self.B
         self.prequant = [np.full((paging.entry_count(N, ratio), dim), np.nan, np.float32) for N in self.n]
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self._host = None
 
     def append(self, sizes):
+        self._host = None  # the pools change
         from paged_compressed_kv_b200 import v4kv
         dev = torch.device("cuda")
         sizes = [min(int(s), N - d) for s, N, d in zip(sizes, self.n, self.done)]
@@ -90,15 +92,25 @@ class Appender:
             self.done[b] += sizes[b]
         assert int(self.status.item()) == 0
 
+    def host_pools(self):
+        """Host copies of the pools, taken once after the last append."""
+        if self._host is None:
+            main = self.main.data.view(torch.int16) if self.main_dtype == "bf16" else self.main.data
+            win = self.win.data.view(torch.int16) if self.win_dtype == "bf16" else self.win.data
+            self._host = {
+                "main": main.cpu().numpy(),
+                "main_scales": self.main.scales.cpu().numpy() if self.main.scales is not None else None,
+                "win": win.cpu().numpy(),
+                "win_scales": self.win.scales.cpu().numpy() if self.win.scales is not None else None,
+            }
+        return self._host
+
     def entries(self, b):
         """Stored entries of sequence b: (codes or bf16 bits [n, D], scales or None)."""
         spb = 256 // self.ratio
         n = paging.entry_count(self.n[b], self.ratio)
-        data = self.main.data
-        if self.main_dtype == "bf16":
-            data = data.view(torch.int16)
-        data = data.cpu().numpy()
-        sc = self.main.scales.cpu().numpy() if self.main.scales is not None else None
+        h = self.host_pools()
+        data, sc = h["main"], h["main_scales"]
         rows = np.stack([data[self.bt[b, j // spb], j % spb] for j in range(n)]) if n else data[:0, 0]
         scs = np.array([sc[self.bt[b, j // spb], j % spb] for j in range(n)]) if sc is not None else None
         return rows, scs
@@ -110,12 +122,12 @@ class Appender:
         if not ts:
             return np.zeros((0, self.dim), np.float32)
         pages = [self.wbt[b, t // 256] for t in ts]
+        h = self.host_pools()
         if self.win_dtype == "fp8":
-            codes = self.win.data.cpu().numpy()
-            sc = self.win.scales.cpu().numpy()
+            codes, sc = h["win"], h["win_scales"]
             return np.stack([codecs.dequantize_entry(codes[p, t % 256][None], sc[p, t % 256])[0]
                              for p, t in zip(pages, ts)])
-        w = self.win.data.view(torch.int16).cpu().numpy().view(np.uint16)
+        w = h["win"].view(np.uint16)
         return codecs.bf16_to_f32(np.stack([w[p, t % 256] for p, t in zip(pages, ts)]))
 
 
