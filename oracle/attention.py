@@ -27,7 +27,10 @@ from .rope import rope_rotate
 
 def attend(q, values, sm_scale, seq_len, theta=1e6, rope_dim=64, rope_offset=448):
     """softmax(sm_scale q V^T) V for q [H, D], V [n, D], then inverse RoPE at
-    position seq_len - 1. fp64 [H, D]. An empty V gives zeros."""
+    position seq_len - 1. fp64 [H, D]. An empty V gives zeros.
+
+    Follows P1 §2.1 (shared K=V entries, inverse RoPE on the output).
+    """
     q = np.asarray(q, dtype=np.float64)
     v = np.asarray(values, dtype=np.float64)
     if v.shape[0] == 0:
@@ -45,6 +48,8 @@ def pool_values(data, scales, dtype, slots_per_page, page, slot):
 
     data: [num_pages, spb, D] uint8 codes (fp8) or uint16 bits (bf16);
     scales: [num_pages, spb] fp32 for fp8, None for bf16.
+
+    Follows P1 §3.1.1 and §3.1.3 (paged pools, bf16 or fp8 with a per-entry scale).
     """
     if dtype == "fp8":
         return codecs.e4m3_decode(data[page, slot]) * np.float64(scales[page, slot])
@@ -52,7 +57,10 @@ def pool_values(data, scales, dtype, slots_per_page, page, slot):
 
 
 def gather(data, scales, dtype, block_table_row, indices):
-    """Values of logical indices through one block-table row, fp64 [n, D]."""
+    """Values of logical indices through one block-table row, fp64 [n, D].
+
+    Follows P1 §3.1.1 (logical index through the block table).
+    """
     spb = data.shape[1]
     out = np.zeros((len(indices), data.shape[2]), dtype=np.float64)
     for i, j in enumerate(indices):
@@ -67,6 +75,8 @@ def decode_one(q, main, window, seq_len, ratio, window_len, sm_scale, topk_row=N
 
     main / window: dicts with keys data, scales, dtype, block_table_row.
     topk_row: optional int array of selected entry indices (-1 = none).
+
+    Follows P1 §2.1, §2.2, §2.3 and §4.1 (entries or the selected set, plus the window).
     """
     n_vis = max(0, seq_len - window_len) // ratio
     if topk_row is None:

@@ -20,7 +20,10 @@ E4M3_MAX = 448.0
 
 
 def f32(x):
-    """Cast to float32 (IEEE round-to-nearest-even)."""
+    """Cast to float32 (IEEE round-to-nearest-even).
+
+    Follows IEEE 754 binary32 rounding (the fp32 steps the pages leave to the implementation).
+    """
     return np.asarray(x, dtype=np.float32)
 
 
@@ -31,6 +34,8 @@ def bf16_bits(x):
 
     bf16 keeps the top 16 bits of the fp32 pattern; the discarded low half
     decides the rounding. NaN stays a (quiet) NaN.
+
+    Follows P1 §3.1.3 (bf16 cache storage); round to nearest even.
     """
     u = f32(x).view(np.uint32).astype(np.uint64)
     low = u & 0xFFFF
@@ -43,20 +48,29 @@ def bf16_bits(x):
 
 
 def bf16_to_f32(bits):
-    """bf16 bit pattern -> float32 (exact)."""
+    """bf16 bit pattern -> float32 (exact).
+
+    Follows P1 §3.1.3 (bf16 cache storage).
+    """
     b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
     return b.view(np.float32)
 
 
 def bf16_round(x):
-    """Round fp32 values to the nearest bf16 value, returned as float32."""
+    """Round fp32 values to the nearest bf16 value, returned as float32.
+
+    Follows P1 §3.1.3 (bf16 cache storage); round to nearest even.
+    """
     return bf16_to_f32(bf16_bits(x))
 
 
 # ---------------------------------------------------------------- e4m3
 
 def e4m3_decode(codes):
-    """fp8-e4m3 byte -> float64 value (exact). NaN for S.1111.111."""
+    """fp8-e4m3 byte -> float64 value (exact). NaN for S.1111.111.
+
+    Follows P1 §3.1.3 (fp8 cache) and the OCP FP8 E4M3 format.
+    """
     c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
     sign = np.where((c >> 7) == 1, -1.0, 1.0)
     e = (c >> 3) & 0xF
@@ -76,6 +90,8 @@ def e4m3_encode(x):
     The rounding is done on the exact fp64 value of the fp32 input: in the
     subnormal range the quantum is 2^-9; in binade [2^e, 2^(e+1)) it is
     2^(e-3).
+
+    Follows P1 §3.1.3 (fp8 cache) and the OCP FP8 E4M3 format.
     """
     x = f32(x)
     a = np.abs(x.astype(np.float64))
@@ -111,6 +127,8 @@ def quantize_entry(x):
     or 1 if amax == 0; code_d = e4m3(x_d / scale) with an IEEE division per
     element. Returns (codes uint8 [..., D], scale float32 [...]).
     Dequantised value of element d: float(code_d) * scale.
+
+    Follows P1 §2 and §3.1.3 (fp8 entries, one fp32 absmax scale each).
     """
     x = f32(x)
     amax = np.max(np.abs(x), axis=-1)
@@ -124,5 +142,7 @@ def dequantize_entry(codes, scale):
 
     Value of element d = e4m3_decode(code_d) * scale, formed exactly in fp64
     (a 4-bit-mantissa code times a 24-bit scale needs at most 28 bits).
+
+    Follows P1 §2 and §3.1.3 (fp8 entries, one fp32 absmax scale each).
     """
     return e4m3_decode(codes) * np.asarray(scale, dtype=np.float64)[..., None]

@@ -38,6 +38,8 @@ def group_weights(gates, bias):
 
     gates: [n] logits of the group's present tokens (n <= r);
     bias:  [r] position bias; token i of the group gets bias[i].
+
+    Follows P1 §2.1 (learned, position-biased weights within a group).
     """
     z = np.asarray(gates, dtype=np.float64) + np.asarray(bias, dtype=np.float64)[: len(gates)]
     z = z - z.max()
@@ -52,6 +54,8 @@ def compress_prequant(x, gates, bias, ratio, n_tokens=None, theta=1e6, rope_dim=
     x: raw tokens [N, D] (any float dtype; bf16 inputs are passed as their
     exact fp32 values); gates [N]; bias [r]. Only the first ``n_tokens`` tokens
     are used (default all).
+
+    Follows P1 §2.1 (c4a / c128a folding) and §3.1.2 (partial groups).
     """
     x = np.asarray(x, dtype=np.float64)
     gates = np.asarray(gates, dtype=np.float64)
@@ -72,6 +76,8 @@ def store_entries(prequant, dtype):
 
     dtype "fp8": (codes uint8 [G, D], scale fp32 [G]);
     dtype "bf16": (bits uint16 [G, D], None).
+
+    Follows P1 §2.1 and §3.1.3 (entries stored as fp8 or bf16).
     """
     if dtype == "fp8":
         return codecs.quantize_entry(prequant)
@@ -79,6 +85,9 @@ def store_entries(prequant, dtype):
 
 
 def window_tokens(x, positions, theta=1e6, rope_dim=64, rope_offset=448):
-    """Window copies: RoPE(x_t, t) in fp64, rounded to fp32 [n, D]."""
+    """Window copies: RoPE(x_t, t) in fp64, rounded to fp32 [n, D].
+
+    Follows P1 §2.3 (the last 128 raw tokens, uncompressed).
+    """
     return rope_rotate(np.asarray(x, dtype=np.float64), np.asarray(positions),
                        theta, rope_dim, rope_offset).astype(np.float32)

@@ -16,7 +16,10 @@ indexer keys, plus the raw-token window, plus the compressor state.
 """
 
 def layer_entries(n_tokens, ratio):
-    """Stored entries of one layer: ceil(N / r)."""
+    """Stored entries of one layer: ceil(N / r).
+
+    Follows P1 §2.1 and §2.2 (ceil(N/4) and ceil(N/128) entries per layer).
+    """
     return -(-int(n_tokens) // int(ratio))
 
 
@@ -29,6 +32,8 @@ def kv_bytes(n_tokens, layer_ratios, dim, entry_elem_bytes, entry_scale_bytes=0,
     indexer keys are kept for the c4a (ratio 4) layers only; ``window`` raw
     tokens per layer; with ``state_rows`` each layer also holds r raw tokens
     (and one fp32 gate each) of compressor state.
+
+    Follows P1 §2 (cache bytes per sequence).
     """
     total = 0.0
     for r in layer_ratios:
@@ -60,10 +65,14 @@ def page_claim_9_62():
 
 
 def saving_ratio():
-    """83.9 GiB (previous model) / 9.62 GiB, the page's "8.7x"."""
+    """83.9 GiB (previous model) / 9.62 GiB, the page's "8.7x".
+
+    Follows P1 §2.2 (the saving against the previous model).
+    """
     return 83.9 / 9.62
 
 
 def gib(nbytes):
+    """Follows P1 §2 (the page quotes sizes in GiB)."""
     return nbytes / float(1 << 30)
 

@@ -28,7 +28,10 @@ from . import codecs
 
 
 def index_scores(q_idx, key_codes, key_scales):
-    """Ranking scores (fp32 [n]) of n fp8 keys against one fp32 query."""
+    """Ranking scores (fp32 [n]) of n fp8 keys against one fp32 query.
+
+    Follows P1 §2.2 (indexer cache scores the c4a entries).
+    """
     q8, qs = codecs.quantize_entry(np.asarray(q_idx, dtype=np.float32))
     qv = codecs.e4m3_decode(q8).astype(np.float32)
     kv = codecs.e4m3_decode(np.asarray(key_codes)).astype(np.float32)
@@ -41,7 +44,10 @@ def index_scores(q_idx, key_codes, key_scales):
 
 def topk(scores, n_vis, k):
     """Indices of the min(k, n_vis) best scores among the first n_vis, by
-    (score descending, index ascending), padded with -1 to length k."""
+    (score descending, index ascending), padded with -1 to length k.
+
+    Follows P1 §2.2 and §4.1 (the selected entries of sparse c4a attention).
+    """
     s = np.asarray(scores[:n_vis], dtype=np.float64) + 0.0   # -0.0 -> +0.0
     idx = np.arange(n_vis)
     order = np.lexsort((idx, -s))          # last key is primary
@@ -52,7 +58,10 @@ def topk(scores, n_vis, k):
 
 
 def reported_scores(scores, qs, sel):
-    """Scores written beside the indices: score * qs in fp32, 0 for padding."""
+    """Scores written beside the indices: score * qs in fp32, 0 for padding.
+
+    Follows P1 §2.2 (indexer scores).
+    """
     out = np.zeros(len(sel), dtype=np.float32)
     valid = sel >= 0
     out[valid] = (np.asarray(scores, dtype=np.float32)[sel[valid]] * np.float32(qs)).astype(np.float32)

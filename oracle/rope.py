@@ -15,7 +15,10 @@ import numpy as np
 
 
 def rope_angles(pos, theta, rope_dim):
-    """Angles [..., rope_dim/2] for integer positions ``pos`` (fp64)."""
+    """Angles [..., rope_dim/2] for integer positions ``pos`` (fp64).
+
+    Follows P1 §2.1 (keys carry RoPE).
+    """
     i = np.arange(rope_dim // 2, dtype=np.float64)
     freq = np.power(np.float64(theta), -2.0 * i / rope_dim)
     return np.asarray(pos, dtype=np.float64)[..., None] * freq
@@ -27,6 +30,8 @@ def rope_rotate(x, pos, theta=1e6, rope_dim=64, rope_offset=448, inverse=False):
     ``pos`` broadcasts against x's leading axes. Pair (a, b) becomes
     (a cos - b sin, a sin + b cos). Dims outside the rope range are unchanged.
     Returns a new fp64 array.
+
+    Follows P1 §2.1 (RoPE on the keys, inverse RoPE on the output).
     """
     y = np.array(x, dtype=np.float64, copy=True)
     if rope_dim == 0:
