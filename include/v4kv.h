@@ -125,7 +125,9 @@ v4kv_status v4kv_slot_mapping(const int32_t* block_table, int32_t max_blocks, in
  * For every group g touched by the new tokens (see v4kv_slot_mapping), with
  * present tokens t in [g*r, min((g+1)*r, end)), end = seq_start + n_new:
  *     w_t = softmax_t(gate_t + pos_bias[t - g*r])     (fp32, expf)
- *     e   = sum_t w_t * x_t                          (fp32, ascending t)
+ *     e   = sum_t w_t * x_t                          (fp32; ratio 4: ascending t;
+ *                                                     ratio 128: 8 runs of 16 tokens,
+ *                                                     each ascending, added in order)
  *     e   = RoPE(e, position g*r)                    (angles in fp64)
  * then e is stored at slot_mapping[cu_entries[b] + (g - seq_start/r)]:
  * fp8 pools quantise per entry (amax, scale = amax/448 or 1 if amax == 0,
