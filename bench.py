@@ -8,17 +8,24 @@ v4kv_slot_mapping -> v4kv_compress_append (1 token each) ->
 v4kv_decode_attention (all visible entries + window). Inputs are synthetic
 (seeded device draws) and resident in HBM; L2 is flushed between steps.
 
+The default run (N = 1) also measures the other workloads and adds them to
+the same JSON line under "configs": the c128a decode (batch 32, context
+log-uniform [128K, 1M]), the compressor write path (8 x 32K tokens in random
+chunks, ratios 4 and 128) and the 61-layer mixed decode step (30 c4a layers
+with the indexer's top-512 + 31 c128a layers, batch 128, context U[1K, 256K]).
+Each sub-record carries its time, algorithmic bytes, GB/s, fraction of the
+HBM peak and the SM clocks sampled while it ran.
+
     python bench.py [--gpus N --steps K --warmup W] [--workload NAME]
 
-Workloads: c4a-b64 (default, above); c128a-b32 (c128a decode, batch 32,
-context log-uniform [128K, 1M]); tiny-c4a (1 sequence of 1024 tokens, 8 heads);
-compressor (the compressor write path alone); mixed-61 (a 61-layer mixed decode
-step with the indexer).
+Workloads: c4a-b64 (default, above); c128a-b32; tiny-c4a (1 sequence of 1024
+tokens, 8 heads); compressor; mixed-61.
     python bench.py --impl reference ...   # the CPU oracle on host cores
 
 Prints one JSON line (rank 0).
 """
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -38,6 +45,8 @@ METRIC = "decode-attention tokens/s and achieved HBM GB/s (% of B200 peak), fp8 
 D = 512
 W = 128
 HEADS = 64
+L2_BYTES = 126e6
+DTYPE = "f16"   # the tensor cores' operand type (fp8 codes convert to f16 exactly)
 
 
 def load_peaks():
@@ -46,6 +55,12 @@ def load_peaks():
         j = json.load(open(p))
         return float(j["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def l2_note(alg_bytes):
+    rel = "exceed" if alg_bytes > L2_BYTES else "are smaller than"
+    return (f"L2 flushed between steps (256 MB write); the step's algorithmic bytes "
+            f"({alg_bytes / 1e6:.0f} MB) {rel} L2 (126 MB)")
 
 
 # ------------------------------------------------------------------ workloads
@@ -75,57 +90,81 @@ def _decode_workload(name):
     raise ValueError(name)
 
 
+def decode_inputs(workload, device, seed_offset=0, seqs=0):
+    """Device-resident caches and per-step inputs of one decode workload, as
+    plain torch tensors (seeded draws only; nothing here calls the library)."""
+    c = decode_workload(workload, seqs)
+    lens = c["lens"].astype(np.int64)
+    ratio = c["ratio"]
+    H = c.get("heads", HEADS)
+    B = len(lens)
+    r = c["r"]
+    g = synth.device_generator(synth.seed_for(workload) + 7919 * seed_offset, device)
+    spb = 256 // ratio
+    n_ent = [-(-int(L) // ratio) for L in lens]
+    nblk = [-(-n // spb) for n in n_ent]
+    P = int(sum(nblk))
+    perm = synth.permutation(r, P)
+    bt = np.full((B, max(nblk)), -1, dtype=np.int32)
+    k = 0
+    for b, nb in enumerate(nblk):
+        bt[b, :nb] = perm[k:k + nb]
+        k += nb
+    data = torch.empty(P, spb, D, dtype=torch.uint8, device=device)
+    synth.fill_fp8_codes(data, g)
+    scales = torch.empty(P, spb, dtype=torch.float32, device=device)
+    synth.fill_uniform(scales, g, 0.5 / 112, 1.5 / 112)
+    # window: pages only for the blocks holding tokens [L - W, L)
+    wfirst = [max(0, int(L) - W) // 256 for L in lens]
+    wlast = [(int(L) - 1) // 256 for L in lens]
+    Pw = int(sum(l - f + 1 for f, l in zip(wfirst, wlast)))
+    wperm = synth.permutation(r, Pw)
+    wbt = np.full((B, max(wlast) + 1), -1, dtype=np.int32)
+    k = 0
+    for b in range(B):
+        for blk in range(wfirst[b], wlast[b] + 1):
+            wbt[b, blk] = wperm[k]
+            k += 1
+    wdata = torch.empty(Pw, 256, D, dtype=torch.bfloat16, device=device)
+    synth.fill_normal_bf16(wdata, g)
+    return dict(
+        name=c["name"], lens=lens, ratio=ratio, H=H, B=B, P=P,
+        data=data, scales=scales, bt=torch.from_numpy(bt).to(device),
+        wdata=wdata, wbt=torch.from_numpy(wbt).to(device),
+        # per-step inputs: the new token at position L - 1, then decode at L
+        q=torch.randn(B, H, D, generator=g, device=device),
+        x=torch.randn(B, D, generator=g, device=device).to(torch.bfloat16),
+        gate=torch.randn(B, generator=g, device=device),
+        bias=torch.randn(ratio, generator=g, device=device) * 0.5,
+        state_x=torch.randn(B, ratio, D, generator=g, device=device).to(torch.bfloat16),
+        state_g=torch.randn(B, ratio, generator=g, device=device),
+    )
+
+
+def decode_algorithmic_bytes(lens, ratio, H):
+    """KV, scales, window, q, output and block-table bytes one decode call must touch."""
+    tot = 0
+    for L in lens:
+        L = int(L)
+        n_vis = max(0, L - W) // ratio
+        tot += n_vis * (D + 4) + min(L, W) * D * 2 + H * D * 4 + H * D * 2
+        tot += 4 * (-(-L // 256))
+    return tot
+
+
 class DecodeStep:
-    """Device-resident caches and per-step inputs of one decode workload."""
+    """A decode workload wrapped for the library: pools, step buffers, workspace."""
 
     def __init__(self, workload, device, seed_offset=0, seqs=0):
         from paged_compressed_kv_b200 import PagedPool, v4kv
-        c = decode_workload(workload, seqs)
+        inp = decode_inputs(workload, device, seed_offset, seqs)
         self.v4kv = v4kv
-        self.name = c["name"]
-        self.lens = c["lens"].astype(np.int64)
-        self.ratio = c["ratio"]
-        self.H = c.get("heads", HEADS)
-        self.B = len(self.lens)
-        r = c["r"]
-        g = synth.device_generator(synth.seed_for(workload) + 7919 * seed_offset, device)
-        spb = 256 // self.ratio
-        n_ent = [-(-int(L) // self.ratio) for L in self.lens]
-        nblk = [-(-n // spb) for n in n_ent]
-        P = int(sum(nblk))
-        perm = synth.permutation(r, P)
-        bt = np.full((self.B, max(nblk)), -1, dtype=np.int32)
-        k = 0
-        for b, nb in enumerate(nblk):
-            bt[b, :nb] = perm[k:k + nb]
-            k += nb
-        self.P = P
-        data = torch.empty(P, spb, D, dtype=torch.uint8, device=device)
-        synth.fill_fp8_codes(data, g)
-        scales = torch.empty(P, spb, dtype=torch.float32, device=device)
-        synth.fill_uniform(scales, g, 0.5 / 112, 1.5 / 112)
-        self.main = PagedPool(data=data, block_table=torch.from_numpy(bt).to(device), scales=scales)
-        # window: pages only for the blocks holding tokens [L - W, L)
-        wfirst = [max(0, int(L) - W) // 256 for L in self.lens]
-        wlast = [(int(L) - 1) // 256 for L in self.lens]
-        Pw = int(sum(l - f + 1 for f, l in zip(wfirst, wlast)))
-        wperm = synth.permutation(r, Pw)
-        wbt = np.full((self.B, max(wlast) + 1), -1, dtype=np.int32)
-        k = 0
-        for b in range(self.B):
-            for blk in range(wfirst[b], wlast[b] + 1):
-                wbt[b, blk] = wperm[k]
-                k += 1
-        wdata = torch.empty(Pw, 256, D, dtype=torch.bfloat16, device=device)
-        synth.fill_normal_bf16(wdata, g)
-        self.win = PagedPool(data=wdata, block_table=torch.from_numpy(wbt).to(device))
-        # per-step inputs: the new token at position L - 1, then decode at L
-        self.q = torch.randn(self.B, self.H, D, generator=g, device=device)
-        self.x = torch.randn(self.B, D, generator=g, device=device).to(torch.bfloat16)
-        self.gate = torch.randn(self.B, generator=g, device=device)
-        self.bias = torch.randn(self.ratio, generator=g, device=device) * 0.5
-        self.state_x = torch.randn(self.B, self.ratio, D, generator=g, device=device).to(torch.bfloat16)
-        self.state_g = torch.randn(self.B, self.ratio, generator=g, device=device)
+        self.name, self.lens, self.ratio = inp["name"], inp["lens"], inp["ratio"]
+        self.H, self.B, self.P = inp["H"], inp["B"], inp["P"]
+        self.main = PagedPool(data=inp["data"], block_table=inp["bt"], scales=inp["scales"])
+        self.win = PagedPool(data=inp["wdata"], block_table=inp["wbt"])
+        self.q, self.x, self.gate, self.bias = inp["q"], inp["x"], inp["gate"], inp["bias"]
+        self.state_x, self.state_g = inp["state_x"], inp["state_g"]
         self.seq_start = torch.from_numpy((self.lens - 1).astype(np.int32)).to(device)
         self.n_new = torch.ones(self.B, dtype=torch.int32, device=device)
         self.cu_seqlens = torch.arange(self.B + 1, dtype=torch.int32, device=device)
@@ -160,14 +199,7 @@ class DecodeStep:
                                         dev_status=self.status, stream=stream)
 
     def algorithmic_bytes(self):
-        """KV, scales, window, q, output and block-table bytes one decode call must touch."""
-        tot = 0
-        for L in self.lens:
-            L = int(L)
-            n_vis = max(0, L - W) // self.ratio
-            tot += n_vis * (D + 4) + min(L, W) * D * 2 + self.H * D * 4 + self.H * D * 2
-            tot += 4 * (-(-L // 256))
-        return tot
+        return decode_algorithmic_bytes(self.lens, self.ratio, self.H)
 
     def h2d_bytes(self):
         return (self.q.numel() * 4 + self.x.numel() * 2 + self.gate.numel() * 4 +
@@ -180,20 +212,23 @@ class DecodeStep:
 # ------------------------------------------------------------------ helpers
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples while the timed region runs."""
+    """nvidia-smi clock / throttle samples (every 50 ms) while the benchmark
+    runs; summary(t0, t1) keeps the samples taken inside [t0, t1] (wall
+    clock, time.time()), widened to the nearest sample on each side."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.rows = []
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -201,35 +236,43 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
-
-    def summary(self):
-        sm, mx, reasons = [], 0.0, set()
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        for l in out.splitlines():
             f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = max(mx, float(f[2]))
-            except ValueError:
+                ts = time.mktime(time.strptime(f[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + f[0].split(".")[1]) if "." in f[0] else 0.0
+                sm, mx = float(f[2]), float(f[3])
+            except (ValueError, IndexError):
                 continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+            reasons = {n for n, v in zip(names, f[6:10]) if v.lower() == "active"}
+            self.rows.append((ts, sm, mx, reasons))
+
+    def summary(self, t0=None, t1=None):
+        rows = self.rows
+        if t0 is not None and rows:
+            inside = [x for x in rows if t0 <= x[0] <= t1]
+            before = [x for x in rows if x[0] < t0][-1:]
+            after = [x for x in rows if x[0] > t1][:1]
+            rows = before + inside + after
+        if not rows:
             return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set()
+        for x in rows:
+            reasons |= x[3]
+        return {"sm_mhz": float(np.median([x[1] for x in rows])),
+                "sm_max_mhz": max(x[2] for x in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
 
 
 def max_over_ranks(values, device, world):
@@ -251,7 +294,63 @@ def l2_flush(buf):
     buf.add_(1)
 
 
-def cores_used():
+def source_digest(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()[:16]
+
+
+SWEEP_SOURCES = ["paged_compressed_kv_b200/csrc/decode_tc.cu", "paged_compressed_kv_b200/csrc/tc.cuh"]
+
+
+def sweep_traffic(workload):
+    """DRAM bytes (read + write) of one sweep launch on this workload, from the
+    committed ncu summary (profiles/decode_tc_traffic.txt), only when that
+    capture was taken on the current sweep source; else None."""
+    p = os.path.join(ROOT, "profiles", "decode_tc_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    digest = source_digest(SWEEP_SOURCES)
+    for line in open(p):
+        f = line.split()
+        if len(f) >= 4 and f[0] == "traffic" and f[1] == workload and f[3] == digest:
+            return float(f[2])
+    return None
+
+
+# ------------------------------------------------------------------ the oracle on host cores
+
+SAMPLE_SEQS = 48   # fixed sample of whole sequences both CPU legs time
+
+
+def oracle_host_pools(inp):
+    """Host copies of one workload's caches (outside any timed region)."""
+    return dict(
+        main={"data": inp["data"].cpu().numpy(), "scales": inp["scales"].cpu().numpy(), "dtype": "fp8"},
+        win={"data": inp["wdata"].view(torch.int16).cpu().numpy().view(np.uint16), "scales": None,
+             "dtype": "bf16"},
+        bt=inp["bt"].cpu().numpy(), wbt=inp["wbt"].cpu().numpy(),
+        q=inp["q"].cpu().numpy().astype(np.float64), lens=inp["lens"], ratio=inp["ratio"])
+
+
+def oracle_sample_order(B):
+    """The sequences both CPU legs time, in order: a fixed seeded permutation."""
+    return np.random.default_rng(0).permutation(B)[:min(SAMPLE_SEQS, B)]
+
+
+def oracle_time(host, seqs):
+    """Run the oracle on the given sequences; (wall s, process CPU s)."""
+    from oracle import attention
+    w0, c0 = time.perf_counter(), time.process_time()
+    for b in seqs:
+        m = dict(host["main"], block_table_row=host["bt"][b])
+        w = dict(host["win"], block_table_row=host["wbt"][b])
+        attention.decode_one(host["q"][b], m, w, int(host["lens"][b]), host["ratio"], W, 1 / math.sqrt(D))
+    return time.perf_counter() - w0, time.process_time() - c0
+
+
+def threads_available():
     try:
         from threadpoolctl import threadpool_info
         n = [i.get("num_threads", 1) for i in threadpool_info()]
@@ -260,37 +359,44 @@ def cores_used():
         return os.cpu_count() or 1
 
 
-def oracle_sample(step, seconds=10.0, max_seqs=None):
-    """Time the CPU oracle on whole sequences of the workload (rank 0 only).
-
-    The caches are copied to the host once (outside the timed region); the
-    oracle then gathers each sample sequence's pages and runs the fp64
-    attention. Returns (sequences per second, sequences timed, seconds)."""
-    from oracle import attention
-    main = {"data": step.main.data.cpu().numpy(), "scales": step.main.scales.cpu().numpy(),
-            "dtype": "fp8"}
-    win = {"data": step.win.data.view(torch.int16).cpu().numpy().view(np.uint16), "scales": None,
-           "dtype": "bf16"}
-    bt = step.main.block_table.cpu().numpy()
-    wbt = step.win.block_table.cpu().numpy()
-    q = step.q.cpu().numpy().astype(np.float64)
-    order = np.random.default_rng(0).permutation(step.B)
-    done, t0 = 0, time.perf_counter()
-    for b in order:
-        m = dict(main, block_table_row=bt[b])
-        w = dict(win, block_table_row=wbt[b])
-        attention.decode_one(q[b], m, w, int(step.lens[b]), step.ratio, W, 1 / math.sqrt(D))
-        done += 1
-        el = time.perf_counter() - t0
-        if el >= seconds or (max_seqs and done >= max_seqs):
-            break
-    el = time.perf_counter() - t0
-    return done / el, done, el
+def cpu_baseline(inp):
+    """The oracle as it stands on the host cores: the fixed sample once with the
+    BLAS threads it has, and its first 8 sequences again on one thread."""
+    host = oracle_host_pools(inp)
+    order = oracle_sample_order(inp["B"])
+    wall, cpu = oracle_time(host, order)
+    one = None
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            w1, _ = oracle_time(host, order[:8])
+        one = 8 / w1
+    except Exception:
+        pass
+    return {"value": len(order) / wall, "unit": "tokens/s", "cores": round(cpu / wall, 2),
+            "kind": "oracle", "threads_available": threads_available(),
+            "value_1thread": one,
+            "sample": f"{len(order)} whole sequences of the same workload (fixed seeded choice; fp64 "
+                      f"numpy oracle, pages gathered on the host), {wall:.1f} s wall; 'cores' = "
+                      f"process CPU time / wall time; value_1thread = its first 8 sequences with "
+                      f"BLAS limited to one thread"}
 
 
 # ------------------------------------------------------------------ arms
 
-def run_ours(args, rank, world, device):
+def time_events(fn, steps, flush, stream):
+    """Median ms of fn() over `steps` runs, L2 flushed between runs."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        ev[i][0].record(stream)
+        fn()
+        ev[i][1].record(stream)
+        l2_flush(flush)
+    torch.cuda.synchronize()
+    return float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+
+def run_ours(args, rank, world, device, clk):
     peak, peak_kind = load_peaks()
     step = DecodeStep(args.workload, device, seed_offset=rank, seqs=args.seqs)
     stream = torch.cuda.current_stream()
@@ -307,22 +413,23 @@ def run_ours(args, rank, world, device):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(device.index) as clk:
-        for i in range(args.steps):
-            s0, s1, s2 = ev[i]
-            s0.record(stream)
-            step.append()
-            s1.record(stream)
-            step.decode()
-            s2.record(stream)
-            l2_flush(flush)
-        torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        s0, s1, s2 = ev[i]
+        s0.record(stream)
+        step.append()
+        s1.record(stream)
+        step.decode()
+        s2.record(stream)
+        l2_flush(flush)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
     if world > 1:
         torch.distributed.barrier()
     step_ms = [a.elapsed_time(c) for a, _, c in ev]
     dec_ms = [b.elapsed_time(c) for _, b, c in ev]
-    t_step = float(np.sum(step_ms)) / args.steps
-    t_dec = float(np.mean(dec_ms))
+    t_step = float(np.median(step_ms))
+    t_dec = float(np.median(dec_ms))
     t_step, t_dec = max_over_ranks([t_step, t_dec], device, world)
 
     # end to end through the public API with host buffers (pinned), copies timed
@@ -352,7 +459,7 @@ def run_ours(args, rank, world, device):
             e2e_ev[i - args.warmup][1].record(stream)
         l2_flush(flush)
     torch.cuda.synchronize()
-    t_e2e = float(np.mean([a.elapsed_time(b) for a, b in e2e_ev]))
+    t_e2e = float(np.median([a.elapsed_time(b) for a, b in e2e_ev]))
     (t_e2e,) = max_over_ranks([t_e2e], device, world)
     if step.status.item() != 0:
         raise RuntimeError(f"device status {step.status.item()}")
@@ -375,61 +482,70 @@ def run_ours(args, rank, world, device):
         "data": "synthetic (seeded device draws: fp8 codes, fp32 scales, bf16 window, fp32 q)",
         "config": {"workload": step.name, "batch": step.B, "heads": step.H, "dim": D,
                    "ratio": step.ratio, "window": W, "parallelism": f"replicas x{world}",
-                   "l2": "flushed between steps (256 MB write), inputs also exceed L2",
-                   "decode_ms": t_dec, "hbm_gbs": achieved},
+                   "l2": l2_note(alg), "decode_ms": t_dec, "hbm_gbs": achieved,
+                   "timing": f"median of {args.steps} steps (CUDA events)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": SWEEP_TRAFFIC.get(args.workload) if not args.seqs else None,
+                     "frac": achieved / peak,
+                     "traffic": sweep_traffic(args.workload) if not args.seqs else None,
                      "kernel": "v4kv_decode_attention (query prep + sweep + merge)",
                      "algorithmic_bytes": alg, "peak_source": peak_kind},
         "e2e": {"value": rate_e2e, "unit": "tokens/s",
                 "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": step.d2h_bytes()},
         "gpu_launches": step.launches_per_step() * args.steps,
     }
-    clocks = clk.summary()
-    if clocks is not None:
-        line["clocks"] = clocks
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, n, el = oracle_sample(step, seconds=args.cpu_seconds)
-        line["cpu_baseline"] = {"value": rate * 1.0, "unit": "tokens/s", "cores": cores_used(),
-                                "kind": "oracle",
-                                "sample": f"{n} whole sequences of the same workload (fp64 numpy "
-                                          f"oracle, pages gathered on the host), {el:.1f} s"}
-    return line
+    line["_window"] = (t_wall0, t_wall1)
+    return line, step
 
 
 def run_reference(args, rank, world):
-    """The oracle as the reference arm: each step times a bounded sample."""
+    """The oracle as the reference arm: each step times a bounded sample of the
+    same fixed sequence sample the cpu_baseline leg times. Inputs are the same
+    seeded device draws as the library's arm; the library itself is not loaded."""
     if rank != 0:
         return None
     torch.set_grad_enabled(False)
-    dev = torch.device("cuda", 0) if torch.cuda.is_available() else None
-    if dev is None:
-        return {"impl": "reference", "unavailable": "needs the workload's caches on a CUDA device"}
-    step = DecodeStep(args.workload, dev, seqs=args.seqs)
+    if not torch.cuda.is_available():
+        return {"impl": "reference", "unavailable": "needs a CUDA device to draw the workload's caches"}
+    dev = torch.device("cuda", 0)
+    inp = decode_inputs(args.workload, dev, seqs=args.seqs)
+    host = oracle_host_pools(inp)
+    del inp["data"], inp["wdata"]
+    order = oracle_sample_order(inp["B"])
     per = max(1, int(args.ref_seqs))
+    cur = 0
+
+    def next_seqs():
+        nonlocal cur
+        s = [order[(cur + i) % len(order)] for i in range(per)]
+        cur += per
+        return s
+
     for _ in range(args.warmup):
-        oracle_sample(step, seconds=1e9, max_seqs=1)
-    rates = []
-    t_all = 0.0
+        oracle_time(host, next_seqs()[:1])
+    cur = 0
+    walls, cpus = [], []
     for _ in range(args.steps):
-        rate, n, el = oracle_sample(step, seconds=1e9, max_seqs=per)
-        rates.append(rate)
-        t_all += el
-    value = float(np.mean(rates))
+        w, c = oracle_time(host, next_seqs())
+        walls.append(w)
+        cpus.append(c)
+    value = per * args.steps / float(np.sum(walls))
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * t_all / args.steps, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": 1e3 * float(np.median(walls)), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded device draws)",
-        "config": {"workload": step.name, "batch": step.B, "heads": step.H, "dim": D,
-                   "ratio": step.ratio, "window": W, "parallelism": "cpu oracle, rank 0"},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
-                         "sample": f"{per} whole sequences per step"},
+        "config": {"workload": inp["name"], "batch": inp["B"], "heads": inp["H"], "dim": D,
+                   "ratio": inp["ratio"], "window": W, "parallelism": "cpu oracle, rank 0"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s",
+                         "cores": round(float(np.sum(cpus)) / float(np.sum(walls)), 2),
+                         "threads_available": threads_available(), "kind": "oracle",
+                         "sample": f"{per} whole sequences per step, cycling through the fixed "
+                                   f"{len(order)}-sequence sample the cpu_baseline leg times"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
-# ------------------------------------------------------------------ other rows (compressor, mixed-61)
+# ------------------------------------------------------------------ other workloads
 
 class CompressStep:
     """Compressor write path: 8 sequences x 32K raw bf16 tokens appended in
@@ -475,6 +591,7 @@ class CompressStep:
             cap = int(sum(sizes)) // ratio + 2 * seqs
             self.call_inputs.append(dict(x=self.x[rows].contiguous(), gate=self.gate[rows].contiguous(),
                                          cu=cu, ss=ss, nn=nn, n=int(sum(sizes)),
+                                         starts=np.array(done), sizes=np.array(sizes),
                                          slots=torch.empty(cap, dtype=torch.int64, device=device),
                                          cue=torch.empty(seqs + 1, dtype=torch.int32, device=device)))
             for b in range(seqs):
@@ -492,14 +609,13 @@ class CompressStep:
     def algorithmic_bytes(self, c):
         ci = self.call_inputs[c]
         n = ci["n"]
-        sizes = ci["nn"].cpu().numpy()
-        starts = ci["ss"].cpu().numpy()
-        touched = sum((-(-(s0 + m) // self.ratio)) - s0 // self.ratio for s0, m in zip(starts, sizes) if m)
-        win = sum(min(int(m), W) for m in sizes)
+        touched = sum((-(-(int(s0) + int(m)) // self.ratio)) - int(s0) // self.ratio
+                      for s0, m in zip(ci["starts"], ci["sizes"]) if m)
+        win = sum(min(int(m), W) for m in ci["sizes"])
         return n * (D * 2 + 4) + touched * (D + 4) + win * D * 2 + self.B * self.ratio * (D * 2 + 4)
 
 
-def run_compress(args, device):
+def run_compress(args, device, clk):
     peak, _ = load_peaks()
     out = {}
     for ratio in (4, 128):
@@ -527,7 +643,9 @@ def run_compress(args, device):
         for _ in range(3):
             graph.replay()
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
-        reps, ms_g = 5, []
+        reps, ms_g = max(5, args.steps), []
+        torch.cuda.synchronize()
+        t0 = time.time()
         for _ in range(reps):
             flush.fill_(1)  # inputs of one pass (~300 MB) exceed L2 anyway
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -536,17 +654,22 @@ def run_compress(args, device):
             e1.record()
             torch.cuda.synchronize()
             ms_g.append(e0.elapsed_time(e1))
+        t1 = time.time()
         del graph
         ms = float(np.median(ms_g))
         byts = sum(st.algorithmic_bytes(c) for c in range(st.calls))
         out[f"r{ratio}"] = {"calls": st.calls, "tokens": st.B * st.N, "ms": ms,
+                            "algorithmic_bytes": byts,
                             "tokens_per_s": st.B * st.N / (ms * 1e-3),
                             "gbs": byts / (ms * 1e-3) / 1e9, "frac": byts / (ms * 1e-3) / 1e9 / peak,
                             "ms_eager": ms_eager,
                             "gbs_eager": byts / (ms_eager * 1e-3) / 1e9,
-                            "status": int(st.status.item())}
+                            "status": int(st.status.item()),
+                            "launches": 2 * st.calls, "_window": (t0, t1)}
+        del st
+        torch.cuda.empty_cache()
     return {"config": "compressor write path, 8 x 32K raw bf16 tokens, random chunks 1..4096, fp8 "
-                      "entries, shuffled pages; ms = one CUDA-graph replay of all calls (median of 5), "
+                      "entries, shuffled pages; ms = one CUDA-graph replay of all calls (median), "
                       "ms_eager = the calls launched one by one from Python", "results": out}
 
 
@@ -566,7 +689,7 @@ class MixedStep:
         self.max_len = int(self.lens.max())
         self.seq_lens = torch.from_numpy(self.lens.astype(np.int32)).to(device)
 
-        def pool(ratio, dim, dtype_fp8=True):
+        def pool(ratio, dim):
             spb = 256 // ratio
             nblk = [-(-(-(-int(L) // ratio)) // spb) for L in self.lens]
             P = int(sum(nblk))
@@ -641,14 +764,14 @@ class MixedStep:
         return idx, att4, att128
 
 
-def run_mixed(args, device):
+def run_mixed(args, device, clk, layers=0, seqs=0):
     peak, _ = load_peaks()
     kw = {}
-    if args.seqs:
-        kw["seqs"] = args.seqs
-    if args.layers:
-        kw["c4a_layers"] = min(30, args.layers)
-        kw["c128a_layers"] = min(31, args.layers)
+    if seqs:
+        kw["seqs"] = seqs
+    if layers:
+        kw["c4a_layers"] = min(30, layers)
+        kw["c128a_layers"] = min(31, layers)
     st = MixedStep(device, **kw)
     nl4, nl128 = len(st.c4a), len(st.c128a)
 
@@ -677,11 +800,13 @@ def run_mixed(args, device):
             with torch.cuda.graph(graphs[name], stream=side):
                 fn()
     torch.cuda.synchronize()
-    tot = {}
+    tot, win = {}, {}
     for name, gr in graphs.items():
         gr.replay()
         gr.replay()
         ms = []
+        torch.cuda.synchronize()
+        t0 = time.time()
         for _ in range(args.steps):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
@@ -689,30 +814,68 @@ def run_mixed(args, device):
             e1.record()
             torch.cuda.synchronize()
             ms.append(e0.elapsed_time(e1))
+        win[name] = (t0, time.time())
         tot[name] = float(np.median(ms))
     graphs.clear()
     idx_b, a4_b, a128_b = st.bytes()
     step_ms = tot["step"]
-    res = {"step_ms": step_ms, "parts_ms_sum": tot["idx"] + tot["att4"] + tot["att128"], "tokens_per_s": st.B / (step_ms * 1e-3),
-           "indexer": {"ms_per_layer": tot["idx"] / nl4, "gbs": idx_b / (tot["idx"] / nl4 * 1e-3) / 1e9},
-           "c4a_attention": {"ms_per_layer": tot["att4"] / nl4, "gbs": a4_b / (tot["att4"] / nl4 * 1e-3) / 1e9},
-           "c128a_attention": {"ms_per_layer": tot["att128"] / nl128, "gbs": a128_b / (tot["att128"] / nl128 * 1e-3) / 1e9},
-           "step_gbs": (nl4 * (idx_b + a4_b) + nl128 * a128_b) / (step_ms * 1e-3) / 1e9,
-           "status": int(st.status.item())}
+
+    def rec(ms_layer, byts, key):
+        gbs = byts / (ms_layer * 1e-3) / 1e9
+        return {"ms_per_layer": ms_layer, "algorithmic_bytes_per_layer": byts, "gbs": gbs,
+                "frac": gbs / peak, "clocks": clk.summary(*win[key]) if clk else None}
+
+    step_bytes = nl4 * (idx_b + a4_b) + nl128 * a128_b
+    res = {"step_ms": step_ms, "parts_ms_sum": tot["idx"] + tot["att4"] + tot["att128"],
+           "tokens_per_s": st.B / (step_ms * 1e-3), "algorithmic_bytes": step_bytes,
+           "indexer": rec(tot["idx"] / nl4, idx_b, "idx"),
+           "c4a_attention": rec(tot["att4"] / nl4, a4_b, "att4"),
+           "c128a_attention": rec(tot["att128"] / nl128, a128_b, "att128"),
+           "step_gbs": step_bytes / (step_ms * 1e-3) / 1e9,
+           "status": int(st.status.item()), "_window": win["step"]}
     res["step_frac"] = res["step_gbs"] / peak
     name = (f"{nl4 + nl128}-layer mixed step ({nl4} c4a with indexer top-512 + {nl128} c128a), "
             f"batch {st.B}, context U[1K, 256K], 64 heads, fp8 KV; CUDA-graph replays, median of "
             f"{args.steps}")
+    del st
+    torch.cuda.empty_cache()
     return {"config": name, "results": res}
 
 
-DTYPE = "f16"
+def run_decode_only(args, device, workload, clk):
+    """Decode call alone (v4kv_decode_attention) on one workload: median of
+    `steps` calls with L2 flushed between them."""
+    peak, _ = load_peaks()
+    step = DecodeStep(workload, device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        step.decode()
+        l2_flush(flush)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    ms = time_events(step.decode, max(args.steps, 20), flush, stream)
+    t1 = time.time()
+    alg = step.algorithmic_bytes()
+    gbs = alg / (ms * 1e-3) / 1e9
+    st = int(step.status.item())
+    res = {"workload": step.name, "decode_ms": ms, "tokens_per_s": step.B / (ms * 1e-3),
+           "algorithmic_bytes": alg, "gbs": gbs, "frac": gbs / peak, "l2": l2_note(alg),
+           "traffic": sweep_traffic(workload), "status": st, "clocks": clk.summary(t0, t1)}
+    del step
+    torch.cuda.empty_cache()
+    return res
 
-# DRAM bytes (read + write) of one sweep launch, from an ncu capture of the same
-# build on the first 32 sequences of the workload (149.8 MB for 150.9 MB of
-# algorithmic bytes), scaled by the algorithmic bytes of the full workload; None
-# where no capture of the current kernel exists
-SWEEP_TRAFFIC = {"c4a-b64": 300.7e6}
+
+def finish_clocks(d, clk):
+    """Replace the wall-clock windows recorded in a result tree by clock summaries."""
+    if isinstance(d, dict):
+        if "_window" in d:
+            w = d.pop("_window")
+            if "clocks" not in d:
+                d["clocks"] = clk.summary(*w)
+        for v in d.values():
+            finish_clocks(v, clk)
 
 
 def main():
@@ -723,9 +886,10 @@ def main():
     ap.add_argument("--workload", default="c4a-b64",
                     choices=["c4a-b64", "c128a-b32", "tiny-c4a", "compressor", "mixed-61"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seqs", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads' sub-records (headline line only)")
     ap.add_argument("--layers", type=int, default=0,
                     help="mixed-61: c4a and c128a layers each (small cases for profiler captures)")
     ap.add_argument("--seqs", type=int, default=0,
@@ -744,15 +908,37 @@ def main():
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     if args.workload in ("compressor", "mixed-61") and world == 1:
-        print(json.dumps(run_compress(args, device) if args.workload == "compressor" else run_mixed(args, device)),
-              flush=True)
+        with ClockSampler(device.index) as clk:
+            res = (run_compress(args, device, clk) if args.workload == "compressor"
+                   else run_mixed(args, device, clk, args.layers, args.seqs))
+        finish_clocks(res, clk)
+        print(json.dumps(res), flush=True)
         return
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     try:
-        line = run_ours(args, rank, world, device)
+        with ClockSampler(device.index) as clk:
+            line, step = run_ours(args, rank, world, device, clk)
+            extra = None
+            if rank == 0 and world == 1 and not args.no_configs and not args.seqs \
+                    and args.workload == "c4a-b64":
+                del step
+                torch.cuda.empty_cache()
+                extra = {
+                    "c128a-b32": run_decode_only(args, device, "c128a-b32", clk),
+                    "compressor": run_compress(args, device, clk),
+                    "mixed-61": run_mixed(args, device, clk),
+                }
+        line["clocks"] = clk.summary(*line.pop("_window"))
+        if extra is not None:
+            finish_clocks(extra, clk)
+            line["configs"] = extra
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            inp = decode_inputs(args.workload, device, seqs=args.seqs)
+            line["cpu_baseline"] = cpu_baseline(inp)
+            del inp
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

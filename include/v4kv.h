@@ -51,6 +51,8 @@ typedef int32_t v4kv_status;
 #define V4KV_DEV_BAD_INDEX 4 /* top-k index outside the stored entries     */
 #define V4KV_DEV_OVERFLOW 8  /* output array too small for what is needed  */
 #define V4KV_DEV_TIMEOUT 16  /* a wait inside a kernel gave up (no progress) */
+#define V4KV_DEV_RANGE 32    /* a bf16 value beyond the f16 range met the     */
+                             /* 64-head tensor-core path and was clamped      */
 
 typedef enum { V4KV_BF16 = 0, V4KV_FP8_E4M3 = 1, V4KV_FP32 = 2 } v4kv_dtype;
 
@@ -203,7 +205,13 @@ v4kv_status v4kv_index_topk(const float* q_idx, const v4kv_paged* idx_cache,
  *     s_hj = sm_scale * q_h . v_j,  p = softmax_j(s),  o_h = sum_j p_hj v_j
  *     out  = inverse RoPE of o at position L - 1, rounded to bf16.
  * Numerics: q and p enter the tensor cores as f16 (q scaled per sequence by a
- * power of two), fp8 values convert exactly, accumulation is fp32.
+ * power of two), fp8 values convert exactly, accumulation is fp32. With 64
+ * heads (the tensor-core path) bf16 entries and window tokens are rounded to
+ * f16 as well: magnitudes of 2^16 or more are clamped to 65504 and flagged
+ * V4KV_DEV_RANGE; magnitudes below 2^-14 keep an absolute error of at most
+ * 2^-25. Other head counts use bf16 values exactly. Any fp8 scale is valid,
+ * including zero (the entry's value is 0) and negative scales.
+ *   sm_scale     softmax scale; 0 selects the default 1/sqrt(512)
  *   q            device [batch, heads, dim], fp32 or bf16 (q_dtype), with RoPE
  *                already applied at position L - 1
  *   heads        1 .. 128; dim (of q, main_cache and window) must be 512

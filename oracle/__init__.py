@@ -27,6 +27,6 @@ footprint   KV-cache bytes per sequence
 
 Pins: every function is checked in ``tests/test_oracle_*.py`` against facts the
 pages or mathematics fix (closed forms, library routines, invariants, brute
-force); nothing there compares the oracle with itself. The one function with no
-such pin is ``footprint.page_claim_9_62`` (see its docstring): parity unpinned.
+force, hand-derived worked examples under ``tests/golden/``); nothing there
+compares the oracle with itself.
 """

@@ -8,7 +8,9 @@ P1 §2 computes the cache of one 1,000,000-token sequence on the 61-layer model
 shared 5,120-element bf16 vector (10,240 bytes) per entry that is about
 2.38 GiB per c4a layer and 0.075 GiB per c128a layer, 73.73 GiB in bf16 as the
 page rounds it. It then states 9.62 GiB for fp8 entries with an fp4 indexer and
-compares with 83.9 GiB for the previous model (an "8.7x" saving).
+compares with 83.9 GiB for the previous model (an "8.7x" saving). The 9.62
+comes from a division by an unexplained 7.66 that no formula on the page
+produces, so it is not restated here; the tests only note it.
 
 ``kv_bytes`` is the general formula: per layer, ceil(N / r) entries of
 (dim * bytes per element + scale bytes), plus for c4a layers ceil(N / 4)
@@ -53,15 +55,6 @@ def page_bf16_breakdown():
     c4a = layer_entries(1_000_000, 4) * 5120 * 2 / gib
     c128a = layer_entries(1_000_000, 128) * 5120 * 2 / gib
     return c4a, 30 * c4a, c128a, 31 * c128a, 30 * c4a + 31 * c128a
-
-
-def page_claim_9_62():
-    """P1 §2's 9.62 GiB: the page divides its bf16 total by an unexplained 7.66.
-
-    Parity unpinned: no formula on the page produces 7.66 (fp8 alone halves
-    the entry bytes), so this only restates the page's own division.
-    """
-    return 73.73 / 7.66
 
 
 def saving_ratio():

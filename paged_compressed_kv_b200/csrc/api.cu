@@ -219,28 +219,51 @@ v4kv_status v4kv_workspace_size(int32_t op, int32_t batch, int32_t heads, int32_
   return V4KV_OK;
 }
 
-v4kv_status v4kv_decode_attention(const void* q, int32_t q_dtype, int32_t batch, int32_t heads,
-                                  const v4kv_paged* main_cache, const v4kv_paged* window,
-                                  const int32_t* seq_lens, int32_t max_seq_len, int32_t ratio,
-                                  int32_t window_len, const int32_t* topk, int32_t k,
-                                  float sm_scale, v4kv_rope rope, void* out, void* workspace,
-                                  size_t workspace_bytes, int32_t* dev_status, void* stream) {
+}  // extern "C"
+
+namespace v4kv {
+
+// Host-side argument checks of decode attention (everything but the
+// workspace), shared by both decode entry points so that they report the
+// same status for the same bad argument.
+v4kv_status decode_check_args(const void* q, int32_t q_dtype, int32_t batch, int32_t heads,
+                              const v4kv_paged* main_cache, const v4kv_paged* window,
+                              const int32_t* seq_lens, int32_t max_seq_len, int32_t ratio,
+                              int32_t window_len, const int32_t* topk, int32_t k, float sm_scale,
+                              v4kv_rope rope, const void* out) {
   if (!q || !seq_lens || !out || batch <= 0 || max_seq_len < 0 || window_len < 0)
     return V4KV_ERR_INVALID_ARG;
   if (q_dtype != V4KV_FP32 && q_dtype != V4KV_BF16) return V4KV_ERR_INVALID_ARG;
   if (heads < 1 || heads > 128) return V4KV_ERR_UNSUPPORTED;
   if (ratio != 4 && ratio != 128) return V4KV_ERR_INVALID_ARG;
   if (topk && (k < 1 || k > 2048)) return V4KV_ERR_INVALID_ARG;
-  if (!topk) k = 0;
   if (!main_cache || !window) return V4KV_ERR_INVALID_ARG;
   if (main_cache->dim != 512 || window->dim != 512) return V4KV_ERR_UNSUPPORTED;
   if (!pool_ok(main_cache, kBlock / ratio, 512, true, true)) return V4KV_ERR_INVALID_ARG;
   if (!pool_ok(window, kBlock, 512, true, true)) return V4KV_ERR_INVALID_ARG;
   if (!rope_ok(rope, 512)) return V4KV_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out)) return V4KV_ERR_INVALID_ARG;
-  if (!(sm_scale > 0.f) || !isfinite(sm_scale)) return V4KV_ERR_INVALID_ARG;
+  if (sm_scale != 0.f && (!(sm_scale > 0.f) || !isfinite(sm_scale))) return V4KV_ERR_INVALID_ARG;
+  return check_device(nullptr);
+}
+
+}  // namespace v4kv
+
+extern "C" {
+
+v4kv_status v4kv_decode_attention(const void* q, int32_t q_dtype, int32_t batch, int32_t heads,
+                                  const v4kv_paged* main_cache, const v4kv_paged* window,
+                                  const int32_t* seq_lens, int32_t max_seq_len, int32_t ratio,
+                                  int32_t window_len, const int32_t* topk, int32_t k,
+                                  float sm_scale, v4kv_rope rope, void* out, void* workspace,
+                                  size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  v4kv_status st = decode_check_args(q, q_dtype, batch, heads, main_cache, window, seq_lens,
+                                     max_seq_len, ratio, window_len, topk, k, sm_scale, rope, out);
+  if (st != V4KV_OK) return st;
+  if (!topk) k = 0;
+  if (sm_scale == 0.f) sm_scale = 1.f / sqrtf(512.f);  // the default scale 1/sqrt(dim)
   int sms = 0;
-  v4kv_status st = check_device(&sms);
+  st = check_device(&sms);
   if (st != V4KV_OK) return st;
   const DecodePlan plan =
       plan_decode(batch, heads, max_seq_len, ratio, window_len, k, main_cache->dtype, 512, sms);

@@ -49,8 +49,8 @@ constexpr uint32_t kVOff = 0;                    // 8 dim atoms x 128 rows x 128
 constexpr uint32_t kQOff = 131072;               // 8 dim atoms x 64 rows x 128 B
 constexpr uint32_t kPOff = 196608;               // 128 rows x 128 B (64 heads f16)
 constexpr int kRing = 6;        // tiles of row addresses the address warp keeps ready
-constexpr uint32_t kMetaOff = 212992;                 // [kRing][128] fp32 item scales (0 = skip)
-constexpr uint32_t kPtrOff = kMetaOff + kRing * 512;  // [kRing][128] item row addresses
+constexpr uint32_t kMetaOff = 212992;                 // [kRing][128] fp32 item scales
+constexpr uint32_t kPtrOff = kMetaOff + kRing * 512;  // [kRing][128] item row addresses (null = skip)
 constexpr uint32_t kMrefOff = kPtrOff + kRing * 1024;  // [64] reference max per head
 constexpr uint32_t kAlphaOff = kMrefOff + 256;   // [64] rescale factors
 constexpr uint32_t kRedOff = kAlphaOff + 256;    // [8][32] per-warp reductions
@@ -254,12 +254,15 @@ __device__ __forceinline__ void fp8x16_to_f16(uint4 raw, uint4& lo, uint4& hi) {
   hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// 8 bf16 -> 8 f16 (round to nearest, saturating to the f16 range)
-__device__ __forceinline__ uint4 bf16x8_to_f16(uint4 raw) {
+// 8 bf16 -> 8 f16 (round to nearest, saturating to the f16 range). `wide`
+// is set when a value's magnitude is 2^16 or more (or not finite): such a
+// value does not fit the f16 operands of the tensor cores and is clamped.
+__device__ __forceinline__ uint4 bf16x8_to_f16(uint4 raw, bool& wide) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
+    wide |= (w[i] & 0x7fffu) >= 0x4780u || ((w[i] >> 16) & 0x7fffu) >= 0x4780u;
     const float a = __uint_as_float(w[i] << 16), b = __uint_as_float(w[i] & 0xffff0000u);
     uint32_t r;
     asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
@@ -552,6 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
     }
     float k0 = a.qk0[b0];
     int q_issued = 1;  // query copies started by this thread (tid 0 only)
+    bool wide = false; // a bf16 value outside the f16 range was clamped
     bool ok = true;
 
     // fp8 rows: lane covers rows 16w + 4r + lane/8 (r = 0..3), 16 bytes at
@@ -620,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
           for (int r = 0; r < 8; ++r) {
             const uint32_t vr = 16 * warp + 2 * r + (lane >> 4);
             *reinterpret_cast<uint4*>(sm + kVOff + atom * 16384 + tc::sw128_off(vr, part & 7)) =
-                bf16x8_to_f16(V4KV_RB(c & 1, r));
+                bf16x8_to_f16(V4KV_RB(c & 1, r), wide);
           }
           tc::fence_proxy_async_smem();
           tc::mbar_arrive(&bars->v_full[c]);
@@ -657,11 +661,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       ok = named_and(1, 256, ok);
       if (!ok) break;
       tc::tc_fence_after();
+      // a row is an item when its address was resolved; its scale may be any
+      // value (value = code * scale): |scale| enters the exponent, its sign the
+      // weight P', and a zero scale gives a zero-valued item that still counts
+      // in the normaliser with score 0
+      const bool valid = rowptr[(i % kRing) * kT + row] != nullptr;
       const float ks = meta[(i % kRing) * kT + row];
-      const bool valid = ks > 0.f;
+      const float aks = fabsf(ks);
       const float cj = valid ? k0 * ks : 0.f;
-      const float lk = valid ? __log2f(ks) : -INFINITY;
-      const float inv_k = valid ? __frcp_rn(ks) : 0.f;
+      const float lk = !valid ? -INFINITY : (aks > 0.f ? __log2f(aks) : 0.f);
+      const float inv_k = !valid ? 0.f : (aks > 0.f ? __frcp_rn(aks) : 1.f);
+      const float sgn = (valid && ks != 0.f) ? copysignf(1.f, ks) : 0.f;
       // u = score in log2 units including log2 ks; d = u - m_ref (in place)
       float d[32];
       const uint32_t s_addr = lane_base + (uint32_t)(i & 1) * kH + 32 * hh;
@@ -763,7 +773,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
           const int h = 8 * c + 2 * e;
           d[h] = fast_exp2(d[h]);
           d[h + 1] = fast_exp2(d[h + 1]);
-          pk[e] = h2u(__floats2half2_rn(d[h], d[h + 1]));
+          pk[e] = h2u(__floats2half2_rn(sgn * d[h], sgn * d[h + 1]));
         }
         *reinterpret_cast<uint4*>(sm + kPOff + tc::sw128_off(row, 4 * hh + c)) =
             make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -852,6 +862,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       *abort_flag = 1;
       flag(a.dev_status, V4KV_DEV_TIMEOUT);
     }
+    if (__any_sync(0xffffffffu, wide) && lane == 0) flag(a.dev_status, V4KV_DEV_RANGE);
     if (tid == 0) {
       // the last query copy has landed before shared memory is released
       // (normally long since; after an abort it may still be in flight)

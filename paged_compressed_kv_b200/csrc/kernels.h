@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/v4kv.h"
+
 namespace v4kv {
 
 struct PoolArgs {
@@ -128,6 +130,14 @@ cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);  // sweep + merge
 size_t decode_tc_workspace_bytes(int batch, int num_sms);
 void decode_tc_layout(DecodeArgs& a, void* workspace);  // needs batch, n_splits
+
+// Host-side argument checks of decode attention, without the workspace
+// (api.cu); V4KV_OK when the call may proceed.
+v4kv_status decode_check_args(const void* q, int32_t q_dtype, int32_t batch, int32_t heads,
+                              const v4kv_paged* main_cache, const v4kv_paged* window,
+                              const int32_t* seq_lens, int32_t max_seq_len, int32_t ratio,
+                              int32_t window_len, const int32_t* topk, int32_t k, float sm_scale,
+                              v4kv_rope rope, const void* out);
 
 // Tensor map over `rows` rows of `row_bytes` bytes (uint8, 2-D, 128-byte
 // swizzle), boxes of `row_bytes` x `box_rows`. base must be 16-byte aligned.

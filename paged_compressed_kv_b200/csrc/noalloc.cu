@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/v4kv.h"
+#include "kernels.h"
 
 namespace {
 
@@ -46,10 +47,14 @@ extern "C" v4kv_status v4kv_decode_attention_noalloc(
     const v4kv_paged* window, const int32_t* seq_lens, int32_t max_seq_len, int32_t ratio,
     int32_t window_len, const int32_t* topk, int32_t k, float sm_scale, v4kv_rope rope, void* out,
     int32_t* dev_status, void* stream) {
-  if (!main_cache) return V4KV_ERR_INVALID_ARG;
+  // the same argument checks (and statuses) as v4kv_decode_attention first
+  v4kv_status st = v4kv::decode_check_args(q, q_dtype, batch, heads, main_cache, window, seq_lens,
+                                           max_seq_len, ratio, window_len, topk, k, sm_scale,
+                                           rope, out);
+  if (st != V4KV_OK) return st;
   size_t need = 0;
-  v4kv_status st = v4kv_workspace_size(V4KV_OP_DECODE, batch, heads, max_seq_len, ratio,
-                                       window_len, topk ? k : 0, main_cache->dtype, 512, &need);
+  st = v4kv_workspace_size(V4KV_OP_DECODE, batch, heads, max_seq_len, ratio, window_len,
+                           topk ? k : 0, main_cache->dtype, 512, &need);
   if (st != V4KV_OK) return st;
   if (need > (size_t)V4KV_NOALLOC_SCRATCH_BYTES) return V4KV_ERR_INVALID_ARG;
   void* scratch = nullptr;

@@ -6,7 +6,6 @@ same name in ``libv4kv.so``. No computation happens in Python and there is no
 fallback: if the shared library is missing, importing this module raises.
 """
 import ctypes
-import math
 import os
 from dataclasses import dataclass
 from typing import Optional
@@ -24,6 +23,8 @@ V4KV_DEV_BAD_PAGE = 1
 V4KV_DEV_BAD_SLOT = 2
 V4KV_DEV_BAD_INDEX = 4
 V4KV_DEV_OVERFLOW = 8
+V4KV_DEV_TIMEOUT = 16
+V4KV_DEV_RANGE = 32
 V4KV_BF16 = 0
 V4KV_FP8_E4M3 = 1
 V4KV_FP32 = 2
@@ -240,7 +241,7 @@ def v4kv_decode_attention(q, main, window, seq_lens, max_seq_len, ratio, window_
         _need(topk, (torch.int32,), "topk", ndim=2)
     rope = rope or Rope()
     if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(q.shape[2])
+        sm_scale = 0.0  # the library's default, 1/sqrt(512)
     mc, wc = main.c(), window.c()
     st = _lib.v4kv_decode_attention(
         q.data_ptr(), V4KV_FP32 if q.dtype == torch.float32 else V4KV_BF16, q.shape[0], q.shape[1],
@@ -265,7 +266,7 @@ def v4kv_decode_attention_noalloc(q, main, window, seq_lens, max_seq_len, ratio,
         _need(topk, (torch.int32,), "topk", ndim=2)
     rope = rope or Rope()
     if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(q.shape[2])
+        sm_scale = 0.0  # the library's default, 1/sqrt(512)
     mc, wc = main.c(), window.c()
     st = _lib.v4kv_decode_attention_noalloc(
         q.data_ptr(), V4KV_FP32 if q.dtype == torch.float32 else V4KV_BF16, q.shape[0], q.shape[1],

@@ -91,3 +91,54 @@ def test_footprint_matches_oracle(n):
     # the page's bf16 configuration
     got = v4kv.v4kv_kv_footprint_bytes(n, layers, 5120, 16)
     assert got == footprint.kv_bytes(n, layers, 5120, 2)
+
+
+def test_noalloc_reports_the_same_status_as_the_workspace_entry_point():
+    # both decode entry points run the same host-side argument checks, so a bad
+    # argument gets the same status from either (no device is needed to see it)
+    from paged_compressed_kv_b200 import v4kv
+    lib = v4kv._lib
+    fake = 0x10000
+    pool = v4kv._Paged(0x10000, 0x20000, 4, 64, 512, 1, 0x30000, 4)
+    win = v4kv._Paged(0x40000, None, 4, 256, 512, 0, 0x50000, 4)
+    narrow = v4kv._Paged(0x10000, 0x20000, 4, 64, 256, 1, 0x30000, 4)
+    rope = v4kv._Rope(1e6, 64, 448)
+    cases = [
+        dict(heads=129),                      # unsupported head count
+        dict(heads=0),
+        dict(ratio=3),                        # not 4 or 128
+        dict(q=0x10001),                      # misaligned query
+        dict(q=None),
+        dict(q_dtype=7),
+        dict(main=narrow),                    # dim 256: unsupported
+        dict(topk=fake, k=4096),              # k above 2048
+        dict(sm_scale=-1.0),
+        dict(batch=0),
+    ]
+    for c in cases:
+        a = dict(q=fake, q_dtype=2, batch=1, heads=8, main=pool, ratio=4, topk=None, k=0,
+                 sm_scale=0.04)
+        a.update(c)
+        ws = lib.v4kv_decode_attention(a["q"], a["q_dtype"], a["batch"], a["heads"],
+                                       ctypes.byref(a["main"]), ctypes.byref(win), fake, 1024,
+                                       a["ratio"], 128, a["topk"], a["k"], a["sm_scale"], rope, fake,
+                                       fake, 1 << 20, None, None)
+        na = lib.v4kv_decode_attention_noalloc(a["q"], a["q_dtype"], a["batch"], a["heads"],
+                                               ctypes.byref(a["main"]), ctypes.byref(win), fake,
+                                               1024, a["ratio"], 128, a["topk"], a["k"],
+                                               a["sm_scale"], rope, fake, None, None)
+        assert ws == na, (c, ws, na)
+        assert ws in (v4kv.V4KV_ERR_INVALID_ARG, v4kv.V4KV_ERR_UNSUPPORTED), (c, ws)
+
+
+def test_library_footprint_against_the_hand_worked_two_layer_model():
+    from paged_compressed_kv_b200 import v4kv
+    for line in open(os.path.join(ROOT, "tests", "golden", "footprint_worked.txt")):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        key, n, state, want = line.split()
+        if int(state):
+            continue  # the library's footprint has no compressor-state term
+        got = v4kv.v4kv_kv_footprint_bytes(int(n), [4, 128], 512, 8, 4, 128, 8, 4, 128, 16)
+        assert got == int(want), key

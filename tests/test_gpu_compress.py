@@ -18,7 +18,7 @@ class Appender:
     """Runs appends of per-sequence chunks through the library."""
 
     def __init__(self, seed, n_tokens, ratio, main_dtype="fp8", W=128, gates=None, dim=D,
-                 rope=True, win_dtype="bf16"):
+                 rope=True, win_dtype="bf16", x=None, bias=None):
         from paged_compressed_kv_b200 import PagedPool, Rope
         self.r = synth.rng(seed)
         self.n = [int(v) for v in n_tokens]
@@ -28,8 +28,12 @@ class Appender:
         self.rope = Rope(rope_offset=dim - 64) if rope else Rope(rope_dim=0)
         self.x = [synth.normal(self.r, (N, dim)) for N in self.n]
         self.x = [codecs.bf16_round(v) for v in self.x]             # exact bf16 values
+        if x is not None:
+            self.x = [codecs.bf16_round(np.asarray(v, dtype=np.float32)) for v in x]
         self.g = gates if gates is not None else [synth.normal(self.r, N) for N in self.n]
         self.bias = synth.normal(self.r, ratio, 0.5)
+        if bias is not None:
+            self.bias = np.asarray(bias, dtype=np.float32)
         spb = 256 // ratio
         nblk = [-(-paging.entry_count(N, ratio) // spb) for N in self.n]
         self.bt, self.P = paging.allocate_block_tables(nblk, synth.permutation(self.r, sum(nblk) + 2))
@@ -290,3 +294,78 @@ def test_slot_mapping_flags_bad_pages_and_overflow():
     v4kv.v4kv_slot_mapping(bt, ss, nn, 4, 3, small, None, dev_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) & 8
+
+
+# Crafted quantiser inputs (scale 1 when amax = 448, so each quotient is the
+# value itself). Expected e4m3 codes are worked by hand from the OCP FP8 E4M3
+# definition (bias 7, 3 mantissa bits, subnormal quantum 2^-9, largest 448):
+#   448 -> 0x7E; 1.0625 (midway 1.0 | 1.125) -> 1.0 = 0x38 (even mantissa);
+#   1.1875 (midway 1.125 | 1.25) -> 1.25 = 0x3A; 1.0703125 -> 1.125 = 0x39;
+#   -1.0625 -> 0xB8; 2^-8 -> 2 * 2^-9 = 0x02; 3 * 2^-10 (midway 1 | 2 quanta)
+#   -> 0x02; 2^-10 (midway 0 | 1 quantum) -> 0x00; -2^-11 -> -0 = 0x80;
+#   2^-9 -> 0x01; 5 * 2^-10 (midway 2 | 3 quanta) -> 0x02; 240 = 1.875 * 2^7
+#   -> 0x77; 232 (midway 224 | 240) -> 224 = 0x76; -0.0 -> 0x80 (or 0x00 when the
+#   fp32 group sum has returned +0, see below).
+CRAFTED = [(448.0, 0x7E), (1.0625, 0x38), (1.1875, 0x3A), (1.0703125, 0x39), (-1.0625, 0xB8),
+           (2.0 ** -8, 0x02), (3 * 2.0 ** -10, 0x02), (2.0 ** -10, 0x00), (-(2.0 ** -11), 0x80),
+           (2.0 ** -9, 0x01), (5 * 2.0 ** -10, 0x02), (240.0, 0x77), (232.0, 0x76)]
+
+
+def test_quantiser_edge_cases_through_the_compressor():
+    # one-hot gates (the group's first token has logit 0, the others -1e30),
+    # zero position bias and no RoPE make every entry exactly its group's first
+    # token, so the quantiser sees chosen values: e4m3 ties to even, subnormal
+    # quotients, -0 and negative underflow, an all-zero entry (scale 1), an
+    # entry whose fp32 scale is itself subnormal (amax 2^-120), and a scale that
+    # is not a power of two
+    r = synth.rng(460)
+    n_groups = 6
+    N = 4 * n_groups
+    x = np.zeros((N, D), dtype=np.float32)
+    e0 = synth.normal(r, D, 8.0)
+    for i, (v, _) in enumerate(CRAFTED):
+        e0[i] = v
+    e0[len(CRAFTED)] = -0.0
+    e0[len(CRAFTED) + 1:] = np.clip(e0[len(CRAFTED) + 1:], -447.0, 447.0)
+    x[0] = e0                                           # entry 0: amax 448, scale 1
+    # entry 1 stays all zero
+    x[8] = synth.normal(r, D, 30.0)                     # entry 2: a general scale
+    x[8, 7] = 100.0
+    x[12] = np.where(r.random(D) < 0.5, -1.0, 1.0) * 2.0 ** -120 * r.integers(1, 5, D)  # entry 3
+    x[16] = -np.abs(synth.normal(r, D, 1e-3))           # entry 4: all negative, small,
+    x[16, :8] = -1e-12 * np.arange(1, 9)                # eight of them far below the quantum
+    x[20] = synth.normal(r, D, 1.0)                     # entry 5
+    x[20, 3] = -0.0
+    gates = np.full(N, -1e30, dtype=np.float32)
+    gates[::4] = 0.0
+    ap = Appender(461, [N], 4, "fp8", gates=[gates], rope=False, x=[x], bias=np.zeros(4))
+    ap.append([N])
+    tok = codecs.bf16_round(x[::4])                     # the exact token values
+    pre = ap.prequant[0]
+    assert np.array_equal(pre, tok)                     # -0 == +0 here
+    rows, scs = ap.entries(0)
+    # bytes and scales: bit-exact against the oracle's quantiser on the
+    # kernel's own pre-quant values ...
+    codes, sc = codecs.quantize_entry(pre)
+    assert np.array_equal(rows, codes)
+    assert np.array_equal(scs.view(np.uint32), sc.view(np.uint32))
+    # ... and on the chosen tokens, except that a -0 token may reach the
+    # quantiser as +0 (the fp32 group sum starts from +0)
+    codes_t, sc_t = codecs.quantize_entry(tok)
+    negzero = (tok == 0) & np.signbit(tok)
+    assert np.array_equal(rows[~negzero], codes_t[~negzero])
+    assert np.all(np.isin(rows[negzero], [0x00, 0x80]))
+    assert np.array_equal(scs.view(np.uint32), sc_t.view(np.uint32))
+    # the hand-worked codes of entry 0 (scale exactly 1)
+    assert scs[0] == 1.0
+    for i, (_, want) in enumerate(CRAFTED):
+        assert rows[0, i] == want, (i, CRAFTED[i], hex(rows[0, i]))
+    # the all-zero entry: scale 1, every code 0
+    assert scs[1] == 1.0 and np.all(rows[1] == 0)
+    # the tiny entry's scale is an fp32 subnormal, computed as amax / 448
+    assert 0 < scs[3] < np.finfo(np.float32).tiny
+    # negative underflow keeps the sign: 0x80, never 0x00, in the all-negative entry
+    q4 = (x[16] / scs[4]).astype(np.float32)
+    under = np.abs(q4) < 2.0 ** -10
+    assert under.sum() >= 8
+    assert np.all(rows[4][under] == 0x80)

@@ -181,3 +181,40 @@ def test_fp8_window(heads):
     got, st = run_decode(case)
     assert st == 0
     check_all(case, got)
+
+
+@pytest.mark.parametrize("heads", [8, 64])
+def test_zero_and_negative_scale_entries(heads):
+    # value = code * scale for any scale: a zero scale is a zero-valued entry
+    # that still takes part in the softmax (score 0), a negative scale flips
+    # the entry's sign; both head-count paths must agree with the oracle
+    case = DecodeCase(214, [3000, 9000], heads, 4)
+    r = synth.rng(215)
+    sc = case.main.scales
+    used = np.unique(case.main.bt[case.main.bt >= 0])
+    for p in used[:: 3]:
+        rows = r.choice(sc.shape[1], 8, replace=False)
+        sc[p, rows[:4]] = 0.0
+        sc[p, rows[4:]] = -sc[p, rows[4:]]
+    got, st = run_decode(case)
+    assert st == 0
+    check_all(case, got)
+
+
+def test_bf16_beyond_f16_range_is_flagged_on_the_tensor_core_path():
+    # 64 heads convert bf16 window tokens to f16: a magnitude of 2^16 or more
+    # cannot be represented there, so it is clamped and flagged
+    # (V4KV_DEV_RANGE = 32); other head counts use the bf16 value exactly
+    from oracle import codecs
+    for heads in (8, 64):
+        case = DecodeCase(216, [2000], heads, 4)
+        L = 2000
+        page = case.win.bt[0, (L - 3) // 256]
+        row = case.win.data[page, (L - 3) % 256]
+        row[:4] = codecs.bf16_bits(np.array([1e5, -7e4, 3e4, 65536.0], dtype=np.float32))
+        got, st = run_decode(case)
+        if heads == 64:
+            assert st & 32
+        else:
+            assert st == 0
+            check_all(case, got)
