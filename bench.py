@@ -823,7 +823,7 @@ def run_mixed(args, device, clk, layers=0, seqs=0):
     def rec(ms_layer, byts, key):
         gbs = byts / (ms_layer * 1e-3) / 1e9
         return {"ms_per_layer": ms_layer, "algorithmic_bytes_per_layer": byts, "gbs": gbs,
-                "frac": gbs / peak, "clocks": clk.summary(*win[key]) if clk else None}
+                "frac": gbs / peak, "_window": win[key]}
 
     step_bytes = nl4 * (idx_b + a4_b) + nl128 * a128_b
     res = {"step_ms": step_ms, "parts_ms_sum": tot["idx"] + tot["att4"] + tot["att128"],
@@ -861,7 +861,7 @@ def run_decode_only(args, device, workload, clk):
     st = int(step.status.item())
     res = {"workload": step.name, "decode_ms": ms, "tokens_per_s": step.B / (ms * 1e-3),
            "algorithmic_bytes": alg, "gbs": gbs, "frac": gbs / peak, "l2": l2_note(alg),
-           "traffic": sweep_traffic(workload), "status": st, "clocks": clk.summary(t0, t1)}
+           "traffic": sweep_traffic(workload), "status": st, "_window": (t0, t1)}
     del step
     torch.cuda.empty_cache()
     return res

@@ -54,13 +54,15 @@ typedef int32_t v4kv_status;
 #define V4KV_DEV_RANGE 32    /* a bf16 value beyond the f16 range met the     */
                              /* 64-head tensor-core path and was clamped      */
 
-typedef enum { V4KV_BF16 = 0, V4KV_FP8_E4M3 = 1, V4KV_FP32 = 2 } v4kv_dtype;
+typedef enum { V4KV_BF16 = 0, V4KV_FP8_E4M3 = 1, V4KV_FP32 = 2, V4KV_FP4_E2M1 = 3 } v4kv_dtype;
 
 /* One paged pool of one cache kind (P1 §3.1.1, §3.1.3).
  *   data   device, [num_pages, slots_per_page, dim] elements of `dtype`
- *          (fp8-e4m3 codes or bf16); one page = one 256-token logical block.
+ *          (fp8-e4m3 codes or bf16; for fp4-e2m1, accepted by the indexer
+ *          only, dim / 2 bytes per slot, dim 2i in the low nibble of byte i);
+ *          one page = one 256-token logical block.
  *   scales device, [num_pages, slots_per_page] fp32, one absmax scale per
- *          fp8 entry (value = float(code) * scale); NULL for bf16.
+ *          fp8 or fp4 entry (value = float(code) * scale); NULL for bf16.
  *   block_table device, [batch, max_blocks] int32: logical block -> page;
  *          -1 marks a block that has no page (skipped on write, an error on
  *          read). Logical index j of a sequence lives in page
@@ -181,7 +183,10 @@ v4kv_status v4kv_compress_append(const void* x, const float* gate, const int32_t
  * -0 == +0) are written to topk_out[b] in that order, padded with -1;
  * score_out (optional) receives score_j * qs (0 for padding).
  *   q_idx        device fp32 [batch, dim]
- *   idx_cache    fp8 indexer pool, slots_per_page = 256 / ratio, dim 128
+ *   idx_cache    fp8 or fp4 indexer pool, slots_per_page = 256 / ratio,
+ *                dim a multiple of 32 in [32, 512] (fp4: P1 §2 keeps the c4a
+ *                indexer in fp4; each product of an e4m3 query value and an
+ *                e2m1 key value is exact, so the chain is the same)
  *   seq_lens     device int32 [batch], L of each sequence (tokens so far)
  *   max_seq_len  host upper bound of seq_lens (sizes the launch)
  *   k            1 .. 2048
@@ -229,6 +234,30 @@ v4kv_status v4kv_decode_attention(const void* q, int32_t q_dtype, int32_t batch,
                                   int32_t window_len, const int32_t* topk, int32_t k,
                                   float sm_scale, v4kv_rope rope, void* out, void* workspace,
                                   size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * v4kv_decode_attention_fp8out -- v4kv_decode_attention with the output
+ * quantised to fp8-e4m3 in the same epilogue as the inverse RoPE (P1 §3.2.1:
+ * inverse RoPE fused with fp8 quantisation, for a next layer that reads fp8).
+ * Each (sequence, head) vector o (fp32, after the inverse RoPE) is quantised
+ * like a cache entry: amax = max_d |o_d|, scale = amax / 448 (IEEE fp32
+ * division; 1 if amax == 0), code_d = e4m3_rn_satfinite(o_d / scale).
+ *   out_codes    device uint8 [batch, heads, 512]
+ *   out_scales   device fp32 [batch, heads]
+ *   prequant_out device fp32 [batch, heads, 512] or NULL: the fp32 values
+ *                handed to the quantiser
+ * Every other argument, the workspace (same size) and the errors are those of
+ * v4kv_decode_attention.
+ */
+v4kv_status v4kv_decode_attention_fp8out(const void* q, int32_t q_dtype, int32_t batch,
+                                         int32_t heads, const v4kv_paged* main_cache,
+                                         const v4kv_paged* window, const int32_t* seq_lens,
+                                         int32_t max_seq_len, int32_t ratio, int32_t window_len,
+                                         const int32_t* topk, int32_t k, float sm_scale,
+                                         v4kv_rope rope, void* out_codes, float* out_scales,
+                                         float* prequant_out, void* workspace,
+                                         size_t workspace_bytes, int32_t* dev_status,
+                                         void* stream);
 
 /*
  * v4kv_decode_attention_noalloc -- v4kv_decode_attention for callers that

@@ -92,3 +92,16 @@ def decode_one(q, main, window, seq_len, ratio, window_len, sm_scale, topk_row=N
         parts.append(gather(window["data"], window["scales"], window["dtype"], window["block_table_row"], wins))
     v = np.concatenate(parts, axis=0) if parts else np.zeros((0, q.shape[1]))
     return attend(q, v, sm_scale, seq_len, theta, rope_dim, rope_offset)
+
+
+def output_fp8(o):
+    """The attention output quantised to fp8-e4m3 per (sequence, head) vector.
+
+    P1 §3.2.1 fuses the output's inverse RoPE with its fp8 quantisation (the
+    next layer reads fp8). The pages fix neither the grouping nor the scale;
+    this follows the cache entries' rule (codecs.quantize_entry) on each
+    head's 512-vector: the fp64 output (after the inverse RoPE) is rounded to
+    fp32, then amax, scale = amax / 448 (1 if amax == 0) and e4m3 codes of the
+    per-element quotients. Returns (codes uint8 [..., D], scale fp32 [...]).
+    """
+    return codecs.quantize_entry(np.asarray(o, dtype=np.float32))

@@ -146,3 +146,89 @@ def dequantize_entry(codes, scale):
     Follows P1 §2 and §3.1.3 (fp8 entries, one fp32 absmax scale each).
     """
     return e4m3_decode(codes) * np.asarray(scale, dtype=np.float64)[..., None]
+
+
+# ---------------------------------------------------------------- e2m1 (fp4)
+# OCP MX FP4 E2M1: 1 sign bit, 2 exponent bits (bias 1), 1 mantissa bit, no
+# infinities or NaN. Code magnitudes 0..7: 0, 0.5 (subnormal), 1, 1.5, 2, 3,
+# 4, 6; the sign is bit 3. P1 §2 stores the c4a indexer keys in fp4 for its
+# 9.62 GiB figure; the pages fix nothing else, so the keys are quantised like
+# the fp8 entries: one fp32 absmax scale per key, scale = amax / 6.
+
+E2M1_MAX = 6.0
+E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def e2m1_decode(codes):
+    """fp4-e2m1 code (low 4 bits) -> float64 value (exact).
+
+    Follows P1 §2 (fp4 indexer) and the OCP MX FP4 E2M1 format.
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64) & 0xF
+    e = (c >> 1) & 0x3
+    m = c & 0x1
+    mag = np.where(e == 0, 0.5 * m, (1.0 + 0.5 * m) * np.exp2((e - 1).astype(np.float64)))
+    return np.where((c >> 3) == 1, -mag, mag)
+
+
+def e2m1_encode(x):
+    """float32 -> fp4-e2m1 code: round to nearest, ties to even, saturate to
+    +-6; the sign bit is kept for zero results (-0 and negative underflow ->
+    0x8). The rounding works on the exact value of the fp32 input: the
+    representable magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6, and at a tie the
+    code with the even mantissa bit (0, 1, 2, 4 and 0.5's neighbour 1) wins.
+
+    Follows P1 §2 (fp4 indexer) and the OCP MX FP4 E2M1 format.
+    """
+    x = f32(x).astype(np.float64)
+    a = np.abs(x)
+    neg = np.signbit(x)
+    # index of the largest representable magnitude <= a, and the next one up
+    lo = np.searchsorted(E2M1_VALUES, a, side="right") - 1
+    lo = np.clip(lo, 0, 7)
+    hi = np.minimum(lo + 1, 7)
+    vlo, vhi = E2M1_VALUES[lo], E2M1_VALUES[hi]
+    up = (a - vlo) > (vhi - a)
+    tie = (a - vlo) == (vhi - a)
+    up = up | (tie & ((lo & 1) == 1))      # ties go to the even code (mantissa bit 0)
+    mag = np.where(up & (hi != lo), hi, lo)
+    mag = np.where(a >= E2M1_MAX, 7, mag)
+    return (np.where(neg, mag | 0x8, mag)).astype(np.uint8)
+
+
+def quantize_entry_fp4(x):
+    """Per-key absmax fp4 quantisation of fp32 vectors (last axis = one key).
+
+    amax = max |x_d| (fp32); scale = amax / 6 (IEEE fp32 division), 1 if
+    amax == 0; code_d = e2m1(x_d / scale) with an IEEE division per element.
+    Returns (codes uint8 [..., D], one code per byte, and scale fp32 [...]).
+
+    Follows P1 §2 (fp4 indexer keys with a per-key scale, read like the fp8 entries).
+    """
+    x = f32(x)
+    amax = np.max(np.abs(x), axis=-1)
+    scale = np.where(amax == 0, np.float32(1.0), amax / np.float32(E2M1_MAX)).astype(np.float32)
+    quot = (x / scale[..., None]).astype(np.float32)
+    return e2m1_encode(quot), scale
+
+
+def pack_fp4(codes):
+    """Two fp4 codes per byte: dim 2i in the low nibble, dim 2i + 1 in the high
+    nibble ([..., D] -> [..., D/2] uint8).
+
+    Follows the storage layout of the fp4 indexer pool (one byte per two dims).
+    """
+    c = np.asarray(codes, dtype=np.uint8)
+    return (c[..., 0::2] & 0xF) | ((c[..., 1::2] & 0xF) << 4)
+
+
+def unpack_fp4(packed):
+    """Inverse of pack_fp4: [..., D/2] bytes -> [..., D] codes.
+
+    Follows the storage layout of the fp4 indexer pool (one byte per two dims).
+    """
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out

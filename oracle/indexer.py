@@ -27,14 +27,20 @@ import numpy as np
 from . import codecs
 
 
-def index_scores(q_idx, key_codes, key_scales):
-    """Ranking scores (fp32 [n]) of n fp8 keys against one fp32 query.
+def index_scores(q_idx, key_codes, key_scales, key_format="fp8"):
+    """Ranking scores (fp32 [n]) of n keys against one fp32 query.
+
+    key_codes [n, D]: one code per element, fp8-e4m3 (key_format "fp8") or
+    fp4-e2m1 (key_format "fp4": P1 §2 keeps the c4a indexer in fp4 for its
+    9.62 GiB figure). Each product of an e4m3 query value and an e4m3 or e2m1
+    key value is exact in fp32, so the chain is the same in both formats.
 
     Follows P1 §2.2 (indexer cache scores the c4a entries).
     """
     q8, qs = codecs.quantize_entry(np.asarray(q_idx, dtype=np.float32))
     qv = codecs.e4m3_decode(q8).astype(np.float32)
-    kv = codecs.e4m3_decode(np.asarray(key_codes)).astype(np.float32)
+    dec = codecs.e2m1_decode if key_format == "fp4" else codecs.e4m3_decode
+    kv = dec(np.asarray(key_codes)).astype(np.float32)
     acc = np.zeros(kv.shape[0], dtype=np.float32)
     for d in range(kv.shape[1]):
         acc = (acc + qv[d] * kv[:, d]).astype(np.float32)

@@ -40,7 +40,8 @@ v4kv_status check_device(int* num_sms) {
 v4kv_status to_status(cudaError_t e) { return e == cudaSuccess ? V4KV_OK : V4KV_ERR_CUDA; }
 
 // checks common to every pool; spb must equal `want_spb`
-bool pool_ok(const v4kv_paged* p, int want_spb, int want_dim, bool allow_bf16, bool allow_fp8) {
+bool pool_ok(const v4kv_paged* p, int want_spb, int want_dim, bool allow_bf16, bool allow_fp8,
+             bool allow_fp4 = false) {
   if (!p || !p->data || !p->block_table) return false;
   if (!aligned16(p->data)) return false;
   if (p->num_pages <= 0 || p->max_blocks <= 0) return false;
@@ -48,6 +49,8 @@ bool pool_ok(const v4kv_paged* p, int want_spb, int want_dim, bool allow_bf16, b
   if (want_dim > 0 && p->dim != want_dim) return false;
   if (p->dtype == V4KV_FP8_E4M3) {
     if (!allow_fp8 || !p->scales) return false;
+  } else if (p->dtype == V4KV_FP4_E2M1) {
+    if (!allow_fp4 || !p->scales) return false;
   } else if (p->dtype == V4KV_BF16) {
     if (!allow_bf16) return false;
   } else {
@@ -179,8 +182,9 @@ v4kv_status v4kv_index_topk(const float* q_idx, const v4kv_paged* idx_cache,
     return V4KV_ERR_INVALID_ARG;
   if (ratio != 4 && ratio != 128) return V4KV_ERR_INVALID_ARG;
   if (k < 1 || k > 2048) return V4KV_ERR_INVALID_ARG;
-  if (!pool_ok(idx_cache, kBlock / ratio, 0, false, true)) return V4KV_ERR_INVALID_ARG;
+  if (!pool_ok(idx_cache, kBlock / ratio, 0, false, true, true)) return V4KV_ERR_INVALID_ARG;
   if (idx_cache->dim < 16 || idx_cache->dim > 512 || idx_cache->dim % 16) return V4KV_ERR_UNSUPPORTED;
+  if (idx_cache->dtype == V4KV_FP4_E2M1 && idx_cache->dim % 32) return V4KV_ERR_UNSUPPORTED;
   const size_t need = index_workspace_bytes(batch, max_seq_len, ratio, window_len);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return V4KV_ERR_INVALID_ARG;
@@ -249,17 +253,22 @@ v4kv_status decode_check_args(const void* q, int32_t q_dtype, int32_t batch, int
 
 }  // namespace v4kv
 
-extern "C" {
+namespace {
 
-v4kv_status v4kv_decode_attention(const void* q, int32_t q_dtype, int32_t batch, int32_t heads,
-                                  const v4kv_paged* main_cache, const v4kv_paged* window,
-                                  const int32_t* seq_lens, int32_t max_seq_len, int32_t ratio,
-                                  int32_t window_len, const int32_t* topk, int32_t k,
-                                  float sm_scale, v4kv_rope rope, void* out, void* workspace,
-                                  size_t workspace_bytes, int32_t* dev_status, void* stream) {
+// decode attention with the output in bf16 (out_fp8 == 0) or as e4m3 codes
+// with one scale per (sequence, head) (out_fp8 == 1)
+v4kv_status decode_impl(const void* q, int32_t q_dtype, int32_t batch, int32_t heads,
+                        const v4kv_paged* main_cache, const v4kv_paged* window,
+                        const int32_t* seq_lens, int32_t max_seq_len, int32_t ratio,
+                        int32_t window_len, const int32_t* topk, int32_t k, float sm_scale,
+                        v4kv_rope rope, void* out, int out_fp8, float* out_scales,
+                        float* prequant_out, void* workspace, size_t workspace_bytes,
+                        int32_t* dev_status, void* stream) {
   v4kv_status st = decode_check_args(q, q_dtype, batch, heads, main_cache, window, seq_lens,
                                      max_seq_len, ratio, window_len, topk, k, sm_scale, rope, out);
   if (st != V4KV_OK) return st;
+  if (out_fp8 && (!out_scales || (prequant_out && !aligned16(prequant_out))))
+    return V4KV_ERR_INVALID_ARG;
   if (!topk) k = 0;
   if (sm_scale == 0.f) sm_scale = 1.f / sqrtf(512.f);  // the default scale 1/sqrt(dim)
   int sms = 0;
@@ -293,6 +302,9 @@ v4kv_status v4kv_decode_attention(const void* q, int32_t q_dtype, int32_t batch,
   a.n_splits = plan.n_splits;
   a.max_len = max_seq_len;
   a.pad_sel = plan.path == 1;
+  a.out_fp8 = out_fp8;
+  a.out_scales = out_scales;
+  a.prequant_out = out_fp8 ? prequant_out : nullptr;
   if (plan.path == 1) {
     decode_tc_layout(a, workspace);
     return to_status(launch_decode_tc(a, (cudaStream_t)stream));
@@ -300,6 +312,35 @@ v4kv_status v4kv_decode_attention(const void* q, int32_t q_dtype, int32_t batch,
   cudaError_t e = launch_decode_simt(a, (cudaStream_t)stream);
   if (e != cudaSuccess) return V4KV_ERR_CUDA;
   return to_status(launch_decode_merge(a, (cudaStream_t)stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+v4kv_status v4kv_decode_attention(const void* q, int32_t q_dtype, int32_t batch, int32_t heads,
+                                  const v4kv_paged* main_cache, const v4kv_paged* window,
+                                  const int32_t* seq_lens, int32_t max_seq_len, int32_t ratio,
+                                  int32_t window_len, const int32_t* topk, int32_t k,
+                                  float sm_scale, v4kv_rope rope, void* out, void* workspace,
+                                  size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  return decode_impl(q, q_dtype, batch, heads, main_cache, window, seq_lens, max_seq_len, ratio,
+                     window_len, topk, k, sm_scale, rope, out, 0, nullptr, nullptr, workspace,
+                     workspace_bytes, dev_status, stream);
+}
+
+v4kv_status v4kv_decode_attention_fp8out(const void* q, int32_t q_dtype, int32_t batch,
+                                         int32_t heads, const v4kv_paged* main_cache,
+                                         const v4kv_paged* window, const int32_t* seq_lens,
+                                         int32_t max_seq_len, int32_t ratio, int32_t window_len,
+                                         const int32_t* topk, int32_t k, float sm_scale,
+                                         v4kv_rope rope, void* out_codes, float* out_scales,
+                                         float* prequant_out, void* workspace,
+                                         size_t workspace_bytes, int32_t* dev_status,
+                                         void* stream) {
+  return decode_impl(q, q_dtype, batch, heads, main_cache, window, seq_lens, max_seq_len, ratio,
+                     window_len, topk, k, sm_scale, rope, out_codes, 1, out_scales, prequant_out,
+                     workspace, workspace_bytes, dev_status, stream);
 }
 
 uint64_t v4kv_kv_footprint_bytes(uint64_t n_tokens, const v4kv_footprint_cfg* c) {

@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
+#include <cuda_fp4.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -104,6 +105,48 @@ __device__ __forceinline__ float block_reduce(float v, float* red) {
   float r = red[0];
   __syncthreads();
   return r;
+}
+
+// Output epilogue of decode attention for n consecutive values of one
+// (sequence, head) vector held by this thread (amax = the vector's absolute
+// maximum, reduced by the caller): bf16, or e4m3 codes with the vector's
+// scale amax / 448 (1 if amax == 0; IEEE division per element, round to
+// nearest even, saturating), optionally also the fp32 values themselves.
+template <int N>
+__device__ __forceinline__ void store_output(const DecodeArgs& a, size_t row, int d0, const float* v,
+                                             float amax, bool scale_writer) {
+  const size_t off = row * 512 + d0;
+  if (a.prequant_out) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4)
+      *reinterpret_cast<float4*>(a.prequant_out + off + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+  }
+  if (a.out_fp8) {
+    const float scale = amax == 0.f ? 1.f : __fdiv_rn(amax, kE4m3Max);
+    uint32_t w[N / 4];
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const uint16_t lo = float2_to_e4m3x2(__fdiv_rn(v[4 * i], scale), __fdiv_rn(v[4 * i + 1], scale));
+      const uint16_t hi = float2_to_e4m3x2(__fdiv_rn(v[4 * i + 2], scale), __fdiv_rn(v[4 * i + 3], scale));
+      w[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    uint8_t* dst = reinterpret_cast<uint8_t*>(a.out) + off;
+    if constexpr (N == 16) {
+      *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < N / 4; ++i) reinterpret_cast<uint32_t*>(dst)[i] = w[i];
+    }
+    if (scale_writer) a.out_scales[row] = scale;
+  } else {
+    uint32_t w[N / 2];
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i)
+      w[i] = (uint32_t)float_to_bf16_bits(v[2 * i]) | ((uint32_t)float_to_bf16_bits(v[2 * i + 1]) << 16);
+    uint16_t* dst = reinterpret_cast<uint16_t*>(a.out) + off;
+#pragma unroll
+    for (int i = 0; i < N / 2; i += 2) *reinterpret_cast<uint2*>(dst + 2 * i) = make_uint2(w[i], w[i + 1]);
+  }
 }
 
 // page of logical index j through a block-table row; -1 if absent

@@ -237,10 +237,12 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
       }
     }
   }
-  uint16_t* dst = reinterpret_cast<uint16_t*>(a.out) + ((size_t)b * a.heads + h) * kDim + d0;
-  const uint32_t w0 = (uint32_t)float_to_bf16_bits(o[0]) | ((uint32_t)float_to_bf16_bits(o[1]) << 16);
-  const uint32_t w1 = (uint32_t)float_to_bf16_bits(o[2]) | ((uint32_t)float_to_bf16_bits(o[3]) << 16);
-  *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
+  float amax = 0.f;
+  if (a.out_fp8) {
+    __shared__ float red[32];
+    amax = block_reduce<true>(fmaxf(fmaxf(fabsf(o[0]), fabsf(o[1])), fmaxf(fabsf(o[2]), fabsf(o[3]))), red);
+  }
+  store_output<4>(a, (size_t)b * a.heads + h, d0, o, amax, threadIdx.x == 0);
 }
 
 DecodePlan plan_decode(int batch, int heads, int max_seq_len, int ratio, int window_len, int k,

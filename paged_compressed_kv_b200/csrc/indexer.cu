@@ -64,6 +64,23 @@ __device__ __forceinline__ float fma4_fp8(float acc, uint32_t k4, uint32_t q01, 
   return acc;
 }
 
+// the same chain over eight consecutive dims whose keys are fp4-e2m1 codes
+// (k8: four bytes, dim 2i in the low nibble of byte i, lowest byte first);
+// q[0..3] the query's f16 pairs of these dims. e2m1 values are exact in f16.
+__device__ __forceinline__ float fma8_fp4(float acc, uint32_t k8, const uint32_t* q) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2_raw kr = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((k8 >> (8 * i)) & 0xffu), __NV_E2M1);
+    const uint32_t kk = (uint32_t)kr.x | ((uint32_t)kr.y << 16);
+    asm("{\n\t.reg .f16 a0, a1, b0, b1;\n\t"
+        "mov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+        "fma.rn.f32.f16 %0, a0, b0, %0;\n\tfma.rn.f32.f16 %0, a1, b1, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(kk), "r"(q[i]));
+  }
+  return acc;
+}
+
 // order-preserving map of fp32 onto uint32 (larger float -> larger key)
 __device__ __forceinline__ uint32_t score_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -101,7 +118,9 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_kernel(IndexArgs a)
   const int j1 = min(n_vis, j0 + kScoreChunk);
   const int32_t* bt = a.cache.block_table + (size_t)b * a.cache.max_blocks;
   const uint8_t* base = reinterpret_cast<const uint8_t*>(a.cache.data);
-  const int nq = dim / 16;  // 16-byte chunks per key
+  const bool fp4 = a.cache.dtype == V4KV_FP4_E2M1;
+  const int rowb = fp4 ? dim / 2 : dim;  // bytes per key
+  const int nq = rowb / 16;              // 16-byte chunks per key
   for (int jj = j0 + threadIdx.x; jj < j1; jj += 2 * blockDim.x) {
     const int ja = jj, jb = jj + blockDim.x;
     const bool hb = jb < j1;
@@ -115,8 +134,24 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_kernel(IndexArgs a)
       const int nc = min(8, nq - c0);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        ra[c] = (c < nc && sa >= 0) ? *reinterpret_cast<const uint4*>(base + sa * dim + 16 * (c0 + c)) : make_uint4(0, 0, 0, 0);
-        rb[c] = (c < nc && sb >= 0) ? *reinterpret_cast<const uint4*>(base + sb * dim + 16 * (c0 + c)) : make_uint4(0, 0, 0, 0);
+        ra[c] = (c < nc && sa >= 0) ? *reinterpret_cast<const uint4*>(base + sa * rowb + 16 * (c0 + c)) : make_uint4(0, 0, 0, 0);
+        rb[c] = (c < nc && sb >= 0) ? *reinterpret_cast<const uint4*>(base + sb * rowb + 16 * (c0 + c)) : make_uint4(0, 0, 0, 0);
+      }
+      if (fp4) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if (c >= nc) break;
+          const uint32_t* qq = &q16[16 * (c0 + c)];  // dims 32 (c0 + c) ..
+          acc_a = fma8_fp4(acc_a, ra[c].x, qq);
+          acc_a = fma8_fp4(acc_a, ra[c].y, qq + 4);
+          acc_a = fma8_fp4(acc_a, ra[c].z, qq + 8);
+          acc_a = fma8_fp4(acc_a, ra[c].w, qq + 12);
+          acc_b = fma8_fp4(acc_b, rb[c].x, qq);
+          acc_b = fma8_fp4(acc_b, rb[c].y, qq + 4);
+          acc_b = fma8_fp4(acc_b, rb[c].z, qq + 8);
+          acc_b = fma8_fp4(acc_b, rb[c].w, qq + 12);
+        }
+        continue;
       }
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -191,8 +226,13 @@ constexpr uint32_t kStageBytes = kTmaBatch * 128;
 constexpr size_t kTmaSmem = 1024 + kTmaStages * kStageBytes + (kBins / 2) * 4 + 64 * 4 +
                             kTmaGroups * 8 + 32 * 4 + kTmaStages * 8 + 16;
 
+// fp4 keys (64 bytes) use the same machinery on the pool seen as 128-byte
+// rows of two keys: a 64-entry group is one box of 32 rows, entry e of a stage
+// is half e % 2 of row e / 2.
+template <bool kFp4>
 __global__ void __launch_bounds__(kTmaBatch) index_score_tma_kernel(const __grid_constant__ CUtensorMap keys,
                                                                     IndexArgs a) {
+  constexpr int kRowsPerBox = kFp4 ? kTmaBox / 2 : kTmaBox;  // 128-byte rows per 64-entry group
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* stages = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* hist2 = reinterpret_cast<uint32_t*>(stages + kTmaStages * kStageBytes);  // 16-bit pairs
@@ -218,7 +258,7 @@ __global__ void __launch_bounds__(kTmaBatch) index_score_tma_kernel(const __grid
       const long long blk = g0 / spb;
       const int32_t* bt = a.cache.block_table + (size_t)b * a.cache.max_blocks;
       const int p = blk < a.cache.max_blocks ? bt[blk] : -1;
-      if (p >= 0 && p < a.cache.num_pages) r = (long long)p * spb + g0 % spb;
+      if (p >= 0 && p < a.cache.num_pages) r = ((long long)p * spb + g0 % spb) / (kFp4 ? 2 : 1);
       else flag(a.dev_status, V4KV_DEV_BAD_PAGE);
     }
     row0[t] = r;
@@ -235,13 +275,13 @@ __global__ void __launch_bounds__(kTmaBatch) index_score_tma_kernel(const __grid
     uint32_t bytes = 0;
     for (int k = 0; k < kTmaBatch / kTmaBox; ++k) {
       const int g = bi * (kTmaBatch / kTmaBox) + k;
-      if (g < ngroups && row0[g] >= 0) bytes += kTmaBox * 128;
+      if (g < ngroups && row0[g] >= 0) bytes += kRowsPerBox * 128;
     }
     tc::mbar_arrive_expect_tx(&full[s], bytes);
     for (int k = 0; k < kTmaBatch / kTmaBox; ++k) {
       const int g = bi * (kTmaBatch / kTmaBox) + k;
       if (g < ngroups && row0[g] >= 0)
-        tc::tma_load_2d(stages_s + s * kStageBytes + k * kTmaBox * 128, &keys, 0, (int)row0[g], &full[s]);
+        tc::tma_load_2d(stages_s + s * kStageBytes + k * kRowsPerBox * 128, &keys, 0, (int)row0[g], &full[s]);
     }
   };
   int issued = 0;  // thread 0: stages issued so far
@@ -268,7 +308,7 @@ __global__ void __launch_bounds__(kTmaBatch) index_score_tma_kernel(const __grid
     const int e = bi * kTmaBatch + t;  // entry offset within the chunk
     const int j = j0 + e;
     const long long r = j < j1 ? row0[e / kTmaBox] : -1;
-    const long long slot = r >= 0 ? r + (e % kTmaBox) : -1;
+    const long long slot = r >= 0 ? r * (kFp4 ? 2 : 1) + (e % kTmaBox) : -1;
     const float ks = slot >= 0 ? a.cache.scales[slot] : 0.f;
     if (!tc::mbar_wait(&full[s], (uint32_t)(bi / kTmaStages) & 1u, abort_sh)) {
       flag(a.dev_status, V4KV_DEV_TIMEOUT);
@@ -276,7 +316,22 @@ __global__ void __launch_bounds__(kTmaBatch) index_score_tma_kernel(const __grid
     }
     if (j < j1) {
       float score = 0.f;
-      if (slot >= 0) {
+      if (slot >= 0 && kFp4) {
+        // row t / 2 of the stage (its swizzle phase (t / 2) % 8), half t % 2
+        const uint8_t* row = stages + s * kStageBytes + (t >> 1) * 128;
+        const int swr = ((t >> 1) & 7) * 16;
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 kv = *reinterpret_cast<const uint4*>(row + ((16 * (4 * (t & 1) + c)) ^ swr));
+          const uint32_t* qq = &q16[16 * c];
+          acc = fma8_fp4(acc, kv.x, qq);
+          acc = fma8_fp4(acc, kv.y, qq + 4);
+          acc = fma8_fp4(acc, kv.z, qq + 8);
+          acc = fma8_fp4(acc, kv.w, qq + 12);
+        }
+        score = __fmul_rn(acc, ks);
+      } else if (slot >= 0) {
         const uint8_t* row = stages + s * kStageBytes + t * 128;
         float acc = 0.f;
 #pragma unroll
@@ -530,19 +585,22 @@ cudaError_t launch_index_topk(IndexArgs a, int max_seq_len, cudaStream_t stream)
   a.hist_ws = reinterpret_cast<uint32_t*>(a.scores_ws + (size_t)a.batch * a.ws_stride);
   cudaError_t e = cudaMemsetAsync(a.hist_ws, 0, (size_t)a.batch * kBins * sizeof(uint32_t), stream);
   if (e != cudaSuccess) return e;
-  // 128-byte keys on pages of whole 64-entry groups go through TMA boxes
+  // 128-dim keys (128 bytes fp8, 64 bytes fp4) on pages of whole 64-entry
+  // groups go through TMA boxes of 128-byte rows
+  const bool fp4 = a.cache.dtype == V4KV_FP4_E2M1;
   const bool tma = a.cache.dim == 128 && a.cache.spb % kTmaBox == 0 &&
                    (reinterpret_cast<uintptr_t>(a.cache.data) & 15) == 0 &&
                    (long long)a.cache.num_pages * a.cache.spb <= 0x7fffffffLL;
   if (nv > 0 && tma) {
     CUtensorMap keys;
-    e = encode_rows_u8(&keys, a.cache.data, (uint64_t)a.cache.num_pages * a.cache.spb, 128, kTmaBox);
+    const uint64_t rows = (uint64_t)a.cache.num_pages * a.cache.spb / (fp4 ? 2 : 1);
+    e = encode_rows_u8(&keys, a.cache.data, rows, 128, fp4 ? kTmaBox / 2 : kTmaBox);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(index_score_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kTmaSmem);
+    auto kern = fp4 ? index_score_tma_kernel<true> : index_score_tma_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTmaSmem);
     if (e != cudaSuccess) return e;
     dim3 grid((nv + kTmaChunk - 1) / kTmaChunk, a.batch);
-    index_score_tma_kernel<<<grid, kTmaBatch, kTmaSmem, stream>>>(keys, a);
+    kern<<<grid, kTmaBatch, kTmaSmem, stream>>>(keys, a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   } else if (nv > 0) {

@@ -28,13 +28,14 @@ V4KV_DEV_RANGE = 32
 V4KV_BF16 = 0
 V4KV_FP8_E4M3 = 1
 V4KV_FP32 = 2
+V4KV_FP4_E2M1 = 3
 V4KV_OP_INDEX_TOPK = 1
 V4KV_OP_DECODE = 2
 
 EXPORTED = [
     "v4kv_status_string", "v4kv_version", "v4kv_slot_mapping", "v4kv_compress_append",
     "v4kv_index_topk", "v4kv_decode_attention", "v4kv_workspace_size", "v4kv_kv_footprint_bytes",
-    "v4kv_decode_attention_noalloc",
+    "v4kv_decode_attention_noalloc", "v4kv_decode_attention_fp8out",
 ]
 
 V4KV_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -86,6 +87,9 @@ def _load():
         "v4kv_decode_attention_noalloc": (I32, [P, I32, I32, I32, ctypes.POINTER(_Paged),
                                                 ctypes.POINTER(_Paged), P, I32, I32, I32, P, I32,
                                                 F32, _Rope, P, P, P]),
+        "v4kv_decode_attention_fp8out": (I32, [P, I32, I32, I32, ctypes.POINTER(_Paged),
+                                               ctypes.POINTER(_Paged), P, I32, I32, I32, P, I32,
+                                               F32, _Rope, P, P, P, P, SZ, P, P]),
         "v4kv_workspace_size": (I32, [I32, I32, I32, I32, I32, I32, I32, I32, I32,
                                       ctypes.POINTER(SZ)]),
         "v4kv_kv_footprint_bytes": (ctypes.c_uint64, [ctypes.c_uint64, ctypes.POINTER(_Footprint)]),
@@ -118,18 +122,25 @@ class PagedPool:
     data: torch.Tensor
     block_table: torch.Tensor
     scales: Optional[torch.Tensor] = None
+    fp4: bool = False  # uint8 data holds packed fp4-e2m1 pairs (indexer pools)
 
     @property
     def dtype_code(self):
+        if self.fp4:
+            return V4KV_FP4_E2M1
         return V4KV_FP8_E4M3 if self.data.dtype == torch.uint8 else V4KV_BF16
+
+    @property
+    def dim(self):
+        return self.data.shape[2] * (2 if self.fp4 else 1)
 
     def c(self):
         d = self.data
         _need(d, (torch.uint8, torch.bfloat16, torch.int16), "pool data", ndim=3)
         _need(self.block_table, (torch.int32,), "block_table", ndim=2)
-        if self.dtype_code == V4KV_FP8_E4M3:
+        if self.dtype_code in (V4KV_FP8_E4M3, V4KV_FP4_E2M1):
             _need(self.scales, (torch.float32,), "scales", ndim=2)
-        return _Paged(d.data_ptr(), _ptr(self.scales), d.shape[0], d.shape[1], d.shape[2],
+        return _Paged(d.data_ptr(), _ptr(self.scales), d.shape[0], d.shape[1], self.dim,
                       self.dtype_code, self.block_table.data_ptr(), self.block_table.shape[1])
 
 
@@ -249,6 +260,33 @@ def v4kv_decode_attention(q, main, window, seq_lens, max_seq_len, ratio, window_
         _ptr(topk), topk.shape[1] if topk is not None else 0, sm_scale, rope.c(), out.data_ptr(),
         workspace.data_ptr(), workspace.numel(), _ptr(dev_status), _stream(stream))
     _check("v4kv_decode_attention", st)
+
+
+def v4kv_decode_attention_fp8out(q, main, window, seq_lens, max_seq_len, ratio, window_len,
+                                 out_codes, out_scales, workspace, topk=None, sm_scale=None,
+                                 rope=None, prequant_out=None, dev_status=None, stream=None):
+    """v4kv_decode_attention with the output quantised to e4m3 per (sequence,
+    head) vector: out_codes uint8 [B, H, 512], out_scales fp32 [B, H]."""
+    _need(q, (torch.float32, torch.bfloat16), "q", ndim=3)
+    _need(seq_lens, (torch.int32,), "seq_lens")
+    _need(out_codes, (torch.uint8,), "out_codes", ndim=3)
+    _need(out_scales, (torch.float32,), "out_scales", ndim=2)
+    _need(workspace, (torch.uint8,), "workspace")
+    if topk is not None:
+        _need(topk, (torch.int32,), "topk", ndim=2)
+    if prequant_out is not None:
+        _need(prequant_out, (torch.float32,), "prequant_out", ndim=3)
+    rope = rope or Rope()
+    if sm_scale is None:
+        sm_scale = 0.0  # the library's default, 1/sqrt(512)
+    mc, wc = main.c(), window.c()
+    st = _lib.v4kv_decode_attention_fp8out(
+        q.data_ptr(), V4KV_FP32 if q.dtype == torch.float32 else V4KV_BF16, q.shape[0], q.shape[1],
+        ctypes.byref(mc), ctypes.byref(wc), seq_lens.data_ptr(), max_seq_len, ratio, window_len,
+        _ptr(topk), topk.shape[1] if topk is not None else 0, sm_scale, rope.c(),
+        out_codes.data_ptr(), out_scales.data_ptr(), _ptr(prequant_out), workspace.data_ptr(),
+        workspace.numel(), _ptr(dev_status), _stream(stream))
+    _check("v4kv_decode_attention_fp8out", st)
 
 
 def v4kv_decode_attention_noalloc(q, main, window, seq_lens, max_seq_len, ratio, window_len, out,

@@ -26,6 +26,10 @@ class NpPool:
 
     def to_cuda(self):
         from paged_compressed_kv_b200 import PagedPool
+        if self.dtype == "fp4":
+            return PagedPool(data=torch.from_numpy(self.data).cuda(),
+                             block_table=torch.from_numpy(self.bt).cuda(),
+                             scales=torch.from_numpy(self.scales).cuda(), fp4=True)
         if self.dtype == "fp8":
             data = torch.from_numpy(self.data).cuda()
             sc = torch.from_numpy(self.scales).cuda()
@@ -58,7 +62,7 @@ def lay_out(rows_per_seq, spb, r, dtype, first_block=None, extra_pages=3, max_bl
     bt = np.full((B, mb), -1, dtype=np.int32)
     vdt = rows_per_seq[0][0].dtype if rows_per_seq else np.uint8
     data = np.zeros((total, spb, D), dtype=vdt)
-    scales = np.zeros((total, spb), dtype=np.float32) if dtype == "fp8" else None
+    scales = np.zeros((total, spb), dtype=np.float32) if dtype in ("fp8", "fp4") else None
     k = 0
     for b, (vals, sc) in enumerate(rows_per_seq):
         f, nb = nblk[b]
@@ -156,7 +160,10 @@ def oracle_index(q_idx, pool, b, L, ratio, W, k):
         p = pool.bt[b, j // spb]
         codes[j] = pool.data[p, j % spb]
         ks[j] = pool.scales[p, j % spb]
-    scores, qs = indexer.index_scores(q_idx, codes, ks)
+    if pool.dtype == "fp4":
+        scores, qs = indexer.index_scores(q_idx, codecs.unpack_fp4(codes), ks, key_format="fp4")
+    else:
+        scores, qs = indexer.index_scores(q_idx, codes, ks)
     sel = indexer.topk(scores, n_vis, k)
     return sel, indexer.reported_scores(scores, qs, sel)
 

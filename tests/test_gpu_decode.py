@@ -218,3 +218,72 @@ def test_bf16_beyond_f16_range_is_flagged_on_the_tensor_core_path():
         else:
             assert st == 0
             check_all(case, got)
+
+
+def test_fp8_window_then_bf16_entries_64_heads():
+    # a segment whose window tiles (fp8) run in the pipelined path and whose
+    # entry tiles (bf16) run one at a time, with several such segments per
+    # sweep block and blocks starting in the middle of a sequence
+    lens = [3000, 700, 128 * 4 + 129, 5000, 1]
+    case = DecodeCase(217, lens, 64, 4, main_dtype="bf16", win_dtype="fp8", window=300)
+    got, st = run_decode(case)
+    assert st == 0
+    check_all(case, got)
+
+
+@pytest.mark.parametrize("heads", [64])
+def test_long_window_fp8_many_segments(heads):
+    # windows of several tiles, fp8 window and fp8 entries: consecutive fp8
+    # segments across segment boundaries in one block
+    r = synth.rng(218)
+    lens = r.integers(1, 2500, 40).tolist()
+    case = DecodeCase(218, lens, heads, 4, win_dtype="fp8", window=700)
+    got, st = run_decode(case)
+    assert st == 0
+    check_all(case, got, seqs=list(range(0, 40, 3)))
+
+
+@pytest.mark.parametrize("heads", [8, 64])
+def test_fp8_output_epilogue(heads):
+    # v4kv_decode_attention_fp8out: the merge epilogue quantises each
+    # (sequence, head) output vector to e4m3 after the inverse RoPE. The fp32
+    # values it hands to the quantiser meet the decode tolerance against the
+    # oracle; codes and scales are bit-exact against the oracle's quantiser on
+    # those same fp32 values; and the bf16 entry point's output is exactly
+    # their bf16 rounding
+    from oracle import attention, codecs
+    from paged_compressed_kv_b200 import v4kv
+    case = DecodeCase(219, [3000, 129, 9000, 0], heads, 4)
+    dev = torch.device("cuda")
+    q = torch.from_numpy(case.q).to(dev)
+    main, win = case.main.to_cuda(), case.win.to_cuda()
+    seq = torch.from_numpy(case.lens.astype(np.int32)).to(dev)
+    ws = v4kv.v4kv_workspace_size(v4kv.V4KV_OP_DECODE, case.B, case.H, case.max_len, case.ratio,
+                                  case.W, 0, main.dtype_code)
+    workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    codes = torch.empty(case.B, case.H, 512, dtype=torch.uint8, device=dev)
+    scales = torch.empty(case.B, case.H, dtype=torch.float32, device=dev)
+    pre = torch.full((case.B, case.H, 512), float("nan"), dtype=torch.float32, device=dev)
+    v4kv.v4kv_decode_attention_fp8out(q, main, win, seq, case.max_len, case.ratio, case.W, codes,
+                                      scales, workspace, prequant_out=pre, dev_status=st)
+    out = torch.empty(case.B, case.H, 512, dtype=torch.bfloat16, device=dev)
+    v4kv.v4kv_decode_attention(q, main, win, seq, case.max_len, case.ratio, case.W, out, workspace,
+                               dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    pre = pre.cpu().numpy()
+    assert not np.isnan(pre).any()
+    want_c, want_s = attention.output_fp8(pre)
+    assert np.array_equal(codes.cpu().numpy(), want_c)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), want_s.view(np.uint32))
+    assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), codecs.bf16_bits(pre))
+    for b in range(case.B):
+        ref = case.oracle(b)
+        d = np.abs(pre[b].astype(np.float64) - ref)
+        mx = np.abs(ref).max() if case.lens[b] else 0.0
+        assert d.max() <= 1e-2 * mx + 1e-30
+        if case.lens[b]:
+            assert d.sum() / np.abs(ref).sum() <= 1e-3
+        else:
+            assert np.all(want_c[b] == 0) and np.all(scales.cpu().numpy()[b] == 1.0)

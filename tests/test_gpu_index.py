@@ -11,7 +11,7 @@ from tests.helpers import lay_out, oracle_index
 pytestmark = pytest.mark.gpu
 
 
-def build(seed, lens, dup_groups=0, dim=128, ratio=4):
+def build(seed, lens, dup_groups=0, dim=128, ratio=4, fp4=False):
     r = synth.rng(seed)
     rows = []
     for L in lens:
@@ -20,8 +20,12 @@ def build(seed, lens, dup_groups=0, dim=128, ratio=4):
         if dup_groups and n:
             base = x[: dup_groups].copy()
             x = base[r.integers(0, dup_groups, n)]
-        rows.append(codecs.quantize_entry(x))
-    pool = lay_out(rows, 256 // ratio, r, "fp8")
+        if fp4:
+            codes, sc = codecs.quantize_entry_fp4(x)
+            rows.append((codecs.pack_fp4(codes), sc))
+        else:
+            rows.append(codecs.quantize_entry(x))
+    pool = lay_out(rows, 256 // ratio, r, "fp4" if fp4 else "fp8")
     q = synth.normal(r, (len(lens), dim))
     return pool, q
 
@@ -32,7 +36,7 @@ def run(pool, q, lens, k, ratio=4, W=128):
     B = len(lens)
     max_len = int(max(lens))
     ws = v4kv.v4kv_workspace_size(v4kv.V4KV_OP_INDEX_TOPK, B, 1, max_len, ratio, W, k,
-                                  v4kv.V4KV_FP8_E4M3, pool.data.shape[2])
+                                  v4kv.V4KV_FP8_E4M3, 128)
     workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
     topk = torch.empty(B, k, dtype=torch.int32, device=dev)
     score = torch.empty(B, k, dtype=torch.float32, device=dev)
@@ -110,5 +114,33 @@ def test_bad_page_is_flagged_and_scored_zero():
     assert st & v4kv.V4KV_DEV_BAD_PAGE
     for b, L in enumerate(lens):
         sel, rs = oracle_index(q[b], zero, b, L, 4, 128, 512)
+        assert np.array_equal(got[b], sel), f"seq {b}"
+        assert np.array_equal(sc[b].view(np.uint32), rs.view(np.uint32)), f"seq {b}"
+
+
+@pytest.mark.parametrize("k", [16, 512])
+def test_fp4_keys_bit_exact(k):
+    # fp4-e2m1 keys with one fp32 scale each (two codes per byte): the
+    # 128-dim keys take the TMA kernel on the pool seen as 128-byte rows of two
+    # keys; indices and reported scores bit-exact against the oracle
+    lens = [0, 100, 128 + 4 * 300, 4096, 20000, 65536]
+    pool, q = build(340 + k, lens, fp4=True)
+    assert pool.data.shape[2] == 64
+    got, sc, st = run(pool, q, lens, k)
+    assert st == 0
+    for b, L in enumerate(lens):
+        sel, rs = oracle_index(q[b], pool, b, L, 4, 128, k)
+        assert np.array_equal(got[b], sel), f"seq {b}"
+        assert np.array_equal(sc[b].view(np.uint32), rs.view(np.uint32)), f"seq {b}"
+
+
+def test_fp4_keys_other_width_generic_kernel():
+    # 256-dim fp4 keys (128 bytes) take the generic scoring kernel
+    lens = [300, 128 + 4 * 1000 + 3, 30000]
+    pool, q = build(350, lens, dim=256, fp4=True)
+    got, sc, st = run(pool, q, lens, 512)
+    assert st == 0
+    for b, L in enumerate(lens):
+        sel, rs = oracle_index(q[b], pool, b, L, 4, 128, 512)
         assert np.array_equal(got[b], sel), f"seq {b}"
         assert np.array_equal(sc[b].view(np.uint32), rs.view(np.uint32)), f"seq {b}"

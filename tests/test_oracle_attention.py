@@ -118,3 +118,36 @@ def test_topk_restricts_the_set():
     vals = np.concatenate([codecs.dequantize_entry(codes[[3, 5, 100]], sc[[3, 5, 100]]),
                            codecs.bf16_to_f32(w[L - 128:]).astype(np.float64)])
     assert np.allclose(out, attention.attend(q, vals, 0.1, L), atol=1e-14)
+
+
+def test_output_fp8_hand_worked_vector():
+    # tests/golden/output_fp8_worked.txt: codes and scale derived by hand from
+    # the e4m3 definition for a vector whose scale is exactly 2^-6
+    import os
+    rows, scale = [], None
+    for line in open(os.path.join(os.path.dirname(__file__), "golden", "output_fp8_worked.txt")):
+        f = line.split("#")[0].split()
+        if not f:
+            continue
+        if f[0] == "scale":
+            scale = float(f[1])
+        else:
+            rows.append((int(f[0]), float(f[1]), int(f[2], 16)))
+    o = np.zeros((1, 512))
+    for i, v, _ in rows:
+        o[0, i] = v
+    codes, sc = attention.output_fp8(o)
+    assert sc[0] == scale
+    for i, _, want in rows:
+        assert codes[0, i] == want, (i, hex(codes[0, i]))
+    assert np.all(codes[0, 7:] == 0)
+
+
+def test_output_fp8_follows_the_fp32_rounding_of_the_output():
+    # the quantiser sees the fp32 value of the fp64 output: an output 1 + 2^-40
+    # quantises exactly like 1.0
+    o = np.zeros((2, 512))
+    o[0, 0], o[1, 0] = 1.0, 1.0 + 2.0 ** -40
+    o[:, 1] = -3.0
+    c, s = attention.output_fp8(o)
+    assert np.array_equal(c[0], c[1]) and s[0] == s[1]

@@ -105,3 +105,66 @@ def test_decode_known_values():
     assert codecs.e4m3_decode(np.uint8(0x7E)) == 448.0
     assert codecs.e4m3_decode(np.uint8(0x01)) == math.ldexp(1.0, -9)
     assert codecs.e4m3_decode(np.uint8(0xB8)) == -1.0
+
+
+def _e2m1_points():
+    import os
+    codes, encs = [], []
+    for line in open(os.path.join(os.path.dirname(__file__), "golden", "e2m1_spec_points.txt")):
+        f = line.split("#")[0].split()
+        if not f:
+            continue
+        if f[0] == "code":
+            codes.append((int(f[1], 16), float(f[2])))
+        else:
+            encs.append((float(f[1]), int(f[2], 16)))
+    return codes, encs
+
+
+def test_e2m1_decode_all_sixteen_codes():
+    codes, _ = _e2m1_points()
+    assert len(codes) == 16
+    for c, v in codes:
+        got = codecs.e2m1_decode(np.array([c]))[0]
+        assert got == v and np.signbit(got) == np.signbit(v), (hex(c), got, v)
+
+
+def test_e2m1_encode_spec_points():
+    _, encs = _e2m1_points()
+    for x, c in encs:
+        got = int(codecs.e2m1_encode(np.array([x], dtype=np.float32))[0])
+        assert got == c, (x, hex(got), hex(c))
+
+
+def test_e2m1_round_trip_and_nearest():
+    # every code decodes to a value that encodes back to it (except -0 / +0,
+    # which keep their sign), and on a dense grid the encoder's choice is
+    # never farther than the other neighbour (the nearest value)
+    for c in range(16):
+        v = codecs.e2m1_decode(np.array([c]))[0]
+        assert int(codecs.e2m1_encode(np.array([v], dtype=np.float32))[0]) == c
+    x = np.linspace(-7, 7, 20001).astype(np.float32)
+    dec = codecs.e2m1_decode(codecs.e2m1_encode(x))
+    grid = np.concatenate([-codecs.E2M1_VALUES[::-1], codecs.E2M1_VALUES])
+    best = np.min(np.abs(x[:, None].astype(np.float64) - grid[None, :]), axis=1)
+    assert np.all(np.abs(np.clip(x, -6, 6) - dec) <= best + 1e-12)
+
+
+def test_fp4_key_quantiser_bound_and_packing():
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((50, 128)).astype(np.float32)
+    x[3] = 0.0
+    codes, sc = codecs.quantize_entry_fp4(x)
+    assert sc[3] == 1.0 and np.all(codes[3] == 0)
+    amax = np.abs(x).max(axis=1)
+    assert np.all(sc[np.arange(50) != 3] == (amax / np.float32(6.0)).astype(np.float32)[np.arange(50) != 3])
+    dq = codecs.e2m1_decode(codes) * sc[:, None].astype(np.float64)
+    # the largest e2m1 gap is 2 (between 4 and 6): error <= 1 * scale; below
+    # 2 it is <= 0.25 * scale
+    err = np.abs(dq - x)
+    assert np.all(err <= sc[:, None] * 1.0 + 1e-12)
+    small = np.abs(x / sc[:, None]) < 2
+    assert np.all(err[small] <= sc[:, None].repeat(128, 1)[small] * 0.25 + 1e-12)
+    assert np.array_equal(codecs.unpack_fp4(codecs.pack_fp4(codes)), codes)
+    p = codecs.pack_fp4(np.array([[0x1, 0xF, 0x7, 0x8]], dtype=np.uint8))
+    assert p.tolist() == [[0xF1, 0x87]]

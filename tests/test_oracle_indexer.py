@@ -96,3 +96,32 @@ def test_shortfall_padding(n_vis, k):
     m = min(n_vis, k)
     assert got[:m].tolist() == list(range(n_vis - 1, n_vis - 1 - m, -1))
     assert np.all(got[m:] == -1)
+
+
+def test_fp4_keys_brute_force_exact_rational():
+    # e2m1 keys (values k/2, integers up to 6) against integer-valued query
+    # codes keep the fp32 chain exact: the scores equal an exact rational
+    # dot product and the ranking an exact sort; a decode of the wrong format
+    # (e4m3 instead of e2m1) or a dropped half-step would fail here
+    rng = np.random.default_rng(17)
+    n, d = 200, 128
+    keys = rng.integers(0, 16, size=(n, d)).astype(np.uint8)
+    kscale = np.exp2(rng.integers(-2, 3, n)).astype(np.float32)
+    q = rng.choice([-448.0, -224.0, 0.0, 112.0, 448.0], size=d).astype(np.float32)
+    q[0] = 448.0
+    scores, qs = indexer.index_scores(q, keys, kscale, key_format="fp4")
+    q8, _ = codecs.quantize_entry(q)
+    vals = [Fraction(0), Fraction(1, 2), Fraction(1), Fraction(3, 2), Fraction(2), Fraction(3),
+            Fraction(4), Fraction(6)]
+    exact = []
+    for j in range(n):
+        s = Fraction(0)
+        for i in range(d):
+            c = int(keys[j, i])
+            kv = -vals[c & 7] if c & 8 else vals[c & 7]
+            s += _exact(q8[i]) * kv
+        s *= Fraction(float(kscale[j]))
+        assert Fraction(float(scores[j])) == s
+        exact.append(s)
+    want = sorted(range(n), key=lambda j: (-exact[j], j))[:64]
+    assert indexer.topk(scores, n, 64)[:64].tolist() == want
