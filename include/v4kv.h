@@ -325,6 +325,54 @@ typedef struct {
 
 uint64_t v4kv_kv_footprint_bytes(uint64_t n_tokens, const v4kv_footprint_cfg* cfg);
 
+/*
+ * Unified page pools (host only; P1 §3.1.3, "unifying page sizes").
+ *
+ * Every cache kind keeps one 256-token logical block per physical page, so
+ * its page size is (256 / ratio) x bytes per entry (P1 §3.1.3 writes it as
+ * block_size x compress_ratio x per_entry_size). Instead of one pool per kind,
+ * the kinds are grouped into a few buckets (three on the page), each a pool of
+ * fixed-size pages: the grouping is planned once ("static planning") and
+ * requests then take whole pages of their kind's bucket ("dynamic
+ * allocation"), with no compaction or migration between pools. These calls
+ * only hand out page indices; the caller owns the device memory of each
+ * bucket (bucket_bytes[b] x pages) and writes the indices into its block
+ * tables. Thread-safe: each pool object serialises its own calls.
+ */
+
+/* Page bytes of a kind: (256 / ratio) x (ceil(dim x elem_bits / 8) +
+ * scale_bytes); ratio 1 for raw-token pools. 0 for invalid arguments. */
+uint64_t v4kv_page_bytes(int32_t ratio, int32_t dim, int32_t elem_bits, int32_t scale_bytes);
+
+/* Group n_kinds page sizes into at most max_buckets buckets. Sizes are split
+ * in ascending order into contiguous groups whose page size is the group's
+ * largest member, minimising the largest ratio (bucket page / kind page) over
+ * the kinds, then the sum of those ratios. Kinds with equal page sizes always
+ * share a bucket. Writes bucket_of[n_kinds] (bucket 0 = the largest pages),
+ * bucket_bytes[*n_buckets] and *n_buckets (<= max_buckets).
+ * V4KV_ERR_INVALID_ARG for a null pointer, a count <= 0 or a zero size. */
+v4kv_status v4kv_plan_buckets(int32_t n_kinds, const uint64_t* page_bytes, int32_t max_buckets,
+                              int32_t* bucket_of, uint64_t* bucket_bytes, int32_t* n_buckets);
+
+typedef struct v4kv_page_pools v4kv_page_pools; /* opaque host object */
+
+/* Create the pools: pages_per_bucket[b] pages of bucket_bytes[b] each, all
+ * free (page indices 0 .. pages_per_bucket[b] - 1, handed out lowest first). */
+v4kv_status v4kv_page_pools_create(int32_t n_buckets, const uint64_t* bucket_bytes,
+                                   const int32_t* pages_per_bucket, v4kv_page_pools** out);
+void v4kv_page_pools_destroy(v4kv_page_pools* pools);
+
+/* Take n pages of `bucket` into pages_out[n]. If fewer than n are free,
+ * nothing is taken and V4KV_ERR_UNSUPPORTED is returned. */
+v4kv_status v4kv_page_alloc(v4kv_page_pools* pools, int32_t bucket, int32_t n, int32_t* pages_out);
+
+/* Return n pages of `bucket`. All or nothing: a page that is not allocated,
+ * out of range or listed twice gives V4KV_ERR_INVALID_ARG and frees none. */
+v4kv_status v4kv_page_free(v4kv_page_pools* pools, int32_t bucket, int32_t n, const int32_t* pages);
+
+/* Free pages left in `bucket` (-1 for a bad bucket or pool). */
+int64_t v4kv_pages_free(v4kv_page_pools* pools, int32_t bucket);
+
 #ifdef __cplusplus
 }
 #endif

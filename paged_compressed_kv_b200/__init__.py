@@ -7,7 +7,7 @@ build step (``paged_compressed_kv_b200.build``) imports without the library.
 """
 
 _EXPORTS = {
-    "EXPORTED", "LIB_PATH", "PagedPool", "Rope", "V4KVError", "v4kv_compress_append",
+    "EXPORTED", "LIB_PATH", "PagedPool", "PagePools", "v4kv_page_bytes", "v4kv_plan_buckets", "Rope", "V4KVError", "v4kv_compress_append",
     "v4kv_decode_attention", "v4kv_decode_attention_fp8out", "v4kv_decode_attention_noalloc", "v4kv_index_topk",
     "v4kv_kv_footprint_bytes", "v4kv_slot_mapping", "v4kv_status_string", "v4kv_version",
     "v4kv_workspace_size",

@@ -36,6 +36,8 @@ EXPORTED = [
     "v4kv_status_string", "v4kv_version", "v4kv_slot_mapping", "v4kv_compress_append",
     "v4kv_index_topk", "v4kv_decode_attention", "v4kv_workspace_size", "v4kv_kv_footprint_bytes",
     "v4kv_decode_attention_noalloc", "v4kv_decode_attention_fp8out",
+    "v4kv_page_bytes", "v4kv_plan_buckets", "v4kv_page_pools_create", "v4kv_page_pools_destroy",
+    "v4kv_page_alloc", "v4kv_page_free", "v4kv_pages_free",
 ]
 
 V4KV_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -93,6 +95,13 @@ def _load():
         "v4kv_workspace_size": (I32, [I32, I32, I32, I32, I32, I32, I32, I32, I32,
                                       ctypes.POINTER(SZ)]),
         "v4kv_kv_footprint_bytes": (ctypes.c_uint64, [ctypes.c_uint64, ctypes.POINTER(_Footprint)]),
+        "v4kv_page_bytes": (ctypes.c_uint64, [I32, I32, I32, I32]),
+        "v4kv_plan_buckets": (I32, [I32, P, I32, P, P, P]),
+        "v4kv_page_pools_create": (I32, [I32, P, P, ctypes.POINTER(ctypes.c_void_p)]),
+        "v4kv_page_pools_destroy": (None, [P]),
+        "v4kv_page_alloc": (I32, [P, I32, I32, P]),
+        "v4kv_page_free": (I32, [P, I32, I32, P]),
+        "v4kv_pages_free": (I64, [P, I32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -321,3 +330,53 @@ def v4kv_kv_footprint_bytes(n_tokens, layer_ratios, dim, entry_bits, entry_scale
     cfg = _Footprint(len(layer_ratios), arr, dim, entry_bits, entry_scale_bytes, indexer_dim,
                      indexer_bits, indexer_scale_bytes, window, window_bits)
     return int(_lib.v4kv_kv_footprint_bytes(n_tokens, ctypes.byref(cfg)))
+
+
+# ------------------------------------------------------------------ page pools (host)
+
+def v4kv_page_bytes(ratio, dim, elem_bits, scale_bytes=0):
+    return int(_lib.v4kv_page_bytes(ratio, dim, elem_bits, scale_bytes))
+
+
+def v4kv_plan_buckets(page_bytes, max_buckets=3):
+    """Group page sizes into at most max_buckets buckets; returns
+    (bucket_of per kind, bucket page bytes)."""
+    n = len(page_bytes)
+    pb = (ctypes.c_uint64 * n)(*page_bytes)
+    bo = (ctypes.c_int32 * n)()
+    bb = (ctypes.c_uint64 * max(1, max_buckets))()
+    nb = ctypes.c_int32(0)
+    _check("v4kv_plan_buckets", _lib.v4kv_plan_buckets(n, pb, max_buckets, bo, bb, ctypes.byref(nb)))
+    return list(bo), list(bb)[: nb.value]
+
+
+class PagePools:
+    """Host-side fixed-size page pools of the planned buckets."""
+
+    def __init__(self, bucket_bytes, pages_per_bucket):
+        n = len(bucket_bytes)
+        h = ctypes.c_void_p()
+        _check("v4kv_page_pools_create", _lib.v4kv_page_pools_create(
+            n, (ctypes.c_uint64 * n)(*bucket_bytes), (ctypes.c_int32 * n)(*pages_per_bucket),
+            ctypes.byref(h)))
+        self._h = h
+
+    def alloc(self, bucket, n):
+        out = (ctypes.c_int32 * max(1, n))()
+        _check("v4kv_page_alloc", _lib.v4kv_page_alloc(self._h, bucket, n, out))
+        return list(out)[:n]
+
+    def free(self, bucket, pages):
+        arr = (ctypes.c_int32 * max(1, len(pages)))(*pages)
+        _check("v4kv_page_free", _lib.v4kv_page_free(self._h, bucket, len(pages), arr))
+
+    def free_pages(self, bucket):
+        return int(_lib.v4kv_pages_free(self._h, bucket))
+
+    def close(self):
+        if self._h:
+            _lib.v4kv_page_pools_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
