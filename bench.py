@@ -720,15 +720,33 @@ class MixedStep:
             synth.fill_normal_bf16(wd, g)
             return PagedPool(data=wd, block_table=torch.from_numpy(wbt).to(device))
 
+        def append_inputs(ratio, P):
+            # the new token of every sequence (position L - 1) and the
+            # compressor state of its unfinished group
+            return dict(x=torch.randn(seqs, D, generator=g, device=device).to(torch.bfloat16),
+                        gate=torch.randn(seqs, generator=g, device=device),
+                        bias=torch.randn(ratio, generator=g, device=device) * 0.5,
+                        sx=torch.randn(seqs, ratio, D, generator=g, device=device).to(torch.bfloat16),
+                        sg=torch.randn(seqs, ratio, generator=g, device=device),
+                        slots=torch.empty(2 * seqs + 1, dtype=torch.int64, device=device),
+                        cue=torch.empty(seqs + 1, dtype=torch.int32, device=device), P=P)
+
         self.c4a = []
         for _ in range(c4a_layers):
-            self.c4a.append(dict(main=pool(4, D), idx=pool(4, 128), win=window(),
+            main = pool(4, D)
+            self.c4a.append(dict(main=main, idx=pool(4, 128), win=window(),
                                  q=torch.randn(seqs, HEADS, D, generator=g, device=device),
-                                 qi=torch.randn(seqs, 128, generator=g, device=device)))
+                                 qi=torch.randn(seqs, 128, generator=g, device=device),
+                                 ap=append_inputs(4, main.data.shape[0])))
         self.c128a = []
         for _ in range(c128a_layers):
-            self.c128a.append(dict(main=pool(128, D), win=window(),
-                                   q=torch.randn(seqs, HEADS, D, generator=g, device=device)))
+            main = pool(128, D)
+            self.c128a.append(dict(main=main, win=window(),
+                                   q=torch.randn(seqs, HEADS, D, generator=g, device=device),
+                                   ap=append_inputs(128, main.data.shape[0])))
+        self.seq_start = torch.from_numpy((self.lens - 1).astype(np.int32)).to(device)
+        self.n_new = torch.ones(seqs, dtype=torch.int32, device=device)
+        self.cu_seqlens = torch.arange(seqs + 1, dtype=torch.int32, device=device)
         self.topk = torch.empty(seqs, k, dtype=torch.int32, device=device)
         self.out = torch.empty(seqs, HEADS, D, dtype=torch.bfloat16, device=device)
         v = v4kv
@@ -737,6 +755,39 @@ class MixedStep:
         wsi = v.v4kv_workspace_size(v.V4KV_OP_INDEX_TOPK, seqs, 1, self.max_len, 4, W, k, v.V4KV_FP8_E4M3, 128)
         self.ws = torch.empty(max(wsa, wsb, wsi, 256), dtype=torch.uint8, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def append(self, L, ratio, stream=None):
+        """One new token per sequence into layer L's cache: slot mapping, then
+        the compressor (entry of the token's group, window row, state)."""
+        a, v = L["ap"], self.v4kv
+        v.v4kv_slot_mapping(L["main"].block_table, self.seq_start, self.n_new, ratio, a["P"],
+                            a["slots"], a["cue"], dev_status=self.status, stream=stream)
+        v.v4kv_compress_append(a["x"], a["gate"], self.cu_seqlens, self.seq_start, a["bias"], ratio,
+                               a["sx"], a["sg"], L["main"], a["slots"], a["cue"], window=L["win"],
+                               window_len=W, dev_status=self.status, stream=stream)
+
+    def full_step(self, overlap, side=None):
+        """The 61-layer decode step with each layer's append. With `overlap`,
+        a c4a layer's indexer runs on the side stream while its compressor
+        append runs on the current stream (P1 §3.2.2: indexer and main-KV
+        compression / window insertion are independent after the
+        projections); attention waits for both."""
+        cur = torch.cuda.current_stream()
+        for l in range(len(self.c4a)):
+            L = self.c4a[l]
+            if overlap:
+                side.wait_stream(cur)
+                with torch.cuda.stream(side):
+                    self.index(l)
+                self.append(L, 4)
+                cur.wait_stream(side)
+            else:
+                self.append(L, 4)
+                self.index(l)
+            self.attend_c4a(l)
+        for l in range(len(self.c128a)):
+            self.append(self.c128a[l], 128)
+            self.attend_c128a(l)
 
     def index(self, l):
         L = self.c4a[l]
@@ -782,12 +833,17 @@ def run_mixed(args, device, clk, layers=0, seqs=0):
         for l in range(nl128):
             st.attend_c128a(l)
 
+    side_stream = torch.cuda.Stream()
     parts = {"step": whole_step,
              "idx": lambda: [st.index(l) for l in range(nl4)],
              "att4": lambda: [st.attend_c4a(l) for l in range(nl4)],
-             "att128": lambda: [st.attend_c128a(l) for l in range(nl128)]}
+             "att128": lambda: [st.attend_c128a(l) for l in range(nl128)],
+             "full_serial": lambda: st.full_step(False),
+             "full_overlap": lambda: st.full_step(True, side_stream)}
     for _ in range(args.warmup):
         whole_step()
+    st.full_step(False)
+    st.full_step(True, side_stream)
     torch.cuda.synchronize()
     # each part is captured once into a CUDA graph and replayed, so the times
     # are the device's, without the Python enqueue of ~150 calls per step
@@ -834,6 +890,11 @@ def run_mixed(args, device, clk, layers=0, seqs=0):
            "step_gbs": step_bytes / (step_ms * 1e-3) / 1e9,
            "status": int(st.status.item()), "_window": win["step"]}
     res["step_frac"] = res["step_gbs"] / peak
+    # the same step with every layer's append (one token per sequence), its
+    # c4a indexers serialised or overlapped with the appends on a second stream
+    res["full_step_serial_ms"] = tot["full_serial"]
+    res["full_step_overlap_ms"] = tot["full_overlap"]
+    res["overlap_saving"] = 1.0 - tot["full_overlap"] / tot["full_serial"]
     name = (f"{nl4 + nl128}-layer mixed step ({nl4} c4a with indexer top-512 + {nl128} c128a), "
             f"batch {st.B}, context U[1K, 256K], 64 heads, fp8 KV; CUDA-graph replays, median of "
             f"{args.steps}")

@@ -83,3 +83,47 @@ def test_mixed_c4a_layer_sampled():
         ref = attention.decode_one(q[b], seq_pool(layer["main"], b), seq_pool(layer["win"], b), L,
                                    4, bench.W, 1.0 / math.sqrt(bench.D), topk_row=topk[b])
         assert_close_bf16(out[b], ref, f"mixed c4a sequence {b} (L = {L})")
+
+
+def test_two_stream_step_equals_the_serial_step():
+    # P1 §3.2.2: a c4a layer's indexer runs on a second stream while its
+    # compressor append runs on the first; attention waits for both. The
+    # overlapped step must give exactly the serial step's outputs (every
+    # layer's append is idempotent for a fixed token, so both orders start
+    # from the same caches).
+    dev = torch.device("cuda", 0)
+    st = bench.MixedStep(dev, seqs=24, c4a_layers=3, c128a_layers=2)
+    side = torch.cuda.Stream()
+
+    def run(overlap):
+        outs = []
+        cur = torch.cuda.current_stream()
+        for l in range(len(st.c4a)):
+            L = st.c4a[l]
+            if overlap:
+                side.wait_stream(cur)
+                with torch.cuda.stream(side):
+                    st.index(l)
+                st.append(L, 4)
+                cur.wait_stream(side)
+            else:
+                st.append(L, 4)
+                st.index(l)
+            st.attend_c4a(l)
+            outs.append((st.topk.clone(), st.out.clone()))
+        for l in range(len(st.c128a)):
+            st.append(st.c128a[l], 128)
+            st.attend_c128a(l)
+            outs.append((None, st.out.clone()))
+        torch.cuda.synchronize()
+        return outs
+
+    serial = run(False)
+    overlap = run(True)
+    again = run(False)
+    assert int(st.status.item()) == 0
+    for (ta, oa), (tb, ob), (tc, oc) in zip(serial, overlap, again):
+        if ta is not None:
+            assert torch.equal(ta, tb) and torch.equal(ta, tc)
+        assert torch.equal(oa.view(torch.int16), ob.view(torch.int16))
+        assert torch.equal(oa.view(torch.int16), oc.view(torch.int16))
