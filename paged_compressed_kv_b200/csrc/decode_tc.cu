@@ -3,49 +3,32 @@
 //
 // Per tile of 128 items (entries or window tokens) of one sequence:
 //   S^T[128 x 64] = V[128 x 512] . Q^T          (M = items, N = heads, K = dims)
-//   P' = 2^(S^T * c_j + log2|ks_j| - m_h)       (CUDA cores, one thread per item)
+//   P' = 2^(S^T * c_j + log2 ks_j - m_h)        (CUDA cores, one thread per item)
 //   O^T[512 x 64] += V^T[512 x 128] . P'^T      (M = dims in 4 tiles of 128)
+// V sits once in shared memory as f16 in 128-byte-swizzled atoms; it is the
+// K-major A operand of the first product and the MN-major A operand of the
+// second. fp8 codes convert to f16 exactly; the entry's fp32 scale ks_j enters
+// the score multiplier c_j and, through log2 ks_j, the exponent, so P' is the
+// weight of the raw code vector. The normaliser is sum_j P'_hj / ks_j.
+// q is scaled per sequence by a power of two into f16 range. m_h is a
+// reference maximum per head, raised only when a score exceeds it by more
+// than 2^8 (P' <= 256), at which point O^T and the partial sums are rescaled.
 //
-// fp8 tiles (the compressed entries; an fp8 window) run a software pipeline:
-//   * The fp8 codes of the tile go from global memory through registers into
-//     tensor memory unchanged (items as lanes, four codes per column). The
-//     first product reads them from there as the A operand (kind::f8f6f4), so
-//     V costs no shared-memory bandwidth in it. The query enters as three
-//     exact e4m3 terms (q = hi + mid + lo after a power-of-two scaling, about
-//     12 significant bits): three MMAs per 32-dim step share the A operand and
-//     accumulate into the same scores.
-//   * The second product needs V^T in f16 from shared memory. The converter
-//     warps read the codes back from tensor memory chunk by chunk (128 dims),
-//     convert them exactly to f16 and store them into a ring of three 32 KB
-//     chunk slots that the second product drains M-tile by M-tile.
-//   * Order on the tensor pipe: QK(t+1), PV(t), QK(t+2), PV(t+1), ... so the
-//     softmax of tile t runs while PV(t-1) and QK(t+1) execute.
-// bf16 tiles (a bf16 window or bf16 entries) run one at a time: the f16 query
-// image and the tile's f16 values fill shared memory and both products read
-// them there (kind::f16).
-//
-// The entry's fp32 scale ks_j enters the score multiplier c_j and, through
-// log2|ks_j|, the exponent, so P' is the weight of the raw code vector; its
-// sign enters P'. The normaliser is sum_j |P'_hj| / |ks_j| (a zero scale is
-// a zero-valued item of score 0). m_h is a reference maximum per head, raised
-// only when a score exceeds it by more than 2^8 (P' <= 256), at which point
-// O^T and the partial sums are rescaled. The normalisers of each row (one per
-// head) live in tensor memory.
-//
-// Warp roles (512 threads): warps 0-3 run the softmax (warp q owns tile rows
-// 32q .. 32q + 31, its tensor-memory lane quarter, all 64 heads); warps 4-11
-// convert (warp w: rows 32(w%4) + 16((w-4)/4) .. + 15); warp 12 allocates
-// tensor memory and one of its lanes issues every MMA; warps 13 and 14
-// resolve the rows of the even and odd tiles up to kRing - 1 ahead and
-// prefetch them into L2; warp 15 copies the query images.
+// Warp roles (352 threads): warps 0-7 are workers. Each runs the softmax of
+// one tile row (its TMEM lane) for 32 of the 64 heads, then gathers and
+// converts 16 rows of the next tile (16-byte coalesced page loads) as the
+// second product releases each V chunk. Warp 8 allocates tensor memory and
+// one of its threads issues the MMAs; warps 9 and 10 resolve the rows of the
+// even and odd tiles up to kRing - 1 ahead and prefetch them into L2. The
+// partial normalisers of each row (one per head) live in tensor memory.
 //
 // Schedule: the kernel is persistent. The tiles of all sequences form one
-// list (each sequence: its window tiles first, then its entries padded to
-// whole tiles); block c processes the tile range [x0[c], x0[c+1]) that the
-// prep kernel balanced by estimated cost. A block writes one partial result
+// list (each sequence: its entries padded to whole tiles, then its window);
+// block c of G processes tiles [c*T/G, (c+1)*T/G), so every SM gets the same
+// number of tiles whatever the length mix. A block writes one partial result
 // (O, m, l) per sequence it touches into slot b + c, which is unique because
-// b + c increases strictly along the tile list; the merge kernel combines
-// the slots of each sequence.
+// b + c increases strictly along the tile list; the merge kernel combines the
+// slots of each sequence.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -57,65 +40,48 @@ namespace {
 constexpr int kH = 64;          // heads (MMA N)
 constexpr int kD = 512;         // dims
 constexpr int kT = 128;         // items per tile (MMA M of the first product)
-constexpr int kThreads = 512;
+constexpr int kThreads = 352;
 constexpr float kTau = 8.f;     // rescale when a score exceeds the reference by 2^8
 constexpr float kNone = -1e30f; // reference maximum before any item
 
-constexpr int kMmaWarp = 12;
-constexpr int kAddrWarp = 13;   // 13 and 14
-constexpr int kLoadWarp = 15;
-
 // shared memory map (bytes from a 1024-aligned base)
-//   fp8 tiles:  Q3 image [0, 96K), chunk ring slots [96K, 192K), P' [192K, 208K)
-//   bf16 tiles: f16 query image [0, 64K), f16 tile [64K, 192K), P' [192K, 208K)
-constexpr uint32_t kQ3Off = 0;         // 3 terms x 4 chunks x (64 rows x 128 B)
-constexpr uint32_t kQ3Bytes = 98304;
-constexpr uint32_t kRingOff = 98304;   // 3 slots x (2 dim atoms x 128 rows x 128 B)
-constexpr uint32_t kSlotBytes = 32768;
-constexpr uint32_t kQhOff = 0;         // f16 query: 8 dim atoms x 64 rows x 128 B
-constexpr uint32_t kVhOff = 65536;     // f16 tile: 8 dim atoms x 128 rows x 128 B
-constexpr uint32_t kPOff = 196608;     // 128 rows x 128 B (64 heads f16)
-constexpr int kRing = 6;               // tiles of row addresses kept ready
+constexpr uint32_t kVOff = 0;                    // 8 dim atoms x 128 rows x 128 B
+constexpr uint32_t kQOff = 131072;               // 8 dim atoms x 64 rows x 128 B
+constexpr uint32_t kPOff = 196608;               // 128 rows x 128 B (64 heads f16)
+constexpr int kRing = 6;        // tiles of row addresses the address warp keeps ready
 constexpr uint32_t kMetaOff = 212992;                 // [kRing][128] fp32 item scales
-constexpr uint32_t kPtrOff = kMetaOff + kRing * 512;  // [kRing][128] row addresses (null = skip)
-constexpr uint32_t kMrefOff = kPtrOff + kRing * 1024; // [64] reference max per head
-constexpr uint32_t kAlphaOff = kMrefOff + 256;        // [64] rescale factors
-constexpr uint32_t kRedOff = kAlphaOff + 256;         // [4][64] per-warp reductions
-constexpr uint32_t kBarOff = kRedOff + 1024;          // mbarriers
-constexpr uint32_t kMiscOff = kBarOff + 512;          // tmem address, flags, range
-constexpr uint32_t kSmemBytes = kMiscOff + 64 + 1024; // + alignment slack
+constexpr uint32_t kPtrOff = kMetaOff + kRing * 512;  // [kRing][128] item row addresses (null = skip)
+constexpr uint32_t kMrefOff = kPtrOff + kRing * 1024;  // [64] reference max per head
+constexpr uint32_t kAlphaOff = kMrefOff + 256;   // [64] rescale factors
+constexpr uint32_t kRedOff = kAlphaOff + 256;    // [8][32] per-warp reductions
+constexpr uint32_t kBarOff = kRedOff + 1024;     // mbarriers
+constexpr uint32_t kInfoOff = kBarOff + 256;     // [kRing] tile info words
+constexpr uint32_t kMiscOff = kInfoOff + 64;     // tmem address, flags, range
+constexpr uint32_t kSmemBytes = kMiscOff + 64 + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory per block");
-static_assert(kRingOff + 3 * kSlotBytes == kPOff && kVhOff + 8 * 16384 == kPOff, "map");
 
-// tensor memory columns: fp8 tile [0, 128), S [128, 192), O^T 4 x 64 at
-// [192, 448), normalisers [448, 512)
+// TMEM columns: S double buffer [0, 128), O^T 4 x 64 at [128, 384), partial
+// normalisers of each lane (64 heads) at [384, 448)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kVCol = 0;
-constexpr uint32_t kSCol = 128;
-constexpr uint32_t kOCol = 192;
-constexpr uint32_t kLCol = 448;
+constexpr uint32_t kOCol = 128;
+constexpr uint32_t kLCol = 384;
 
 struct Bars {
-  uint64_t addr_ready[kRing];  // 32 arrivals (an address warp)
-  uint64_t addr_free[kRing];   // 384 arrivals (converters and softmax)
-  uint64_t vt_full;            // 256: an fp8 tile is in tensor memory
-  uint64_t qk8_done;           // commit: the fp8 tile's first product has read it
-  uint64_t s_full;             // commit: scores of the next tile ready
-  uint64_t s_free;             // 128: the softmax holds the scores in registers
-  uint64_t p_full;             // 128: P' of the next tile stored
-  uint64_t pv_done;            // commit: the tile's second product is complete
-  uint64_t v_full[3];          // 256: a ring slot holds its f16 chunk
-  uint64_t v_empty[3];         // commit: the M-tile that read the slot is complete
-  uint64_t sv_full;            // 256: a bf16 tile is in shared memory as f16
-  uint64_t ring_free;          // commit before a bf16 tile: every earlier MMA complete
-  uint64_t ser_done;           // commit: a bf16 tile's products are complete
-  uint64_t q3_ready;           // tx: a Q3 image landed
-  uint64_t qh_ready;           // tx: an f16 query image landed
-  uint64_t q_free;             // commit: the last first product of a run read its image
-  uint64_t o_free;             // 128: the segment epilogue has read O^T
-  uint64_t drain;              // commit: every MMA issued
+  uint64_t addr_ready[kRing];
+  uint64_t addr_free[kRing];
+  uint64_t v_full[4];
+  uint64_t v_empty[4];
+  uint64_t s_full[2];
+  uint64_t p_full;
+  uint64_t pv_done;
+  uint64_t q_ready;
+  uint64_t drain;
 };
-static_assert(sizeof(Bars) <= 512, "barrier area");
+static_assert(sizeof(Bars) <= 256, "barrier area");
+
+// tile info word written by the address warp
+constexpr uint32_t kInfoFp8 = 1;    // rows are fp8 codes (else bf16)
+constexpr uint32_t kInfoFirst = 2;  // first tile of a segment (new sequence)
 
 // 2^x on the special-function unit (ftz: results below 2^-126 become 0)
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -135,6 +101,18 @@ __device__ __forceinline__ float from_ordered_key(int k) {
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+__device__ __forceinline__ bool named_and(int id, int n, bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred a, b;\n\t"
+      "setp.ne.u32 a, %1, 0;\n\t"
+      "bar.red.and.pred b, %2, %3, a;\n\t"
+      "selp.u32 %0, 1, 0, b;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)p), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ bool named_or(int id, int n, bool p) {
   uint32_t r;
   asm volatile(
@@ -148,117 +126,44 @@ __device__ __forceinline__ bool named_or(int id, int n, bool p) {
   return r != 0;
 }
 
-// One sequence's items: window tiles first (tokens [w0, L)), then its
-// selected entries padded to whole tiles.
 struct Seq {
-  int L, n_sel, n_win, w0, nwt, nmt;
+  int L, n_sel, n_sel_pad, n_win, w0, n_items;
 };
 
-__device__ __forceinline__ Seq seq_of(const DecodeArgs& a, int b) {
+__device__ __forceinline__ Seq seq_of(const DecodeArgs& a, int b, int32_t* st) {
   Seq s;
-  const int L = min(max(0, a.seq_lens[b]), a.max_len);
-  s.L = L;
-  const int n_vis = max(0, L - a.window_len) / a.ratio;
+  int L = a.seq_lens[b];
+  if (L > a.max_len) {
+    if (threadIdx.x == 0) flag(st, V4KV_DEV_OVERFLOW);
+    L = a.max_len;
+  }
+  s.L = max(0, L);
+  const int n_vis = max(0, s.L - a.window_len) / a.ratio;
   s.n_sel = a.topk ? a.k : n_vis;
-  s.w0 = max(0, L - a.window_len);
-  s.n_win = L - s.w0;
-  s.nwt = (s.n_win + kT - 1) / kT;
-  s.nmt = (s.n_sel + kT - 1) / kT;
+  s.n_sel_pad = (s.n_sel + kT - 1) / kT * kT;
+  s.w0 = max(0, s.L - a.window_len);
+  s.n_win = s.L - s.w0;
+  s.n_items = s.n_sel_pad + s.n_win;
   return s;
 }
 
-__device__ __forceinline__ int tiles_of(const Seq& s) { return s.nwt + s.nmt; }
-
-// tile lt of a sequence holds fp8 codes (else bf16)
-__device__ __forceinline__ bool tile_fp8(const DecodeArgs& a, const Seq& s, int lt) {
-  return (lt < s.nwt ? a.window.dtype : a.main.dtype) == V4KV_FP8_E4M3;
+// one bulk L2 prefetch of `bytes` (a multiple of 16, 16-byte aligned) through
+// the copy engine: a single instruction per row instead of one per cache line
+// keeps the load/store path free for the converters
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-// Estimated cost of a sequence's tiles in the sweep: fp8 tiles 4, bf16 tiles
-// 12 (they run one at a time), and 4 for opening a segment (query copy,
-// epilogue).
-constexpr int kCostFp8 = 4, kCostBf16 = 12, kCostSeg = 4;
-
-__device__ __forceinline__ long long seq_cost(const DecodeArgs& a, const Seq& s) {
-  if (tiles_of(s) == 0) return 0;
-  const int cw = a.window.dtype == V4KV_FP8_E4M3 ? kCostFp8 : kCostBf16;
-  const int cm = a.main.dtype == V4KV_FP8_E4M3 ? kCostFp8 : kCostBf16;
-  return kCostSeg + (long long)s.nwt * cw + (long long)s.nmt * cm;
-}
-
-// tile of sequence s at which `off` cost units (from the sequence's start)
-// fall, clamped to the sequence's tiles
-__device__ __forceinline__ int tile_at_cost(const DecodeArgs& a, const Seq& s, long long off) {
-  const int cw = a.window.dtype == V4KV_FP8_E4M3 ? kCostFp8 : kCostBf16;
-  const int cm = a.main.dtype == V4KV_FP8_E4M3 ? kCostFp8 : kCostBf16;
-  off -= kCostSeg;
-  if (off <= 0) return 0;
-  if (off < (long long)s.nwt * cw) return (int)(off / cw);
-  const long long k = s.nwt + (off - (long long)s.nwt * cw) / cm;
-  return (int)min(k, (long long)(tiles_of(s) - 1));
-}
-
-// Walks a block's tile range: sequence b, tile lt of nt in that sequence.
-struct Cursor {
-  int b, lt, nt;
-  Seq s;
-};
-
-__device__ __forceinline__ void cursor_set(Cursor& c, const DecodeArgs& a, int b, int lt) {
-  c.b = b;
-  c.lt = lt;
-  c.s = seq_of(a, b);
-  c.nt = tiles_of(c.s);
-}
-
-__device__ __forceinline__ void cursor_next(Cursor& c, const DecodeArgs& a) {
-  ++c.lt;
-  while (c.lt >= c.nt && c.b + 1 < a.batch) {
-    ++c.b;
-    c.lt = 0;
-    c.s = seq_of(a, c.b);
-    c.nt = tiles_of(c.s);
-  }
-}
-
-// Where tile i of a block's range stands: its kind and whether it opens or
-// closes its segment (the block's part of one sequence) and its run (the
-// segment's consecutive tiles of one kind, which share a query image).
-struct TileFlags {
-  bool fp8, seg_first, seg_last, run_first, run_last;
-};
-
-__device__ __forceinline__ TileFlags flags_of(const DecodeArgs& a, const Cursor& c, int i,
-                                              int n_tiles) {
-  TileFlags f;
-  f.fp8 = tile_fp8(a, c.s, c.lt);
-  f.seg_first = i == 0 || c.lt == 0;
-  f.seg_last = i == n_tiles - 1 || c.lt == c.nt - 1;
-  f.run_first = f.seg_first || tile_fp8(a, c.s, c.lt - 1) != f.fp8;
-  f.run_last = f.seg_last || tile_fp8(a, c.s, c.lt + 1) != f.fp8;
-  return f;
-}
-
-// mbar_wait for a whole warp: every lane waits and the warp agrees on the
-// result, so that it stays converged for the .sync.aligned instructions after
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, int phase, volatile int* abort) {
-  return __all_sync(0xffffffffu, tc::mbar_wait(bar, (uint32_t)(phase & 1), abort));
-}
-
-__device__ __forceinline__ void prefetch_l2_line(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
-// Address warp: lane l resolves rows l, l+32, l+64, l+96 of tile lt of
-// sequence b into the row-address and scale tables (nullptr for a skipped
-// item), then asks L2 for the rows' cache lines so that the converters'
+// Address warp: lane l resolves rows l, l+32, l+64, l+96 of the tile that
+// starts at item tile0 into the row-address and scale tables (nullptr / 0 for
+// a skipped item), then asks L2 for the rows' cache lines so that the workers'
 // loads find them there. The loads go in phases (top-k indices, block-table
 // entries, scales), each phase's four loads independent of one another, so a
 // tile costs three memory latencies rather than twelve. Problems are flagged
 // as V4KV_DEV_* bits.
-__device__ __forceinline__ void resolve_tile(const DecodeArgs& a, int b, const Seq& s, int lt,
+__device__ __forceinline__ void resolve_tile(const DecodeArgs& a, int b, const Seq& s, int tile0,
                                              int lane, const uint8_t** rp, float* ms) {
-  const bool main_tile = lt >= s.nwt;  // a tile is all entries or all window
+  const bool main_tile = tile0 < s.n_sel_pad;  // a tile is all entries or all window
   const int spb = main_tile ? a.main.spb : a.window.spb;
   const int max_blocks = main_tile ? a.main.max_blocks : a.window.max_blocks;
   const int num_pages = main_tile ? a.main.num_pages : a.window.num_pages;
@@ -272,12 +177,12 @@ __device__ __forceinline__ void resolve_tile(const DecodeArgs& a, int b, const S
   long long j[4];
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
+    const int it = tile0 + lane + 32 * r;
     j[r] = -1;
     if (main_tile) {
-      const int it = (lt - s.nwt) * kT + lane + 32 * r;
       if (it < s.n_sel) j[r] = a.topk ? (long long)a.topk[(size_t)b * a.k + it] : (long long)it;
     } else {
-      const int w = lt * kT + lane + 32 * r;
+      const int w = it - s.n_sel_pad;
       if (w < s.n_win) j[r] = s.w0 + w;
     }
   }
@@ -325,7 +230,7 @@ __device__ __forceinline__ void resolve_tile(const DecodeArgs& a, int b, const S
 #pragma unroll
   for (int r = 0; r < 4; ++r)
     if (p[r])
-      for (int k = 0; k < lines; ++k) prefetch_l2_line(p[r] + 128 * k);
+      prefetch_l2_bulk(p[r], 128 * lines);
   if (err) flag(a.dev_status, err);
 }
 
@@ -339,10 +244,17 @@ __device__ __forceinline__ uint4 ldg_stream(const uint8_t* p) {
 
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
-// 4 fp8 codes (one word, lowest byte first) -> 4 f16 values as two words
-__device__ __forceinline__ void fp8x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  lo = h2u(e4m3x2_to_half2((uint16_t)(w & 0xffffu)));
-  hi = h2u(e4m3x2_to_half2((uint16_t)(w >> 16)));
+// 16 fp8 codes -> 16 f16 values as two 16-byte halves
+__device__ __forceinline__ void fp8x16_to_f16(uint4 raw, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    o[2 * i] = h2u(e4m3x2_to_half2((uint16_t)(w[i] & 0xffffu)));
+    o[2 * i + 1] = h2u(e4m3x2_to_half2((uint16_t)(w[i] >> 16)));
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 // 8 bf16 -> 8 f16 (round to nearest, saturating to the f16 range). `wide`
@@ -354,18 +266,80 @@ __device__ __forceinline__ uint4 bf16x8_to_f16(uint4 raw, bool& wide) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     wide |= (w[i] & 0x7fffu) >= 0x4780u || ((w[i] >> 16) & 0x7fffu) >= 0x4780u;
-    const float x = __uint_as_float(w[i] << 16), y = __uint_as_float(w[i] & 0xffff0000u);
+    const float a = __uint_as_float(w[i] << 16), b = __uint_as_float(w[i] & 0xffff0000u);
     uint32_t r;
-    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(y), "f"(x));
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
     o[i] = r;
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-constexpr uint32_t kQhImg = kH * kD * 2;  // one f16 query image
-constexpr uint32_t kQ3Img = kQ3Bytes;     // one three-term fp8 query image
-constexpr int kMaxSplits = 160;           // sweep blocks at most (the plan caps the grid)
-constexpr int kPrepCache = 2048;          // batches whose prefix sums the prep keeps in shared memory
+
+__device__ __forceinline__ int tiles_of(const Seq& s) {
+  return s.n_sel_pad / kT + (s.n_win + kT - 1) / kT;
+}
+
+// Estimated cost of a sequence's tiles in the sweep (units of a quarter of an
+// fp8 tile): fp8 tiles 4, bf16 tiles 8 (twice the bytes and a slower
+// conversion), and 4 for opening a segment (query copy, epilogue).
+constexpr int kCostFp8 = 4, kCostBf16 = 8, kCostSeg = 4;
+
+__device__ __forceinline__ long long seq_cost(const DecodeArgs& a, const Seq& s) {
+  const int nm = s.n_sel_pad / kT, nw = (s.n_win + kT - 1) / kT;
+  if (nm + nw == 0) return 0;
+  const int cm = a.main.dtype == V4KV_FP8_E4M3 ? kCostFp8 : kCostBf16;
+  const int cw = a.window.dtype == V4KV_FP8_E4M3 ? kCostFp8 : kCostBf16;
+  return kCostSeg + (long long)nm * cm + (long long)nw * cw;
+}
+
+// tile of sequence s at which `off` cost units (from the sequence's start)
+// fall, clamped to the sequence's tiles
+__device__ __forceinline__ int tile_at_cost(const DecodeArgs& a, const Seq& s, long long off) {
+  const int nm = s.n_sel_pad / kT, nw = (s.n_win + kT - 1) / kT;
+  const int cm = a.main.dtype == V4KV_FP8_E4M3 ? kCostFp8 : kCostBf16;
+  const int cw = a.window.dtype == V4KV_FP8_E4M3 ? kCostFp8 : kCostBf16;
+  off -= kCostSeg;
+  if (off <= 0) return 0;
+  if (off < (long long)nm * cm) return (int)(off / cm);
+  const long long k = nm + (off - (long long)nm * cm) / cw;
+  return (int)min(k, (long long)(nm + nw - 1));
+}
+
+// Walks the global tile list: sequence b, tile lt of nt in that sequence.
+struct Cursor {
+  int b, lt, nt;
+  Seq s;
+};
+
+__device__ __forceinline__ void cursor_set(Cursor& c, const DecodeArgs& a, int b, int lt) {
+  c.b = b;
+  c.lt = lt;
+  c.s = seq_of(a, b, nullptr);
+  c.nt = tiles_of(c.s);
+}
+
+__device__ __forceinline__ void cursor_next(Cursor& c, const DecodeArgs& a) {
+  ++c.lt;
+  while (c.lt >= c.nt && c.b + 1 < a.batch) {
+    ++c.b;
+    c.lt = 0;
+    c.s = seq_of(a, c.b, nullptr);
+    c.nt = tiles_of(c.s);
+  }
+}
+
+constexpr uint32_t kQBytes = kH * kD * 2;  // one query image (f16)
+constexpr int kMaxSplits = 160;            // sweep blocks at most (the plan caps the grid)
+constexpr int kPrepCache = 2048;           // batches whose prefix sums the prep keeps in shared memory
+
+// Start the bulk copy of sequence b's query image into shared memory; the
+// copy completes phase by transaction count on `bar`.
+__device__ __forceinline__ void issue_q(const DecodeArgs& a, int b, uint32_t qdst, uint64_t* bar) {
+  tc::mbar_arrive_expect_tx(bar, kQBytes);
+  const uint8_t* src = a.qh + (size_t)b * kQBytes;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) tc::bulk_load(qdst + k * (kQBytes / 4), src + k * (kQBytes / 4), kQBytes / 4, bar);
+}
 
 // Sum 32 per-lane values over the 32 lanes of a warp (reduce-scatter): lane l
 // ends with the sum of value `rev` where the lane bits pick halves (bit 4: 16
@@ -389,75 +363,6 @@ __device__ __forceinline__ int warp_reduce_scatter32(float* v, int lane, float* 
   return base;
 }
 
-// Column (0..31) of a 128-dim chunk of the fp8 tile in tensor memory that
-// holds the four codes of dims d4 .. d4 + 3 (d4 a multiple of 4). A converter
-// thread writes, for p = lane % 4, the words of its 16-byte loads at bytes
-// 16p .. 16p + 15 and 64 + 16p .. 64 + 16p + 15 of the chunk into the
-// columns its .16x256b registers map to (8k + 2p + e for its word 2k + e), so
-// the columns hold the dims in this order; the Q3 image orders its K axis the
-// same way.
-__device__ __forceinline__ int chunk_dim_col(int d4) {
-  const int hi = d4 >= 64;
-  const int rel = d4 - 64 * hi;
-  const int p = rel >> 4;
-  const int j = 4 * hi + ((rel & 15) >> 2);
-  return 8 * (j >> 1) + 2 * p + (j & 1);
-}
-
-// Converter: the codes of rows rA and rB of the tile whose row addresses are
-// rp, each 128-dim chunk c as the 16 registers of a .16x256b store (bytes
-// 16p .. 16p + 15 and 64 + 16p .. 64 + 16p + 15 of the chunk)
-__device__ __forceinline__ void conv_load(const uint8_t* const* rp, int rA, int rB, int p,
-                                          uint32_t (&raw)[4][16]) {
-  const uint8_t* pa = rp[rA];
-  const uint8_t* pb = rp[rB];
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint4 a0 = make_uint4(0, 0, 0, 0), b0 = a0, a1 = a0, b1 = a0;
-    if (pa) {
-      a0 = ldg_stream(pa + 128 * c + 16 * p);
-      b0 = ldg_stream(pa + 128 * c + 64 + 16 * p);
-    }
-    if (pb) {
-      a1 = ldg_stream(pb + 128 * c + 16 * p);
-      b1 = ldg_stream(pb + 128 * c + 64 + 16 * p);
-    }
-    uint32_t* r = raw[c];
-    r[0] = a0.x; r[1] = a0.y; r[2] = a1.x; r[3] = a1.y;
-    r[4] = a0.z; r[5] = a0.w; r[6] = a1.z; r[7] = a1.w;
-    r[8] = b0.x; r[9] = b0.y; r[10] = b1.x; r[11] = b1.y;
-    r[12] = b0.z; r[13] = b0.w; r[14] = b1.z; r[15] = b1.w;
-  }
-}
-
-// Converter: one chunk (16 registers in .16x256b order) of rows rA, rB as f16
-// into ring position gpos, once the second product has released the slot
-__device__ __forceinline__ bool conv_store(uint8_t* sm, Bars* bars, volatile int* abort_flag,
-                                           const uint32_t (&r)[16], int gpos, int rA, int rB, int p) {
-  const int slot = gpos % 3, use = gpos / 3;
-  if (use > 0 && !warp_wait(&bars->v_empty[slot], use - 1, abort_flag)) return false;
-  uint8_t* base = sm + kRingOff + slot * kSlotBytes;
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {     // bytes 16p.. (atom 0) and 64 + 16p.. (atom 1)
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {         // rows rA, rB
-      const int row = rr ? rB : rA;
-      uint32_t h[8];
-#pragma unroll
-      for (int k = 0; k < 2; ++k)            // words 4(2 half + k) + 2 rr + 0/1
-#pragma unroll
-        for (int e = 0; e < 2; ++e)
-          fp8x4_to_f16(r[4 * (2 * half + k) + 2 * rr + e], h[4 * k + 2 * e], h[4 * k + 2 * e + 1]);
-      uint8_t* at = base + half * 16384;
-      *reinterpret_cast<uint4*>(at + tc::sw128_off(row, 2 * p)) = make_uint4(h[0], h[1], h[2], h[3]);
-      *reinterpret_cast<uint4*>(at + tc::sw128_off(row, 2 * p + 1)) = make_uint4(h[4], h[5], h[6], h[7]);
-    }
-  }
-  tc::fence_proxy_async_smem();
-  tc::mbar_arrive(&bars->v_full[slot]);
-  return true;
-}
-
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
@@ -469,6 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   Bars* bars = reinterpret_cast<Bars*>(sm + kBarOff);
   float* meta = reinterpret_cast<float*>(sm + kMetaOff);
   const uint8_t** rowptr = reinterpret_cast<const uint8_t**>(sm + kPtrOff);
+  uint32_t* info = reinterpret_cast<uint32_t*>(sm + kInfoOff);
   float* mref = reinterpret_cast<float*>(sm + kMrefOff);
   float* alpha = reinterpret_cast<float*>(sm + kAlphaOff);
   float* red = reinterpret_cast<float*>(sm + kRedOff);
@@ -484,35 +390,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   if (tid == 0) {
     for (int k = 0; k < kRing; ++k) {
       tc::mbar_init(&bars->addr_ready[k], 32);
-      tc::mbar_init(&bars->addr_free[k], 384);
+      tc::mbar_init(&bars->addr_free[k], 256);
     }
-    tc::mbar_init(&bars->vt_full, 256);
-    tc::mbar_init(&bars->qk8_done, 1);
-    tc::mbar_init(&bars->s_full, 1);
-    tc::mbar_init(&bars->s_free, 128);
-    tc::mbar_init(&bars->p_full, 128);
+    for (int c = 0; c < 4; ++c) {
+      tc::mbar_init(&bars->v_full[c], 256);
+      tc::mbar_init(&bars->v_empty[c], 1);
+    }
+    tc::mbar_init(&bars->s_full[0], 1);
+    tc::mbar_init(&bars->s_full[1], 1);
+    tc::mbar_init(&bars->p_full, 256);
     tc::mbar_init(&bars->pv_done, 1);
-    for (int s = 0; s < 3; ++s) {
-      tc::mbar_init(&bars->v_full[s], 256);
-      tc::mbar_init(&bars->v_empty[s], 1);
-    }
-    tc::mbar_init(&bars->sv_full, 256);
-    tc::mbar_init(&bars->ring_free, 1);
-    tc::mbar_init(&bars->ser_done, 1);
-    tc::mbar_init(&bars->q3_ready, 1);
-    tc::mbar_init(&bars->qh_ready, 1);
-    tc::mbar_init(&bars->q_free, 1);
-    tc::mbar_init(&bars->o_free, 128);
+    tc::mbar_init(&bars->q_ready, 1);
     tc::mbar_init(&bars->drain, 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == kMmaWarp) tc::tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == 8) tc::tmem_alloc(tmem_slot, kTmemCols);
   if (tid < kH) mref[tid] = kNone;
   tc::pdl_wait();  // the tile prefix sums and query images are complete from here on
   tc::pdl_launch_dependents();
 
   // ---- this block's tile range [x0, x1) and the sequence of its first tile
+  // (the prep kernel balanced the ranges by estimated cost)
   if (tid == 0) {
     const int x0 = a.cta_x0[cta], x1 = a.cta_x0[cta + 1];
     const int b0 = x0 < x1 ? a.cta_b0[cta] : a.batch;
@@ -520,6 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
     range[1] = (b0 < a.batch) ? x1 : x0;
     range[2] = b0;
     range[3] = b0 < a.batch ? x0 - a.cum[b0] : 0;
+    if (b0 < a.batch && x0 < x1) issue_q(a, b0, sbase + kQOff, &bars->q_ready);
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -529,195 +429,102 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   const int b0 = range[2], lt0 = range[3];
   const uint32_t tmem = *tmem_slot;
   if (x0 >= x1) {
-    if (warp == kMmaWarp) tc::tmem_free(tmem, kTmemCols);
+    // nothing to do: release tensor memory and leave
+    if (warp == 8) tc::tmem_free(tmem, kTmemCols);
     return;
   }
 
-  if (warp == kAddrWarp || warp == kAddrWarp + 1) {
+  if (warp >= 9) {
     // ======================= address resolution + L2 prefetch, up to kRing - 1 tiles ahead
-    // (warp 13 the even tiles, warp 14 the odd ones)
-    const int aw = warp - kAddrWarp;
+    // (warp 9 the even tiles, warp 10 the odd ones)
+    const int aw = warp - 9;
     Cursor cu;
     cursor_set(cu, a, b0, lt0);
     if (aw) cursor_next(cu, a);
     for (int t = aw; t < n_tiles; t += 2) {
       const int buf = t % kRing;
-      if (t >= kRing && !warp_wait(&bars->addr_free[buf], (t - kRing) / kRing, abort_flag)) break;
-      resolve_tile(a, cu.b, cu.s, cu.lt, lane, rowptr + buf * kT, meta + buf * kT);
+      if (t >= kRing && !tc::mbar_wait(&bars->addr_free[buf], ((t - kRing) / kRing) & 1, abort_flag)) break;
+      if (t > 0 && cu.lt == 0) {
+        // a new sequence starts: pull its query image into L2 as well
+        const uint8_t* qp = a.qh + (size_t)cu.b * kQBytes;
+        if (lane < 4) prefetch_l2_bulk(qp + lane * (kQBytes / 4), kQBytes / 4);
+      }
+      const int tile0 = cu.lt * kT;
+      resolve_tile(a, cu.b, cu.s, tile0, lane, rowptr + buf * kT, meta + buf * kT);
+      if (lane == 0) {
+        const bool main_tile = tile0 < cu.s.n_sel_pad;
+        const bool fp8 = (main_tile ? a.main.dtype : a.window.dtype) == V4KV_FP8_E4M3;
+        info[buf] = (fp8 ? kInfoFp8 : 0u) | ((t == 0 || cu.lt == 0) ? kInfoFirst : 0u);
+      }
       __syncwarp();
       tc::mbar_arrive(&bars->addr_ready[buf]);
       cursor_next(cu, a);
       cursor_next(cu, a);
     }
-  } else if (warp == kLoadWarp) {
-    // ======================= query images: one per run of same-kind tiles
-    // (Q3 for fp8 runs, the f16 image for bf16 runs), each copied once the
-    // run before it has finished reading the region
-    Cursor cu;
-    cursor_set(cu, a, b0, lt0);
-    int runs = 0, n_ser = 0, last3 = -1, lasth = -1;
-    bool ok = true;
-    for (int i = 0; i < n_tiles && ok; ++i) {
-      const TileFlags f = flags_of(a, cu, i, n_tiles);
-      if (f.run_first) {
-        if (runs > 0) ok = warp_wait(&bars->q_free, runs - 1, abort_flag);
-        // the Q3 image also covers the first chunk of the f16 tile area
-        if (ok && f.fp8 && n_ser > 0) ok = warp_wait(&bars->ser_done, n_ser - 1, abort_flag);
-        if (!ok) break;
-        if (lane == 0) {
-          if (f.fp8) {
-            tc::mbar_arrive_expect_tx(&bars->q3_ready, kQ3Img);
-            const uint8_t* src = a.q3 + (size_t)cu.b * kQ3Img;
-            for (int k = 0; k < 6; ++k)
-              tc::bulk_load(sbase + kQ3Off + k * (kQ3Img / 6), src + k * (kQ3Img / 6), kQ3Img / 6,
-                            &bars->q3_ready);
-          } else {
-            tc::mbar_arrive_expect_tx(&bars->qh_ready, kQhImg);
-            const uint8_t* src = a.qh + (size_t)cu.b * kQhImg;
-            for (int k = 0; k < 4; ++k)
-              tc::bulk_load(sbase + kQhOff + k * (kQhImg / 4), src + k * (kQhImg / 4), kQhImg / 4,
-                            &bars->qh_ready);
-          }
-        }
-        if (f.fp8) ++last3; else ++lasth;
-        ++runs;
-      }
-      if (!f.fp8) ++n_ser;
-      cursor_next(cu, a);
-    }
-    // every copy has landed before shared memory is released (normally long
-    // since; after an abort one may still be in flight)
-    volatile int never = 0;
-    if (last3 >= 0 && !tc::mbar_wait(&bars->q3_ready, last3 & 1, &never)) flag(a.dev_status, V4KV_DEV_TIMEOUT);
-    if (lasth >= 0 && !tc::mbar_wait(&bars->qh_ready, lasth & 1, &never)) flag(a.dev_status, V4KV_DEV_TIMEOUT);
-    if (!ok) {
-      *abort_flag = 1;
-      flag(a.dev_status, V4KV_DEV_TIMEOUT);
-    }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == 8) {
     // ======================= MMA issuer
     // The whole warp runs the loop, so descriptors, addresses and wait results
     // stay warp-uniform; one lane, elected once, issues every MMA and commit
     // (a commit tracks the MMAs of the thread that issues it).
     const bool leader = tc::elect_one();
     const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
-    const uint32_t id8 = tc::idesc_f16(128, kH, 0, 0);   // e4m3 x e4m3 -> f32 (format fields 0)
     const uint32_t iq = tc::idesc_f16(128, kH, 0, 0);
     const uint32_t ip = tc::idesc_f16(128, kH, 1, 1);
-    const uint64_t q3_desc = tc::sw128_desc(sbase + kQ3Off, 16, 1024);     // Q3 terms, K-major
-    const uint64_t qh_desc = tc::sw128_desc(sbase + kQhOff, 16, 1024);     // f16 Q, K-major
-    const uint64_t vk_desc = tc::sw128_desc(sbase + kVhOff, 16, 1024);     // f16 tile, K-major
-    const uint64_t vm_desc = tc::sw128_desc(sbase + kVhOff, 16384, 1024);  // f16 tile^T, MN-major
-    const uint64_t rm_desc = tc::sw128_desc(sbase + kRingOff, 16384, 1024);  // ring slot^T, MN-major
-    const uint64_t p_desc = tc::sw128_desc(sbase + kPOff, 0, 1024);        // P^T, MN-major
-    Cursor cu;
-    cursor_set(cu, a, b0, lt0);
+    // descriptors at the operands' bases; a step adds its byte offset / 16
+    const uint64_t vk_desc = tc::sw128_desc(sbase + kVOff, 16, 1024);     // V, K-major
+    const uint64_t qk_desc = tc::sw128_desc(sbase + kQOff, 16, 1024);     // Q, K-major
+    const uint64_t vm_desc = tc::sw128_desc(sbase + kVOff, 16384, 1024);  // V^T, MN-major
+    const uint64_t p_desc = tc::sw128_desc(sbase + kPOff, 0, 1024);       // P^T, MN-major
     bool ok = true;
-    int n8 = 0, nser = 0, nrun3 = 0, nrunh = 0, nseg = 0;
-    int pend = -1, pend_chunk = 0, pend_seg = 0;
-    bool pend_first = false;
-    auto wait = [&](uint64_t* bar, int phase) -> bool {
-      return __all_sync(0xffffffffu, tc::mbar_wait_spin(bar, phase & 1, abort_flag));
-    };
-    // second product of fp8 tile j (its chunks at ring positions g0 .. g0 + 3)
-    auto pv8 = [&](int j, int g0, bool first, int seg) -> bool {
-      if (!wait(&bars->p_full, j)) return false;
-      if (first && seg > 0 && !wait(&bars->o_free, seg - 1)) return false;
-      for (int mt = 0; mt < 4; ++mt) {
-        const int g = g0 + mt, slot = g % 3;
-        if (!wait(&bars->v_full[slot], g / 3)) return false;
+    int seg = 0;
+    for (int i = 0; i < n_tiles && ok; ++i) {
+      const uint32_t par = i & 1;
+      const uint32_t s_col = (uint32_t)(i & 1) * kH;
+      bool first = i == 0;
+      for (int c = 0; c < 4 && ok; ++c) {
+        ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->v_full[c], par, abort_flag));
+        if (!ok) break;
+        if (c == 0) {
+          // the converters read this tile's info word before arriving
+          first = (info[i % kRing] & kInfoFirst) != 0;
+          if (first) {
+            // the segment's query image has landed in shared memory
+            ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->q_ready, seg & 1, abort_flag));
+            if (!ok) break;
+            ++seg;
+          }
+        }
         tc::tc_fence_after();
         if (leader) {
+#pragma unroll
+          for (int k8 = 0; k8 < 8; ++k8) {
+            const int kk = 8 * c + k8;  // 16-dim step: atom kk/4, 32-byte column kk%4
+            tc::mma_f16(tm + s_col, vk_desc + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
+                        qk_desc + (uint64_t)((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), iq,
+                        kk > 0 ? 1u : 0u);
+          }
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (leader) tc::mma_commit(&bars->s_full[i & 1]);
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->p_full, par, abort_flag));
+      if (!ok) break;
+      tc::tc_fence_after();
+      if (leader) {
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            tc::mma_f16(tm + kOCol + kH * mt,
-                        rm_desc + (uint64_t)((slot * kSlotBytes + kk * 2048) >> 4),
+            tc::mma_f16(tm + kOCol + kH * mt, vm_desc + (uint64_t)((2 * mt * 16384 + kk * 2048) >> 4),
                         p_desc + (uint64_t)((kk * 2048) >> 4), ip, (!first || kk > 0) ? 1u : 0u);
-          tc::mma_commit(&bars->v_empty[slot]);
+          tc::mma_commit(&bars->v_empty[mt]);
         }
-        __syncwarp();
+        tc::mma_commit(&bars->pv_done);
       }
-      if (leader) tc::mma_commit(&bars->pv_done);
       __syncwarp();
-      return true;
-    };
-    for (int i = 0; i < n_tiles && ok; ++i) {
-      const TileFlags f = flags_of(a, cu, i, n_tiles);
-      if (f.seg_first && i > 0) ++nseg;
-      if (f.fp8) {
-        // ---- first product of fp8 tile i: A = codes in tensor memory, B = Q3 terms
-        ok = wait(&bars->vt_full, n8);
-        if (ok && f.run_first) ok = wait(&bars->q3_ready, nrun3);
-        if (ok && i > 0) ok = wait(&bars->s_free, i - 1);
-        if (!ok) break;
-        tc::tc_fence_after();
-        if (leader) {
-#pragma unroll 1
-          for (int ks = 0; ks < 16; ++ks) {
-#pragma unroll
-            for (int term = 0; term < 3; ++term)
-              tc::mma_f8_ts(tm + kSCol, tm + kVCol + 8 * ks,
-                            q3_desc + (uint64_t)(((term * 4 + (ks >> 2)) * 8192 + (ks & 3) * 32) >> 4),
-                            id8, (ks > 0 || term > 0) ? 1u : 0u);
-          }
-          tc::mma_commit(&bars->s_full);
-          tc::mma_commit(&bars->qk8_done);
-          if (f.run_last) tc::mma_commit(&bars->q_free);
-        }
-        __syncwarp();
-        if (f.run_first) ++nrun3;
-        // ---- second product of the previous fp8 tile
-        if (pend >= 0 && !(ok = pv8(pend, pend_chunk, pend_first, pend_seg))) break;
-        pend = i;
-        pend_chunk = 4 * n8;
-        pend_first = f.seg_first;
-        pend_seg = nseg;
-        ++n8;
-      } else {
-        // ---- bf16 tile: drain, then both products from shared memory
-        if (pend >= 0) {
-          if (!(ok = pv8(pend, pend_chunk, pend_first, pend_seg))) break;
-          pend = -1;
-        }
-        if (leader) tc::mma_commit(&bars->ring_free);
-        __syncwarp();
-        ok = wait(&bars->sv_full, nser);
-        if (ok && f.run_first) ok = wait(&bars->qh_ready, nrunh);
-        if (ok && i > 0) ok = wait(&bars->s_free, i - 1);
-        if (!ok) break;
-        tc::tc_fence_after();
-        if (leader) {
-#pragma unroll 4
-          for (int kk = 0; kk < 32; ++kk)
-            tc::mma_f16(tm + kSCol, vk_desc + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
-                        qh_desc + (uint64_t)((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), iq,
-                        kk > 0 ? 1u : 0u);
-          tc::mma_commit(&bars->s_full);
-          if (f.run_last) tc::mma_commit(&bars->q_free);
-        }
-        __syncwarp();
-        if (f.run_first) ++nrunh;
-        ok = wait(&bars->p_full, i);
-        if (ok && f.seg_first && nseg > 0) ok = wait(&bars->o_free, nseg - 1);
-        if (!ok) break;
-        tc::tc_fence_after();
-        if (leader) {
-#pragma unroll
-          for (int mt = 0; mt < 4; ++mt) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              tc::mma_f16(tm + kOCol + kH * mt, vm_desc + (uint64_t)((2 * mt * 16384 + kk * 2048) >> 4),
-                          p_desc + (uint64_t)((kk * 2048) >> 4), ip, (!f.seg_first || kk > 0) ? 1u : 0u);
-          }
-          tc::mma_commit(&bars->pv_done);
-          tc::mma_commit(&bars->ser_done);
-        }
-        __syncwarp();
-        ++nser;
-      }
-      cursor_next(cu, a);
     }
-    if (ok && pend >= 0) ok = pv8(pend, pend_chunk, pend_first, pend_seg);
     if (!ok && leader) {
       *abort_flag = 1;
       flag(a.dev_status, V4KV_DEV_TIMEOUT);
@@ -729,161 +536,127 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
     volatile int never = 0;
     if (!tc::mbar_wait(&bars->drain, 0, &never) && leader) flag(a.dev_status, V4KV_DEV_TIMEOUT);
     __syncwarp();
-  } else if (warp >= 4) {
-    // ======================= converters (warps 4-11)
-    // Warp (q, g) = (warp % 4, (warp - 4) / 4) owns tile rows R0 .. R0 + 15,
-    // R0 = 32q + 16g. In the .16x256b shape, lane l holds rows R0 + l/4 and
-    // R0 + l/4 + 8 and, of every 128-dim chunk, the bytes 16p .. 16p + 15 and
-    // 64 + 16p .. 64 + 16p + 15 (p = l % 4): 64 contiguous bytes of a row per
-    // warp load, the same 16 bytes per thread in registers, tensor memory and
-    // the f16 ring.
-    const int q = warp & 3, g = (warp - 4) >> 2;
-    const int R0 = 32 * q + 16 * g;
-    const int rA = R0 + (lane >> 2), rB = rA + 8, p = lane & 3;
-    const uint32_t tl = tmem + ((uint32_t)R0 << 16);
-    uint32_t raw[4][16];     // a tile's codes, per chunk in the .16x256b register order
-    uint32_t held[16];       // chunk 3 of the last fp8 tile, read back from tensor memory
-    int held_g = -1;         // its ring position (-1: none)
-    bool have_raw = false;
-    bool wide = false;       // a bf16 value outside the f16 range was clamped
-    bool ok = true;
-    int n8 = 0, nser = 0;
-    bool ser_pending = false;  // a bf16 tile has used the ring area since the last ring write
-
-    Cursor cu;
-    cursor_set(cu, a, b0, lt0);
-    for (int i = 0; i < n_tiles && ok; ++i) {
-      const TileFlags f = flags_of(a, cu, i, n_tiles);
-      if (f.fp8) {
-        if (!have_raw) {
-          if (!(ok = warp_wait(&bars->addr_ready[i % kRing], i / kRing, abort_flag))) break;
-          conv_load(rowptr + (i % kRing) * kT, rA, rB, p, raw);
-        }
-        // the tensor-memory tile is free once the previous fp8 tile's first
-        // product has read it (this warp read its own rows back already)
-        if (n8 > 0 && !(ok = warp_wait(&bars->qk8_done, n8 - 1, abort_flag))) break;
-        tc::tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tc::tmem_st16x256_x4(tl + kVCol + 32 * c, raw[c]);
-        tc::tmem_wait_st();
-        tc::tc_fence_before();
-        tc::mbar_arrive(&bars->vt_full);
-        tc::mbar_arrive(&bars->addr_free[i % kRing]);
-        have_raw = false;
-        // the next fp8 tile's codes fly while this one is converted
-        if (i + 1 < n_tiles) {
-          Cursor nx = cu;
-          cursor_next(nx, a);
-          if (tile_fp8(a, nx.s, nx.lt)) {
-            if (!(ok = warp_wait(&bars->addr_ready[(i + 1) % kRing], (i + 1) / kRing, abort_flag))) break;
-            conv_load(rowptr + ((i + 1) % kRing) * kT, rA, rB, p, raw);
-            have_raw = true;
-          }
-        }
-        if (ser_pending) {
-          if (!(ok = warp_wait(&bars->ser_done, nser - 1, abort_flag))) break;
-          ser_pending = false;
-        }
-        // the previous fp8 tile's last chunk (its slot frees when the second
-        // product of that tile has read its first chunk)
-        if (held_g >= 0) {
-          if (!(ok = conv_store(sm, bars, abort_flag, held, held_g, rA, rB, p))) break;
-          held_g = -1;
-        }
-        // chunks 0-2 of this tile from tensor memory into the ring, chunk 3
-        // into registers (so that the next tile may overwrite tensor memory)
-        for (int c = 0; c < 3 && ok; ++c) {
-          uint32_t r[16];
-          tc::tmem_ld16x256_x4(tl + kVCol + 32 * c, r);
-          tc::tmem_wait_ld();
-          ok = conv_store(sm, bars, abort_flag, r, 4 * n8 + c, rA, rB, p);
-        }
-        if (!ok) break;
-        tc::tmem_ld16x256_x4(tl + kVCol + 96, held);
-        tc::tmem_wait_ld();
-        tc::tc_fence_before();
-        held_g = 4 * n8 + 3;
-        ++n8;
-      } else {
-        // ---- bf16 tile into the f16 area, once every earlier MMA has completed
-        if (held_g >= 0) {
-          if (!(ok = conv_store(sm, bars, abort_flag, held, held_g, rA, rB, p))) break;
-          held_g = -1;
-        }
-        if (!(ok = warp_wait(&bars->ring_free, nser, abort_flag))) break;
-        if (!(ok = warp_wait(&bars->addr_ready[i % kRing], i / kRing, abort_flag))) break;
-        const uint8_t* const* rp = rowptr + (i % kRing) * kT;
-        // lane covers rows R0 + 2r + lane/16 (r = 0..7), 16 bytes at
-        // 16 * (lane % 16) of each 256-byte (128-dim) chunk
-        const int part = lane & 15;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint4 v[8];
-#pragma unroll
-          for (int r = 0; r < 8; ++r) {
-            const uint8_t* pr = rp[R0 + 2 * r + (lane >> 4)];
-            v[r] = pr ? ldg_stream(pr + 256 * c + 16 * part) : make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int r = 0; r < 8; ++r) {
-            const uint32_t vr = R0 + 2 * r + (lane >> 4);
-            const uint32_t atom = 2 * c + (part >> 3);
-            *reinterpret_cast<uint4*>(sm + kVhOff + atom * 16384 + tc::sw128_off(vr, part & 7)) =
-                bf16x8_to_f16(v[r], wide);
-          }
-        }
-        tc::fence_proxy_async_smem();
-        tc::mbar_arrive(&bars->sv_full);
-        tc::mbar_arrive(&bars->addr_free[i % kRing]);
-        ++nser;
-        ser_pending = true;
-      }
-      cursor_next(cu, a);
-    }
-    if (ok && held_g >= 0) ok = conv_store(sm, bars, abort_flag, held, held_g, rA, rB, p);
-    if (!ok) {
-      *abort_flag = 1;
-      flag(a.dev_status, V4KV_DEV_TIMEOUT);
-    }
-    if (__any_sync(0xffffffffu, wide) && lane == 0) flag(a.dev_status, V4KV_DEV_RANGE);
   } else {
-    // ======================= softmax (warps 0-3)
-    // Thread (warp q, lane l) owns tile row 32q + l (its TMEM lane) for all 64
-    // heads; its partial normalisers live in tensor memory (columns kLCol ..).
-    // The four warps meet at named barrier 1 after every bounded wait, so they
-    // leave together when one gives up.
-    const int q = warp;
-    const int row = 32 * q + lane;
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-    const uint32_t l_addr = lane_base + kLCol;
+    // ======================= workers (warps 0-7): softmax and gather + convert
+    // Softmax: thread (warp w, lane l) owns tile row j = 32 (w % 4) + l (its
+    // TMEM lane) and heads 32 hh .. 32 hh + 31 (hh = w / 4); its partial
+    // normalisers live in tensor memory (columns kLCol + 32 hh ..). Conversion: warp w writes rows 16w ..
+    // 16w + 15 of every V chunk. Per tile: softmax(i), then the conversion of
+    // tile i + 1 as the second product of tile i frees each V chunk; the codes
+    // of tile i + 1 are loaded before softmax(i).
+    const int hh = warp >> 2;
+    const int row = 32 * (warp & 3) + lane;   // tile row = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    uint4 rawv[4][4];
+    const uint32_t l_addr = lane_base + kLCol + 32 * hh;
     {
       uint32_t z[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) z[e] = 0u;
       tc::tmem_st32(l_addr, z);
-      tc::tmem_st32(l_addr + 32, z);
       tc::tmem_wait_st();
+    }
+    float k0 = a.qk0[b0];
+    int q_issued = 1;  // query copies started by this thread (tid 0 only)
+    bool wide = false; // a bf16 value outside the f16 range was clamped
+    bool ok = true;
+
+    // fp8 rows: lane covers rows 16w + 4r + lane/8 (r = 0..3), 16 bytes at
+    // 16*(lane%8) of each 128-byte dim chunk
+    auto load_fp8 = [&](int t) {
+      const uint8_t** rp = rowptr + (t % kRing) * kT;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const uint8_t* p = rp[16 * warp + 4 * r + (lane >> 3)];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          rawv[c][r] = p ? ldg_stream(p + 128 * c + 16 * (lane & 7)) : make_uint4(0, 0, 0, 0);
+      }
+    };
+    // convert tile t into the V buffer; chunk c waits for the second product of
+    // tile t - 1 to release it (v_empty)
+    auto convert = [&](int t, bool fp8) -> bool {
+      if (fp8) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (t > 0 && !tc::mbar_wait(&bars->v_empty[c], (t - 1) & 1, abort_flag)) return false;
+          const int part = lane & 7;                 // 16-dim piece within the chunk
+          const uint32_t atom = 2 * c + (part >> 2);
+          const uint32_t q = 2 * (part & 3);
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const uint32_t vr = 16 * warp + 4 * r + (lane >> 3);
+            uint4 lo, hi;
+            fp8x16_to_f16(rawv[c][r], lo, hi);
+            uint8_t* base = sm + kVOff + atom * 16384;
+            if (part & 4) {
+              *reinterpret_cast<uint4*>(base + tc::sw128_off(vr, q + 1)) = hi;
+              *reinterpret_cast<uint4*>(base + tc::sw128_off(vr, q)) = lo;
+            } else {
+              *reinterpret_cast<uint4*>(base + tc::sw128_off(vr, q)) = lo;
+              *reinterpret_cast<uint4*>(base + tc::sw128_off(vr, q + 1)) = hi;
+            }
+          }
+          tc::fence_proxy_async_smem();
+          tc::mbar_arrive(&bars->v_full[c]);
+        }
+      } else {
+        // bf16 rows: lane covers rows 16w + 2r + lane/16 (r = 0..7), 16 bytes at
+        // 16*(lane%16) of each 256-byte dim chunk; chunk c + 1 is loaded while
+        // chunk c is converted (the two buffers reuse the code registers)
+        const uint8_t** rp = rowptr + (t % kRing) * kT;
+#define V4KV_RB(k, r) rawv[2 * (k) + ((r) >> 2)][(r) & 3]
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const uint8_t* p = rp[16 * warp + 2 * r + (lane >> 4)];
+          V4KV_RB(0, r) = p ? ldg_stream(p + 16 * (lane & 15)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c + 1 < 4) {
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+              const uint8_t* p = rp[16 * warp + 2 * r + (lane >> 4)];
+              V4KV_RB((c + 1) & 1, r) = p ? ldg_stream(p + 256 * (c + 1) + 16 * (lane & 15)) : make_uint4(0, 0, 0, 0);
+            }
+          }
+          if (t > 0 && !tc::mbar_wait(&bars->v_empty[c], (t - 1) & 1, abort_flag)) return false;
+          const int part = lane & 15;                // 8-dim piece within the chunk
+          const uint32_t atom = 2 * c + (part >> 3);
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            const uint32_t vr = 16 * warp + 2 * r + (lane >> 4);
+            *reinterpret_cast<uint4*>(sm + kVOff + atom * 16384 + tc::sw128_off(vr, part & 7)) =
+                bf16x8_to_f16(V4KV_RB(c & 1, r), wide);
+          }
+          tc::fence_proxy_async_smem();
+          tc::mbar_arrive(&bars->v_full[c]);
+        }
+#undef V4KV_RB
+      }
+      return true;
+    };
+
+    // tile 0
+    {
+      ok = tc::mbar_wait(&bars->addr_ready[0], 0, abort_flag);
+      const bool fp8 = ok && (info[0] & kInfoFp8) != 0;
+      if (ok && fp8) load_fp8(0);
+      if (ok) ok = convert(0, fp8);
     }
     Cursor cu;
     cursor_set(cu, a, b0, lt0);
-    bool ok = true;
+    bool seg_first = true;  // the current tile opens a segment
     for (int i = 0; i < n_tiles && ok; ++i) {
-      const TileFlags f = flags_of(a, cu, i, n_tiles);
-      const float k0 = f.fp8 ? a.qk08[cu.b] : a.qk0[cu.b];
-      ok = tc::mbar_wait(&bars->addr_ready[i % kRing], (i / kRing) & 1, abort_flag) &&
-           tc::mbar_wait_spin(&bars->s_full, i & 1, abort_flag, 32);
-      ok = !named_or(1, 128, !ok);
+      const bool seg_last = i == n_tiles - 1 || cu.lt == cu.nt - 1;
+      // S(i) complete implies PV(i-1) complete (the MMAs run in issue order),
+      // so waiting for pv_done(i-1) here costs nothing and frees P and O^T
+      ok = ok && tc::mbar_wait_spin(&bars->s_full[i & 1], (i >> 1) & 1, abort_flag, 32) &&
+           (i == 0 || tc::mbar_wait(&bars->pv_done, (i - 1) & 1, abort_flag));
+      // the eight worker warps leave together (they meet at named barriers)
+      ok = named_and(1, 256, ok);
       if (!ok) break;
       tc::tc_fence_after();
-      float u[64];  // scores in log2 units including log2|ks|, then u - m_ref
-      {
-        uint32_t* r = reinterpret_cast<uint32_t*>(u);
-        tc::tmem_ld32(lane_base + kSCol, r);
-        tc::tmem_ld32(lane_base + kSCol + 32, r + 32);
-        tc::tmem_wait_ld();
-      }
-      tc::tc_fence_before();
-      tc::mbar_arrive(&bars->s_free);
       // a row is an item when its address was resolved; its scale may be any
       // value (value = code * scale): |scale| enters the exponent, its sign the
       // weight P', and a zero scale gives a zero-valued item that still counts
@@ -895,59 +668,81 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       const float lk = !valid ? -INFINITY : (aks > 0.f ? __log2f(aks) : 0.f);
       const float inv_k = !valid ? 0.f : (aks > 0.f ? __frcp_rn(aks) : 1.f);
       const float sgn = (valid && ks != 0.f) ? copysignf(1.f, ks) : 0.f;
+      // u = score in log2 units including log2 ks; d = u - m_ref (in place)
+      float d[32];
+      const uint32_t s_addr = lane_base + (uint32_t)(i & 1) * kH + 32 * hh;
+      {
+        uint32_t r32[32];
+        tc::tmem_ld32(s_addr, r32);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 32; ++h) d[h] = fmaf(__uint_as_float(r32[h]), cj, lk);
+      }
+      if (seg_last && i + 1 < n_tiles && tid == 0) {
+        // QK(i) is complete (S(i) was read), so Q is free: copy the next
+        // segment's query image while the rest of this tile runs
+        Cursor nx = cu;
+        cursor_next(nx, a);
+        issue_q(a, nx.b, sbase + kQOff, &bars->q_ready);
+        ++q_issued;
+      }
       float dmax = -INFINITY;
       {
-        const float4* mr4 = reinterpret_cast<const float4*>(mref);
+        const float4* mr4 = reinterpret_cast<const float4*>(mref + 32 * hh);
 #pragma unroll
-        for (int h4 = 0; h4 < 16; ++h4) {
+        for (int h4 = 0; h4 < 8; ++h4) {
           const float4 m4 = mr4[h4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) u[4 * h4 + e] = fmaf(u[4 * h4 + e], cj, lk);
-          dmax = fmaxf(dmax, fmaxf(fmaxf(u[4 * h4] - m4.x, u[4 * h4 + 1] - m4.y),
-                                   fmaxf(u[4 * h4 + 2] - m4.z, u[4 * h4 + 3] - m4.w)));
+          d[4 * h4] -= m4.x;
+          d[4 * h4 + 1] -= m4.y;
+          d[4 * h4 + 2] -= m4.z;
+          d[4 * h4 + 3] -= m4.w;
+          dmax = fmaxf(dmax, fmaxf(fmaxf(d[4 * h4], d[4 * h4 + 1]), fmaxf(d[4 * h4 + 2], d[4 * h4 + 3])));
         }
       }
-      bool waited = false;  // pv_done of tile i - 1 has been waited for
-      if (named_or(1, 128, dmax > kTau)) {
-        // rare: raise the reference of every head to its running maximum; the
-        // earlier tiles' products must be complete before O^T is rescaled
-        if (i > 0) {
-          ok = tc::mbar_wait(&bars->pv_done, (i - 1) & 1, abort_flag);
-          ok = !named_or(1, 128, !ok);
-          if (!ok) break;
-          waited = true;
-          tc::tc_fence_after();
+      if (named_or(1, 256, dmax > kTau)) {
+        // rare: raise the reference of every head to its running maximum.
+        // u is recomputed from S (still in tensor memory) to keep it exact.
+        {
+          uint32_t r32[32];
+          tc::tmem_ld32(s_addr, r32);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < 32; ++h) d[h] = fmaf(__uint_as_float(r32[h]), cj, lk);
         }
 #pragma unroll
-        for (int h = 0; h < 64; ++h) {
-          const int wm = __reduce_max_sync(0xffffffffu, ordered_key(u[h]));
-          if (lane == 0) red[q * 64 + h] = from_ordered_key(wm);
+        for (int h = 0; h < 32; ++h) {
+          const int wm = __reduce_max_sync(0xffffffffu, ordered_key(d[h]));
+          if (lane == 0) red[warp * 32 + h] = from_ordered_key(wm);
         }
-        named_sync(1, 128);
+        named_sync(1, 256);
         if (tid < kH) {
+          const int half = tid >> 5, hx = tid & 31;
           const float old = mref[tid];
           float nm = old;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) nm = fmaxf(nm, red[64 * w + tid]);
+          for (int w = 0; w < 4; ++w) nm = fmaxf(nm, red[(4 * half + w) * 32 + hx]);
           alpha[tid] = exp2f(old - nm);
           mref[tid] = nm;
         }
-        named_sync(1, 128);
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
+        named_sync(1, 256);
+#pragma unroll
+        for (int h = 0; h < 32; ++h) d[h] -= mref[32 * hh + h];
+        {
           uint32_t lv[32];
-          tc::tmem_ld32(l_addr + 32 * half, lv);
+          tc::tmem_ld32(l_addr, lv);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int h = 0; h < 32; ++h)
-            lv[h] = __float_as_uint(__uint_as_float(lv[h]) * alpha[32 * half + h]);
-          tc::tmem_st32(l_addr + 32 * half, lv);
+            lv[h] = __float_as_uint(__uint_as_float(lv[h]) * alpha[32 * hh + h]);
+          tc::tmem_st32(l_addr, lv);
+          tc::tmem_wait_st();
         }
-        tc::tmem_wait_st();
-        if (!f.seg_first) {
-          // O^T rows of this lane (dims 128 mt + row) times alpha per head column
+        if (!seg_first) {
+          // O^T rows of this lane (dims 128 mt + row, mt = 2hh, 2hh + 1) times
+          // alpha per head column
 #pragma unroll 1
-          for (int mt = 0; mt < 4; ++mt) {
+          for (int m2 = 0; m2 < 2; ++m2) {
+            const int mt = 2 * hh + m2;
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
               uint32_t r32[32];
@@ -962,62 +757,67 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
           }
           tc::tmem_wait_st();
         }
-        named_sync(1, 128);  // red and alpha are free again
       }
-      // P' row of this item (64 heads f16, eight 16-byte chunks of the swizzled
-      // MN-major row) once the previous tile's second product has read P'
-      if (i > 0 && !waited) {
-        ok = tc::mbar_wait(&bars->pv_done, (i - 1) & 1, abort_flag);
-        ok = !named_or(1, 128, !ok);
-        if (!ok) break;
-      }
-      {
-        const float4* mr4 = reinterpret_cast<const float4*>(mref);
+      // P' row of this item: heads 32 hh .. 32 hh + 31 in f16, 8 heads per
+      // 16-byte chunk (chunks 4 hh .. 4 hh + 3 of the MN-major swizzled row);
+      // d keeps the fp32 weights for the normaliser update after the arrive
 #pragma unroll
-        for (int h4 = 0; h4 < 16; ++h4) {
-          const float4 m4 = mr4[h4];
-          u[4 * h4] = fast_exp2(u[4 * h4] - m4.x);
-          u[4 * h4 + 1] = fast_exp2(u[4 * h4 + 1] - m4.y);
-          u[4 * h4 + 2] = fast_exp2(u[4 * h4 + 2] - m4.z);
-          u[4 * h4 + 3] = fast_exp2(u[4 * h4 + 3] - m4.w);
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int h = 8 * c + 2 * e;
-          pk[e] = h2u(__floats2half2_rn(sgn * u[h], sgn * u[h + 1]));
+          d[h] = fast_exp2(d[h]);
+          d[h + 1] = fast_exp2(d[h + 1]);
+          pk[e] = h2u(__floats2half2_rn(sgn * d[h], sgn * d[h + 1]));
         }
-        *reinterpret_cast<uint4*>(sm + kPOff + tc::sw128_off(row, c)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(sm + kPOff + tc::sw128_off(row, 4 * hh + c)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       tc::mbar_arrive(&bars->p_full);
       tc::mbar_arrive(&bars->addr_free[i % kRing]);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      // the next tile's codes (fp8) fly while PV(i) runs. They are requested
+      // only now: a barrier or a release arrival waits for every load this
+      // thread has in flight, so loads issued before the softmax would hold
+      // it back by a memory latency.
+      bool nxt_fp8 = false;
+      if (i + 1 < n_tiles) {
+        ok = tc::mbar_wait(&bars->addr_ready[(i + 1) % kRing], ((i + 1) / kRing) & 1, abort_flag);
+        ok = named_and(1, 256, ok);  // the workers leave together
+        if (!ok) break;
+        nxt_fp8 = (info[(i + 1) % kRing] & kInfoFp8) != 0;
+        if (nxt_fp8) load_fp8(i + 1);
+      }
+      {
         uint32_t lv[32];
-        tc::tmem_ld32(l_addr + 32 * half, lv);
+        tc::tmem_ld32(l_addr, lv);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < 32; ++h)
-          lv[h] = __float_as_uint(fmaf(u[32 * half + h], inv_k, __uint_as_float(lv[h])));
-        tc::tmem_st32(l_addr + 32 * half, lv);
+        for (int h = 0; h < 32; ++h) lv[h] = __float_as_uint(fmaf(d[h], inv_k, __uint_as_float(lv[h])));
+        tc::tmem_st32(l_addr, lv);
+        tc::tmem_wait_st();
       }
-      tc::tmem_wait_st();
+      // convert tile i + 1 as PV(i) frees the V chunks (before the epilogue,
+      // so that QK(i + 1) overlaps it; PV(i + 1) cannot start before the
+      // epilogue has read O^T, since it needs this tile loop's next P')
+      if (i + 1 < n_tiles && !(ok = convert(i + 1, nxt_fp8))) break;
 
-      if (f.seg_last) {
-        // ---- segment epilogue: partial result of (sequence b, block cta) in
-        // slot b + cta, O^T un-normalised, relative to the reference maximum
+      if (seg_last) {
+        const int b_done = cu.b;
+        cursor_next(cu, a);
+        if (i + 1 < n_tiles) k0 = a.qk0[cu.b];
         ok = tc::mbar_wait(&bars->pv_done, i & 1, abort_flag);
-        ok = !named_or(1, 128, !ok);
+        ok = named_and(1, 256, ok);
         if (!ok) break;
         tc::tc_fence_after();
-        const size_t prow = ((size_t)cu.b + cta) * kH;
+        // partial result of (sequence b_done, block cta) in slot b_done + cta:
+        // O^T un-normalised, relative to the reference maximum
+        const size_t prow = ((size_t)b_done + cta) * kH;
 #pragma unroll 1
-        for (int mt = 0; mt < 4; ++mt) {
+        for (int m2 = 0; m2 < 2; ++m2) {
+          const int mt = 2 * hh + m2;
 #pragma unroll 1
           for (int half = 0; half < 2; ++half) {
             uint32_t r32[32];
@@ -1029,50 +829,59 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
           }
         }
         // normaliser: sum the 128 rows' partial sums per head
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
+        {
           float lsum[32];
           {
             uint32_t lv[32];
-            tc::tmem_ld32(l_addr + 32 * half, lv);
+            tc::tmem_ld32(l_addr, lv);
             tc::tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) lsum[e] = __uint_as_float(lv[e]);
           }
           float two[1];
           const int hb = warp_reduce_scatter32(lsum, lane, two);
-          red[q * 64 + 32 * half + hb] = two[0];
-        }
-        named_sync(1, 128);
-        if (tid < kH) {
-          const float l = red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid];
-          a.part_ml[(prow + tid) * 2] = mref[tid];
-          a.part_ml[(prow + tid) * 2 + 1] = l;
-          mref[tid] = kNone;
-        }
-        {
-          uint32_t z[32];
+          named_sync(1, 256);  // red is free (no slow path in flight)
+          red[warp * 32 + hb] = two[0];
+          named_sync(1, 256);
+          if (tid < kH) {
+            const int half = tid >> 5, hx = tid & 31;
+            const float l = red[(4 * half) * 32 + hx] + red[(4 * half + 1) * 32 + hx] +
+                            red[(4 * half + 2) * 32 + hx] + red[(4 * half + 3) * 32 + hx];
+            a.part_ml[(prow + tid) * 2] = mref[tid];
+            a.part_ml[(prow + tid) * 2 + 1] = l;
+            mref[tid] = kNone;
+          }
+          {
+            uint32_t z[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) z[e] = 0u;
-          tc::tmem_st32(l_addr, z);
-          tc::tmem_st32(l_addr + 32, z);
-          tc::tmem_wait_st();
+            for (int e = 0; e < 32; ++e) z[e] = 0u;
+            tc::tmem_st32(l_addr, z);
+            tc::tmem_wait_st();
+          }
+          named_sync(1, 256);
         }
-        named_sync(1, 128);
-        tc::tc_fence_before();
-        tc::mbar_arrive(&bars->o_free);
+        seg_first = true;
+      } else {
+        cursor_next(cu, a);
+        seg_first = false;
       }
-      cursor_next(cu, a);
     }
     if (!ok) {
       *abort_flag = 1;
       flag(a.dev_status, V4KV_DEV_TIMEOUT);
     }
+    if (__any_sync(0xffffffffu, wide) && lane == 0) flag(a.dev_status, V4KV_DEV_RANGE);
+    if (tid == 0) {
+      // the last query copy has landed before shared memory is released
+      // (normally long since; after an abort it may still be in flight)
+      volatile int never = 0;
+      if (!tc::mbar_wait(&bars->q_ready, (q_issued - 1) & 1, &never)) flag(a.dev_status, V4KV_DEV_TIMEOUT);
+    }
   }
 
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == 8) {
     tc::tc_fence_after();
     tc::tmem_free(tmem, kTmemCols);
   }
@@ -1156,19 +965,12 @@ __global__ void __launch_bounds__(256) decode_tc_merge_kernel(DecodeArgs a) {
   store_output<16>(a, (size_t)b * kH + h, d0, acc, amax, lane == 0);
 }
 
-// grid (batch + 1), 256 threads. Block b < batch writes sequence b's query
-// images for the sweep's B operands:
-//   * f16, scaled by 2^e so that max|q| * 2^e < 2^15, eight 64-dim atoms of
-//     64 head rows x 128 B in the 128-byte swizzle (one linear copy puts it in
-//     place), and qk0[b] = sm_scale * log2(e) * 2^-e;
-//   * three e4m3 terms: x = q * 2^e8 with max|x| in [128, 256), hi = e4m3(x),
-//     mid = e4m3(x - hi), lo = e4m3(x - hi - mid) (round to nearest even; the
-//     residuals are exact in fp32), each as four 128-dim chunks of 64 head
-//     rows x 128 B in the 128-byte swizzle, the K axis of a chunk in the order
-//     the converters leave the codes in tensor memory (chunk_dim_col); and
-//     qk08[b] = sm_scale * log2(e) * 2^-e8.
-// Block `batch` writes the tile prefix sums, the cost prefix sums and every
-// sweep block's range.
+// grid (batch + 1), 256 threads. Block b < batch writes sequence b's query as
+// the shared-memory image of the first product's B operand: f16, scaled by
+// 2^e so that max|q| * 2^e < 2^15, eight 64-dim atoms of 64 head rows x 128 B
+// in the 128-byte swizzle, so that one linear copy puts it in place; and
+// qk0[b] = sm_scale * log2(e) * 2^-e. Block `batch` writes the tile prefix
+// sums cum[0..batch].
 __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
   tc::pdl_wait();  // q and the lengths (written by earlier work in the stream) are complete
   tc::pdl_launch_dependents();
@@ -1194,7 +996,7 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
       long long cost = 0;
       if (bb < a.batch) {
         if (a.seq_lens[bb] > a.max_len) flag(a.dev_status, V4KV_DEV_OVERFLOW);
-        const Seq sq = seq_of(a, bb);
+        const Seq sq = seq_of(a, bb, nullptr);
         n = tiles_of(sq);
         cost = seq_cost(a, sq);
       }
@@ -1244,7 +1046,7 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
           if (costcum[m] <= target) l = m; else r = m - 1;
         }
         b0 = l;
-        const Seq sq = seq_of(a, b0);
+        const Seq sq = seq_of(a, b0, nullptr);
         x0 = cum[b0] + tile_at_cost(a, sq, target - costcum[b0]);
       }
       a.cta_x0[c] = x0;
@@ -1305,17 +1107,14 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
   __syncthreads();
   float amax = 0.f;
   for (int w = 0; w < 8; ++w) amax = fmaxf(amax, red[w]);
-  int e = 0, e8 = 0;
+  int e = 0;
   if (amax > 0.f) {
     int k;
-    frexpf(amax, &k);  // 2^(k-1) <= amax < 2^k
+    frexpf(amax, &k);  // amax < 2^k
     e = 15 - k;
-    e8 = 8 - k;        // max|q| * 2^e8 in [128, 256)
   }
   const float qs = ldexpf(1.f, e);
-  const float qs8 = ldexpf(1.f, e8);
-  uint8_t* img = a.qh + (size_t)b * kQhImg;
-  uint8_t* img3 = a.q3 + (size_t)b * kQ3Img;
+  uint8_t* img = a.qh + (size_t)b * kQBytes;
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
     const int u = t + 256 * k;
@@ -1325,37 +1124,8 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
     for (int i = 0; i < 4; ++i) hv[i] = h2u(__floats2half2_rn(x[k][2 * i] * qs, x[k][2 * i + 1] * qs));
     *reinterpret_cast<uint4*>(img + (c8 >> 3) * 8192 + tc::sw128_off(h, c8 & 7)) =
         make_uint4(hv[0], hv[1], hv[2], hv[3]);
-    // the three fp8 terms of these 8 dims (dims 8 c8 .. 8 c8 + 7 lie in
-    // 128-dim chunk c8 / 16, as two groups of four)
-    const int c = c8 >> 4, dl = 8 * (c8 & 15);
-#pragma unroll
-    for (int g = 0; g < 2; ++g) {
-      uint32_t w3[3] = {0u, 0u, 0u};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float xv = x[k][4 * g + i] * qs8;
-        const uint8_t hi = (uint8_t)__nv_cvt_float_to_fp8(xv, __NV_SATFINITE, __NV_E4M3);
-        const float r1 = xv - e4m3_to_float(hi);
-        const uint8_t mid = (uint8_t)__nv_cvt_float_to_fp8(r1, __NV_SATFINITE, __NV_E4M3);
-        const float r2 = r1 - e4m3_to_float(mid);
-        const uint8_t lo = (uint8_t)__nv_cvt_float_to_fp8(r2, __NV_SATFINITE, __NV_E4M3);
-        w3[0] |= (uint32_t)hi << (8 * i);
-        w3[1] |= (uint32_t)mid << (8 * i);
-        w3[2] |= (uint32_t)lo << (8 * i);
-      }
-      // byte position of the column in the chunk's 128-byte K row
-      const int kb = 4 * chunk_dim_col(dl + 4 * g);
-#pragma unroll
-      for (int term = 0; term < 3; ++term) {
-        uint8_t* at = img3 + (term * 4 + c) * 8192 + tc::sw128_off(h, kb >> 4) + (kb & 15);
-        *reinterpret_cast<uint32_t*>(at) = w3[term];
-      }
-    }
   }
-  if (t == 0) {
-    a.qk0[b] = a.sm_scale * 1.4426950408889634f * ldexpf(1.f, -e);
-    a.qk08[b] = a.sm_scale * 1.4426950408889634f * ldexpf(1.f, -e8);
-  }
+  if (t == 0) a.qk0[b] = a.sm_scale * 1.4426950408889634f * ldexpf(1.f, -e);
   // cos/sin of the inverse RoPE at the query position, for the merge
   if (t < kRopeTable && 2 * t < a.rope.rope_dim) {
     const int Lb = min(a.seq_lens[b], a.max_len);
@@ -1365,27 +1135,23 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
   }
 }
 
-// workspace of the tensor-core path: query images (f16 and three-term fp8),
-// their multipliers, partial results (o, m, l) per slot, tile prefix sums
+// workspace of the tensor-core path: query images, their multipliers, partial
+// results (o, m, l) per slot, tile prefix sums
 size_t decode_tc_workspace_bytes(int batch, int num_sms) {
   const size_t slots = (size_t)batch + num_sms;
   const size_t qk0 = ((size_t)batch * sizeof(float) + 255) / 256 * 256;
-  return (size_t)batch * kQhImg + (size_t)batch * kQ3Img + 2 * qk0 +
-         slots * kH * (size_t)(kD + 2) * sizeof(float) + ((size_t)batch + 1) * sizeof(int32_t) + 256 +
-         ((size_t)batch + 1) * sizeof(long long) + (2 * (size_t)num_sms + 1) * sizeof(int32_t) + 256 +
-         (size_t)batch * sizeof(int2) + 256 + (size_t)batch * kRopeTable * sizeof(float2) + 256;
+  return (size_t)batch * kQBytes + qk0 + slots * kH * (size_t)(kD + 2) * sizeof(float) +
+         ((size_t)batch + 1) * sizeof(int32_t) + 256 + ((size_t)batch + 1) * sizeof(long long) +
+         (2 * (size_t)num_sms + 1) * sizeof(int32_t) + 256 + (size_t)batch * sizeof(int2) + 256 +
+         (size_t)batch * kRopeTable * sizeof(float2) + 256;
 }
 
 void decode_tc_layout(DecodeArgs& a, void* workspace) {
   uint8_t* w = static_cast<uint8_t*>(workspace);
   const size_t slots = (size_t)a.batch + a.n_splits;
   a.qh = w;
-  w += (size_t)a.batch * kQhImg;
-  a.q3 = w;
-  w += (size_t)a.batch * kQ3Img;
+  w += (size_t)a.batch * kQBytes;
   a.qk0 = reinterpret_cast<float*>(w);
-  w += ((size_t)a.batch * sizeof(float) + 255) / 256 * 256;
-  a.qk08 = reinterpret_cast<float*>(w);
   w += ((size_t)a.batch * sizeof(float) + 255) / 256 * 256;
   a.part_o = reinterpret_cast<float*>(w);
   a.part_ml = a.part_o + slots * kH * kD;

@@ -107,9 +107,7 @@ struct DecodeArgs {
   float* prequant_out;  // optional [batch, heads, dim] fp32: the values handed to the quantiser
   int32_t* cum; // tensor-core path: [batch + 1] tile prefix sums (workspace)
   uint8_t* qh;  // tensor-core path: [batch] f16 query images, 64 KB each (workspace)
-  uint8_t* q3;  // tensor-core path: [batch] three-term fp8 query images, 96 KB each
   float* qk0;   // tensor-core path: [batch] score multipliers of the f16 images
-  float* qk08;  // tensor-core path: [batch] score multipliers of the fp8 images
   long long* costcum;  // tensor-core path: [batch + 1] cost prefix sums (workspace)
   int32_t* cta_x0;     // tensor-core path: [n_splits + 1] first tile of each block's range
   int32_t* cta_b0;     // tensor-core path: [n_splits] sequence of that first tile
