@@ -90,13 +90,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-__device__ __forceinline__ int ordered_key(float f) {
-  int k = __float_as_int(f);
-  return k >= 0 ? k : (k ^ 0x7fffffff);
-}
-__device__ __forceinline__ float from_ordered_key(int k) {
-  return __int_as_float(k >= 0 ? k : (k ^ 0x7fffffff));
-}
 
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -130,14 +123,10 @@ struct Seq {
   int L, n_sel, n_sel_pad, n_win, w0, n_items;
 };
 
-__device__ __forceinline__ Seq seq_of(const DecodeArgs& a, int b, int32_t* st) {
+// the tile plan of a sequence of length L (already clamped to [0, max_len])
+__device__ __forceinline__ Seq seq_from_len(const DecodeArgs& a, int L) {
   Seq s;
-  int L = a.seq_lens[b];
-  if (L > a.max_len) {
-    if (threadIdx.x == 0) flag(st, V4KV_DEV_OVERFLOW);
-    L = a.max_len;
-  }
-  s.L = max(0, L);
+  s.L = L;
   const int n_vis = max(0, s.L - a.window_len) / a.ratio;
   s.n_sel = a.topk ? a.k : n_vis;
   s.n_sel_pad = (s.n_sel + kT - 1) / kT * kT;
@@ -147,17 +136,28 @@ __device__ __forceinline__ Seq seq_of(const DecodeArgs& a, int b, int32_t* st) {
   return s;
 }
 
+__device__ __forceinline__ Seq seq_of(const DecodeArgs& a, int b, int32_t* st) {
+  int L = a.seq_lens[b];
+  if (L > a.max_len) {
+    if (threadIdx.x == 0) flag(st, V4KV_DEV_OVERFLOW);
+    L = a.max_len;
+  }
+  return seq_from_len(a, max(0, L));
+}
+
+__device__ __forceinline__ void prefetch_l2_line(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // one bulk L2 prefetch of `bytes` (a multiple of 16, 16-byte aligned) through
-// the copy engine: a single instruction per row instead of one per cache line
-// keeps the load/store path free for the converters
+// the copy engine
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 // Address warp: lane l resolves rows l, l+32, l+64, l+96 of the tile that
 // starts at item tile0 into the row-address and scale tables (nullptr / 0 for
-// a skipped item), then asks L2 for the rows' cache lines so that the workers'
-// loads find them there. The loads go in phases (top-k indices, block-table
+// a skipped item). The loads go in phases (top-k indices, block-table
 // entries, scales), each phase's four loads independent of one another, so a
 // tile costs three memory latencies rather than twelve. Problems are flagged
 // as V4KV_DEV_* bits.
@@ -226,11 +226,6 @@ __device__ __forceinline__ void resolve_tile(const DecodeArgs& a, int b, const S
     rp[lane + 32 * r] = p[r];
     ms[lane + 32 * r] = ks[r];
   }
-  const int lines = fp8 ? kD / 128 : 2 * kD / 128;
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-    if (p[r])
-      prefetch_l2_bulk(p[r], 128 * lines);
   if (err) flag(a.dev_status, err);
 }
 
@@ -311,10 +306,10 @@ struct Cursor {
   Seq s;
 };
 
-__device__ __forceinline__ void cursor_set(Cursor& c, const DecodeArgs& a, int b, int lt) {
+__device__ __forceinline__ void cursor_set(Cursor& c, const DecodeArgs& a, int b, int lt, int L) {
   c.b = b;
   c.lt = lt;
-  c.s = seq_of(a, b, nullptr);
+  c.s = seq_from_len(a, L);
   c.nt = tiles_of(c.s);
 }
 
@@ -341,9 +336,11 @@ __device__ __forceinline__ void issue_q(const DecodeArgs& a, int b, uint32_t qds
   for (int k = 0; k < 4; ++k) tc::bulk_load(qdst + k * (kQBytes / 4), src + k * (kQBytes / 4), kQBytes / 4, bar);
 }
 
-// Sum 32 per-lane values over the 32 lanes of a warp (reduce-scatter): lane l
-// ends with the sum of value `rev` where the lane bits pick halves (bit 4: 16
-// values, bit 3: 8, ... bit 0: 1). Returns that value's index.
+// Sum (or maximum, kMax) of 32 per-lane values over the 32 lanes of a warp
+// (reduce-scatter): lane l ends with the result for the value whose index the
+// lane bits pick (bit 4: the upper 16 values, bit 3: 8, ... bit 0: 1), and
+// returns that index. 31 shuffles per lane.
+template <bool kMax>
 __device__ __forceinline__ int warp_reduce_scatter32(float* v, int lane, float* out1) {
   int base = 0;
 #pragma unroll
@@ -355,7 +352,8 @@ __device__ __forceinline__ int warp_reduce_scatter32(float* v, int lane, float* 
     for (int k = 0; k < n; ++k) {
       const float mine = upper ? v[n + k] : v[k];
       const float other = upper ? v[k] : v[n + k];
-      v[k] = mine + __shfl_xor_sync(0xffffffffu, other, off);
+      const float x = __shfl_xor_sync(0xffffffffu, other, off);
+      v[k] = kMax ? fmaxf(mine, x) : mine + x;
     }
     if (upper) base += n;
   }
@@ -380,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   float* red = reinterpret_cast<float*>(sm + kRedOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kMiscOff + 4);
-  int* range = reinterpret_cast<int*>(sm + kMiscOff + 16);  // x0, x1, b0, lt0
+  int* range = reinterpret_cast<int*>(sm + kMiscOff + 16);  // x0, x1, b0, lt0, L0
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x;
@@ -413,20 +411,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   // ---- this block's tile range [x0, x1) and the sequence of its first tile
   // (the prep kernel balanced the ranges by estimated cost)
   if (tid == 0) {
-    const int x0 = a.cta_x0[cta], x1 = a.cta_x0[cta + 1];
-    const int b0 = x0 < x1 ? a.cta_b0[cta] : a.batch;
-    range[0] = x0;
-    range[1] = (b0 < a.batch) ? x1 : x0;
-    range[2] = b0;
-    range[3] = b0 < a.batch ? x0 - a.cum[b0] : 0;
-    if (b0 < a.batch && x0 < x1) issue_q(a, b0, sbase + kQOff, &bars->q_ready);
+    // one record per block (independent loads): no chain of dependent loads
+    // before the first tile's addresses can be resolved
+    const int4 rec = a.cta_rec[cta];
+    range[0] = rec.x;
+    range[1] = rec.y;
+    range[2] = rec.z;
+    range[3] = rec.w;
+    range[4] = a.cta_L0[cta];
+    if (rec.x < rec.y) issue_q(a, rec.z, sbase + kQOff, &bars->q_ready);
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const int x0 = range[0], x1 = range[1];
   const int n_tiles = x1 - x0;
-  const int b0 = range[2], lt0 = range[3];
+  const int b0 = range[2], lt0 = range[3], L0 = range[4];
   const uint32_t tmem = *tmem_slot;
   if (x0 >= x1) {
     // nothing to do: release tensor memory and leave
@@ -439,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
     // (warp 9 the even tiles, warp 10 the odd ones)
     const int aw = warp - 9;
     Cursor cu;
-    cursor_set(cu, a, b0, lt0);
+    cursor_set(cu, a, b0, lt0, L0);
     if (aw) cursor_next(cu, a);
     for (int t = aw; t < n_tiles; t += 2) {
       const int buf = t % kRing;
@@ -451,6 +451,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       }
       const int tile0 = cu.lt * kT;
       resolve_tile(a, cu.b, cu.s, tile0, lane, rowptr + buf * kT, meta + buf * kT);
+      if (t >= 2) {
+        // rows into L2 for the workers' loads. Tiles 0 and 1 are loaded at
+        // once by the workers; prefetching them too would only add to the
+        // burst of requests every block makes at its start.
+        const bool main_tile = tile0 < cu.s.n_sel_pad;
+        const bool fp8 = (main_tile ? a.main.dtype : a.window.dtype) == V4KV_FP8_E4M3;
+        const uint8_t* const* rp = rowptr + buf * kT;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const uint8_t* pr = rp[lane + 32 * r];
+          if (pr)
+            for (int k = 0; k < (fp8 ? kD / 128 : 2 * kD / 128); ++k) prefetch_l2_line(pr + 128 * k);
+        }
+      }
       if (lane == 0) {
         const bool main_tile = tile0 < cu.s.n_sel_pad;
         const bool fp8 = (main_tile ? a.main.dtype : a.window.dtype) == V4KV_FP8_E4M3;
@@ -645,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       if (ok) ok = convert(0, fp8);
     }
     Cursor cu;
-    cursor_set(cu, a, b0, lt0);
+    cursor_set(cu, a, b0, lt0, L0);
     bool seg_first = true;  // the current tile opens a segment
     for (int i = 0; i < n_tiles && ok; ++i) {
       const bool seg_last = i == n_tiles - 1 || cu.lt == cu.nt - 1;
@@ -687,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
         ++q_issued;
       }
       float dmax = -INFINITY;
-      {
+      if (!seg_first) {
         const float4* mr4 = reinterpret_cast<const float4*>(mref + 32 * hh);
 #pragma unroll
         for (int h4 = 0; h4 < 8; ++h4) {
@@ -699,20 +713,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
           dmax = fmaxf(dmax, fmaxf(fmaxf(d[4 * h4], d[4 * h4 + 1]), fmaxf(d[4 * h4 + 2], d[4 * h4 + 3])));
         }
       }
-      if (named_or(1, 256, dmax > kTau)) {
-        // rare: raise the reference of every head to its running maximum.
-        // u is recomputed from S (still in tensor memory) to keep it exact.
-        {
+      // A segment's first tile sets the references to its per-head maxima
+      // (d still holds u, the normalisers are zero and O^T is written afresh);
+      // a later tile raises them, rarely, when a score exceeds its reference
+      // by 2^kTau.
+      if (seg_first || named_or(1, 256, dmax > kTau)) {
+        if (!seg_first) {
+          // u is recomputed from S (still in tensor memory) to keep it exact
           uint32_t r32[32];
           tc::tmem_ld32(s_addr, r32);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int h = 0; h < 32; ++h) d[h] = fmaf(__uint_as_float(r32[h]), cj, lk);
         }
+        {
+          // per-head maximum over the warp's 32 rows: a transposing
+          // shuffle reduction leaves head hb's maximum in this lane
+          float t32[32], one[1];
 #pragma unroll
-        for (int h = 0; h < 32; ++h) {
-          const int wm = __reduce_max_sync(0xffffffffu, ordered_key(d[h]));
-          if (lane == 0) red[warp * 32 + h] = from_ordered_key(wm);
+          for (int h = 0; h < 32; ++h) t32[h] = d[h];
+          const int hb = warp_reduce_scatter32<true>(t32, lane, one);
+          red[warp * 32 + hb] = one[0];
         }
         named_sync(1, 256);
         if (tid < kH) {
@@ -727,17 +748,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
         named_sync(1, 256);
 #pragma unroll
         for (int h = 0; h < 32; ++h) d[h] -= mref[32 * hh + h];
-        {
-          uint32_t lv[32];
-          tc::tmem_ld32(l_addr, lv);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < 32; ++h)
-            lv[h] = __float_as_uint(__uint_as_float(lv[h]) * alpha[32 * hh + h]);
-          tc::tmem_st32(l_addr, lv);
-          tc::tmem_wait_st();
-        }
         if (!seg_first) {
+          {
+            uint32_t lv[32];
+            tc::tmem_ld32(l_addr, lv);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < 32; ++h)
+              lv[h] = __float_as_uint(__uint_as_float(lv[h]) * alpha[32 * hh + h]);
+            tc::tmem_st32(l_addr, lv);
+            tc::tmem_wait_st();
+          }
           // O^T rows of this lane (dims 128 mt + row, mt = 2hh, 2hh + 1) times
           // alpha per head column
 #pragma unroll 1
@@ -839,7 +860,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
             for (int e = 0; e < 32; ++e) lsum[e] = __uint_as_float(lv[e]);
           }
           float two[1];
-          const int hb = warp_reduce_scatter32(lsum, lane, two);
+          const int hb = warp_reduce_scatter32<false>(lsum, lane, two);
           named_sync(1, 256);  // red is free (no slow path in flight)
           red[warp * 32 + hb] = two[0];
           named_sync(1, 256);
@@ -896,48 +917,68 @@ __global__ void __launch_bounds__(256) decode_tc_merge_kernel(DecodeArgs a) {
   tc::pdl_wait();  // the sweep's partial results are complete from here on
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = 8 * blockIdx.x + warp, b = blockIdx.y;
+  const int Lb = min(a.seq_lens[b], a.max_len);  // independent of the loads below
   const int2 sl = a.seq_slots[b];
   const int lo = sl.x, hi = sl.y;
+  // per block: (m, l) in one load; the weights go to shared memory
   float M = -INFINITY;
-  for (int c = lo + lane; c <= hi; c += 32) {
-    const bool empty = a.cta_x0[c + 1] <= a.cta_x0[c];
-    const float m = empty ? -INFINITY : a.part_ml[(((size_t)b + c) * kH + h) * 2];
-    w_sh[warp][c - lo] = m;
-    M = fmaxf(M, m);
+  float2 ml_keep[(kMaxSplits + 31) / 32];
+#pragma unroll
+  for (int k = 0; k < (kMaxSplits + 31) / 32; ++k) {
+    const int c = lo + lane + 32 * k;
+    float2 ml = make_float2(-INFINITY, 0.f);
+    if (c <= hi && a.cta_x0[c + 1] > a.cta_x0[c])
+      ml = reinterpret_cast<const float2*>(a.part_ml)[((size_t)b + c) * kH + h];
+    ml_keep[k] = ml;
+    M = fmaxf(M, ml.x);
   }
   M = warp_max(M);
   float L = 0.f;
-  for (int c = lo + lane; c <= hi; c += 32) {
-    const float m = w_sh[warp][c - lo];
-    const float w = m == -INFINITY ? 0.f : exp2f(m - M);
-    w_sh[warp][c - lo] = w;
-    if (w > 0.f) L = fmaf(w, a.part_ml[(((size_t)b + c) * kH + h) * 2 + 1], L);
+#pragma unroll
+  for (int k = 0; k < (kMaxSplits + 31) / 32; ++k) {
+    const int c = lo + lane + 32 * k;
+    if (c <= hi) {
+      const float w = ml_keep[k].x == -INFINITY ? 0.f : exp2f(ml_keep[k].x - M);
+      w_sh[warp][c - lo] = w;
+      L = fmaf(w, ml_keep[k].y, L);
+    }
   }
   L = warp_sum(L);
   __syncwarp();
+  // weighted sum of the blocks' rows, four blocks' loads in flight at a time
   const int d0 = 16 * lane;
   float acc[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-  for (int c = lo; c <= hi; ++c) {
-    const float w = w_sh[warp][c - lo];
-    if (w == 0.f) continue;
-    const float4* o4 = reinterpret_cast<const float4*>(a.part_o + (((size_t)b + c) * kH + h) * kD + d0);
-    float4 v[4];
+  for (int c = lo; c <= hi; c += 4) {
+    float4 v[4][4];
+    float w[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) v[q] = o4[q];
+    for (int j = 0; j < 4; ++j) {
+      w[j] = c + j <= hi ? w_sh[warp][c + j - lo] : 0.f;
+      if (w[j] != 0.f) {
+        const float4* o4 =
+            reinterpret_cast<const float4*>(a.part_o + (((size_t)b + c + j) * kH + h) * kD + d0);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      acc[4 * q] = fmaf(w, v[q].x, acc[4 * q]);
-      acc[4 * q + 1] = fmaf(w, v[q].y, acc[4 * q + 1]);
-      acc[4 * q + 2] = fmaf(w, v[q].z, acc[4 * q + 2]);
-      acc[4 * q + 3] = fmaf(w, v[q].w, acc[4 * q + 3]);
+        for (int q = 0; q < 4; ++q) v[j][q] = o4[q];
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[j][q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[4 * q] = fmaf(w[j], v[j][q].x, acc[4 * q]);
+        acc[4 * q + 1] = fmaf(w[j], v[j][q].y, acc[4 * q + 1]);
+        acc[4 * q + 2] = fmaf(w[j], v[j][q].z, acc[4 * q + 2]);
+        acc[4 * q + 3] = fmaf(w[j], v[j][q].w, acc[4 * q + 3]);
+      }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
   for (int e = 0; e < 16; ++e) acc[e] *= inv;
-  const int Lb = min(a.seq_lens[b], a.max_len);
   if (a.rope.rope_dim > 0 && Lb > 0) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -983,10 +1024,12 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
     // c/G of the total
     __shared__ long long csum[8];
     __shared__ int x0_sh[kMaxSplits + 1];
+    __shared__ int b0_sh[kMaxSplits];
     // the prefix sums also go to shared memory (when they fit) for the
     // binary searches below, which would otherwise chain global loads
     __shared__ int cum_sh[kPrepCache + 1];
     __shared__ long long ccum_sh[kPrepCache + 1];
+    __shared__ int len_sh[kPrepCache];  // clamped lengths
     const bool cached = a.batch <= kPrepCache;
     int carry = 0;
     long long ccarry = 0;
@@ -999,6 +1042,7 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
         const Seq sq = seq_of(a, bb, nullptr);
         n = tiles_of(sq);
         cost = seq_cost(a, sq);
+        if (cached) len_sh[bb] = sq.L;
       }
       int incl = n;
       long long cincl = cost;
@@ -1046,14 +1090,20 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
           if (costcum[m] <= target) l = m; else r = m - 1;
         }
         b0 = l;
-        const Seq sq = seq_of(a, b0, nullptr);
+        const Seq sq = cached ? seq_from_len(a, len_sh[b0]) : seq_of(a, b0, nullptr);
         x0 = cum[b0] + tile_at_cost(a, sq, target - costcum[b0]);
       }
       a.cta_x0[c] = x0;
-      if (c < G) a.cta_b0[c] = b0;
       x0_sh[c] = x0;
+      if (c < G) b0_sh[c] = b0;
     }
     __syncthreads();
+    for (int c = t; c < G; c += 256) {
+      const int x0 = x0_sh[c], x1 = x0_sh[c + 1], b0 = b0_sh[c];
+      const bool live = x0 < x1 && b0 < a.batch;
+      a.cta_rec[c] = live ? make_int4(x0, x1, b0, x0 - cum[b0]) : make_int4(x0, x0, a.batch, 0);
+      a.cta_L0[c] = live ? (cached ? len_sh[b0] : seq_of(a, b0, nullptr).L) : 0;
+    }
     // blocks whose ranges [x0[c], x0[c+1]) meet each sequence's tiles [c0, c1)
     for (int bb = t; bb < a.batch; bb += 256) {
       const int c0 = cum[bb], c1 = cum[bb + 1];
@@ -1142,7 +1192,8 @@ size_t decode_tc_workspace_bytes(int batch, int num_sms) {
   const size_t qk0 = ((size_t)batch * sizeof(float) + 255) / 256 * 256;
   return (size_t)batch * kQBytes + qk0 + slots * kH * (size_t)(kD + 2) * sizeof(float) +
          ((size_t)batch + 1) * sizeof(int32_t) + 256 + ((size_t)batch + 1) * sizeof(long long) +
-         (2 * (size_t)num_sms + 1) * sizeof(int32_t) + 256 + (size_t)batch * sizeof(int2) + 256 +
+         ((size_t)num_sms + 1) * sizeof(int32_t) + 16 + (size_t)num_sms * (sizeof(int4) + sizeof(int32_t)) +
+         256 + (size_t)batch * sizeof(int2) + 256 +
          (size_t)batch * kRopeTable * sizeof(float2) + 256;
 }
 
@@ -1160,8 +1211,11 @@ void decode_tc_layout(DecodeArgs& a, void* workspace) {
   c = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(c) + 255) & ~uintptr_t(255));
   a.costcum = reinterpret_cast<long long*>(c);
   a.cta_x0 = reinterpret_cast<int32_t*>(a.costcum + a.batch + 1);
-  a.cta_b0 = a.cta_x0 + a.n_splits + 1;
-  uint8_t* q = reinterpret_cast<uint8_t*>(a.cta_b0 + a.n_splits);
+  uint8_t* rc = reinterpret_cast<uint8_t*>(a.cta_x0 + a.n_splits + 1);
+  rc = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(rc) + 15) & ~uintptr_t(15));
+  a.cta_rec = reinterpret_cast<int4*>(rc);
+  a.cta_L0 = reinterpret_cast<int32_t*>(a.cta_rec + a.n_splits);
+  uint8_t* q = reinterpret_cast<uint8_t*>(a.cta_L0 + a.n_splits);
   q = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(q) + 255) & ~uintptr_t(255));
   a.seq_slots = reinterpret_cast<int2*>(q);
   uint8_t* r = reinterpret_cast<uint8_t*>(a.seq_slots + a.batch);

@@ -110,7 +110,9 @@ struct DecodeArgs {
   float* qk0;   // tensor-core path: [batch] score multipliers of the f16 images
   long long* costcum;  // tensor-core path: [batch + 1] cost prefix sums (workspace)
   int32_t* cta_x0;     // tensor-core path: [n_splits + 1] first tile of each block's range
-  int32_t* cta_b0;     // tensor-core path: [n_splits] sequence of that first tile
+  int4* cta_rec;       // tensor-core path: [n_splits] {x0, x1, b0, lt0}: a block's tile range,
+                       // the sequence of its first tile and that tile's index in the sequence
+  int32_t* cta_L0;     // tensor-core path: [n_splits] length of that sequence (clamped)
   int2* seq_slots;     // tensor-core path: [batch] first and last block meeting the sequence
   float2* rope_tab;    // tensor-core path: [batch][kRopeTable] (cos, sin) at position L - 1
 };
