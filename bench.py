@@ -4,8 +4,9 @@ Default workload (one GPU): c4a decode, batch 64, context lengths uniform on
 [4K, 64K], 64 query heads, shared KV dim 512 stored as fp8-e4m3 with one fp32
 scale per entry, 128-token bf16 window, physical pages randomly permuted.
 One step = the whole hot path for one new token per sequence:
-v4kv_slot_mapping -> v4kv_compress_append (1 token each) ->
-v4kv_decode_attention (all visible entries + window). Inputs are synthetic
+v4kv_compress_append (1 token each; the slots come from the block tables
+inside the compressor) -> v4kv_decode_attention (all visible entries +
+window). Inputs are synthetic
 (seeded device draws) and resident in HBM; L2 is flushed between steps.
 
 The default run (N = 1) also measures the other workloads and adds them to
@@ -169,8 +170,6 @@ class DecodeStep:
         self.n_new = torch.ones(self.B, dtype=torch.int32, device=device)
         self.cu_seqlens = torch.arange(self.B + 1, dtype=torch.int32, device=device)
         self.seq_lens = torch.from_numpy(self.lens.astype(np.int32)).to(device)
-        self.slots = torch.empty(2 * self.B + 1, dtype=torch.int64, device=device)
-        self.cu_e = torch.empty(self.B + 1, dtype=torch.int32, device=device)
         self.out = torch.empty(self.B, self.H, D, dtype=torch.bfloat16, device=device)
         self.max_len = int(self.lens.max())
         ws = v4kv.v4kv_workspace_size(v4kv.V4KV_OP_DECODE, self.B, self.H, self.max_len, self.ratio,
@@ -179,18 +178,16 @@ class DecodeStep:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
     def launches_per_step(self):
-        # slot mapping 1, compressor 1 (entries, window rows and state in one
-        # launch), decode 3 for 64 heads (query prep, sweep, merge) or 2 otherwise
-        return 5 if self.H == 64 else 4
+        # compressor 1 (slots, entries, window rows and state in one launch),
+        # decode 3 for 64 heads (query prep, sweep, merge) or 2 otherwise
+        return 4 if self.H == 64 else 3
 
     def append(self, stream=None):
-        v = self.v4kv
-        v.v4kv_slot_mapping(self.main.block_table, self.seq_start, self.n_new, self.ratio, self.P,
-                            self.slots, self.cu_e, dev_status=self.status, stream=stream)
-        v.v4kv_compress_append(self.x, self.gate, self.cu_seqlens, self.seq_start, self.bias,
-                               self.ratio, self.state_x, self.state_g, self.main, self.slots,
-                               self.cu_e, window=self.win, window_len=W, dev_status=self.status,
-                               stream=stream)
+        # the compressor derives the new token's slot from the block table
+        self.v4kv.v4kv_compress_append(self.x, self.gate, self.cu_seqlens, self.seq_start, self.bias,
+                                       self.ratio, self.state_x, self.state_g, self.main, None, None,
+                                       window=self.win, window_len=W, dev_status=self.status,
+                                       stream=stream)
 
     def decode(self, stream=None, q=None, out=None):
         self.v4kv.v4kv_decode_attention(self.q if q is None else q, self.main, self.win,
@@ -588,22 +585,19 @@ class CompressStep:
             cu = torch.tensor(np.concatenate([[0], np.cumsum(sizes)]), dtype=torch.int32, device=device)
             ss = torch.tensor(done, dtype=torch.int32, device=device)
             nn = torch.tensor(sizes, dtype=torch.int32, device=device)
-            cap = int(sum(sizes)) // ratio + 2 * seqs
             self.call_inputs.append(dict(x=self.x[rows].contiguous(), gate=self.gate[rows].contiguous(),
                                          cu=cu, ss=ss, nn=nn, n=int(sum(sizes)),
-                                         starts=np.array(done), sizes=np.array(sizes),
-                                         slots=torch.empty(cap, dtype=torch.int64, device=device),
-                                         cue=torch.empty(seqs + 1, dtype=torch.int32, device=device)))
+                                         starts=np.array(done), sizes=np.array(sizes)))
             for b in range(seqs):
                 done[b] += sizes[b]
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
     def call(self, c):
+        """One append: the compressor derives the slots from the block table
+        itself (no slot mapping argument, one launch)."""
         v, ci = self.v4kv, self.call_inputs[c]
-        v.v4kv_slot_mapping(self.main.block_table, ci["ss"], ci["nn"], self.ratio, self.P, ci["slots"],
-                            ci["cue"], dev_status=self.status)
         v.v4kv_compress_append(ci["x"], ci["gate"], ci["cu"], ci["ss"], self.bias, self.ratio,
-                               self.state_x, self.state_g, self.main, ci["slots"], ci["cue"],
+                               self.state_x, self.state_g, self.main, None, None,
                                window=self.win, window_len=W, dev_status=self.status)
 
     def algorithmic_bytes(self, c):
@@ -665,12 +659,13 @@ def run_compress(args, device, clk):
                             "ms_eager": ms_eager,
                             "gbs_eager": byts / (ms_eager * 1e-3) / 1e9,
                             "status": int(st.status.item()),
-                            "launches": 2 * st.calls, "_window": (t0, t1)}
+                            "launches": st.calls, "_window": (t0, t1)}
         del st
         torch.cuda.empty_cache()
     return {"config": "compressor write path, 8 x 32K raw bf16 tokens, random chunks 1..4096, fp8 "
-                      "entries, shuffled pages; ms = one CUDA-graph replay of all calls (median), "
-                      "ms_eager = the calls launched one by one from Python", "results": out}
+                      "entries, shuffled pages, slots from the block tables inside the compressor; "
+                      "ms = one CUDA-graph replay of all calls (median), ms_eager = the calls launched "
+                      "one by one from Python", "results": out}
 
 
 class MixedStep:
@@ -727,9 +722,7 @@ class MixedStep:
                         gate=torch.randn(seqs, generator=g, device=device),
                         bias=torch.randn(ratio, generator=g, device=device) * 0.5,
                         sx=torch.randn(seqs, ratio, D, generator=g, device=device).to(torch.bfloat16),
-                        sg=torch.randn(seqs, ratio, generator=g, device=device),
-                        slots=torch.empty(2 * seqs + 1, dtype=torch.int64, device=device),
-                        cue=torch.empty(seqs + 1, dtype=torch.int32, device=device), P=P)
+                        sg=torch.randn(seqs, ratio, generator=g, device=device), P=P)
 
         self.c4a = []
         for _ in range(c4a_layers):
@@ -757,13 +750,12 @@ class MixedStep:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
     def append(self, L, ratio, stream=None):
-        """One new token per sequence into layer L's cache: slot mapping, then
-        the compressor (entry of the token's group, window row, state)."""
+        """One new token per sequence into layer L's cache: the compressor
+        (entry of the token's group, window row, state), slots derived from
+        the block table inside it."""
         a, v = L["ap"], self.v4kv
-        v.v4kv_slot_mapping(L["main"].block_table, self.seq_start, self.n_new, ratio, a["P"],
-                            a["slots"], a["cue"], dev_status=self.status, stream=stream)
         v.v4kv_compress_append(a["x"], a["gate"], self.cu_seqlens, self.seq_start, a["bias"], ratio,
-                               a["sx"], a["sg"], L["main"], a["slots"], a["cue"], window=L["win"],
+                               a["sx"], a["sg"], L["main"], None, None, window=L["win"],
                                window_len=W, dev_status=self.status, stream=stream)
 
     def full_step(self, overlap, side=None):

@@ -156,7 +156,11 @@ v4kv_status v4kv_slot_mapping(const int32_t* block_table, int32_t max_blocks, in
  *   slot_mapping device int64 and cu_entries device int32 [batch + 1], as
  *                produced by v4kv_slot_mapping(ratio) for this append;
  *                slot_mapping must hold all cu_entries[batch] slots
- *                (total_tokens / ratio + 2 * batch always suffices)
+ *                (total_tokens / ratio + 2 * batch always suffices). Both
+ *                NULL: the kernel derives the same slots from
+ *                main_cache->block_table itself (one launch instead of two;
+ *                batch < 1024, else V4KV_ERR_UNSUPPORTED). Exactly one NULL
+ *                is V4KV_ERR_INVALID_ARG.
  *   window       window pool (bf16 or fp8, slots_per_page 256) or NULL
  *   prequant_out device fp32 [cu_entries[batch], dim] or NULL: the fp32
  *                values handed to the quantiser (after RoPE)

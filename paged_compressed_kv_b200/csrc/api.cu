@@ -131,9 +131,12 @@ v4kv_status v4kv_compress_append(const void* x, const float* gate, const int32_t
                                  float* prequant_out, int32_t* dev_status, void* stream) {
   if (batch <= 0 || total_tokens < 0) return V4KV_ERR_INVALID_ARG;
   if (ratio != 4 && ratio != 128) return V4KV_ERR_INVALID_ARG;
-  if (!cu_seqlens || !seq_start || !pos_bias || !state_x || !state_gate || !cu_entries)
-    return V4KV_ERR_INVALID_ARG;
-  if (total_tokens > 0 && (!x || !gate || !slot_mapping)) return V4KV_ERR_INVALID_ARG;
+  if (!cu_seqlens || !seq_start || !pos_bias || !state_x || !state_gate) return V4KV_ERR_INVALID_ARG;
+  // the slot mapping comes from v4kv_slot_mapping, or (both NULL) is computed
+  // inside the kernel from main_cache's block table, for batch < 1024
+  if (!slot_mapping != !cu_entries) return V4KV_ERR_INVALID_ARG;
+  if (!slot_mapping && batch >= 1024) return V4KV_ERR_UNSUPPORTED;
+  if (total_tokens > 0 && (!x || !gate)) return V4KV_ERR_INVALID_ARG;
   if (!main_cache) return V4KV_ERR_INVALID_ARG;
   const int dim = main_cache->dim;
   if (dim < 8 || dim > 1024 || dim % 8) return V4KV_ERR_INVALID_ARG;

@@ -210,8 +210,8 @@ __device__ __forceinline__ void weighted_rows(const CompressArgs& a, int b, int 
 // RoPE at the group's first position, optional pre-quantisation copy, and
 // the store into the entry's slot
 template <int KC>
-__device__ __forceinline__ void finish_entry(const CompressArgs& a, int i, int t0, int lane, int nch,
-                                             float (&e)[KC][8]) {
+__device__ __forceinline__ void finish_entry(const CompressArgs& a, int i, int b, int t0, int lane,
+                                             int nch, float (&e)[KC][8]) {
   rope_warp<KC>(e, lane, nch, a.rope, (long long)t0);
   if (a.prequant_out) {
 #pragma unroll
@@ -223,9 +223,18 @@ __device__ __forceinline__ void finish_entry(const CompressArgs& a, int i, int t
       *reinterpret_cast<float4*>(po + 4) = make_float4(e[k][4], e[k][5], e[k][6], e[k][7]);
     }
   }
-  const long long slot = a.slot_mapping[i];
+  long long slot;
+  if (a.slot_mapping) {
+    slot = a.slot_mapping[i];
+  } else {
+    // the slot mapping of this entry (group t0 / r of sequence b) inline
+    const long long g = t0 / a.ratio;
+    const int p = page_of(a.main.block_table + (size_t)b * a.main.max_blocks, a.main.max_blocks, g,
+                          a.main.spb, a.main.num_pages, lane == 0 ? a.dev_status : nullptr);
+    slot = p < 0 ? -1 : (long long)p * a.main.spb + g % a.main.spb;
+  }
   const long long cap = (long long)a.main.num_pages * a.main.spb;
-  if (slot < 0) return;  // unmapped page (already flagged by the slot mapping)
+  if (slot < 0) return;  // unmapped page (flagged by the slot mapping)
   if (slot >= cap) {
     if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
     return;
@@ -292,11 +301,39 @@ __global__ void __launch_bounds__(kWarps * 32) compress_append_kernel(CompressAr
   }
   const int eb = blockIdx.x - window_blocks;
   const bool cached = a.batch + 1 <= kCuSmem;
-  if (cached) {
+  if (!a.cu_entries) {
+    // no slot mapping given: the entry counts (groups touched by each
+    // sequence's new tokens) and their prefix sums, computed here
+    __shared__ int wsum[kWarps];
+    int carry = 0;
+    for (int base = 0; base < a.batch; base += kWarps * 32) {
+      const int bb = base + threadIdx.x;
+      int n = 0;
+      if (bb < a.batch) {
+        const int s0 = a.seq_start[bb], m = a.cu_seqlens[bb + 1] - a.cu_seqlens[bb];
+        n = m > 0 ? (s0 + m + a.ratio - 1) / a.ratio - s0 / a.ratio : 0;
+      }
+      int x = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) wsum[warp] = x;
+      __syncthreads();
+      int before = carry;
+      for (int w2 = 0; w2 < warp; ++w2) before += wsum[w2];
+      if (bb < a.batch) cu_sh[bb] = before + x - n;
+      for (int w2 = 0; w2 < kWarps; ++w2) carry += wsum[w2];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) cu_sh[a.batch] = carry;
+    __syncthreads();
+  } else if (cached) {
     for (int k = threadIdx.x; k <= a.batch; k += blockDim.x) cu_sh[k] = a.cu_entries[k];
     __syncthreads();
   }
-  const int32_t* cu = cached ? cu_sh : a.cu_entries;
+  const int32_t* cu = (cached || !a.cu_entries) ? cu_sh : a.cu_entries;
   const int total = cu[a.batch];
   const int i = kBlockGroup ? eb : eb * kWarps + warp;
   if (i >= total) return;  // uniform over the warp (and over the block for block groups)
@@ -309,7 +346,6 @@ __global__ void __launch_bounds__(kWarps * 32) compress_append_kernel(CompressAr
   const bool first_of_seq = i == cu[b];
 
   float* w = w_sh[warp];
-  group_weights<kNQ>(a, b, s, t0, np, lane, w);
   float acc[KC][8];
 #pragma unroll
   for (int k = 0; k < KC; ++k)
@@ -317,12 +353,38 @@ __global__ void __launch_bounds__(kWarps * 32) compress_append_kernel(CompressAr
     for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
 
   if constexpr (!kBlockGroup) {
-    weighted_rows<KC, kRB>(a, b, s, t0, 0, np, w, lane, nch, acc);
-    finish_entry<KC>(a, i, t0, lane, nch, acc);
+    // the group's first kRB rows are requested before the gate softmax, so
+    // that the two memory latencies overlap
+    uint4 q[kRB][KC];
+#pragma unroll
+    for (int j = 0; j < kRB; ++j) {
+      const int tt = t0 + j;
+      if (j < np) {
+        const uint16_t* row = tt < s ? a.state_x + ((size_t)b * r + j) * a.dim
+                                     : a.x + (size_t)(a.cu_seqlens[b] + (tt - s)) * a.dim;
+        load_row<KC>(row, lane, nch, q[j]);
+      }
+    }
+    group_weights<kNQ>(a, b, s, t0, np, lane, w);
+#pragma unroll
+    for (int j = 0; j < kRB; ++j) {
+      if (j >= np) break;
+      const float wt = w[j];
+#pragma unroll
+      for (int k = 0; k < KC; ++k) {
+        float v[8];
+        unpack_bf16x8(q[j][k], v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wt, v[e], acc[k][e]);
+      }
+    }
+    if (np > kRB) weighted_rows<KC, kRB>(a, b, s, t0, kRB, np, w, lane, nch, acc);
+    finish_entry<KC>(a, i, b, t0, lane, nch, acc);
     // this warp consumed every old state row and gate it read (the sums and
     // the softmax reductions depend on them), so the state may be rewritten
     if (first_of_seq) copy_state<KC, kRB>(a, b, s, end, 0, r, lane, nch);
   } else {
+    group_weights<kNQ>(a, b, s, t0, np, lane, w);
     const int rpw = (r + kWarps - 1) / kWarps;
     weighted_rows<KC, kRB>(a, b, s, t0, min(np, warp * rpw), min(np, (warp + 1) * rpw), w, lane, nch,
                            acc);
@@ -342,7 +404,7 @@ __global__ void __launch_bounds__(kWarps * 32) compress_append_kernel(CompressAr
 #pragma unroll
           for (int e = 0; e < 8; ++e) acc[k][e] += part[ww][8 * (lane + 32 * k) + e];
       }
-      finish_entry<KC>(a, i, t0, lane, nch, acc);
+      finish_entry<KC>(a, i, b, t0, lane, nch, acc);
     }
     if (first_of_seq) copy_state<KC, kRB>(a, b, s, end, warp * rpw, (warp + 1) * rpw, lane, nch);
   }

@@ -214,15 +214,18 @@ def v4kv_compress_append(x, gate, cu_seqlens, seq_start, pos_bias, ratio, state_
     _need(pos_bias, (torch.float32,), "pos_bias")
     _need(state_x, (torch.bfloat16,), "state_x", ndim=3)
     _need(state_gate, (torch.float32,), "state_gate", ndim=2)
-    _need(slot_mapping, (torch.int64,), "slot_mapping")
-    _need(cu_entries, (torch.int32,), "cu_entries")
+    if (slot_mapping is None) != (cu_entries is None):
+        raise ValueError("slot_mapping and cu_entries: both or neither")
+    if slot_mapping is not None:
+        _need(slot_mapping, (torch.int64,), "slot_mapping")
+        _need(cu_entries, (torch.int32,), "cu_entries")
     rope = rope or Rope()
     mc = main.c()
     wc = window.c() if window is not None else None
     st = _lib.v4kv_compress_append(
         x.data_ptr(), gate.data_ptr(), cu_seqlens.data_ptr(), seq_start.data_ptr(),
         seq_start.numel(), x.shape[0], pos_bias.data_ptr(), ratio, rope.c(), state_x.data_ptr(),
-        state_gate.data_ptr(), ctypes.byref(mc), slot_mapping.data_ptr(), cu_entries.data_ptr(),
+        state_gate.data_ptr(), ctypes.byref(mc), _ptr(slot_mapping), _ptr(cu_entries),
         ctypes.byref(wc) if wc is not None else None, window_len, _ptr(prequant_out),
         _ptr(dev_status), _stream(stream))
     _check("v4kv_compress_append", st)

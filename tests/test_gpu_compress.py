@@ -61,7 +61,9 @@ class Appender:
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self._host = None
 
-    def append(self, sizes):
+    def append(self, sizes, inline_slots=False):
+        """One append call. inline_slots: no v4kv_slot_mapping call; the
+        compressor derives the slots from the block table itself."""
         self._host = None  # the pools change
         from paged_compressed_kv_b200 import v4kv
         dev = torch.device("cuda")
@@ -76,13 +78,16 @@ class Appender:
         cu_e = torch.zeros(self.B + 1, dtype=torch.int32, device=dev)
         ss = torch.from_numpy(seq_start).to(dev)
         nn = torch.from_numpy(n_new).to(dev)
-        v4kv.v4kv_slot_mapping(self.main.block_table, ss, nn, self.ratio, self.P, slots, cu_e,
-                               dev_status=self.status)
-        # slots must equal the oracle's slot mapping bit for bit
         want, want_cu = paging.slot_mapping(self.bt, seq_start, n_new, self.ratio, 256 // self.ratio)
-        got_cu = cu_e.cpu().numpy()
-        assert np.array_equal(got_cu, want_cu)
-        assert np.array_equal(slots[: len(want)].cpu().numpy(), want)
+        if inline_slots:
+            slots = cu_e = None
+        else:
+            v4kv.v4kv_slot_mapping(self.main.block_table, ss, nn, self.ratio, self.P, slots, cu_e,
+                                   dev_status=self.status)
+            # slots must equal the oracle's slot mapping bit for bit
+            got_cu = cu_e.cpu().numpy()
+            assert np.array_equal(got_cu, want_cu)
+            assert np.array_equal(slots[: len(want)].cpu().numpy(), want)
         pre = torch.full((max(1, len(want)), self.dim), np.nan, dtype=torch.float32, device=dev)
         v4kv.v4kv_compress_append(
             synth.bf16_tensor(xs).to(dev).reshape(-1, self.dim), torch.from_numpy(gs).to(dev),
@@ -208,6 +213,42 @@ def test_chunked_equals_one_shot_bitwise(ratio):
         rb, sb = b.entries(s)
         assert np.array_equal(ra, rb) and np.array_equal(sa, sb)
         assert np.array_equal(a.prequant[s].view(np.uint32), b.prequant[s].view(np.uint32))
+
+
+@pytest.mark.parametrize("ratio", [4, 128])
+def test_inline_slot_mapping_equals_explicit_bitwise(ratio):
+    """The compressor without a slot mapping (slots from the block table, in
+    the kernel) writes the same bytes, state and pre-quantisation values as
+    with the v4kv_slot_mapping output, over random chunks (P1 §3.1.1)."""
+    n = [5000, 2049, 777, 9000, 1]
+    a = Appender(430, n, ratio)
+    b = Appender(430, n, ratio)
+    r = synth.rng(431)
+    while any(d < N for d, N in zip(a.done, a.n)):
+        sizes = [int(r.integers(0, 900)) for _ in n]
+        a.append(sizes)
+        b.append(sizes, inline_slots=True)
+    check_against_oracle(b)
+    for s in range(len(n)):
+        ra, sa = a.entries(s)
+        rb, sb = b.entries(s)
+        assert np.array_equal(ra, rb) and np.array_equal(sa, sb)
+        assert np.array_equal(a.prequant[s].view(np.uint32), b.prequant[s].view(np.uint32))
+        assert np.array_equal(a.window_values(s), b.window_values(s))
+    assert torch.equal(a.state_x, b.state_x) and torch.equal(a.state_g, b.state_g)
+
+
+def test_inline_slot_mapping_arguments():
+    """Exactly one of slot_mapping / cu_entries missing is an argument error."""
+    from paged_compressed_kv_b200 import v4kv
+    ap = Appender(432, [10], 4)
+    dev = torch.device("cuda")
+    cu_e = torch.zeros(2, dtype=torch.int32, device=dev)
+    with pytest.raises(ValueError):
+        v4kv.v4kv_compress_append(
+            torch.zeros(10, D, dtype=torch.bfloat16, device=dev), torch.zeros(10, device=dev),
+            torch.tensor([0, 10], dtype=torch.int32, device=dev), torch.zeros(1, dtype=torch.int32, device=dev),
+            torch.zeros(4, device=dev), 4, ap.state_x, ap.state_g, ap.main, None, cu_e)
 
 
 def test_one_hot_gates_store_the_selected_token():
