@@ -22,6 +22,18 @@ Readings adopted (the pages are garbled or silent on these points):
     it has, and rewritten as more tokens arrive (ceil(N/r) stored entries);
   * window token t = RoPE(x_t, t), stored bf16 (or quantised per token).
 
+Variants (P1 §2.1, §3.1.2, §3.2.1), each optional:
+  * overlapping window (c4a: "an 8-token overlapping state"): entry g folds the
+    tokens [g*r - r, g*r + r) that exist, with a position bias of 2r values,
+    bias[t - (g*r - r)]; the stride stays r, so there are still ceil(N/r)
+    entries, and the RoPE position stays g*r;
+  * RMSNorm in the compressor fusion (compressor -> RMSNorm -> RoPE -> insert):
+    e <- e * w / sqrt(mean_d(e_d^2) + eps) with a per-dim weight w (eps 1e-6),
+    after the weighted sum and before RoPE;
+  * per-channel gates: one logit a_{t,d} per token and dim; the softmax over the
+    entry's tokens is taken separately for every dim d, with the same position
+    bias for all dims.
+
 The oracle works on a sequence's whole token history, so it has no rolling
 state: an append split into chunks must give exactly what one append gives.
 Arithmetic is fp64; the value handed to the quantiser is that fp64 value
@@ -47,25 +59,64 @@ def group_weights(gates, bias):
     return u / u.sum()
 
 
+def entry_tokens(g, ratio, n, overlap=False):
+    """The tokens [lo, hi) entry g folds, and the bias index of token lo.
+
+    Without overlap: the group [g*r, (g+1)*r); with it: [g*r - r, g*r + r).
+    Tokens that do not exist (t < 0 or t >= n) are left out; token t takes
+    bias[t - start] where start = g*r (or g*r - r with overlap).
+
+    Follows P1 §2.1 (groups of r tokens) and §3.1.2 (c4a's 8-token overlap).
+    """
+    start = g * ratio - (ratio if overlap else 0)
+    lo, hi = max(0, start), min(g * ratio + ratio, n)
+    return lo, hi, lo - start
+
+
+def rms_norm(e, weight, eps=1e-6):
+    """e * w / sqrt(mean_d(e_d^2) + eps) over the last axis (fp64).
+
+    Follows P1 §3.2.1 (RMSNorm in the compressor fusion, before RoPE).
+    """
+    e = np.asarray(e, dtype=np.float64)
+    ms = np.mean(e * e, axis=-1, keepdims=True)
+    return e * np.asarray(weight, dtype=np.float64) / np.sqrt(ms + eps)
+
+
 def compress_prequant(x, gates, bias, ratio, n_tokens=None, theta=1e6, rope_dim=64,
-                      rope_offset=448):
+                      rope_offset=448, overlap=False, norm_weight=None, norm_eps=1e-6):
     """Pre-quantisation entries of one sequence, fp32 [ceil(N/r), D].
 
     x: raw tokens [N, D] (any float dtype; bf16 inputs are passed as their
-    exact fp32 values); gates [N]; bias [r]. Only the first ``n_tokens`` tokens
-    are used (default all).
+    exact fp32 values); gates [N] (one logit per token) or [N, D] (per-channel
+    gates); bias [r] (or [2r] with overlap). Only the first ``n_tokens`` tokens
+    are used (default all). overlap: the 8-token c4a window; norm_weight: [D]
+    RMSNorm weights (None: no norm).
 
-    Follows P1 §2.1 (c4a / c128a folding) and §3.1.2 (partial groups).
+    Follows P1 §2.1 (c4a / c128a folding), §3.1.2 (partial groups, the
+    overlapping state) and §3.2.1 (RMSNorm before RoPE).
     """
     x = np.asarray(x, dtype=np.float64)
     gates = np.asarray(gates, dtype=np.float64)
+    per_dim = gates.ndim == 2
     n = x.shape[0] if n_tokens is None else int(n_tokens)
     n_groups = -(-n // ratio)
     out = np.zeros((n_groups, x.shape[1]), dtype=np.float64)
     for g in range(n_groups):
-        lo, hi = g * ratio, min((g + 1) * ratio, n)
-        w = group_weights(gates[lo:hi], bias)
-        out[g] = w @ x[lo:hi]
+        lo, hi, b0 = entry_tokens(g, ratio, n, overlap)
+        b = np.asarray(bias, dtype=np.float64)[b0:b0 + hi - lo]
+        if per_dim:
+            # the softmax over the entry's tokens, separately for every dim
+            z = gates[lo:hi] + b[:, None]
+            z = z - z.max(axis=0, keepdims=True)
+            u = np.exp(z)
+            w = u / u.sum(axis=0, keepdims=True)
+            out[g] = np.sum(w * x[lo:hi], axis=0)
+        else:
+            w = group_weights(gates[lo:hi], b)
+            out[g] = w @ x[lo:hi]
+    if n_groups and norm_weight is not None:
+        out = rms_norm(out, norm_weight, norm_eps)
     if n_groups:
         out = rope_rotate(out, np.arange(n_groups) * ratio, theta, rope_dim, rope_offset)
     return out.astype(np.float32)

@@ -1,10 +1,15 @@
 """Pins for oracle.compressor: the hand-derived example, one-hot gates reducing
-to token selection, uniform gates giving the mean, softmax shift invariance."""
+to token selection, uniform gates giving the mean, softmax shift invariance;
+for the variants, the overlapping window reducing to the plain grouping when
+the history is excluded and to the window mean / one token by brute force,
+RMSNorm against torch's rms_norm and closed forms, per-channel gates reducing
+to scalar gates and to scalar loops."""
 import math
 import os
 
 import numpy as np
 
+import synth
 from oracle import codecs, compressor
 from oracle.rope import rope_rotate
 
@@ -88,3 +93,91 @@ def test_entry_count_and_partial_group():
     e = compressor.compress_prequant(x, g, np.zeros(128), 128, n_tokens=1000, rope_dim=0)
     alone = compressor.compress_prequant(x[896:1000], g[896:1000], np.zeros(128), 128, rope_dim=0)
     assert np.array_equal(e[7], alone[0])
+
+
+# ---- variants: overlapping c4a window, RMSNorm, per-channel gates
+
+
+def test_overlap_with_excluded_history_is_the_plain_grouping():
+    # bias -1e30 on the r tokens before the group makes their weights exactly 0,
+    # so the overlapping entry equals the non-overlapping one with bias[r:]
+    r = synth.rng(70)
+    x = synth.normal(r, (37, 16))
+    g = synth.normal(r, 37)
+    b = synth.normal(r, 8, 0.5)
+    b_ex = b.copy()
+    b_ex[:4] = -1e30
+    e_ov = compressor.compress_prequant(x, g, b_ex, 4, rope_dim=0, overlap=True)
+    e_pl = compressor.compress_prequant(x, g, b[4:], 4, rope_dim=0)
+    assert np.array_equal(e_ov, e_pl)
+
+
+def test_overlap_brute_force_window_mean_and_one_hot():
+    r = synth.rng(71)
+    n, d = 23, 8
+    x = synth.normal(r, (n, d))
+    # uniform gates and zero bias: entry g is the mean of tokens [4g - 4, 4g + 4) that exist
+    e = compressor.compress_prequant(x, np.zeros(n), np.zeros(8), 4, rope_dim=0, overlap=True)
+    for g in range(e.shape[0]):
+        toks = [t for t in range(4 * g - 4, 4 * g + 4) if 0 <= t < n]
+        want = np.float32(sum(x[t].astype(np.float64) for t in toks) / len(toks))
+        assert np.allclose(e[g], want, rtol=1e-6, atol=1e-7), g
+    # one-hot gates picking a token of the previous group: the entry is that token
+    gates = np.full(n, -1e30)
+    gates[5] = 0.0                      # token 5 lies in entry 2's window [4, 12)
+    e = compressor.compress_prequant(x, gates, np.zeros(8), 4, rope_dim=0, overlap=True)
+    assert np.array_equal(e[2], x[5].astype(np.float32))
+
+
+def test_rms_norm_against_torch_and_closed_forms():
+    import torch
+    r = synth.rng(72)
+    v = synth.normal(r, (5, 64)).astype(np.float64)
+    w = 1.0 + synth.normal(r, 64, 0.1)
+    got = compressor.rms_norm(v, w, 1e-6)
+    want = torch.nn.functional.rms_norm(torch.from_numpy(v), (64,), torch.from_numpy(w.astype(np.float64)),
+                                        eps=1e-6).numpy()
+    assert np.allclose(got, want, rtol=1e-12, atol=0)
+    # a constant vector c: each element becomes c / sqrt(c^2 + eps) times the weight
+    c = 3.0
+    out = compressor.rms_norm(np.full(8, c), np.ones(8), 1e-6)
+    assert np.allclose(out, c / np.sqrt(c * c + 1e-6), rtol=1e-15)
+
+
+def test_norm_applies_before_rope():
+    # RMSNorm (weights 1) keeps the vector's direction and RoPE keeps its norm:
+    # the rope dims of the normed, rotated entry have the norm the pre-RoPE
+    # normed vector has, and the other dims equal the normed vector
+    r = synth.rng(73)
+    x = synth.normal(r, (8, 512))
+    g = synth.normal(r, 8)
+    w = np.ones(512)
+    e_n = compressor.compress_prequant(x, g, np.zeros(4), 4, norm_weight=w)
+    e_raw = compressor.compress_prequant(x, g, np.zeros(4), 4, rope_dim=0).astype(np.float64)
+    normed = compressor.rms_norm(e_raw, w)
+    assert np.allclose(e_n[:, :448], normed[:, :448], rtol=1e-6, atol=1e-6)
+    assert np.allclose(np.linalg.norm(e_n[:, 448:], axis=1), np.linalg.norm(normed[:, 448:], axis=1), rtol=1e-5)
+
+
+def test_per_channel_gates_reduce_to_scalar_gates_and_brute_force():
+    r = synth.rng(74)
+    n, d = 13, 6
+    x = synth.normal(r, (n, d))
+    g = synth.normal(r, n)
+    b = synth.normal(r, 4, 0.5)
+    # the same logit on every channel: the scalar-gate entries, bit for bit
+    same = np.repeat(g[:, None], d, axis=1)
+    assert np.array_equal(compressor.compress_prequant(x, same, b, 4, rope_dim=0),
+                          compressor.compress_prequant(x, g, b, 4, rope_dim=0))
+    # independent channel logits: scalar loops
+    gd = synth.normal(r, (n, d))
+    e = compressor.compress_prequant(x, gd, b, 4, rope_dim=0)
+    for gi in range(e.shape[0]):
+        lo, hi = 4 * gi, min(4 * gi + 4, n)
+        for c in range(d):
+            z = [gd[t, c] + b[t - lo] for t in range(lo, hi)]
+            m = max(z)
+            u = [np.exp(v - m) for v in z]
+            s = sum(u)
+            want = sum(u[k] / s * float(x[lo + k, c]) for k in range(hi - lo))
+            assert abs(float(e[gi, c]) - want) <= 1e-6 * max(1.0, abs(want)), (gi, c)
