@@ -175,6 +175,43 @@ v4kv_status v4kv_compress_append(const void* x, const float* gate, const int32_t
                                  float* prequant_out, int32_t* dev_status, void* stream);
 
 /*
+ * v4kv_compress_append_ex -- v4kv_compress_append with the compressor
+ * variants the pages describe (P1 §2.1; §3.1.2 "an 8-token overlapping
+ * state" for c4a; §3.2.1 RMSNorm in the compressor fusion). opts NULL or all
+ * zero is v4kv_compress_append.
+ *   overlap          1: entry g folds the present tokens [g*r - r, g*r + r)
+ *                    (ratio 4 only, else V4KV_ERR_UNSUPPORTED); pos_bias then
+ *                    holds 2r values, token t taking pos_bias[t - (g*r - r)];
+ *                    the state holds 2r rows per sequence (state_x
+ *                    [batch, 2r, dim], state_gate [batch, 2r]); the RoPE
+ *                    position stays g*r
+ *   gate_per_channel 1: gate is fp32 [total_tokens, dim], one logit per token
+ *                    and dim, and the softmax over an entry's tokens is taken
+ *                    per dim; state_gate is then [batch, rows, dim]; gate and
+ *                    state_gate 16-byte aligned
+ *   norm_weight      fp32 [dim], 16-byte aligned, or NULL: the summed entry
+ *                    becomes e * w / sqrt(mean(e^2) + norm_eps) before RoPE
+ *                    (norm_eps 0 means 1e-6)
+ * With overlap or per-channel gates one block builds each entry (a slower
+ * kernel than the plain path); RMSNorm alone keeps the plain kernels.
+ */
+typedef struct v4kv_compress_opts {
+  int32_t overlap;
+  int32_t gate_per_channel;
+  const float* norm_weight;
+  float norm_eps;
+} v4kv_compress_opts;
+
+v4kv_status v4kv_compress_append_ex(const void* x, const float* gate, const int32_t* cu_seqlens,
+                                    const int32_t* seq_start, int32_t batch, int32_t total_tokens,
+                                    const float* pos_bias, int32_t ratio, v4kv_rope rope,
+                                    void* state_x, float* state_gate, const v4kv_paged* main_cache,
+                                    const int64_t* slot_mapping, const int32_t* cu_entries,
+                                    const v4kv_paged* window, int32_t window_len,
+                                    float* prequant_out, const v4kv_compress_opts* opts,
+                                    int32_t* dev_status, void* stream);
+
+/*
  * v4kv_index_topk -- indexer scores and exact top-k over a c4a layer's
  * visible entries (P1 §2.2 indexer cache; P1 §4.1 sparse attention over
  * the selected c4a entries).

@@ -129,8 +129,29 @@ v4kv_status v4kv_compress_append(const void* x, const float* gate, const int32_t
                                  const int64_t* slot_mapping, const int32_t* cu_entries,
                                  const v4kv_paged* window, int32_t window_len,
                                  float* prequant_out, int32_t* dev_status, void* stream) {
+  return v4kv_compress_append_ex(x, gate, cu_seqlens, seq_start, batch, total_tokens, pos_bias,
+                                 ratio, rope, state_x, state_gate, main_cache, slot_mapping,
+                                 cu_entries, window, window_len, prequant_out, nullptr, dev_status,
+                                 stream);
+}
+
+v4kv_status v4kv_compress_append_ex(const void* x, const float* gate, const int32_t* cu_seqlens,
+                                    const int32_t* seq_start, int32_t batch, int32_t total_tokens,
+                                    const float* pos_bias, int32_t ratio, v4kv_rope rope,
+                                    void* state_x, float* state_gate, const v4kv_paged* main_cache,
+                                    const int64_t* slot_mapping, const int32_t* cu_entries,
+                                    const v4kv_paged* window, int32_t window_len,
+                                    float* prequant_out, const v4kv_compress_opts* opts,
+                                    int32_t* dev_status, void* stream) {
   if (batch <= 0 || total_tokens < 0) return V4KV_ERR_INVALID_ARG;
   if (ratio != 4 && ratio != 128) return V4KV_ERR_INVALID_ARG;
+  const int overlap = opts ? opts->overlap : 0;
+  const int per_channel = opts ? opts->gate_per_channel : 0;
+  const float* norm_w = opts ? opts->norm_weight : nullptr;
+  if ((overlap != 0 && overlap != 1) || (per_channel != 0 && per_channel != 1)) return V4KV_ERR_INVALID_ARG;
+  if (overlap && ratio != 4) return V4KV_ERR_UNSUPPORTED;  // the overlapping window is c4a's
+  if (norm_w && (!aligned16(norm_w) || !(opts->norm_eps >= 0.f))) return V4KV_ERR_INVALID_ARG;
+  if (per_channel && ((gate && !aligned16(gate)) || !aligned16(state_gate))) return V4KV_ERR_INVALID_ARG;
   if (!cu_seqlens || !seq_start || !pos_bias || !state_x || !state_gate) return V4KV_ERR_INVALID_ARG;
   // the slot mapping comes from v4kv_slot_mapping, or (both NULL) is computed
   // inside the kernel from main_cache's block table, for batch < 1024
@@ -170,6 +191,11 @@ v4kv_status v4kv_compress_append(const void* x, const float* gate, const int32_t
   a.ratio = ratio;
   a.dim = dim;
   a.window_len = window ? window_len : 0;
+  a.overlap = overlap;
+  a.gate_dim = per_channel ? dim : 1;
+  a.state_rows = overlap ? 2 * ratio : ratio;
+  a.norm_w = norm_w;
+  a.norm_eps = norm_w ? (opts->norm_eps > 0.f ? opts->norm_eps : 1e-6f) : 0.f;
   // every sequence touches at most ceil(n/r) + 1 groups
   const long long max_groups = (long long)total_tokens / ratio + 2LL * batch;
   if (max_groups > 0x7fffffffLL) return V4KV_ERR_INVALID_ARG;

@@ -207,11 +207,36 @@ __device__ __forceinline__ void weighted_rows(const CompressArgs& a, int b, int 
   }
 }
 
-// RoPE at the group's first position, optional pre-quantisation copy, and
-// the store into the entry's slot
+// RMSNorm of one vector held by a warp: e * w / sqrt(mean(e^2) + eps)
+template <int KC>
+__device__ __forceinline__ void rms_norm_warp(float (&e)[KC][8], int lane, int nch, const float* w,
+                                              float eps, int dim) {
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < KC; ++k)
+    if (lane + 32 * k < nch)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss = fmaf(e[k][i], e[k][i], ss);
+  ss = warp_sum(ss);
+  const float inv = __fdiv_rn(1.f, __fsqrt_rn(__fdiv_rn(ss, (float)dim) + eps));
+#pragma unroll
+  for (int k = 0; k < KC; ++k) {
+    const int c = lane + 32 * k;
+    if (c >= nch) continue;
+    const float4 w0 = *reinterpret_cast<const float4*>(w + 8 * c);
+    const float4 w1 = *reinterpret_cast<const float4*>(w + 8 * c + 4);
+    const float ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) e[k][i] = e[k][i] * inv * ww[i];
+  }
+}
+
+// RMSNorm (when weights are given), RoPE at the group's first position,
+// optional pre-quantisation copy, and the store into the entry's slot
 template <int KC>
 __device__ __forceinline__ void finish_entry(const CompressArgs& a, int i, int b, int t0, int lane,
                                              int nch, float (&e)[KC][8]) {
+  if (a.norm_w) rms_norm_warp<KC>(e, lane, nch, a.norm_w, a.norm_eps, a.dim);
   rope_warp<KC>(e, lane, nch, a.rope, (long long)t0);
   if (a.prequant_out) {
 #pragma unroll
@@ -279,27 +304,11 @@ __device__ __forceinline__ int seq_of(const int32_t* cu, int batch, int i) {
   return lo;
 }
 
-// KC: 8-dim chunks per lane (dim <= 256 * KC). kBlockGroup: one block per
-// group (ratio > 32) instead of one warp per group.
-template <int KC, bool kBlockGroup>
-__global__ void __launch_bounds__(kWarps * 32) compress_append_kernel(CompressArgs a,
-                                                                     int window_blocks,
-                                                                     int window_blocks_per_seq) {
-  constexpr int kRB = (KC <= 2 && kBlockGroup) ? 8 : 4;  // rows in flight per warp
-  constexpr int kNQ = kBlockGroup ? kMaxRatio / 32 : 1;  // gates per lane
-  __shared__ float w_sh[kWarps][kNQ * 32];
-  __shared__ float part[kBlockGroup ? kWarps : 1][kBlockGroup ? KC * 256 : 1];
-  __shared__ int cu_sh[kCuSmem];
-  tc::pdl_wait();  // the slot mapping (and whatever produced x) is complete from here on
-  tc::pdl_launch_dependents();
+// The entry prefix sums of the call (entries touched per sequence), in cu_sh
+// when they fit or are computed here (no slot mapping given); returns the
+// array to use. All threads of the block call it.
+__device__ __forceinline__ const int32_t* entry_prefix(const CompressArgs& a, int* cu_sh) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nch = a.dim >> 3;
-  if ((int)blockIdx.x < window_blocks) {
-    window_row<KC>(a, blockIdx.x / window_blocks_per_seq,
-                   (blockIdx.x % window_blocks_per_seq) * kWarps + warp, lane, nch);
-    return;
-  }
-  const int eb = blockIdx.x - window_blocks;
   const bool cached = a.batch + 1 <= kCuSmem;
   if (!a.cu_entries) {
     // no slot mapping given: the entry counts (groups touched by each
@@ -329,11 +338,38 @@ __global__ void __launch_bounds__(kWarps * 32) compress_append_kernel(CompressAr
     }
     if (threadIdx.x == 0) cu_sh[a.batch] = carry;
     __syncthreads();
-  } else if (cached) {
+    return cu_sh;
+  }
+  if (cached) {
     for (int k = threadIdx.x; k <= a.batch; k += blockDim.x) cu_sh[k] = a.cu_entries[k];
     __syncthreads();
+    return cu_sh;
   }
-  const int32_t* cu = (cached || !a.cu_entries) ? cu_sh : a.cu_entries;
+  return a.cu_entries;
+}
+
+// KC: 8-dim chunks per lane (dim <= 256 * KC). kBlockGroup: one block per
+// group (ratio > 32) instead of one warp per group.
+template <int KC, bool kBlockGroup>
+__global__ void __launch_bounds__(kWarps * 32) compress_append_kernel(CompressArgs a,
+                                                                     int window_blocks,
+                                                                     int window_blocks_per_seq) {
+  constexpr int kRB = (KC <= 2 && kBlockGroup) ? 8 : 4;  // rows in flight per warp
+  constexpr int kNQ = kBlockGroup ? kMaxRatio / 32 : 1;  // gates per lane
+  __shared__ float w_sh[kWarps][kNQ * 32];
+  __shared__ float part[kBlockGroup ? kWarps : 1][kBlockGroup ? KC * 256 : 1];
+  __shared__ int cu_sh[kCuSmem];
+  tc::pdl_wait();  // the slot mapping (and whatever produced x) is complete from here on
+  tc::pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nch = a.dim >> 3;
+  if ((int)blockIdx.x < window_blocks) {
+    window_row<KC>(a, blockIdx.x / window_blocks_per_seq,
+                   (blockIdx.x % window_blocks_per_seq) * kWarps + warp, lane, nch);
+    return;
+  }
+  const int eb = blockIdx.x - window_blocks;
+  const int32_t* cu = entry_prefix(a, cu_sh);
   const int total = cu[a.batch];
   const int i = kBlockGroup ? eb : eb * kWarps + warp;
   if (i >= total) return;  // uniform over the warp (and over the block for block groups)
@@ -410,6 +446,248 @@ __global__ void __launch_bounds__(kWarps * 32) compress_append_kernel(CompressAr
   }
 }
 
+
+// ---------------------------------------------------------------- variants
+// One block per entry. Token k of the entry's span (k = t - start, start =
+// g*r, or g*r - r with the overlapping window) belongs to warp k / rpw, rpw =
+// ceil(span / 8); for every dim the softmax over the present tokens runs in
+// two passes through shared memory (the maxima, then the weighted sums, each
+// warp over its tokens in ascending order, added in warp order), so the
+// arithmetic depends only on a token's place in the span. Per-token gates are
+// the case of one logit for all dims.
+
+// logit of token tt (of sequence b, seq_start s) for dims 8c .. 8c + 7
+__device__ __forceinline__ void gate_chunk(const CompressArgs& a, int b, int s, int old_base, int tt, int c,
+                                           float (&z)[8]) {
+  const int rows = a.state_rows;
+  if (a.gate_dim == 1) {
+    const float g = tt < s ? a.state_gate[(size_t)b * rows + (tt - old_base)]
+                           : a.gate[a.cu_seqlens[b] + (tt - s)];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) z[i] = g;
+  } else {
+    const float* row = tt < s ? a.state_gate + ((size_t)b * rows + (tt - old_base)) * a.dim
+                              : a.gate + (size_t)(a.cu_seqlens[b] + (tt - s)) * a.dim;
+    const float4 u = *reinterpret_cast<const float4*>(row + 8 * c);
+    const float4 v = *reinterpret_cast<const float4*>(row + 8 * c + 4);
+    z[0] = u.x; z[1] = u.y; z[2] = u.z; z[3] = u.w; z[4] = v.x; z[5] = v.y; z[6] = v.z; z[7] = v.w;
+  }
+}
+
+template <int KC>
+__device__ void variant_entry(const CompressArgs& a, int i, int b, const int32_t* cu, float* sh_m,
+                              float* sh_s, float* sh_v) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nch = a.dim >> 3;
+  const int r = a.ratio;
+  const int s = a.seq_start[b];
+  const int end = s + (a.cu_seqlens[b + 1] - a.cu_seqlens[b]);
+  const int t0 = (s / r + (i - cu[b])) * r;
+  const int span = a.overlap ? 2 * r : r;
+  const int start = t0 - (a.overlap ? r : 0);
+  const int lo = max(0, start), hi = min(t0 + r, end);
+  const int old_base = (s / r) * r - (a.overlap ? r : 0);
+  const int rpw = (span + kWarps - 1) / kWarps;
+  const int k0 = max(warp * rpw, lo - start), k1 = min((warp + 1) * rpw, hi - start);
+  // pass 1: this warp's maxima per dim
+  float m[KC][8];
+#pragma unroll
+  for (int k = 0; k < KC; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m[k][e] = -INFINITY;
+  for (int kk = k0; kk < k1; ++kk) {
+    const float bias = a.pos_bias[kk];
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      const int c = lane + 32 * k;
+      if (c >= nch) continue;
+      float z[8];
+      gate_chunk(a, b, s, old_base, start + kk, c, z);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m[k][e] = fmaxf(m[k][e], z[e] + bias);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < KC; ++k) {
+    const int c = lane + 32 * k;
+    if (c >= nch) continue;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sh_m[warp * a.dim + 8 * c + e] = m[k][e];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < KC; ++k) {
+    const int c = lane + 32 * k;
+    if (c >= nch) continue;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float mm = -INFINITY;
+      for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sh_m[w * a.dim + 8 * c + e]);
+      m[k][e] = mm;
+    }
+  }
+  // pass 2: this warp's sums of exp(z - m) and of exp(z - m) * x per dim
+  float su[KC][8], sv[KC][8];
+#pragma unroll
+  for (int k = 0; k < KC; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) su[k][e] = sv[k][e] = 0.f;
+  for (int kk = k0; kk < k1; ++kk) {
+    const int tt = start + kk;
+    const float bias = a.pos_bias[kk];
+    const uint16_t* xrow = tt < s ? a.state_x + ((size_t)b * a.state_rows + (tt - old_base)) * a.dim
+                                  : a.x + (size_t)(a.cu_seqlens[b] + (tt - s)) * a.dim;
+    uint4 q[KC];
+    load_row<KC>(xrow, lane, nch, q);
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      const int c = lane + 32 * k;
+      if (c >= nch) continue;
+      float z[8], x[8];
+      gate_chunk(a, b, s, old_base, tt, c, z);
+      unpack_bf16x8(q[k], x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float u = expf(z[e] + bias - m[k][e]);
+        su[k][e] += u;
+        sv[k][e] = fmaf(u, x[e], sv[k][e]);
+      }
+    }
+  }
+  __syncthreads();  // every warp has read the maxima
+#pragma unroll
+  for (int k = 0; k < KC; ++k) {
+    const int c = lane + 32 * k;
+    if (c >= nch) continue;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      sh_s[warp * a.dim + 8 * c + e] = su[k][e];
+      sh_v[warp * a.dim + 8 * c + e] = sv[k][e];
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float acc[KC][8];
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      const int c = lane + 32 * k;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float S = 0.f, V = 0.f;
+        if (c < nch)
+          for (int w = 0; w < kWarps; ++w) {
+            S += sh_s[w * a.dim + 8 * c + e];
+            V += sh_v[w * a.dim + 8 * c + e];
+          }
+        acc[k][e] = c < nch ? __fdiv_rn(V, S) : 0.f;
+      }
+    }
+    finish_entry<KC>(a, i, b, t0, lane, nch, acc);
+  }
+  __syncthreads();  // the scratch is free again
+}
+
+// state rows after the call: the tokens [max(0, base), end), base = the last
+// group start (minus r with the overlapping window), at row t - base; a token
+// from before the call moves from its old row t - old_base >= t - base, so
+// rows are copied in ascending order by one warp
+template <int KC>
+__device__ void variant_state(const CompressArgs& a, int b) {
+  const int lane = threadIdx.x & 31;
+  const int nch = a.dim >> 3;
+  const int r = a.ratio;
+  const int s = a.seq_start[b];
+  const int end = s + (a.cu_seqlens[b + 1] - a.cu_seqlens[b]);
+  const int ov = a.overlap ? r : 0;
+  const int base = (end / r) * r - ov, old_base = (s / r) * r - ov;
+  for (int tt = max(0, base); tt < end; ++tt) {
+    const int row = tt - base;
+    const uint16_t* src = tt < s ? a.state_x + ((size_t)b * a.state_rows + (tt - old_base)) * a.dim
+                                 : a.x + (size_t)(a.cu_seqlens[b] + (tt - s)) * a.dim;
+    uint4 q[KC];
+    load_row<KC>(src, lane, nch, q);
+    float gsc = 0.f;
+    float4 gv[KC][2];
+    if (a.gate_dim == 1) {
+      gsc = tt < s ? a.state_gate[(size_t)b * a.state_rows + (tt - old_base)]
+                   : a.gate[a.cu_seqlens[b] + (tt - s)];
+    } else {
+      const float* grow = tt < s ? a.state_gate + ((size_t)b * a.state_rows + (tt - old_base)) * a.dim
+                                 : a.gate + (size_t)(a.cu_seqlens[b] + (tt - s)) * a.dim;
+#pragma unroll
+      for (int k = 0; k < KC; ++k) {
+        const int c = lane + 32 * k;
+        if (c < nch) {
+          gv[k][0] = *reinterpret_cast<const float4*>(grow + 8 * c);
+          gv[k][1] = *reinterpret_cast<const float4*>(grow + 8 * c + 4);
+        }
+      }
+    }
+    __syncwarp();  // every lane has read the source row before it is overwritten
+    uint16_t* dst = a.state_x_out + ((size_t)b * a.state_rows + row) * a.dim;
+#pragma unroll
+    for (int k = 0; k < KC; ++k)
+      if (lane + 32 * k < nch) *reinterpret_cast<uint4*>(dst + 8 * (lane + 32 * k)) = q[k];
+    if (a.gate_dim == 1) {
+      if (lane == 0) a.state_gate_out[(size_t)b * a.state_rows + row] = gsc;
+    } else {
+      float* gdst = a.state_gate_out + ((size_t)b * a.state_rows + row) * a.dim;
+#pragma unroll
+      for (int k = 0; k < KC; ++k) {
+        const int c = lane + 32 * k;
+        if (c < nch) {
+          *reinterpret_cast<float4*>(gdst + 8 * c) = gv[k][0];
+          *reinterpret_cast<float4*>(gdst + 8 * c + 4) = gv[k][1];
+        }
+      }
+    }
+    __syncwarp();
+  }
+}
+
+template <int KC>
+__global__ void __launch_bounds__(kWarps * 32) compress_variant_kernel(CompressArgs a, int window_blocks,
+                                                                      int window_blocks_per_seq) {
+  extern __shared__ float vsm[];  // 3 x kWarps x dim: maxima, sums, weighted sums
+  __shared__ int cu_sh[kCuSmem];
+  tc::pdl_wait();  // x, the gates and the state (earlier work in the stream) are complete
+  tc::pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nch = a.dim >> 3;
+  if ((int)blockIdx.x < window_blocks) {
+    window_row<KC>(a, blockIdx.x / window_blocks_per_seq,
+                   (blockIdx.x % window_blocks_per_seq) * kWarps + warp, lane, nch);
+    return;
+  }
+  const int32_t* cu = entry_prefix(a, cu_sh);
+  const int i = blockIdx.x - window_blocks;
+  if (i >= cu[a.batch]) return;
+  const int b = seq_of(cu, a.batch, i);
+  // The old state is read by the sequence's first entry of the call, and with
+  // the overlapping window also by its second: one block builds both and then
+  // rewrites the state.
+  if (a.overlap && i == cu[b] + 1) return;
+  float* sh_m = vsm;
+  float* sh_s = vsm + kWarps * a.dim;
+  float* sh_v = vsm + 2 * kWarps * a.dim;
+  variant_entry<KC>(a, i, b, cu, sh_m, sh_s, sh_v);
+  if (i == cu[b]) {
+    if (a.overlap && i + 1 < cu[b + 1]) variant_entry<KC>(a, i + 1, b, cu, sh_m, sh_s, sh_v);
+    if (warp == 0) variant_state<KC>(a, b);
+  }
+}
+
+template <int KC>
+cudaError_t launch_variant_kc(const CompressArgs& a, int max_groups, int window_blocks, int per_seq,
+                              cudaStream_t stream) {
+  const size_t smem = (size_t)3 * kWarps * a.dim * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(compress_variant_kernel<KC>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(compress_variant_kernel<KC>, dim3(window_blocks + max_groups), dim3(kWarps * 32),
+                    smem, stream, a, window_blocks, per_seq);
+}
+
 template <int KC>
 cudaError_t launch_kc(const CompressArgs& a, int max_groups, int window_blocks, int per_seq,
                       cudaStream_t stream) {
@@ -434,6 +712,13 @@ cudaError_t launch_compress_append(const CompressArgs& a, int max_groups, int to
   if (wb + max_groups > 0x7fffffffLL) return cudaErrorInvalidValue;
   if (wb + max_groups == 0) return cudaSuccess;
   const int kc = (a.dim + 255) / 256;
+  if (a.overlap || a.gate_dim != 1) {
+    // the variant kernel (one block per entry); RMSNorm alone runs in the
+    // regular kernels
+    if (kc <= 1) return launch_variant_kc<1>(a, max_groups, (int)wb, per_seq, stream);
+    if (kc <= 2) return launch_variant_kc<2>(a, max_groups, (int)wb, per_seq, stream);
+    return launch_variant_kc<4>(a, max_groups, (int)wb, per_seq, stream);
+  }
   if (kc <= 1) return launch_kc<1>(a, max_groups, (int)wb, per_seq, stream);
   if (kc <= 2) return launch_kc<2>(a, max_groups, (int)wb, per_seq, stream);
   return launch_kc<4>(a, max_groups, (int)wb, per_seq, stream);

@@ -51,6 +51,12 @@ struct CompressArgs {
   int ratio;
   int dim;
   int window_len;
+  // variants (all off by default)
+  int overlap;          // 1: entry g folds tokens [g*r - r, g*r + r) (pos_bias has 2r values)
+  int gate_dim;         // 1: one logit per token; dim: one per token and dim
+  int state_rows;       // rows of the state per sequence: r, or 2r with the overlap
+  const float* norm_w;  // [dim] RMSNorm weights, or null
+  float norm_eps;
 };
 
 struct IndexArgs {

@@ -34,6 +34,7 @@ V4KV_OP_DECODE = 2
 
 EXPORTED = [
     "v4kv_status_string", "v4kv_version", "v4kv_slot_mapping", "v4kv_compress_append",
+    "v4kv_compress_append_ex",
     "v4kv_index_topk", "v4kv_decode_attention", "v4kv_workspace_size", "v4kv_kv_footprint_bytes",
     "v4kv_decode_attention_noalloc", "v4kv_decode_attention_fp8out",
     "v4kv_page_bytes", "v4kv_plan_buckets", "v4kv_page_pools_create", "v4kv_page_pools_destroy",
@@ -61,6 +62,11 @@ class _Rope(ctypes.Structure):
                 ("rope_offset", ctypes.c_int32)]
 
 
+class _CompressOpts(ctypes.Structure):
+    _fields_ = [("overlap", ctypes.c_int32), ("gate_per_channel", ctypes.c_int32),
+                ("norm_weight", ctypes.c_void_p), ("norm_eps", ctypes.c_float)]
+
+
 class _Footprint(ctypes.Structure):
     _fields_ = [("n_layers", ctypes.c_int32), ("layer_ratios", ctypes.POINTER(ctypes.c_int32)),
                 ("dim", ctypes.c_int32), ("entry_bits", ctypes.c_int32),
@@ -81,6 +87,9 @@ def _load():
         "v4kv_compress_append": (I32, [P, P, P, P, I32, I32, P, I32, _Rope, P, P,
                                        ctypes.POINTER(_Paged), P, P, ctypes.POINTER(_Paged), I32,
                                        P, P, P]),
+        "v4kv_compress_append_ex": (I32, [P, P, P, P, I32, I32, P, I32, _Rope, P, P,
+                                          ctypes.POINTER(_Paged), P, P, ctypes.POINTER(_Paged), I32,
+                                          P, ctypes.POINTER(_CompressOpts), P, P]),
         "v4kv_index_topk": (I32, [P, ctypes.POINTER(_Paged), P, I32, I32, I32, I32, I32, P, P, P,
                                   SZ, P, P]),
         "v4kv_decode_attention": (I32, [P, I32, I32, I32, ctypes.POINTER(_Paged),
@@ -206,14 +215,19 @@ def v4kv_slot_mapping(block_table, seq_start, n_new, ratio, num_pages, slot_out,
 
 def v4kv_compress_append(x, gate, cu_seqlens, seq_start, pos_bias, ratio, state_x, state_gate,
                          main, slot_mapping, cu_entries, window=None, window_len=128,
-                         rope=None, prequant_out=None, dev_status=None, stream=None):
+                         rope=None, prequant_out=None, dev_status=None, stream=None,
+                         overlap=False, gate_per_channel=False, norm_weight=None, norm_eps=0.0):
+    """v4kv_compress_append; with any of overlap, gate_per_channel, norm_weight
+    set, v4kv_compress_append_ex with those options."""
     _need(x, (torch.bfloat16,), "x", ndim=2)
     _need(gate, (torch.float32,), "gate")
     _need(cu_seqlens, (torch.int32,), "cu_seqlens")
     _need(seq_start, (torch.int32,), "seq_start")
     _need(pos_bias, (torch.float32,), "pos_bias")
     _need(state_x, (torch.bfloat16,), "state_x", ndim=3)
-    _need(state_gate, (torch.float32,), "state_gate", ndim=2)
+    _need(state_gate, (torch.float32,), "state_gate", ndim=3 if gate_per_channel else 2)
+    if norm_weight is not None:
+        _need(norm_weight, (torch.float32,), "norm_weight")
     if (slot_mapping is None) != (cu_entries is None):
         raise ValueError("slot_mapping and cu_entries: both or neither")
     if slot_mapping is not None:
@@ -222,13 +236,18 @@ def v4kv_compress_append(x, gate, cu_seqlens, seq_start, pos_bias, ratio, state_
     rope = rope or Rope()
     mc = main.c()
     wc = window.c() if window is not None else None
-    st = _lib.v4kv_compress_append(
-        x.data_ptr(), gate.data_ptr(), cu_seqlens.data_ptr(), seq_start.data_ptr(),
-        seq_start.numel(), x.shape[0], pos_bias.data_ptr(), ratio, rope.c(), state_x.data_ptr(),
-        state_gate.data_ptr(), ctypes.byref(mc), _ptr(slot_mapping), _ptr(cu_entries),
-        ctypes.byref(wc) if wc is not None else None, window_len, _ptr(prequant_out),
-        _ptr(dev_status), _stream(stream))
-    _check("v4kv_compress_append", st)
+    args = (x.data_ptr(), gate.data_ptr(), cu_seqlens.data_ptr(), seq_start.data_ptr(),
+            seq_start.numel(), x.shape[0], pos_bias.data_ptr(), ratio, rope.c(), state_x.data_ptr(),
+            state_gate.data_ptr(), ctypes.byref(mc), _ptr(slot_mapping), _ptr(cu_entries),
+            ctypes.byref(wc) if wc is not None else None, window_len, _ptr(prequant_out))
+    if overlap or gate_per_channel or norm_weight is not None:
+        opts = _CompressOpts(int(bool(overlap)), int(bool(gate_per_channel)), _ptr(norm_weight),
+                             float(norm_eps))
+        st = _lib.v4kv_compress_append_ex(*args, ctypes.byref(opts), _ptr(dev_status), _stream(stream))
+        _check("v4kv_compress_append_ex", st)
+    else:
+        st = _lib.v4kv_compress_append(*args, _ptr(dev_status), _stream(stream))
+        _check("v4kv_compress_append", st)
 
 
 def v4kv_workspace_size(op, batch, heads, max_seq_len, ratio, window_len, k, main_dtype, dim=512):

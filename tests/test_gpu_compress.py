@@ -18,7 +18,8 @@ class Appender:
     """Runs appends of per-sequence chunks through the library."""
 
     def __init__(self, seed, n_tokens, ratio, main_dtype="fp8", W=128, gates=None, dim=D,
-                 rope=True, win_dtype="bf16", x=None, bias=None):
+                 rope=True, win_dtype="bf16", x=None, bias=None, overlap=False, per_channel=False,
+                 norm=False):
         from paged_compressed_kv_b200 import PagedPool, Rope
         self.r = synth.rng(seed)
         self.n = [int(v) for v in n_tokens]
@@ -30,8 +31,15 @@ class Appender:
         self.x = [codecs.bf16_round(v) for v in self.x]             # exact bf16 values
         if x is not None:
             self.x = [codecs.bf16_round(np.asarray(v, dtype=np.float32)) for v in x]
-        self.g = gates if gates is not None else [synth.normal(self.r, N) for N in self.n]
-        self.bias = synth.normal(self.r, ratio, 0.5)
+        self.overlap, self.per_channel = overlap, per_channel
+        if gates is not None:
+            self.g = gates
+        elif per_channel:
+            self.g = [synth.normal(self.r, (N, dim)) for N in self.n]
+        else:
+            self.g = [synth.normal(self.r, N) for N in self.n]
+        self.bias = synth.normal(self.r, 2 * ratio if overlap else ratio, 0.5)
+        self.norm_w = (1.0 + synth.normal(self.r, dim, 0.1)).astype(np.float32) if norm else None
         if bias is not None:
             self.bias = np.asarray(bias, dtype=np.float32)
         spb = 256 // ratio
@@ -54,8 +62,10 @@ class Appender:
         else:
             self.win = PagedPool(data=torch.zeros(self.Pw, 256, dim, dtype=torch.bfloat16, device=dev),
                                  block_table=torch.from_numpy(self.wbt).to(dev))
-        self.state_x = torch.zeros(self.B, ratio, dim, dtype=torch.bfloat16, device=dev)
-        self.state_g = torch.zeros(self.B, ratio, dtype=torch.float32, device=dev)
+        rows = 2 * ratio if overlap else ratio
+        self.state_x = torch.zeros(self.B, rows, dim, dtype=torch.bfloat16, device=dev)
+        self.state_g = torch.zeros((self.B, rows, dim) if per_channel else (self.B, rows),
+                                   dtype=torch.float32, device=dev)
         self.done = [0] * self.B
         self.prequant = [np.full((paging.entry_count(N, ratio), dim), np.nan, np.float32) for N in self.n]
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -93,7 +103,9 @@ class Appender:
             synth.bf16_tensor(xs).to(dev).reshape(-1, self.dim), torch.from_numpy(gs).to(dev),
             torch.from_numpy(cu).to(dev), ss, torch.from_numpy(self.bias).to(dev), self.ratio,
             self.state_x, self.state_g, self.main, slots, cu_e, window=self.win, window_len=self.W,
-            rope=self.rope, prequant_out=pre, dev_status=self.status)
+            rope=self.rope, prequant_out=pre, dev_status=self.status, overlap=self.overlap,
+            gate_per_channel=self.per_channel,
+            norm_weight=None if self.norm_w is None else torch.from_numpy(self.norm_w).to(dev))
         pre = pre.cpu().numpy()
         for b in range(self.B):
             first, end = paging.touched_range(self.done[b], sizes[b], self.ratio)
@@ -145,7 +157,8 @@ def check_against_oracle(ap):
     for b in range(ap.B):
         N = ap.n[b]
         ref = compressor.compress_prequant(ap.x[b], ap.g[b], ap.bias, ap.ratio, rope_dim=rope_dim,
-                                           rope_offset=ap.rope.rope_offset)
+                                           rope_offset=ap.rope.rope_offset, overlap=ap.overlap,
+                                           norm_weight=ap.norm_w)
         got = ap.prequant[b]
         assert not np.isnan(got).any()
         amax = np.abs(ref).max(axis=1, keepdims=True)
@@ -176,10 +189,14 @@ def check_against_oracle(ap):
             xmax = np.abs(ap.x[b][w0:]).max(axis=1, keepdims=True) if N else 0.0
             bound = np.abs(wref) * 2.0**-7 + xmax * 2.0**-20 + 1e-30
             assert np.all(np.abs(wgot - wref) <= bound), f"seq {b}: window"
-        # state: the unfinished group's raw tokens and gates
-        gs = (N // ap.ratio) * ap.ratio
-        st = ap.state_x[b, : N - gs].float().cpu().numpy()
-        assert np.array_equal(st, ap.x[b][gs:N]), f"seq {b}: state"
+        # state: the raw tokens and gates of the unfinished group (and, with
+        # the overlapping window, of the group before it) at row t - base
+        base = (N // ap.ratio) * ap.ratio - (ap.ratio if ap.overlap else 0)
+        lo = max(0, base)
+        st = ap.state_x[b, lo - base: N - base].float().cpu().numpy()
+        assert np.array_equal(st, ap.x[b][lo:N]), f"seq {b}: state"
+        sg = ap.state_g[b, lo - base: N - base].cpu().numpy()
+        assert np.array_equal(sg, np.asarray(ap.g[b][lo:N], dtype=np.float32)), f"seq {b}: state gates"
 
 
 @pytest.mark.parametrize("ratio", [4, 128])
@@ -410,3 +427,47 @@ def test_quantiser_edge_cases_through_the_compressor():
     under = np.abs(q4) < 2.0 ** -10
     assert under.sum() >= 8
     assert np.all(rows[4][under] == 0x80)
+
+
+VARIANTS = [
+    (4, dict(overlap=True)),
+    (4, dict(per_channel=True)),
+    (128, dict(per_channel=True)),
+    (4, dict(norm=True)),
+    (128, dict(norm=True)),
+    (4, dict(overlap=True, per_channel=True, norm=True)),
+]
+
+
+@pytest.mark.parametrize("ratio,opts", VARIANTS)
+def test_variants_match_oracle_and_chunking(ratio, opts):
+    """The compressor variants (P1 §2.1, §3.1.2, §3.2.1): the overlapping c4a
+    window, per-channel gates, RMSNorm before RoPE. Random chunks against the
+    oracle (pre-quantisation values, fp8 bytes on the GPU's own values,
+    window, state), and chunked appends bitwise equal to one-shot ones."""
+    n = [3000, 517, 5, 1200, 257] if ratio == 4 else [3000, 517, 5, 1200, 300]
+    a = Appender(440 + ratio, n, ratio, **opts)
+    a.append(n)
+    b = Appender(440 + ratio, n, ratio, **opts)
+    r = synth.rng(441)
+    while any(d < N for d, N in zip(b.done, b.n)):
+        b.append([int(r.integers(0, 700)) for _ in n])
+    check_against_oracle(a)
+    check_against_oracle(b)
+    for s in range(len(n)):
+        ra, sa = a.entries(s)
+        rb, sb = b.entries(s)
+        assert np.array_equal(ra, rb) and np.array_equal(sa, sb)
+        assert np.array_equal(a.prequant[s].view(np.uint32), b.prequant[s].view(np.uint32))
+
+
+def test_variant_arguments():
+    """The overlapping window is c4a's only; odd option values are rejected."""
+    from paged_compressed_kv_b200 import v4kv
+    ap = Appender(450, [10], 128)
+    dev = torch.device("cuda")
+    with pytest.raises(v4kv.V4KVError):
+        v4kv.v4kv_compress_append(
+            torch.zeros(10, D, dtype=torch.bfloat16, device=dev), torch.zeros(10, device=dev),
+            torch.tensor([0, 10], dtype=torch.int32, device=dev), torch.zeros(1, dtype=torch.int32, device=dev),
+            torch.zeros(256, device=dev), 128, ap.state_x, ap.state_g, ap.main, None, None, overlap=True)
