@@ -577,9 +577,10 @@ class CompressStep:
     random chunks of 1..4096 (one chunk per sequence per call), ratio 4 or 128,
     fp8 entries into shuffled pages, window copies of each chunk's last 128."""
 
-    def __init__(self, device, ratio, seqs=8, tokens=32768):
+    def __init__(self, device, ratio, seqs=8, tokens=32768, overlap=False, norm=False):
         from paged_compressed_kv_b200 import PagedPool, v4kv
         self.v4kv, self.ratio, self.B, self.N = v4kv, ratio, seqs, tokens
+        self.overlap = overlap
         r = synth.rng(synth.seed_for("compressor") + ratio)
         g = synth.device_generator(synth.seed_for("compressor") + ratio, device)
         self.chunks = [synth.chunk_sizes(r, tokens) for _ in range(seqs)]
@@ -600,9 +601,11 @@ class CompressStep:
         self.x = torch.empty(seqs * tokens, D, dtype=torch.bfloat16, device=device)
         synth.fill_normal_bf16(self.x, g)
         self.gate = torch.randn(seqs * tokens, generator=g, device=device)
-        self.bias = torch.randn(ratio, generator=g, device=device) * 0.5
-        self.state_x = torch.zeros(seqs, ratio, D, dtype=torch.bfloat16, device=device)
-        self.state_g = torch.zeros(seqs, ratio, dtype=torch.float32, device=device)
+        self.bias = torch.randn(2 * ratio if overlap else ratio, generator=g, device=device) * 0.5
+        rows = 2 * ratio if overlap else ratio
+        self.state_x = torch.zeros(seqs, rows, D, dtype=torch.bfloat16, device=device)
+        self.state_g = torch.zeros(seqs, rows, dtype=torch.float32, device=device)
+        self.norm_w = (1.0 + 0.1 * torch.randn(D, generator=g, device=device)) if norm else None
         # per call: chunk rows gathered contiguously (inputs resident before timing)
         self.call_inputs = []
         done = [0] * seqs
@@ -626,7 +629,8 @@ class CompressStep:
         v, ci = self.v4kv, self.call_inputs[c]
         v.v4kv_compress_append(ci["x"], ci["gate"], ci["cu"], ci["ss"], self.bias, self.ratio,
                                self.state_x, self.state_g, self.main, None, None,
-                               window=self.win, window_len=W, dev_status=self.status)
+                               window=self.win, window_len=W, dev_status=self.status,
+                               overlap=self.overlap, norm_weight=self.norm_w)
 
     def algorithmic_bytes(self, c):
         ci = self.call_inputs[c]
@@ -634,14 +638,18 @@ class CompressStep:
         touched = sum((-(-(int(s0) + int(m)) // self.ratio)) - int(s0) // self.ratio
                       for s0, m in zip(ci["starts"], ci["sizes"]) if m)
         win = sum(min(int(m), W) for m in ci["sizes"])
-        return n * (D * 2 + 4) + touched * (D + 4) + win * D * 2 + self.B * self.ratio * (D * 2 + 4)
+        rows = 2 * self.ratio if self.overlap else self.ratio
+        return n * (D * 2 + 4) + touched * (D + 4) + win * D * 2 + self.B * rows * (D * 2 + 4)
 
 
 def run_compress(args, device, clk):
     peak, _ = load_peaks()
     out = {}
-    for ratio in (4, 128):
-        st = CompressStep(device, ratio)
+    # the plain compressor for both ratios, then c4a with the overlapping
+    # 8-token window and RMSNorm (the variant kernel)
+    for key, ratio, var in (("r4", 4, {}), ("r128", 128, {}),
+                            ("r4_overlap_norm", 4, dict(overlap=True, norm=True))):
+        st = CompressStep(device, ratio, **var)
         for c in range(st.calls):  # warm-up pass (also fills the cache once)
             st.call(c)
         torch.cuda.synchronize()
@@ -680,7 +688,7 @@ def run_compress(args, device, clk):
         del graph
         ms = float(np.median(ms_g))
         byts = sum(st.algorithmic_bytes(c) for c in range(st.calls))
-        out[f"r{ratio}"] = {"calls": st.calls, "tokens": st.B * st.N, "ms": ms,
+        out[key] = {"calls": st.calls, "tokens": st.B * st.N, "ms": ms,
                             "algorithmic_bytes": byts,
                             "tokens_per_s": st.B * st.N / (ms * 1e-3),
                             "gbs": byts / (ms * 1e-3) / 1e9, "frac": byts / (ms * 1e-3) / 1e9 / peak,

@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(kWarps * 32) compress_append_kernel(CompressAr
 
 
 // ---------------------------------------------------------------- variants
-// One block per entry. Token k of the entry's span (k = t - start, start =
+// c128a with per-channel gates: one block per entry. Token k of the entry's span (k = t - start, start =
 // g*r, or g*r - r with the overlapping window) belongs to warp k / rpw, rpw =
 // ceil(span / 8); for every dim the softmax over the present tokens runs in
 // two passes through shared memory (the maxima, then the weighted sums, each
@@ -677,9 +677,141 @@ __global__ void __launch_bounds__(kWarps * 32) compress_variant_kernel(CompressA
   }
 }
 
+
+// c4a variants, one warp per entry: the span (4 or 8 tokens) fits in a lane's
+// registers. Per-token gates: the weights once per token (lane t), added in
+// ascending t; per-channel gates: per dim, the maximum over the tokens, then
+// the sums of exp(z - m) and of exp(z - m) * x in ascending t.
+template <int KC>
+__device__ void warp_variant_entry(const CompressArgs& a, int i, int b, const int32_t* cu) {
+  constexpr int kSpan = 8;  // 2r for r = 4
+  const int lane = threadIdx.x & 31;
+  const int nch = a.dim >> 3;
+  const int r = a.ratio;
+  const int s = a.seq_start[b];
+  const int end = s + (a.cu_seqlens[b + 1] - a.cu_seqlens[b]);
+  const int t0 = (s / r + (i - cu[b])) * r;
+  const int start = t0 - (a.overlap ? r : 0);
+  const int lo = max(0, start), hi = min(t0 + r, end);
+  const int np = hi - lo, k0 = lo - start;
+  const int old_base = (s / r) * r - (a.overlap ? r : 0);
+  uint4 q[kSpan][KC];
+#pragma unroll
+  for (int j = 0; j < kSpan; ++j) {
+    if (j < np) {
+      const int tt = lo + j;
+      const uint16_t* row = tt < s ? a.state_x + ((size_t)b * a.state_rows + (tt - old_base)) * a.dim
+                                   : a.x + (size_t)(a.cu_seqlens[b] + (tt - s)) * a.dim;
+      load_row<KC>(row, lane, nch, q[j]);
+    }
+  }
+  float acc[KC][8];
+  if (a.gate_dim == 1) {
+    // lane t < np: logit of token lo + t plus its bias; softmax across lanes
+    float z = -INFINITY;
+    if (lane < np) {
+      const int tt = lo + lane;
+      const float g = tt < s ? a.state_gate[(size_t)b * a.state_rows + (tt - old_base)]
+                             : a.gate[a.cu_seqlens[b] + (tt - s)];
+      z = g + a.pos_bias[k0 + lane];
+    }
+    const float m = warp_max(z);
+    const float u = lane < np ? expf(z - m) : 0.f;
+    const float sum = warp_sum(u);
+    const float w = lane < np ? __fdiv_rn(u, sum) : 0.f;
+#pragma unroll
+    for (int k = 0; k < KC; ++k)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
+#pragma unroll
+    for (int j = 0; j < kSpan; ++j) {
+      const float wt = __shfl_sync(0xffffffffu, w, j);
+      if (j >= np) break;
+#pragma unroll
+      for (int k = 0; k < KC; ++k) {
+        float v[8];
+        unpack_bf16x8(q[j][k], v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wt, v[e], acc[k][e]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      const int c = lane + 32 * k;
+      float m[8], su[8], sv[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        m[e] = -INFINITY;
+        su[e] = sv[e] = 0.f;
+      }
+      if (c < nch) {
+#pragma unroll
+        for (int j = 0; j < kSpan; ++j) {
+          if (j >= np) break;
+          float z[8];
+          gate_chunk(a, b, s, old_base, lo + j, c, z);
+          const float bias = a.pos_bias[k0 + j];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], z[e] + bias);
+        }
+#pragma unroll
+        for (int j = 0; j < kSpan; ++j) {
+          if (j >= np) break;
+          float z[8], v[8];
+          gate_chunk(a, b, s, old_base, lo + j, c, z);
+          unpack_bf16x8(q[j][k], v);
+          const float bias = a.pos_bias[k0 + j];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float u = expf(z[e] + bias - m[e]);
+            su[e] += u;
+            sv[e] = fmaf(u, v[e], sv[e]);
+          }
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[k][e] = c < nch ? __fdiv_rn(sv[e], su[e]) : 0.f;
+    }
+  }
+  finish_entry<KC>(a, i, b, t0, lane, nch, acc);
+}
+
+template <int KC>
+__global__ void __launch_bounds__(kWarps * 32) compress_variant_warp_kernel(CompressArgs a,
+                                                                           int window_blocks,
+                                                                           int window_blocks_per_seq) {
+  __shared__ int cu_sh[kCuSmem];
+  tc::pdl_wait();  // x, the gates and the state (earlier work in the stream) are complete
+  tc::pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nch = a.dim >> 3;
+  if ((int)blockIdx.x < window_blocks) {
+    window_row<KC>(a, blockIdx.x / window_blocks_per_seq,
+                   (blockIdx.x % window_blocks_per_seq) * kWarps + warp, lane, nch);
+    return;
+  }
+  const int32_t* cu = entry_prefix(a, cu_sh);
+  const int i = (blockIdx.x - window_blocks) * kWarps + warp;
+  if (i >= cu[a.batch]) return;  // uniform over the warp
+  const int b = seq_of(cu, a.batch, i);
+  // the warp of the sequence's first entry also builds the second (both read
+  // the old state with the overlapping window) and then rewrites the state
+  if (a.overlap && i == cu[b] + 1) return;
+  warp_variant_entry<KC>(a, i, b, cu);
+  if (i == cu[b]) {
+    if (a.overlap && i + 1 < cu[b + 1]) warp_variant_entry<KC>(a, i + 1, b, cu);
+    variant_state<KC>(a, b);
+  }
+}
+
 template <int KC>
 cudaError_t launch_variant_kc(const CompressArgs& a, int max_groups, int window_blocks, int per_seq,
                               cudaStream_t stream) {
+  if (a.ratio <= kWarps)  // c4a: one warp per entry
+    return launch_pdl(compress_variant_warp_kernel<KC>,
+                      dim3(window_blocks + (max_groups + kWarps - 1) / kWarps), dim3(kWarps * 32), 0,
+                      stream, a, window_blocks, per_seq);
   const size_t smem = (size_t)3 * kWarps * a.dim * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(compress_variant_kernel<KC>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
