@@ -142,3 +142,27 @@ def window_tokens(x, positions, theta=1e6, rope_dim=64, rope_offset=448):
     """
     return rope_rotate(np.asarray(x, dtype=np.float64), np.asarray(positions),
                        theta, rope_dim, rope_offset).astype(np.float32)
+
+
+def qk_prepare(q, k_new, positions, norm_weight=None, norm_eps=1e-6, theta=1e6, rope_dim=64,
+               rope_offset=448):
+    """The inputs of one decode step before attention (P1 §3.2.1, the fused
+    "Q norm + KV RoPE + K insert"): each query head's vector is RMS-normalised
+    (when weights are given) and rotated by RoPE at its sequence's position; the
+    new token's K = V row is rotated at the same position for the window.
+
+    q [B, H, D], k_new [B, D] (or None), positions [B] -> (q_out fp32
+    [B, H, D], k_out fp32 [B, D] or None); fp64 arithmetic rounded once.
+
+    Follows P1 §3.2.1 (Q/K insertion fusion) with S38's RMSNorm and S5's RoPE.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    pos = np.asarray(positions).reshape(-1, 1)
+    if norm_weight is not None:
+        q = rms_norm(q, norm_weight, norm_eps)
+    q_out = rope_rotate(q, pos, theta, rope_dim, rope_offset).astype(np.float32)
+    k_out = None
+    if k_new is not None:
+        k_out = rope_rotate(np.asarray(k_new, dtype=np.float64), np.asarray(positions), theta, rope_dim,
+                            rope_offset).astype(np.float32)
+    return q_out, k_out

@@ -181,3 +181,27 @@ def test_per_channel_gates_reduce_to_scalar_gates_and_brute_force():
             s = sum(u)
             want = sum(u[k] / s * float(x[lo + k, c]) for k in range(hi - lo))
             assert abs(float(e[gi, c]) - want) <= 1e-6 * max(1.0, abs(want)), (gi, c)
+
+
+def test_qk_prepare_reduces_to_norm_and_rope():
+    r = synth.rng(75)
+    q = synth.normal(r, (3, 4, 512))
+    k = synth.normal(r, (3, 512))
+    pos = np.array([0, 17, 100000])
+    w = 1.0 + synth.normal(r, 512, 0.1)
+    qo, ko = compressor.qk_prepare(q, k, pos, w)
+    # position 0: RoPE is the identity, so the result is the norm alone
+    assert np.allclose(qo[0], compressor.rms_norm(q[0].astype(np.float64), w), rtol=1e-6, atol=1e-7)
+    assert np.array_equal(ko[0], k[0].astype(np.float32))
+    # RoPE keeps each rope pair's length and leaves the other dims alone
+    nq = compressor.rms_norm(q[1].astype(np.float64), w)
+    assert np.allclose(qo[1][:, :448], nq[:, :448], rtol=1e-6, atol=1e-7)
+    a, b = qo[2][:, 448::2].astype(np.float64), qo[2][:, 449::2].astype(np.float64)
+    nq2 = compressor.rms_norm(q[2].astype(np.float64), w)
+    a0, b0 = nq2[:, 448::2], nq2[:, 449::2]
+    assert np.allclose(a * a + b * b, a0 * a0 + b0 * b0, rtol=1e-5)
+    # the K row is the window copy of the token (the compressor's window path)
+    assert np.array_equal(ko[1], compressor.window_tokens(k[1][None], [17])[0])
+    # no weights: RoPE only
+    qo2, _ = compressor.qk_prepare(q, None, pos)
+    assert np.array_equal(qo2[0], q[0].astype(np.float32))
