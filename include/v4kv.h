@@ -212,6 +212,33 @@ v4kv_status v4kv_compress_append_ex(const void* x, const float* gate, const int3
                                     int32_t* dev_status, void* stream);
 
 /*
+ * v4kv_qk_prepare -- the decode step's query heads and new window row in one
+ * launch (P1 §3.2.1, "fused Q norm + KV RoPE + K insert": one warp per query
+ * head or K row, no communication between them).
+ * For every sequence b and head h:
+ *     q_out[b][h] = RoPE(RMSNorm(q_in[b][h]), positions[b])
+ * with RMSNorm(v) = v * w / sqrt(mean(v^2) + q_norm_eps) (skipped when
+ * q_norm_weight is NULL; q_norm_eps 0 means 1e-6) and RoPE as in
+ * v4kv_compress_append (angles in fp64, the rotation in fp32). When k_new and
+ * window are given, the new token's K = V row is rotated at positions[b] and
+ * stored in the window pool (page window->block_table[b][pos / 256], slot
+ * pos % 256; bf16, or fp8 with its own scale; a -1 page is skipped), exactly
+ * as the compressor stores its window rows.
+ *   q_in          device fp32 [batch, heads, dim], 16-byte aligned
+ *   q_out         device [batch, heads, dim], fp32 or bf16 (q_out_dtype)
+ *   q_norm_weight device fp32 [dim] or NULL
+ *   positions     device int32 [batch], the new token's position (L - 1)
+ *   k_new         device bf16 [batch, dim] or NULL
+ *   window        window pool (slots_per_page 256) or NULL
+ * Rejects dim > 1024 or dim % 8, unaligned buffers, rope dims outside dim.
+ * Out-of-range window blocks or pages are flagged in dev_status and skipped.
+ */
+v4kv_status v4kv_qk_prepare(const float* q_in, int32_t batch, int32_t heads, int32_t dim,
+                            const float* q_norm_weight, float q_norm_eps, const int32_t* positions,
+                            v4kv_rope rope, void* q_out, int32_t q_out_dtype, const void* k_new,
+                            const v4kv_paged* window, int32_t* dev_status, void* stream);
+
+/*
  * v4kv_index_topk -- indexer scores and exact top-k over a c4a layer's
  * visible entries (P1 §2.2 indexer cache; P1 §4.1 sparse attention over
  * the selected c4a entries).

@@ -10,7 +10,7 @@ _EXPORTS = {
     "EXPORTED", "LIB_PATH", "PagedPool", "PagePools", "v4kv_page_bytes", "v4kv_plan_buckets", "Rope", "V4KVError", "v4kv_compress_append",
     "v4kv_decode_attention", "v4kv_decode_attention_fp8out", "v4kv_decode_attention_noalloc", "v4kv_index_topk",
     "v4kv_kv_footprint_bytes", "v4kv_slot_mapping", "v4kv_status_string", "v4kv_version",
-    "v4kv_workspace_size",
+    "v4kv_workspace_size", "v4kv_qk_prepare",
 }
 
 

@@ -202,6 +202,39 @@ v4kv_status v4kv_compress_append_ex(const void* x, const float* gate, const int3
   return to_status(launch_compress_append(a, (int)max_groups, total_tokens, (cudaStream_t)stream));
 }
 
+v4kv_status v4kv_qk_prepare(const float* q_in, int32_t batch, int32_t heads, int32_t dim,
+                            const float* q_norm_weight, float q_norm_eps, const int32_t* positions,
+                            v4kv_rope rope, void* q_out, int32_t q_out_dtype, const void* k_new,
+                            const v4kv_paged* window, int32_t* dev_status, void* stream) {
+  if (batch <= 0 || heads <= 0 || !q_in || !q_out || !positions) return V4KV_ERR_INVALID_ARG;
+  if (dim < 8 || dim > 1024 || dim % 8) return V4KV_ERR_INVALID_ARG;
+  if (q_out_dtype != V4KV_FP32 && q_out_dtype != V4KV_BF16) return V4KV_ERR_INVALID_ARG;
+  if (!aligned16(q_in) || !aligned16(q_out) || (q_norm_weight && !aligned16(q_norm_weight)))
+    return V4KV_ERR_INVALID_ARG;
+  if (q_norm_weight && !(q_norm_eps >= 0.f)) return V4KV_ERR_INVALID_ARG;
+  if (k_new && !aligned16(k_new)) return V4KV_ERR_INVALID_ARG;
+  if (window && !pool_ok(window, kBlock, dim, true, true)) return V4KV_ERR_INVALID_ARG;
+  if (!rope_ok(rope, dim)) return V4KV_ERR_INVALID_ARG;
+  if ((long long)heads + 1 > 65535LL * 8) return V4KV_ERR_INVALID_ARG;
+  v4kv_status st = check_device(nullptr);
+  if (st != V4KV_OK) return st;
+  QkPrepArgs p{};
+  p.q_in = q_in;
+  p.q_out = q_out;
+  p.q_out_bf16 = q_out_dtype == V4KV_BF16;
+  p.norm_w = q_norm_weight;
+  p.norm_eps = q_norm_weight ? (q_norm_eps > 0.f ? q_norm_eps : 1e-6f) : 0.f;
+  p.k_new = static_cast<const uint16_t*>(k_new);
+  p.positions = positions;
+  p.window = to_args(window);
+  p.rope = to_rope(rope);
+  p.dev_status = dev_status;
+  p.batch = batch;
+  p.heads = heads;
+  p.dim = dim;
+  return to_status(launch_qk_prepare(p, (cudaStream_t)stream));
+}
+
 v4kv_status v4kv_index_topk(const float* q_idx, const v4kv_paged* idx_cache,
                             const int32_t* seq_lens, int32_t batch, int32_t max_seq_len,
                             int32_t ratio, int32_t window_len, int32_t k, int32_t* topk_out,

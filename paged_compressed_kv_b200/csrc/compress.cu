@@ -831,6 +831,77 @@ cudaError_t launch_kc(const CompressArgs& a, int max_groups, int window_blocks, 
   return launch_pdl(compress_append_kernel<KC, false>, grid, block, 0, stream, a, window_blocks, per_seq);
 }
 
+
+// ---------------------------------------------------------------- Q/K preparation
+// The decode step's query heads and new window row in one launch, one warp per
+// item (horizontal fusion): warp j < heads RMS-normalises head j of sequence b
+// (when weights are given) and rotates it by RoPE at positions[b]; warp j ==
+// heads rotates the new K = V row and stores it in the window (bf16, or fp8
+// per token), the same arithmetic as the compressor's window rows.
+template <int KC>
+__global__ void __launch_bounds__(kWarps * 32) qk_prepare_kernel(QkPrepArgs p) {
+  tc::pdl_wait();  // q and the new rows (earlier work in the stream) are complete
+  tc::pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x, j = blockIdx.y * kWarps + warp;
+  const int nch = p.dim >> 3;
+  const long long pos = p.positions[b];
+  if (j < p.heads) {
+    const float* src = p.q_in + ((size_t)b * p.heads + j) * p.dim;
+    float e[KC][8];
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      const int c = lane + 32 * k;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) e[k][i] = 0.f;
+      if (c < nch) {
+        const float4 u = *reinterpret_cast<const float4*>(src + 8 * c);
+        const float4 v = *reinterpret_cast<const float4*>(src + 8 * c + 4);
+        e[k][0] = u.x; e[k][1] = u.y; e[k][2] = u.z; e[k][3] = u.w;
+        e[k][4] = v.x; e[k][5] = v.y; e[k][6] = v.z; e[k][7] = v.w;
+      }
+    }
+    if (p.norm_w) rms_norm_warp<KC>(e, lane, nch, p.norm_w, p.norm_eps, p.dim);
+    rope_warp<KC>(e, lane, nch, p.rope, pos);
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      const int c = lane + 32 * k;
+      if (c >= nch) continue;
+      const size_t o = ((size_t)b * p.heads + j) * p.dim + 8 * c;
+      if (p.q_out_bf16) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          w[i] = (uint32_t)float_to_bf16_bits(e[k][2 * i]) | ((uint32_t)float_to_bf16_bits(e[k][2 * i + 1]) << 16);
+        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.q_out) + o) = make_uint4(w[0], w[1], w[2], w[3]);
+      } else {
+        float* dst = static_cast<float*>(p.q_out) + o;
+        *reinterpret_cast<float4*>(dst) = make_float4(e[k][0], e[k][1], e[k][2], e[k][3]);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(e[k][4], e[k][5], e[k][6], e[k][7]);
+      }
+    }
+  } else if (j == p.heads && p.k_new && p.window.data) {
+    const int32_t* row = p.window.block_table + (size_t)b * p.window.max_blocks;
+    const long long blk = pos / kLogicalBlock;
+    if (pos < 0 || blk >= p.window.max_blocks) {
+      if (lane == 0) flag(p.dev_status, V4KV_DEV_BAD_SLOT);
+      return;
+    }
+    const int pg = row[blk];
+    if (pg < 0) return;  // no page for this block: nothing to keep
+    if (pg >= p.window.num_pages) {
+      if (lane == 0) flag(p.dev_status, V4KV_DEV_BAD_PAGE);
+      return;
+    }
+    uint4 q[KC];
+    load_row<KC>(p.k_new + (size_t)b * p.dim, lane, nch, q);
+    float e[KC][8];
+#pragma unroll
+    for (int k = 0; k < KC; ++k) unpack_bf16x8(q[k], e[k]);
+    rope_warp<KC>(e, lane, nch, p.rope, pos);
+    store_entry_warp<KC>(p.window, (long long)pg * kLogicalBlock + (pos % kLogicalBlock), lane, nch, e);
+  }
+}
 }  // namespace
 
 cudaError_t launch_compress_append(const CompressArgs& a, int max_groups, int total_tokens,
@@ -854,6 +925,18 @@ cudaError_t launch_compress_append(const CompressArgs& a, int max_groups, int to
   if (kc <= 1) return launch_kc<1>(a, max_groups, (int)wb, per_seq, stream);
   if (kc <= 2) return launch_kc<2>(a, max_groups, (int)wb, per_seq, stream);
   return launch_kc<4>(a, max_groups, (int)wb, per_seq, stream);
+}
+
+}  // namespace v4kv
+
+namespace v4kv {
+
+cudaError_t launch_qk_prepare(const QkPrepArgs& p, cudaStream_t stream) {
+  const dim3 grid(p.batch, (p.heads + 1 + kWarps - 1) / kWarps), block(kWarps * 32);
+  const int kc = (p.dim + 255) / 256;
+  if (kc <= 1) return launch_pdl(qk_prepare_kernel<1>, grid, block, 0, stream, p);
+  if (kc <= 2) return launch_pdl(qk_prepare_kernel<2>, grid, block, 0, stream, p);
+  return launch_pdl(qk_prepare_kernel<4>, grid, block, 0, stream, p);
 }
 
 }  // namespace v4kv

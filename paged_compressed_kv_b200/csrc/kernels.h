@@ -59,6 +59,22 @@ struct CompressArgs {
   float norm_eps;
 };
 
+struct QkPrepArgs {
+  const float* q_in;        // [batch, heads, dim]
+  void* q_out;              // [batch, heads, dim] fp32 or bf16
+  int q_out_bf16;
+  const float* norm_w;      // [dim] or null
+  float norm_eps;
+  const uint16_t* k_new;    // [batch, dim] bf16 or null
+  const int32_t* positions; // [batch]
+  PoolArgs window;          // data null: no K insert
+  RopeArgs rope;
+  int32_t* dev_status;
+  int batch;
+  int heads;
+  int dim;
+};
+
 struct IndexArgs {
   const float* q_idx;
   const int32_t* seq_lens;
@@ -128,6 +144,7 @@ cudaError_t launch_slot_mapping(const int32_t* bt, int max_blocks, int batch,
                                 int num_pages, int32_t* cu_out, int64_t* slot_out, long long cap,
                                 int32_t* st, cudaStream_t stream);
 
+cudaError_t launch_qk_prepare(const QkPrepArgs& p, cudaStream_t stream);
 cudaError_t launch_compress_append(const CompressArgs& a, int max_groups, int total_tokens,
                                    cudaStream_t stream);
 

@@ -34,7 +34,7 @@ V4KV_OP_DECODE = 2
 
 EXPORTED = [
     "v4kv_status_string", "v4kv_version", "v4kv_slot_mapping", "v4kv_compress_append",
-    "v4kv_compress_append_ex",
+    "v4kv_compress_append_ex", "v4kv_qk_prepare",
     "v4kv_index_topk", "v4kv_decode_attention", "v4kv_workspace_size", "v4kv_kv_footprint_bytes",
     "v4kv_decode_attention_noalloc", "v4kv_decode_attention_fp8out",
     "v4kv_page_bytes", "v4kv_plan_buckets", "v4kv_page_pools_create", "v4kv_page_pools_destroy",
@@ -90,6 +90,8 @@ def _load():
         "v4kv_compress_append_ex": (I32, [P, P, P, P, I32, I32, P, I32, _Rope, P, P,
                                           ctypes.POINTER(_Paged), P, P, ctypes.POINTER(_Paged), I32,
                                           P, ctypes.POINTER(_CompressOpts), P, P]),
+        "v4kv_qk_prepare": (I32, [P, I32, I32, I32, P, F32, P, _Rope, P, I32, P,
+                                  ctypes.POINTER(_Paged), P, P]),
         "v4kv_index_topk": (I32, [P, ctypes.POINTER(_Paged), P, I32, I32, I32, I32, I32, P, P, P,
                                   SZ, P, P]),
         "v4kv_decode_attention": (I32, [P, I32, I32, I32, ctypes.POINTER(_Paged),
@@ -248,6 +250,30 @@ def v4kv_compress_append(x, gate, cu_seqlens, seq_start, pos_bias, ratio, state_
     else:
         st = _lib.v4kv_compress_append(*args, _ptr(dev_status), _stream(stream))
         _check("v4kv_compress_append", st)
+
+
+def v4kv_qk_prepare(q_in, positions, q_out, q_norm_weight=None, q_norm_eps=0.0, k_new=None, window=None,
+                    rope=None, dev_status=None, stream=None):
+    """Per-head RMSNorm (optional) and RoPE of q at each sequence's position,
+    and the new K row rotated into the window pool, in one launch."""
+    _need(q_in, (torch.float32,), "q_in", ndim=3)
+    _need(positions, (torch.int32,), "positions")
+    _need(q_out, (torch.float32, torch.bfloat16), "q_out", ndim=3)
+    if q_out.shape != q_in.shape:
+        raise ValueError("q_out must have q_in's shape")
+    if q_norm_weight is not None:
+        _need(q_norm_weight, (torch.float32,), "q_norm_weight")
+    if k_new is not None:
+        _need(k_new, (torch.bfloat16,), "k_new", ndim=2)
+    rope = rope or Rope()
+    wc = window.c() if window is not None else None
+    B, H, dim = q_in.shape
+    st = _lib.v4kv_qk_prepare(q_in.data_ptr(), B, H, dim, _ptr(q_norm_weight), float(q_norm_eps),
+                              positions.data_ptr(), rope.c(), q_out.data_ptr(),
+                              V4KV_BF16 if q_out.dtype == torch.bfloat16 else V4KV_FP32, _ptr(k_new),
+                              ctypes.byref(wc) if wc is not None else None, _ptr(dev_status),
+                              _stream(stream))
+    _check("v4kv_qk_prepare", st)
 
 
 def v4kv_workspace_size(op, batch, heads, max_seq_len, ratio, window_len, k, main_dtype, dim=512):

@@ -471,3 +471,59 @@ def test_variant_arguments():
             torch.zeros(10, D, dtype=torch.bfloat16, device=dev), torch.zeros(10, device=dev),
             torch.tensor([0, 10], dtype=torch.int32, device=dev), torch.zeros(1, dtype=torch.int32, device=dev),
             torch.zeros(256, device=dev), 128, ap.state_x, ap.state_g, ap.main, None, None, overlap=True)
+
+
+def test_qk_prepare_matches_oracle_and_the_compressor_window_row():
+    """v4kv_qk_prepare (P1 §3.2.1 Q/K insertion fusion): per-head RMSNorm and
+    RoPE of q against the oracle; the new K row in the window is bitwise the
+    row the compressor writes for the same token."""
+    from paged_compressed_kv_b200 import PagedPool, Rope, v4kv
+    dev = torch.device("cuda")
+    r = synth.rng(460)
+    B, H = 5, 64
+    q = synth.normal(r, (B, H, D))
+    kx = codecs.bf16_round(synth.normal(r, (B, D)))
+    pos = np.array([0, 1, 255, 256 + 77, 100000], dtype=np.int32)
+    w = (1.0 + synth.normal(r, D, 0.1)).astype(np.float32)
+    wblk = [int(p // 256) + 1 for p in pos]
+    wbt, Pw = paging.allocate_block_tables(wblk, synth.permutation(r, sum(wblk) + 1))
+    win = PagedPool(data=torch.zeros(Pw, 256, D, dtype=torch.bfloat16, device=dev),
+                    block_table=torch.from_numpy(wbt).to(dev))
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    q_out = torch.empty(B, H, D, dtype=torch.float32, device=dev)
+    v4kv.v4kv_qk_prepare(torch.from_numpy(q).to(dev), torch.from_numpy(pos).to(dev), q_out,
+                         q_norm_weight=torch.from_numpy(w).to(dev), k_new=synth.bf16_tensor(kx).to(dev),
+                         window=win, dev_status=st)
+    qo_ref, ko_ref = compressor.qk_prepare(q, kx, pos, w)
+    got = q_out.cpu().numpy()
+    amax = np.abs(qo_ref).max(axis=2, keepdims=True)
+    assert np.all(np.abs(got - qo_ref) <= 1e-5 * amax), float(np.abs(got - qo_ref).max())
+    assert int(st.item()) == 0
+    # the same token appended alone through the compressor (its window row)
+    win2 = PagedPool(data=torch.zeros(Pw, 256, D, dtype=torch.bfloat16, device=dev),
+                     block_table=torch.from_numpy(wbt).to(dev))
+    # (its entries all land on one scratch page: only the window is compared)
+    main = PagedPool(data=torch.zeros(1, 64, D, dtype=torch.uint8, device=dev),
+                     block_table=torch.zeros(B, 400, dtype=torch.int32, device=dev),
+                     scales=torch.zeros(1, 64, dtype=torch.float32, device=dev))
+    v4kv.v4kv_compress_append(
+        synth.bf16_tensor(kx).to(dev), torch.zeros(B, device=dev),
+        torch.arange(B + 1, dtype=torch.int32, device=dev), torch.from_numpy(pos).to(dev),
+        torch.zeros(4, device=dev), 4, torch.zeros(B, 4, D, dtype=torch.bfloat16, device=dev),
+        torch.zeros(B, 4, device=dev), main, None, None, window=win2, window_len=128, dev_status=st)
+    a1 = win.data.view(torch.int16).cpu().numpy()
+    a2 = win2.data.view(torch.int16).cpu().numpy()
+    for b in range(B):
+        p = int(pos[b])
+        pg = wbt[b, p // 256]
+        assert np.array_equal(a1[pg, p % 256], a2[pg, p % 256]), b
+        ref = codecs.bf16_bits(ko_ref[b:b + 1])[0].view(np.int16)
+        xmax = float(np.abs(kx[b]).max())
+        d = np.abs(codecs.bf16_to_f32(a1[pg, p % 256].view(np.uint16)) - codecs.bf16_to_f32(ref.view(np.uint16)))
+        assert np.all(d <= np.abs(ko_ref[b]) * 2.0**-7 + xmax * 2.0**-20 + 1e-30)
+    # bf16 output and no norm: RoPE only
+    q_bf = torch.empty(B, H, D, dtype=torch.bfloat16, device=dev)
+    v4kv.v4kv_qk_prepare(torch.from_numpy(q).to(dev), torch.from_numpy(pos).to(dev), q_bf, dev_status=st)
+    qo2, _ = compressor.qk_prepare(q, None, pos)
+    got2 = q_bf.float().cpu().numpy()
+    assert np.all(np.abs(got2 - qo2) <= np.abs(qo2) * 2.0**-7 + np.abs(q).max(axis=2, keepdims=True) * 2.0**-20)
