@@ -278,6 +278,9 @@ __device__ __forceinline__ int tiles_of(const Seq& s) {
 // fp8 tile): fp8 tiles 4, bf16 tiles 8 (twice the bytes and a slower
 // conversion), and 4 for opening a segment (query copy, epilogue).
 constexpr int kCostFp8 = 4, kCostBf16 = 8, kCostSeg = 4;
+// estimated cost of splitting a sequence over blocks: the partial results'
+// stores and the merge (about three fp8 tiles)
+constexpr int kCostMerge = 12;
 
 __device__ __forceinline__ long long seq_cost(const DecodeArgs& a, const Seq& s) {
   const int nm = s.n_sel_pad / kT, nw = (s.n_win + kT - 1) / kT;
@@ -359,6 +362,51 @@ __device__ __forceinline__ int warp_reduce_scatter32(float* v, int lane, float* 
   }
   out1[0] = v[0];
   return base;
+}
+
+// A block writes the output of a sequence whose every tile it ran itself
+// (and the merge kernel skips such a sequence) when the output is bf16 and the
+// rope pairs' cos/sin are all in the prep kernel's table.
+__device__ __forceinline__ bool direct_output(const DecodeArgs& a) {
+  return !a.out_fp8 && a.rope.rope_dim <= 2 * kRopeTable;
+}
+
+// That output (called by a softmax thread at the segment's end, O^T complete
+// in tensor memory): O^T rows of this thread's lane (dims 128 mt + row,
+// mt = 2 hh, 2 hh + 1) times inv_l per head, the inverse RoPE at position
+// L - 1 on the rope pairs (the pair's other dim is in the neighbouring lane),
+// bf16 into out16 (the sequence's [64 heads][512 dims]). This is the merge
+// kernel's arithmetic for a sequence with one partial result (weight 1).
+__device__ __noinline__ void write_whole_output(uint16_t* out16, const float2* cs_tab, int rope_dim,
+                                                int rope_offset, uint32_t lane_base, int hh, int row,
+                                                const float* inv_l) {
+#pragma unroll 1
+  for (int m2 = 0; m2 < 2; ++m2) {
+    const int mt = 2 * hh + m2;
+    const int d = 128 * mt + row, de = d & ~1;
+    const bool rot = cs_tab && de >= rope_offset && de + 1 < rope_offset + rope_dim;
+    float c = 1.f, sn = 0.f;
+    if (rot) {
+      const float2 cs = cs_tab[(de - rope_offset) >> 1];
+      c = cs.x;
+      sn = cs.y;
+    }
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+      uint32_t r32[32];
+      tc::tmem_ld32(lane_base + kOCol + kH * mt + 32 * half, r32);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int h = 0; h < 32; ++h) {
+        float v = __uint_as_float(r32[h]) * inv_l[32 * half + h];
+        const float p = __shfl_xor_sync(0xffffffffu, v, 1);
+        if (rot)
+          v = (d & 1) ? __fadd_rn(__fmul_rn(p, -sn), __fmul_rn(v, c))
+                      : __fsub_rn(__fmul_rn(v, c), __fmul_rn(p, -sn));
+        out16[(size_t)(32 * half + h) * kD + d] = float_to_bf16_bits(v);
+      }
+    }
+  }
 }
 
 }  // namespace
@@ -826,29 +874,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       if (i + 1 < n_tiles && !(ok = convert(i + 1, nxt_fp8))) break;
 
       if (seg_last) {
-        const int b_done = cu.b;
+        // a segment that covers its whole sequence writes the output itself
+        // (bf16; the merge skips such sequences), any other one a partial result
+        // (every segment but the block's first opens at the sequence's first
+        // tile; the first one does when the block's range starts there)
+        const bool whole = (cu.b != range[2] || range[3] == 0) && cu.lt == cu.nt - 1 && direct_output(a);
+        const int b_done = cu.b, L_done = cu.s.L;
         cursor_next(cu, a);
         if (i + 1 < n_tiles) k0 = a.qk0[cu.b];
         ok = tc::mbar_wait(&bars->pv_done, i & 1, abort_flag);
         ok = named_and(1, 256, ok);
         if (!ok) break;
         tc::tc_fence_after();
-        // partial result of (sequence b_done, block cta) in slot b_done + cta:
-        // O^T un-normalised, relative to the reference maximum
         const size_t prow = ((size_t)b_done + cta) * kH;
-#pragma unroll 1
-        for (int m2 = 0; m2 < 2; ++m2) {
-          const int mt = 2 * hh + m2;
-#pragma unroll 1
-          for (int half = 0; half < 2; ++half) {
-            uint32_t r32[32];
-            tc::tmem_ld32(lane_base + kOCol + kH * mt + 32 * half, r32);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int h = 0; h < 32; ++h)
-              a.part_o[(prow + 32 * half + h) * kD + 128 * mt + row] = __uint_as_float(r32[h]);
-          }
-        }
         // normaliser: sum the 128 rows' partial sums per head
         {
           float lsum[32];
@@ -868,8 +906,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
             const int half = tid >> 5, hx = tid & 31;
             const float l = red[(4 * half) * 32 + hx] + red[(4 * half + 1) * 32 + hx] +
                             red[(4 * half + 2) * 32 + hx] + red[(4 * half + 3) * 32 + hx];
-            a.part_ml[(prow + tid) * 2] = mref[tid];
-            a.part_ml[(prow + tid) * 2 + 1] = l;
+            if (whole) {
+              alpha[tid] = l > 0.f ? 1.f / l : 0.f;  // the merge's weight for a single slot is 1
+            } else {
+              a.part_ml[(prow + tid) * 2] = mref[tid];
+              a.part_ml[(prow + tid) * 2 + 1] = l;
+            }
             mref[tid] = kNone;
           }
           {
@@ -880,6 +922,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
             tc::tmem_wait_st();
           }
           named_sync(1, 256);
+        }
+        if (whole) {
+          const int Lb = min(L_done, a.max_len);
+          const bool rope = a.rope.rope_dim > 0 && Lb > 0;
+          write_whole_output(reinterpret_cast<uint16_t*>(a.out) + (size_t)b_done * kH * kD,
+                             rope ? a.rope_tab + (size_t)b_done * kRopeTable : nullptr, a.rope.rope_dim,
+                             a.rope.rope_offset, lane_base, hh, row, alpha);
+        } else {
+          // partial result of (sequence b_done, block cta) in slot b_done + cta:
+          // O^T un-normalised, relative to the reference maximum
+#pragma unroll 1
+          for (int m2 = 0; m2 < 2; ++m2) {
+            const int mt = 2 * hh + m2;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+              uint32_t r32[32];
+              tc::tmem_ld32(lane_base + kOCol + kH * mt + 32 * half, r32);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int h = 0; h < 32; ++h)
+                a.part_o[(prow + 32 * half + h) * kD + 128 * mt + row] = __uint_as_float(r32[h]);
+            }
+          }
         }
         seg_first = true;
       } else {
@@ -920,6 +985,7 @@ __global__ void __launch_bounds__(256) decode_tc_merge_kernel(DecodeArgs a) {
   const int Lb = min(a.seq_lens[b], a.max_len);  // independent of the loads below
   const int2 sl = a.seq_slots[b];
   const int lo = sl.x, hi = sl.y;
+  if (lo == hi && direct_output(a)) return;  // one block ran the whole sequence and wrote its output
   // per block: (m, l) in one load; the weights go to shared memory
   float M = -INFINITY;
   float2 ml_keep[(kMaxSplits + 31) / 32];
@@ -1033,6 +1099,7 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
     const bool cached = a.batch <= kPrepCache;
     int carry = 0;
     long long ccarry = 0;
+    long long cmax = 0;  // the largest sequence cost (this thread's share)
     for (int base = 0; base < a.batch; base += 256) {
       const int bb = base + t;
       int n = 0;
@@ -1042,6 +1109,7 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
         const Seq sq = seq_of(a, bb, nullptr);
         n = tiles_of(sq);
         cost = seq_cost(a, sq);
+        cmax = max(cmax, cost);
         if (cached) len_sh[bb] = sq.L;
       }
       int incl = n;
@@ -1076,13 +1144,29 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(DecodeArgs a) {
         ccum_sh[a.batch] = ccarry;
       }
     }
+    // the largest sequence cost, over the block
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+    if (lane == 0) csum[warp] = cmax;
     __syncthreads();  // the prefix sums are visible to the whole block
+    for (int w = 0; w < 8; ++w) cmax = max(cmax, csum[w]);
     const int* cum = cached ? cum_sh : a.cum;
     const long long* costcum = cached ? ccum_sh : a.costcum;
     const int G = a.n_splits;
+    // One sequence per block when every sequence fits one block at a cost
+    // no greater than an even split plus the split's own cost (partial
+    // results and their merge): each block then writes its sequence's output
+    // itself. Otherwise block c starts where the cost prefix reaches c/G of
+    // the total.
+    const bool whole = a.batch <= G && cmax * G <= ccarry + (long long)kCostMerge * G;
     for (int c = t; c <= G; c += 256) {
       int x0 = carry, b0 = a.batch;
-      if (c < G && ccarry > 0) {
+      if (whole) {
+        if (c < a.batch) {
+          x0 = cum[c];
+          b0 = c;
+        }
+      } else if (c < G && ccarry > 0) {
         const long long target = (long long)c * ccarry / G;
         int l = 0, r = a.batch - 1;  // last sequence whose cost prefix is <= target
         while (l < r) {

@@ -287,3 +287,44 @@ def test_fp8_output_epilogue(heads):
             assert d.sum() / np.abs(ref).sum() <= 1e-3
         else:
             assert np.all(want_c[b] == 0) and np.all(scales.cpu().numpy()[b] == 1.0)
+
+
+def test_whole_sequence_blocks_write_the_merge_result_bitwise():
+    # When every sequence fits one sweep block at little cost (here 100
+    # sequences of a top-256 selection plus the window), each block writes its
+    # own sequence's output and the merge kernel skips the sequence. That output
+    # must be, bit for bit, the bf16 rounding of the merge kernel's fp32 result
+    # (the fp8-output entry point always merges and returns those fp32 values),
+    # inverse RoPE included, and meet the tolerance against the oracle.
+    from oracle import codecs
+    from paged_compressed_kv_b200 import v4kv
+    r = synth.rng(221)
+    lens = r.integers(1200, 1600, 100).tolist()
+    case = DecodeCase(221, lens, 64, 4)
+    k = 256
+    topk = np.full((case.B, k), -1, dtype=np.int64)
+    for b, L in enumerate(lens):
+        nv = max(0, L - 128) // 4
+        topk[b, :] = r.permutation(nv)[:k]
+    got, st = run_decode(case, topk=topk)
+    assert st == 0
+    dev = torch.device("cuda")
+    q = torch.from_numpy(case.q).to(dev)
+    main, win = case.main.to_cuda(), case.win.to_cuda()
+    seq = torch.from_numpy(case.lens.astype(np.int32)).to(dev)
+    tk = torch.from_numpy(topk.astype(np.int32)).to(dev)
+    ws = v4kv.v4kv_workspace_size(v4kv.V4KV_OP_DECODE, case.B, case.H, case.max_len, case.ratio,
+                                  case.W, k, main.dtype_code)
+    workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    codes = torch.empty(case.B, case.H, 512, dtype=torch.uint8, device=dev)
+    scales = torch.empty(case.B, case.H, dtype=torch.float32, device=dev)
+    pre = torch.full((case.B, case.H, 512), float("nan"), dtype=torch.float32, device=dev)
+    v4kv.v4kv_decode_attention_fp8out(q, main, win, seq, case.max_len, case.ratio, case.W, codes, scales,
+                                      workspace, topk=tk, prequant_out=pre, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    pre = pre.cpu().numpy()
+    got_bits = torch.from_numpy(got).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got_bits, codecs.bf16_bits(pre))
+    check_all(case, got, topk=topk, seqs=list(range(0, case.B, 11)))
