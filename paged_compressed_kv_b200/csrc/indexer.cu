@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_kernel(IndexArgs a)
   __shared__ __align__(16) uint32_t q16[kIdxMaxDim / 2];  // query codes as f16 pairs
   __shared__ uint32_t hist[kBins];
   __shared__ float red[32];
+  tc::pdl_launch_dependents();  // the select kernel may launch; it waits for this grid's results
   const int b = blockIdx.y;
   const int L = seq_len_of(a, b);
   const int n_vis = visible(L, a.window_len, a.ratio);
@@ -234,6 +235,7 @@ __global__ void __launch_bounds__(kTmaBatch) index_score_tma_kernel(const __grid
                                                                     IndexArgs a) {
   constexpr int kRowsPerBox = kFp4 ? kTmaBox / 2 : kTmaBox;  // 128-byte rows per 64-entry group
   extern __shared__ uint8_t dsm_raw[];
+  tc::pdl_launch_dependents();  // the select kernel may launch; it waits for this grid's results
   uint8_t* stages = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* hist2 = reinterpret_cast<uint32_t*>(stages + kTmaStages * kStageBytes);  // 16-bit pairs
   uint32_t* q16 = hist2 + kBins / 2;
@@ -472,6 +474,10 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexArgs 
     above_sh = 0;
   }
   __syncthreads();
+  // everything above reads only the call's inputs, so it overlaps the scoring
+  // kernel's tail (programmatic dependent launch); the scores and the
+  // histogram are complete from here on
+  tc::pdl_wait();
 
   if (n <= k) {
     for (int j = threadIdx.x; j < n; j += blockDim.x) sel[j] = comp_key(score_key(sc[j]), j);
@@ -609,8 +615,7 @@ cudaError_t launch_index_topk(IndexArgs a, int max_seq_len, cudaStream_t stream)
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  index_select_kernel<<<a.batch, kSelectThreads, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(index_select_kernel, dim3(a.batch), dim3(kSelectThreads), 0, stream, a);
 }
 
 }  // namespace v4kv
