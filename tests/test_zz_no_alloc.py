@@ -70,3 +70,34 @@ def test_noalloc_rejects_sizes_beyond_the_scratch():
     with pytest.raises(v4kv.V4KVError) as e:
         v4kv.v4kv_decode_attention_noalloc(q, main, win, seq, 1_000_000, 4, 128, out)
     assert e.value.status == v4kv.V4KV_ERR_INVALID_ARG
+
+
+def test_noalloc_call_allocates_nothing_under_graph_capture():
+    # The defining property: the call allocates no device memory. During a
+    # CUDA-graph capture in global mode any device allocation in the process
+    # fails the capture, so a warm call that captures cleanly allocates
+    # nothing; its replay must give the warm call's output bit for bit.
+    from paged_compressed_kv_b200 import v4kv
+    dev = torch.device("cuda")
+    case = DecodeCase(604, [5000, 700, 12000], 64, 4)
+    q = torch.from_numpy(case.q).to(dev)
+    main, win = case.main.to_cuda(), case.win.to_cuda()
+    seq = torch.from_numpy(case.lens.astype(np.int32)).to(dev)
+    warm = torch.empty(case.B, case.H, 512, dtype=torch.bfloat16, device=dev)
+    got = torch.full_like(warm, float("nan"))
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    v4kv.v4kv_decode_attention_noalloc(q, main, win, seq, case.max_len, case.ratio, case.W, warm,
+                                       dev_status=st)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side, capture_error_mode="global"):
+            v4kv.v4kv_decode_attention_noalloc(q, main, win, seq, case.max_len, case.ratio, case.W, got,
+                                               dev_status=st)
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(got.view(torch.int16), warm.view(torch.int16))
