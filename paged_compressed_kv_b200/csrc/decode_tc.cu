@@ -24,11 +24,13 @@
 //
 // Schedule: the kernel is persistent. The tiles of all sequences form one
 // list (each sequence: its entries padded to whole tiles, then its window);
-// block c of G processes tiles [c*T/G, (c+1)*T/G), so every SM gets the same
-// number of tiles whatever the length mix. A block writes one partial result
+// the prep kernel gives block c of G the range of tiles where the estimated
+// cost prefix runs from c/G to (c+1)/G of the total, or, when every sequence
+// fits one block cheaply, sequence c whole. A block writes one partial result
 // (O, m, l) per sequence it touches into slot b + c, which is unique because
 // b + c increases strictly along the tile list; the merge kernel combines the
-// slots of each sequence.
+// slots of each sequence. A block that runs every tile of a sequence writes
+// that sequence's output itself and the merge skips it.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
