@@ -328,3 +328,48 @@ def test_whole_sequence_blocks_write_the_merge_result_bitwise():
     got_bits = torch.from_numpy(got).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(got_bits, codecs.bf16_bits(pre))
     check_all(case, got, topk=topk, seqs=list(range(0, case.B, 11)))
+
+
+def test_whole_sequence_plan_with_wide_rope_and_empty_sequences():
+    # The one-sequence-per-block plan when the output cannot be written by the
+    # sweep (rope dims beyond the prep kernel's 32-pair cos/sin table): every
+    # sequence then goes through the merge, which must not skip any. Empty
+    # sequences in the batch own empty blocks and come out as zeros.
+    from oracle import attention
+    from paged_compressed_kv_b200 import Rope, v4kv
+    r = synth.rng(222)
+    lens = r.integers(1200, 1600, 100).tolist()
+    for b in (3, 50, 99):
+        lens[b] = 0
+    case = DecodeCase(222, lens, 64, 4)
+    k = 256
+    topk = np.full((case.B, k), -1, dtype=np.int64)
+    for b, L in enumerate(lens):
+        nv = max(0, L - 128) // 4
+        topk[b, : min(k, nv)] = r.permutation(nv)[:k]
+    rope = Rope(rope_dim=128, rope_offset=384)
+    dev = torch.device("cuda")
+    q = torch.from_numpy(case.q).to(dev)
+    main, win = case.main.to_cuda(), case.win.to_cuda()
+    seq = torch.from_numpy(case.lens.astype(np.int32)).to(dev)
+    out = torch.full((case.B, case.H, 512), float("nan"), dtype=torch.bfloat16, device=dev)
+    ws = v4kv.v4kv_workspace_size(v4kv.V4KV_OP_DECODE, case.B, case.H, case.max_len, case.ratio,
+                                  case.W, k, main.dtype_code)
+    workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    v4kv.v4kv_decode_attention(q, main, win, seq, case.max_len, case.ratio, case.W, out, workspace,
+                               topk=torch.from_numpy(topk.astype(np.int32)).to(dev), rope=rope,
+                               dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got = out.float().cpu().numpy()
+    assert not np.isnan(got).any()
+    for b in (3, 50, 99):
+        assert np.all(got[b] == 0)
+    for b in range(0, case.B, 9):
+        if lens[b] == 0:
+            continue
+        ref = attention.decode_one(case.q[b].astype(np.float64), case.main.seq(b), case.win.seq(b), lens[b],
+                                   4, case.W, 1 / math.sqrt(512), topk_row=topk[b], rope_dim=128,
+                                   rope_offset=384)
+        assert_close_bf16(got[b], ref, f"seq {b} L={lens[b]}")
