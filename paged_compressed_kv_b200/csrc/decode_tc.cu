@@ -330,6 +330,7 @@ __device__ __forceinline__ void cursor_next(Cursor& c, const DecodeArgs& a) {
 
 constexpr uint32_t kQBytes = kH * kD * 2;  // one query image (f16)
 constexpr int kMaxSplits = 160;            // sweep blocks at most (the plan caps the grid)
+constexpr int kMergeWarps = 4;             // heads per merge block (a warp each)
 constexpr int kPrepCache = 2048;           // batches whose prefix sums the prep keeps in shared memory
 
 // Start the bulk copy of sequence b's query image into shared memory; the
@@ -975,30 +976,55 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
   }
 }
 
-// grid (heads / 8, batch), 256 threads: warp w merges head 8 * blockIdx.x + w
-// of sequence b over the blocks whose tile ranges met it (lane l: dims 16l ..
-// 16l + 15), normalises, applies the inverse RoPE at position L - 1 (cos/sin
-// from the prep kernel's table) and stores bf16.
-__global__ void __launch_bounds__(256) decode_tc_merge_kernel(DecodeArgs a) {
-  __shared__ float w_sh[8][kMaxSplits];  // per warp: the blocks' weights
+// grid (heads / kMergeWarps, batch), a warp per head: warp w merges head
+// kMergeWarps * blockIdx.x + w of sequence b over the blocks whose tile ranges
+// met it (lane l: dims 16l .. 16l + 15), normalises, applies the inverse RoPE
+// at position L - 1 (cos/sin from the prep kernel's table) and stores bf16
+// (or e4m3 with a scale per head).
+template <int kMergeFirst>
+__global__ void __launch_bounds__(kMergeWarps * 32) decode_tc_merge_kernel(DecodeArgs a) {
+  __shared__ float w_sh[kMergeWarps][kMaxSplits];  // per warp: the blocks' weights
+  __shared__ float2 cs_sh[kRopeTable];             // the sequence's inverse-RoPE cos / sin
   tc::pdl_wait();  // the sweep's partial results are complete from here on
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = 8 * blockIdx.x + warp, b = blockIdx.y;
-  const int Lb = min(a.seq_lens[b], a.max_len);  // independent of the loads below
+  const int h = kMergeWarps * blockIdx.x + warp, b = blockIdx.y;
+  const int d0 = 16 * lane;
+  // independent loads first: the sequence's blocks and length, and its
+  // inverse-RoPE table (read at the end)
   const int2 sl = a.seq_slots[b];
+  const int Lb = min(a.seq_lens[b], a.max_len);
+  if (threadIdx.x < kRopeTable) cs_sh[threadIdx.x] = a.rope_tab[(size_t)b * kRopeTable + threadIdx.x];
   const int lo = sl.x, hi = sl.y;
   if (lo == hi && direct_output(a)) return;  // one block ran the whole sequence and wrote its output
-  // per block: (m, l) in one load; the weights go to shared memory
-  float M = -INFINITY;
+  // per block: (m, l) and whether the block has tiles, loaded together; the
+  // first four blocks' rows are requested at the same time (they do not
+  // depend on the weights, which only select them)
   float2 ml_keep[(kMaxSplits + 31) / 32];
+  bool has_keep[(kMaxSplits + 31) / 32];
 #pragma unroll
   for (int k = 0; k < (kMaxSplits + 31) / 32; ++k) {
     const int c = lo + lane + 32 * k;
-    float2 ml = make_float2(-INFINITY, 0.f);
-    if (c <= hi && a.cta_x0[c + 1] > a.cta_x0[c])
-      ml = reinterpret_cast<const float2*>(a.part_ml)[((size_t)b + c) * kH + h];
-    ml_keep[k] = ml;
-    M = fmaxf(M, ml.x);
+    ml_keep[k] = make_float2(-INFINITY, 0.f);
+    has_keep[k] = false;
+    if (c <= hi) {
+      ml_keep[k] = reinterpret_cast<const float2*>(a.part_ml)[((size_t)b + c) * kH + h];
+      has_keep[k] = a.cta_x0[c + 1] > a.cta_x0[c];
+    }
+  }
+  float4 v0[kMergeFirst][4];
+#pragma unroll
+  for (int j = 0; j < kMergeFirst; ++j) {
+    if (lo + j <= hi) {
+      const float4* o4 = reinterpret_cast<const float4*>(a.part_o + (((size_t)b + lo + j) * kH + h) * kD + d0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v0[j][q] = o4[q];
+    }
+  }
+  float M = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < (kMaxSplits + 31) / 32; ++k) {
+    if (!has_keep[k]) ml_keep[k] = make_float2(-INFINITY, 0.f);
+    M = fmaxf(M, ml_keep[k].x);
   }
   M = warp_max(M);
   float L = 0.f;
@@ -1013,37 +1039,39 @@ __global__ void __launch_bounds__(256) decode_tc_merge_kernel(DecodeArgs a) {
   }
   L = warp_sum(L);
   __syncwarp();
-  // weighted sum of the blocks' rows, four blocks' loads in flight at a time
-  const int d0 = 16 * lane;
+  // weighted sum of the blocks' rows in block order (a block with weight 0
+  // adds 0 * 0, as every block's row would)
   float acc[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-  for (int c = lo; c <= hi; c += 4) {
-    float4 v[4][4];
-    float w[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      w[j] = c + j <= hi ? w_sh[warp][c + j - lo] : 0.f;
-      if (w[j] != 0.f) {
-        const float4* o4 =
-            reinterpret_cast<const float4*>(a.part_o + (((size_t)b + c + j) * kH + h) * kD + d0);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) v[j][q] = o4[q];
-      } else {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) v[j][q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
+  auto add_rows = [&](int c, int nj, float4 (*v)[4]) {
+#pragma unroll 4
+    for (int j = 0; j < nj; ++j) {
+      const float w = c + j <= hi ? w_sh[warp][c + j - lo] : 0.f;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        acc[4 * q] = fmaf(w[j], v[j][q].x, acc[4 * q]);
-        acc[4 * q + 1] = fmaf(w[j], v[j][q].y, acc[4 * q + 1]);
-        acc[4 * q + 2] = fmaf(w[j], v[j][q].z, acc[4 * q + 2]);
-        acc[4 * q + 3] = fmaf(w[j], v[j][q].w, acc[4 * q + 3]);
+        const float4 x = w != 0.f ? v[j][q] : make_float4(0.f, 0.f, 0.f, 0.f);
+        acc[4 * q] = fmaf(w, x.x, acc[4 * q]);
+        acc[4 * q + 1] = fmaf(w, x.y, acc[4 * q + 1]);
+        acc[4 * q + 2] = fmaf(w, x.z, acc[4 * q + 2]);
+        acc[4 * q + 3] = fmaf(w, x.w, acc[4 * q + 3]);
       }
+    }
+  };
+  add_rows(lo, kMergeFirst, v0);
+  for (int c = lo + kMergeFirst; c <= hi; c += kMergeFirst) {
+    float4 v[kMergeFirst][4];
+#pragma unroll
+    for (int j = 0; j < kMergeFirst; ++j) {
+      if (c + j <= hi) {
+        const float4* o4 = reinterpret_cast<const float4*>(a.part_o + (((size_t)b + c + j) * kH + h) * kD + d0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[j][q] = o4[q];
+      }
+    }
+    add_rows(c, kMergeFirst, v);
   }
+  __syncthreads();  // the RoPE table is in shared memory
   const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
   for (int e = 0; e < 16; ++e) acc[e] *= inv;
@@ -1055,9 +1083,8 @@ __global__ void __launch_bounds__(256) decode_tc_merge_kernel(DecodeArgs a) {
         const int i = (d - a.rope.rope_offset) >> 1;
         float c, s;
         if (i < kRopeTable) {
-          const float2 cs = a.rope_tab[(size_t)b * kRopeTable + i];
-          c = cs.x;
-          s = cs.y;
+          c = cs_sh[i].x;
+          s = cs_sh[i].y;
         } else {
           rope_cs(a.rope, i, (long long)Lb - 1, &c, &s);
         }
@@ -1317,7 +1344,13 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   e = launch_pdl(decode_tc_kernel, dim3(a.n_splits), dim3(kThreads), kSmemBytes, stream, a);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_tc_merge_kernel, dim3(kH / 8, a.batch), dim3(256), 0, stream, a);
+  // a merge warp holds the rows of kMergeFirst blocks in flight (the first
+  // ones requested with the blocks' (m, l)): four when the grid of the wider
+  // kernel (about four blocks per SM) fits one wave, else two (seven per SM)
+  const dim3 mgrid(kH / kMergeWarps, a.batch);
+  if ((long long)a.batch * (kH / kMergeWarps) <= 4LL * a.n_splits)
+    return launch_pdl(decode_tc_merge_kernel<4>, mgrid, dim3(kMergeWarps * 32), 0, stream, a);
+  return launch_pdl(decode_tc_merge_kernel<2>, mgrid, dim3(kMergeWarps * 32), 0, stream, a);
 }
 
 }  // namespace v4kv
