@@ -985,31 +985,34 @@ template <int kMergeFirst>
 __global__ void __launch_bounds__(kMergeWarps * 32) decode_tc_merge_kernel(DecodeArgs a) {
   __shared__ float w_sh[kMergeWarps][kMaxSplits];  // per warp: the blocks' weights
   __shared__ float2 cs_sh[kRopeTable];             // the sequence's inverse-RoPE cos / sin
-  tc::pdl_wait();  // the sweep's partial results are complete from here on
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = kMergeWarps * blockIdx.x + warp, b = blockIdx.y;
   const int d0 = 16 * lane;
-  // independent loads first: the sequence's blocks and length, and its
-  // inverse-RoPE table (read at the end)
+  // What the prep kernel wrote is read before the wait: the sweep launched
+  // this grid only after its own wait for the prep kernel, so those writes
+  // are complete, and these loads overlap the sweep's last blocks. The
+  // sequence's blocks and length, which of them have tiles, and the
+  // inverse-RoPE table (read at the end).
   const int2 sl = a.seq_slots[b];
   const int Lb = min(a.seq_lens[b], a.max_len);
   if (threadIdx.x < kRopeTable) cs_sh[threadIdx.x] = a.rope_tab[(size_t)b * kRopeTable + threadIdx.x];
   const int lo = sl.x, hi = sl.y;
-  if (lo == hi && direct_output(a)) return;  // one block ran the whole sequence and wrote its output
-  // per block: (m, l) and whether the block has tiles, loaded together; the
-  // first four blocks' rows are requested at the same time (they do not
-  // depend on the weights, which only select them)
-  float2 ml_keep[(kMaxSplits + 31) / 32];
   bool has_keep[(kMaxSplits + 31) / 32];
 #pragma unroll
   for (int k = 0; k < (kMaxSplits + 31) / 32; ++k) {
     const int c = lo + lane + 32 * k;
+    has_keep[k] = c <= hi && a.cta_x0[c + 1] > a.cta_x0[c];
+  }
+  tc::pdl_wait();  // the sweep's partial results are complete from here on
+  if (lo == hi && direct_output(a)) return;  // one block ran the whole sequence and wrote its output
+  // per block: (m, l); the first blocks' rows are requested at the same time
+  // (they do not depend on the weights, which only select them)
+  float2 ml_keep[(kMaxSplits + 31) / 32];
+#pragma unroll
+  for (int k = 0; k < (kMaxSplits + 31) / 32; ++k) {
+    const int c = lo + lane + 32 * k;
     ml_keep[k] = make_float2(-INFINITY, 0.f);
-    has_keep[k] = false;
-    if (c <= hi) {
-      ml_keep[k] = reinterpret_cast<const float2*>(a.part_ml)[((size_t)b + c) * kH + h];
-      has_keep[k] = a.cta_x0[c + 1] > a.cta_x0[c];
-    }
+    if (c <= hi) ml_keep[k] = reinterpret_cast<const float2*>(a.part_ml)[((size_t)b + c) * kH + h];
   }
   float4 v0[kMergeFirst][4];
 #pragma unroll
