@@ -147,10 +147,6 @@ __device__ __forceinline__ Seq seq_of(const DecodeArgs& a, int b, int32_t* st) {
   return seq_from_len(a, max(0, L));
 }
 
-__device__ __forceinline__ void prefetch_l2_line(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
 // one bulk L2 prefetch of `bytes` (a multiple of 16, 16-byte aligned) through
 // the copy engine
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
@@ -503,9 +499,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
       const int tile0 = cu.lt * kT;
       resolve_tile(a, cu.b, cu.s, tile0, lane, rowptr + buf * kT, meta + buf * kT);
       if (t >= 2) {
-        // rows into L2 for the workers' loads. Tiles 0 and 1 are loaded at
-        // once by the workers; prefetching them too would only add to the
-        // burst of requests every block makes at its start.
+        // rows into L2 for the workers' loads, one bulk prefetch per row (a
+        // per-line prefetch issues four times the instructions, which hold up
+        // the softmax's shared- and tensor-memory operations). Tiles 0 and 1
+        // are loaded at once by the workers; prefetching them too would only
+        // add to the burst of requests every block makes at its start.
         const bool main_tile = tile0 < cu.s.n_sel_pad;
         const bool fp8 = (main_tile ? a.main.dtype : a.window.dtype) == V4KV_FP8_E4M3;
         const uint8_t* const* rp = rowptr + buf * kT;
@@ -513,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(DecodeArgs a) {
         for (int r = 0; r < 4; ++r) {
           const uint8_t* pr = rp[lane + 32 * r];
           if (pr)
-            for (int k = 0; k < (fp8 ? kD / 128 : 2 * kD / 128); ++k) prefetch_l2_line(pr + 128 * k);
+            prefetch_l2_bulk(pr, fp8 ? kD : 2 * kD);
         }
       }
       if (lane == 0) {
