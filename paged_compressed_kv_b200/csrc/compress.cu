@@ -5,9 +5,10 @@
 //
 // One launch does all three. Its first blocks copy window rows (one warp per
 // token). The rest build entries:
-//   ratio <= 32: one warp per group, eight groups per block;
-//   larger ratios: one block per group, each warp summing a run of rows,
-//                  the eight partial sums added in warp order.
+//   ratio 4: one warp per group, eight groups per block, the group's rows
+//            staged in shared memory with cp.async;
+//   ratio 128: one block per group, each warp summing a run of rows,
+//              the eight partial sums added in warp order.
 // Every row is an 8-dim chunk per lane (chunk c = lane + 32k), so a lane
 // always touches the same columns of every row it reads or writes.
 //
@@ -44,19 +45,37 @@ __device__ __forceinline__ void load_row(const uint16_t* row, int lane, int nch,
   }
 }
 
+// (cos, sin) of rope pair `lane` at position `pos` (identity past the last
+// pair): the first 32 pairs' values, one per lane, which rope_warp uses
+__device__ __forceinline__ void rope_pair_lane(const RopeArgs& rp, int lane, long long pos, float* c,
+                                               float* s) {
+  *c = 1.f;
+  *s = 0.f;
+  if (lane < (rp.rope_dim >> 1)) rope_cs(rp, lane, pos, c, s);
+}
+
 // rotate the rope pairs among this lane's dims at position `pos`. Pair p's
 // (cos, sin) is evaluated once per warp, by lane p % 32, and fetched with
-// shuffles, so every lane must call this.
+// shuffles, so every lane must call this. (c0, s0) are this lane's values
+// for the first 32 pairs (rope_pair_lane), evaluated by the caller, which
+// can then do it while it waits for memory.
 template <int KC>
 __device__ __forceinline__ void rope_warp(float (&e)[KC][8], int lane, int nch, const RopeArgs& rp,
-                                          long long pos) {
+                                          long long pos, float c0, float s0) {
   if (rp.rope_dim == 0) return;
   const int npairs = rp.rope_dim >> 1;
   for (int base = 0; base < npairs; base += 32) {
-    float c = 1.f, s = 0.f;
-    if (base + lane < npairs) rope_cs(rp, base + lane, pos, &c, &s);
+    float c = c0, s = s0;
+    if (base > 0) {
+      c = 1.f;
+      s = 0.f;
+      if (base + lane < npairs) rope_cs(rp, base + lane, pos, &c, &s);
+    }
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
+      // chunks 32k .. 32k + 31 hold dims [256k, 256k + 256): skip them (the
+      // whole warp) when none is rotated
+      if (256 * k >= rp.rope_offset + rp.rope_dim || 256 * (k + 1) <= rp.rope_offset) continue;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int d = 8 * (lane + 32 * k) + 2 * j;
@@ -68,6 +87,36 @@ __device__ __forceinline__ void rope_warp(float (&e)[KC][8], int lane, int nch, 
       }
     }
   }
+}
+
+template <int KC>
+__device__ __forceinline__ void rope_warp(float (&e)[KC][8], int lane, int nch, const RopeArgs& rp,
+                                          long long pos) {
+  if (rp.rope_dim == 0) return;
+  float c0, s0;
+  rope_pair_lane(rp, lane, pos, &c0, &s0);
+  rope_warp<KC>(e, lane, nch, rp, pos, c0, s0);
+}
+
+// v / scale as far as its e4m3 code is concerned, y = 1 / scale rounded to
+// nearest. The product v * y is within 2 fp32 ulps of v / scale (two
+// roundings of relative size 2^-24 each), and the correctly rounded quotient
+// within half an ulp of it, so both give the same e4m3 code unless v / scale
+// lies near the midpoint between two neighbouring codes. The code of a
+// normal-range value (binades 2^-6 .. 2^8) depends only on the 3 leading
+// mantissa bits and the rounding bit below them, so a midpoint is a pattern of
+// 0x80000 in the 20 low mantissa bits; within 8 ulps of it, and below the
+// normal e4m3 range or for infinities and NaNs, the IEEE quotient is formed
+// instead. The codes are therefore those of float2_to_e4m3x2(v / scale).
+__device__ __forceinline__ float e4m3_quotient(float v, float scale, float y) {
+  const float q = __fmul_rn(v, y);
+  const uint32_t u = __float_as_uint(q) & 0x7fffffffu;
+  // outside [2^-6, inf): the unsigned difference wraps past the range
+  const bool outside = u - 0x3c800000u >= 0x7f800000u - 0x3c800000u;
+  // low 20 mantissa bits within 8 of 0x80000
+  const bool near_mid = ((u + 8u - 0x80000u) & 0xfffffu) <= 16u;
+  if (outside || near_mid) return __fdiv_rn(v, scale);
+  return q;
 }
 
 // quantise (fp8: absmax over the warp's whole vector) or round (bf16) one
@@ -84,6 +133,7 @@ __device__ __forceinline__ void store_entry_warp(const PoolArgs& pool, long long
         for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(e[k][i]));
     const float amax = warp_max(m);
     const float scale = amax == 0.f ? 1.f : __fdiv_rn(amax, kE4m3Max);
+    const float y = __frcp_rn(scale);
     uint8_t* base = reinterpret_cast<uint8_t*>(pool.data) + slot * pool.dim;
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
@@ -92,7 +142,8 @@ __device__ __forceinline__ void store_entry_warp(const PoolArgs& pool, long long
       uint16_t q[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        q[i] = float2_to_e4m3x2(__fdiv_rn(e[k][2 * i], scale), __fdiv_rn(e[k][2 * i + 1], scale));
+        q[i] = float2_to_e4m3x2(e4m3_quotient(e[k][2 * i], scale, y),
+                                e4m3_quotient(e[k][2 * i + 1], scale, y));
       *reinterpret_cast<uint2*>(base + 8 * c) =
           make_uint2((uint32_t)q[0] | ((uint32_t)q[1] << 16), (uint32_t)q[2] | ((uint32_t)q[3] << 16));
     }
@@ -142,71 +193,6 @@ __device__ __forceinline__ void window_row(const CompressArgs& a, int b, int u, 
   store_entry_warp<KC>(a.window, (long long)p * kLogicalBlock + (t % kLogicalBlock), lane, nch, e);
 }
 
-// the group's softmax weights over its np present tokens (gate + position
-// bias), written to w[0..np) by one warp
-template <int NQ>
-__device__ __forceinline__ void group_weights(const CompressArgs& a, int b, int s, int t0, int np,
-                                              int lane, float* w) {
-  const int r = a.ratio;
-  float z[NQ];
-  float m = -INFINITY;
-#pragma unroll
-  for (int q = 0; q < NQ; ++q) {
-    const int t = lane + 32 * q;
-    z[q] = -INFINITY;
-    if (t < np) {
-      const int tt = t0 + t;
-      const float g = tt < s ? a.state_gate[(size_t)b * r + t] : a.gate[a.cu_seqlens[b] + (tt - s)];
-      z[q] = g + a.pos_bias[t];
-      m = fmaxf(m, z[q]);
-    }
-  }
-  m = warp_max(m);
-  float part = 0.f;
-#pragma unroll
-  for (int q = 0; q < NQ; ++q) {
-    z[q] = lane + 32 * q < np ? expf(z[q] - m) : 0.f;
-    part += z[q];
-  }
-  const float sum = warp_sum(part);
-#pragma unroll
-  for (int q = 0; q < NQ; ++q)
-    if (lane + 32 * q < np) w[lane + 32 * q] = __fdiv_rn(z[q], sum);
-  __syncwarp();
-}
-
-// acc += sum over rows [lo, hi) of the group (ascending) of w[t] * row t
-template <int KC, int RB>
-__device__ __forceinline__ void weighted_rows(const CompressArgs& a, int b, int s, int t0, int lo,
-                                              int hi, const float* w, int lane, int nch,
-                                              float (&acc)[KC][8]) {
-  const int r = a.ratio;
-  for (int t = lo; t < hi; t += RB) {
-    uint4 q[RB][KC];
-#pragma unroll
-    for (int j = 0; j < RB; ++j) {
-      const int tt = t0 + t + j;
-      if (t + j < hi) {
-        const uint16_t* row = tt < s ? a.state_x + ((size_t)b * r + (t + j)) * a.dim
-                                     : a.x + (size_t)(a.cu_seqlens[b] + (tt - s)) * a.dim;
-        load_row<KC>(row, lane, nch, q[j]);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < RB; ++j) {
-      if (t + j >= hi) break;
-      const float wt = w[t + j];
-#pragma unroll
-      for (int k = 0; k < KC; ++k) {
-        float v[8];
-        unpack_bf16x8(q[j][k], v);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wt, v[e], acc[k][e]);
-      }
-    }
-  }
-}
-
 // RMSNorm of one vector held by a warp: e * w / sqrt(mean(e^2) + eps)
 template <int KC>
 __device__ __forceinline__ void rms_norm_warp(float (&e)[KC][8], int lane, int nch, const float* w,
@@ -231,13 +217,35 @@ __device__ __forceinline__ void rms_norm_warp(float (&e)[KC][8], int lane, int n
   }
 }
 
-// RMSNorm (when weights are given), RoPE at the group's first position,
-// optional pre-quantisation copy, and the store into the entry's slot
+// slot of entry i (group t0 / r of sequence b): from the slot mapping, or
+// (none passed) from the block table; -1 when there is nothing to store
+// (an unmapped page, flagged by the slot mapping, or a bad slot, flagged here)
+__device__ __forceinline__ long long entry_slot(const CompressArgs& a, int i, int b, int t0, int lane) {
+  long long slot;
+  if (a.slot_mapping) {
+    slot = a.slot_mapping[i];
+  } else {
+    const long long g = t0 / a.ratio;
+    const int p = page_of(a.main.block_table + (size_t)b * a.main.max_blocks, a.main.max_blocks, g,
+                          a.main.spb, a.main.num_pages, lane == 0 ? a.dev_status : nullptr);
+    slot = p < 0 ? -1 : (long long)p * a.main.spb + g % a.main.spb;
+  }
+  if (slot >= (long long)a.main.num_pages * a.main.spb) {
+    if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
+    return -1;
+  }
+  return slot < 0 ? -1 : slot;
+}
+
+// RMSNorm (when weights are given), RoPE at the group's first position
+// (rope_c, rope_s: rope_pair_lane at t0), optional pre-quantisation copy, and
+// the store into `slot` (entry_slot)
 template <int KC>
-__device__ __forceinline__ void finish_entry(const CompressArgs& a, int i, int b, int t0, int lane,
-                                             int nch, float (&e)[KC][8]) {
+__device__ __forceinline__ void finish_entry(const CompressArgs& a, int i, int t0, int lane, int nch,
+                                             float (&e)[KC][8], float rope_c, float rope_s,
+                                             long long slot) {
   if (a.norm_w) rms_norm_warp<KC>(e, lane, nch, a.norm_w, a.norm_eps, a.dim);
-  rope_warp<KC>(e, lane, nch, a.rope, (long long)t0);
+  rope_warp<KC>(e, lane, nch, a.rope, (long long)t0, rope_c, rope_s);
   if (a.prequant_out) {
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
@@ -248,23 +256,16 @@ __device__ __forceinline__ void finish_entry(const CompressArgs& a, int i, int b
       *reinterpret_cast<float4*>(po + 4) = make_float4(e[k][4], e[k][5], e[k][6], e[k][7]);
     }
   }
-  long long slot;
-  if (a.slot_mapping) {
-    slot = a.slot_mapping[i];
-  } else {
-    // the slot mapping of this entry (group t0 / r of sequence b) inline
-    const long long g = t0 / a.ratio;
-    const int p = page_of(a.main.block_table + (size_t)b * a.main.max_blocks, a.main.max_blocks, g,
-                          a.main.spb, a.main.num_pages, lane == 0 ? a.dev_status : nullptr);
-    slot = p < 0 ? -1 : (long long)p * a.main.spb + g % a.main.spb;
-  }
-  const long long cap = (long long)a.main.num_pages * a.main.spb;
-  if (slot < 0) return;  // unmapped page (flagged by the slot mapping)
-  if (slot >= cap) {
-    if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
-    return;
-  }
-  store_entry_warp<KC>(a.main, slot, lane, nch, e);
+  if (slot >= 0) store_entry_warp<KC>(a.main, slot, lane, nch, e);
+}
+
+// finish_entry with the slot and the rope values evaluated here
+template <int KC>
+__device__ __forceinline__ void finish_entry(const CompressArgs& a, int i, int b, int t0, int lane,
+                                             int nch, float (&e)[KC][8]) {
+  float c0 = 1.f, s0 = 0.f;
+  if (a.rope.rope_dim) rope_pair_lane(a.rope, lane, (long long)t0, &c0, &s0);
+  finish_entry<KC>(a, i, t0, lane, nch, e, c0, s0, entry_slot(a, i, b, t0, lane));
 }
 
 // state rows [lo, hi) of sequence b after this call: tokens gs + i of the
@@ -348,104 +349,382 @@ __device__ __forceinline__ const int32_t* entry_prefix(const CompressArgs& a, in
   return a.cu_entries;
 }
 
-// KC: 8-dim chunks per lane (dim <= 256 * KC). kBlockGroup: one block per
-// group (ratio > 32) instead of one warp per group.
-template <int KC, bool kBlockGroup>
-__global__ void __launch_bounds__(kWarps * 32) compress_append_kernel(CompressArgs a,
-                                                                     int window_blocks,
-                                                                     int window_blocks_per_seq) {
-  constexpr int kRB = (KC <= 2 && kBlockGroup) ? 8 : 4;  // rows in flight per warp
-  constexpr int kNQ = kBlockGroup ? kMaxRatio / 32 : 1;  // gates per lane
-  __shared__ float w_sh[kWarps][kNQ * 32];
-  __shared__ float part[kBlockGroup ? kWarps : 1][kBlockGroup ? KC * 256 : 1];
+// cp.async of one 16-byte chunk into this thread's shared memory (cached in
+// L2 only); the thread that copies a chunk is the one that reads it back,
+// after cp_async_wait_all
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+constexpr int kGroupRows = 4;  // rows of a group on the warp-per-group path (ratio 4)
+
+// Per-call tables in shared memory for the kernels with a compile-time ratio
+// kR: the entry prefix sums (cu_sh, batch + 1 values) and, per sequence, its
+// seq_start and cu_seqlens (meta_sh[b] = {seq_start[b], cu_seqlens[b]},
+// meta_sh[batch].y = cu_seqlens[batch]). With batch <= 32 one warp builds
+// them while the others wait at the barrier. Returns false when batch + 1 >
+// kCuSmem: then the slot mapping's prefix sums and the global arrays serve.
+template <int kR>
+__device__ __forceinline__ bool seq_tables(const CompressArgs& a, int* cu_sh, int2* meta_sh) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (a.batch + 1 > kCuSmem) return false;
+  if (a.batch <= 32) {
+    if (warp == 0) {
+      int n = 0;
+      if (lane < a.batch) {
+        const int s0 = a.seq_start[lane], c0 = a.cu_seqlens[lane], c1 = a.cu_seqlens[lane + 1];
+        const int m = c1 - c0;
+        n = m > 0 ? (s0 + m + kR - 1) / kR - s0 / kR : 0;
+        meta_sh[lane] = make_int2(s0, c0);
+        if (lane == a.batch - 1) meta_sh[a.batch] = make_int2(0, c1);
+      }
+      if (a.cu_entries) {
+        if (lane <= a.batch) cu_sh[lane] = a.cu_entries[lane];
+      } else {
+        int x = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (lane < a.batch) cu_sh[lane] = x - n;
+        if (lane == a.batch - 1) cu_sh[a.batch] = x;
+      }
+    }
+    __syncthreads();
+    return true;
+  }
+  for (int k = threadIdx.x; k <= a.batch; k += blockDim.x)
+    meta_sh[k] = make_int2(k < a.batch ? a.seq_start[k] : 0, a.cu_seqlens[k]);
+  if (a.cu_entries) {
+    for (int k = threadIdx.x; k <= a.batch; k += blockDim.x) cu_sh[k] = a.cu_entries[k];
+    __syncthreads();
+    return true;
+  }
+  __shared__ int wsum[kWarps];
+  int carry = 0;
+  for (int base = 0; base < a.batch; base += kWarps * 32) {
+    const int bb = base + threadIdx.x;
+    int n = 0;
+    if (bb < a.batch) {
+      const int s0 = a.seq_start[bb], m = a.cu_seqlens[bb + 1] - a.cu_seqlens[bb];
+      n = m > 0 ? (s0 + m + kR - 1) / kR - s0 / kR : 0;
+    }
+    int x = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    int before = carry;
+    for (int w2 = 0; w2 < warp; ++w2) before += wsum[w2];
+    if (bb < a.batch) cu_sh[bb] = before + x - n;
+    for (int w2 = 0; w2 < kWarps; ++w2) carry += wsum[w2];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) cu_sh[a.batch] = carry;
+  __syncthreads();
+  return true;
+}
+
+// Ratio 4: one warp per group, eight groups per block; the leading blocks
+// copy window rows. The group's rows go into the warp's shared memory with
+// cp.async (lane l copies and later reads chunks l, l + 32, ...). Then, while
+// they are in flight, the warp issues the loads of the gates, the position
+// bias and the entry's block-table entry, evaluates the RoPE cos / sin at the
+// group's position, and only then consumes the loads: the group costs one
+// memory latency after the per-call tables. KC: 8-dim chunks per lane (dim <=
+// 256 * KC); kFull: dim == 256 * KC (no partial chunk rows). Dynamic shared
+// memory: kWarps * kGroupRows * KC * 512 B.
+template <int KC, bool kFull>
+__global__ void __launch_bounds__(kWarps * 32, KC <= 2 ? 4 : 2)
+    compress_group_warp_kernel(CompressArgs a, int window_blocks, int window_blocks_per_seq) {
+  constexpr int r = kGroupRows;
+  constexpr int spb = kLogicalBlock / kGroupRows;  // entries per page
+  extern __shared__ uint4 rows_sh[];  // [kWarps][kGroupRows][KC][32]
   __shared__ int cu_sh[kCuSmem];
+  __shared__ int2 meta_sh[kCuSmem];
   tc::pdl_wait();  // the slot mapping (and whatever produced x) is complete from here on
   tc::pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nch = a.dim >> 3;
+  const int nch = kFull ? 32 * KC : a.dim >> 3;
   if ((int)blockIdx.x < window_blocks) {
     window_row<KC>(a, blockIdx.x / window_blocks_per_seq,
                    (blockIdx.x % window_blocks_per_seq) * kWarps + warp, lane, nch);
     return;
   }
-  const int eb = blockIdx.x - window_blocks;
-  const int32_t* cu = entry_prefix(a, cu_sh);
+  const bool cached = seq_tables<r>(a, cu_sh, meta_sh);
+  const int32_t* cu = cached ? cu_sh : a.cu_entries;
   const int total = cu[a.batch];
-  const int i = kBlockGroup ? eb : eb * kWarps + warp;
-  if (i >= total) return;  // uniform over the warp (and over the block for block groups)
+  const int i = (blockIdx.x - window_blocks) * kWarps + warp;
+  if (i >= total) return;  // uniform over the warp
   const int b = seq_of(cu, a.batch, i);
-  const int r = a.ratio;
-  const int s = a.seq_start[b];
-  const int end = s + (a.cu_seqlens[b + 1] - a.cu_seqlens[b]);
-  const int t0 = (s / r + (i - cu[b])) * r;
+  const int s = cached ? meta_sh[b].x : a.seq_start[b];
+  const int c0 = cached ? meta_sh[b].y : a.cu_seqlens[b];
+  const int end = s + ((cached ? meta_sh[b + 1].y : a.cu_seqlens[b + 1]) - c0);
+  const int g = s / r + (i - cu[b]);  // the entry's group index in the sequence
+  const int t0 = g * r;
   const int np = min(t0 + r, end) - t0;
-  const bool first_of_seq = i == cu[b];
 
-  float* w = w_sh[warp];
+  // 1. the rows, into shared memory
+  uint4* stage = rows_sh + (size_t)warp * kGroupRows * KC * 32;
+#pragma unroll
+  for (int j = 0; j < kGroupRows; ++j) {
+    if (j < np) {
+      const int tt = t0 + j;
+      const uint16_t* row = tt < s ? a.state_x + ((size_t)b * r + j) * a.dim
+                                   : a.x + (size_t)(c0 + (tt - s)) * a.dim;
+#pragma unroll
+      for (int k = 0; k < KC; ++k)
+        if (kFull || lane + 32 * k < nch)
+          cp_async16(stage + (j * KC + k) * 32 + lane, row + 8 * (lane + 32 * k));
+    }
+  }
+  // 2. gate, position bias and page loads, consumed after the RoPE values
+  float gate = 0.f, bias = 0.f;
+  if (lane < np) {
+    const int tt = t0 + lane;
+    gate = tt < s ? a.state_gate[(size_t)b * r + lane] : a.gate[c0 + (tt - s)];
+    bias = a.pos_bias[lane];
+  }
+  const int blk = g / spb;
+  long long slot = -1;
+  int page = -1;
+  if (a.slot_mapping) slot = a.slot_mapping[i];
+  else if (blk < a.main.max_blocks) page = a.main.block_table[(size_t)b * a.main.max_blocks + blk];
+  float rc = 1.f, rs = 0.f;
+  if (a.rope.rope_dim) rope_pair_lane(a.rope, lane, (long long)t0, &rc, &rs);
+  if (!a.slot_mapping) {
+    if (blk >= a.main.max_blocks) {
+      if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
+    } else if (page < 0 || page >= a.main.num_pages) {
+      if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_PAGE);
+    } else {
+      slot = (long long)page * spb + g % spb;
+    }
+  }
+  if (slot >= (long long)a.main.num_pages * spb) {
+    if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
+    slot = -1;
+  }
+  // 3. the gate softmax over the np present tokens; lane j holds w[j]
+  const float z = lane < np ? gate + bias : -INFINITY;
+  const float m = warp_max(z);
+  const float ez = lane < np ? expf(z - m) : 0.f;
+  const float wl = __fdiv_rn(ez, warp_sum(ez));
+
   float acc[KC][8];
 #pragma unroll
   for (int k = 0; k < KC; ++k)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
-
-  if constexpr (!kBlockGroup) {
-    // the group's first kRB rows are requested before the gate softmax, so
-    // that the two memory latencies overlap
-    uint4 q[kRB][KC];
+  cp_async_wait_all();
 #pragma unroll
-    for (int j = 0; j < kRB; ++j) {
-      const int tt = t0 + j;
-      if (j < np) {
-        const uint16_t* row = tt < s ? a.state_x + ((size_t)b * r + j) * a.dim
-                                     : a.x + (size_t)(a.cu_seqlens[b] + (tt - s)) * a.dim;
-        load_row<KC>(row, lane, nch, q[j]);
-      }
-    }
-    group_weights<kNQ>(a, b, s, t0, np, lane, w);
-#pragma unroll
-    for (int j = 0; j < kRB; ++j) {
-      if (j >= np) break;
-      const float wt = w[j];
-#pragma unroll
-      for (int k = 0; k < KC; ++k) {
-        float v[8];
-        unpack_bf16x8(q[j][k], v);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wt, v[e], acc[k][e]);
-      }
-    }
-    if (np > kRB) weighted_rows<KC, kRB>(a, b, s, t0, kRB, np, w, lane, nch, acc);
-    finish_entry<KC>(a, i, b, t0, lane, nch, acc);
-    // this warp consumed every old state row and gate it read (the sums and
-    // the softmax reductions depend on them), so the state may be rewritten
-    if (first_of_seq) copy_state<KC, kRB>(a, b, s, end, 0, r, lane, nch);
-  } else {
-    group_weights<kNQ>(a, b, s, t0, np, lane, w);
-    const int rpw = (r + kWarps - 1) / kWarps;
-    weighted_rows<KC, kRB>(a, b, s, t0, min(np, warp * rpw), min(np, (warp + 1) * rpw), w, lane, nch,
-                           acc);
+  for (int j = 0; j < kGroupRows; ++j) {
+    const float wt = __shfl_sync(0xffffffffu, wl, j);
+    if (j >= np) break;
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
-      float* p = &part[warp][8 * (lane + 32 * k)];
-      *reinterpret_cast<float4*>(p) = make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]);
-      *reinterpret_cast<float4*>(p + 4) = make_float4(acc[k][4], acc[k][5], acc[k][6], acc[k][7]);
+      if (!kFull && lane + 32 * k >= nch) continue;
+      float v[8];
+      unpack_bf16x8(stage[(j * KC + k) * 32 + lane], v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wt, v[e], acc[k][e]);
     }
-    __syncthreads();  // partial sums in place; every read of the old state is done
-    if (warp == 0) {
-#pragma unroll
-      for (int k = 0; k < KC; ++k) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[k][e] = part[0][8 * (lane + 32 * k) + e];
-        for (int ww = 1; ww < kWarps; ++ww)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[k][e] += part[ww][8 * (lane + 32 * k) + e];
-      }
-      finish_entry<KC>(a, i, b, t0, lane, nch, acc);
-    }
-    if (first_of_seq) copy_state<KC, kRB>(a, b, s, end, warp * rpw, (warp + 1) * rpw, lane, nch);
   }
+  finish_entry<KC>(a, i, t0, lane, nch, acc, rc, rs, slot);
+  // this warp consumed every old state row and gate it read (the sums and
+  // the softmax reductions depend on them), so the state may be rewritten
+  if (i == cu[b]) copy_state<KC, 2>(a, b, s, end, 0, r, lane, nch);
 }
 
+// Ratio 128: one block per group; the leading blocks copy window rows. Warp
+// w sums rows [16w, 16w + 16) of the group: the first eight go into its
+// shared memory with cp.async, the other eight into registers, all sixteen
+// requested at once, before the gate loads; warp 0 also issues the entry's
+// block-table load and evaluates the RoPE cos / sin while they are in
+// flight. The eight partial sums are added in warp order. KC: 8-dim chunks
+// per lane (dim <= 256 * KC); kFull: dim == 256 * KC. Dynamic shared memory:
+// kWarps * 8 * KC * 512 B.
+constexpr int kBlockRatio = 128;
+constexpr int kStagedRows = 8;  // rows per warp through shared memory (the rest in registers)
+
+template <int KC, bool kFull>
+__global__ void __launch_bounds__(kWarps * 32, KC <= 2 ? 2 : 1)
+    compress_group_block_kernel(CompressArgs a, int window_blocks, int window_blocks_per_seq) {
+  constexpr int r = kBlockRatio;
+  constexpr int spb = kLogicalBlock / kBlockRatio;
+  constexpr int rpw = r / kWarps;                 // 16 rows per warp
+  constexpr int kRegRows = rpw - kStagedRows;     // 8
+  constexpr int kNQ = r / 32;                     // gates per lane
+  extern __shared__ uint4 rows_sh[];  // [kWarps][kStagedRows][KC][32]; then the partial sums
+  __shared__ int cu_sh[kCuSmem];
+  __shared__ int2 meta_sh[kCuSmem];
+  tc::pdl_wait();  // the slot mapping (and whatever produced x) is complete from here on
+  tc::pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nch = kFull ? 32 * KC : a.dim >> 3;
+  if ((int)blockIdx.x < window_blocks) {
+    window_row<KC>(a, blockIdx.x / window_blocks_per_seq,
+                   (blockIdx.x % window_blocks_per_seq) * kWarps + warp, lane, nch);
+    return;
+  }
+  const bool cached = seq_tables<r>(a, cu_sh, meta_sh);
+  const int32_t* cu = cached ? cu_sh : a.cu_entries;
+  const int total = cu[a.batch];
+  const int i = blockIdx.x - window_blocks;
+  if (i >= total) return;  // uniform over the block
+  const int b = seq_of(cu, a.batch, i);
+  const int s = cached ? meta_sh[b].x : a.seq_start[b];
+  const int c0 = cached ? meta_sh[b].y : a.cu_seqlens[b];
+  const int end = s + ((cached ? meta_sh[b + 1].y : a.cu_seqlens[b + 1]) - c0);
+  const int g = s / r + (i - cu[b]);
+  const int t0 = g * r;
+  const int np = min(t0 + r, end) - t0;
+  const int lo = min(np, warp * rpw), mid = min(np, lo + kStagedRows), hi = min(np, lo + rpw);
+
+  // 1. this warp's rows: [lo, mid) into shared memory, [mid, hi) into registers
+  uint4* stage = rows_sh + (size_t)warp * kStagedRows * KC * 32;
+  auto row_ptr = [&](int j) {
+    const int tt = t0 + j;
+    return tt < s ? a.state_x + ((size_t)b * r + j) * a.dim : a.x + (size_t)(c0 + (tt - s)) * a.dim;
+  };
+  for (int j = lo; j < mid; ++j) {
+    const uint16_t* row = row_ptr(j);
+#pragma unroll
+    for (int k = 0; k < KC; ++k)
+      if (kFull || lane + 32 * k < nch)
+        cp_async16(stage + ((j - lo) * KC + k) * 32 + lane, row + 8 * (lane + 32 * k));
+  }
+  uint4 q[kRegRows][KC];
+#pragma unroll
+  for (int j = 0; j < kRegRows; ++j)
+    if (mid + j < hi) load_row<KC>(row_ptr(mid + j), lane, nch, q[j]);
+  // 2. gates and position bias (every warp forms the whole softmax); warp 0:
+  // the page and the RoPE values
+  float gate[kNQ], bias[kNQ];
+#pragma unroll
+  for (int u = 0; u < kNQ; ++u) {
+    const int t = lane + 32 * u;
+    gate[u] = 0.f;
+    bias[u] = 0.f;
+    if (t < np) {
+      const int tt = t0 + t;
+      gate[u] = tt < s ? a.state_gate[(size_t)b * r + t] : a.gate[c0 + (tt - s)];
+      bias[u] = a.pos_bias[t];
+    }
+  }
+  long long slot = -1;
+  float rc = 1.f, rs = 0.f;
+  if (warp == 0) {
+    const int blk = g / spb;
+    int page = -1;
+    if (a.slot_mapping) slot = a.slot_mapping[i];
+    else if (blk < a.main.max_blocks) page = a.main.block_table[(size_t)b * a.main.max_blocks + blk];
+    if (a.rope.rope_dim) rope_pair_lane(a.rope, lane, (long long)t0, &rc, &rs);
+    if (!a.slot_mapping) {
+      if (blk >= a.main.max_blocks) {
+        if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
+      } else if (page < 0 || page >= a.main.num_pages) {
+        if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_PAGE);
+      } else {
+        slot = (long long)page * spb + g % spb;
+      }
+    }
+    if (slot >= (long long)a.main.num_pages * spb) {
+      if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
+      slot = -1;
+    }
+  }
+  // 3. softmax weights: w[t] held by lane t % 32 in wq[t / 32]
+  float z[kNQ], m = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < kNQ; ++u) {
+    z[u] = lane + 32 * u < np ? gate[u] + bias[u] : -INFINITY;
+    m = fmaxf(m, z[u]);
+  }
+  m = warp_max(m);
+  float part_sum = 0.f;
+#pragma unroll
+  for (int u = 0; u < kNQ; ++u) {
+    z[u] = lane + 32 * u < np ? expf(z[u] - m) : 0.f;
+    part_sum += z[u];
+  }
+  const float sum = warp_sum(part_sum);
+  float wq[kNQ];
+#pragma unroll
+  for (int u = 0; u < kNQ; ++u) wq[u] = __fdiv_rn(z[u], sum);
+  auto weight = [&](int t) {  // t warp-uniform
+    float v = wq[0];
+#pragma unroll
+    for (int u = 1; u < kNQ; ++u)
+      if ((t >> 5) == u) v = wq[u];
+    return __shfl_sync(0xffffffffu, v, t & 31);
+  };
+
+  float acc[KC][8];
+#pragma unroll
+  for (int k = 0; k < KC; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
+  cp_async_wait_all();
+  for (int j = lo; j < mid; ++j) {
+    const float wt = weight(j);
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      if (!kFull && lane + 32 * k >= nch) continue;
+      float v[8];
+      unpack_bf16x8(stage[((j - lo) * KC + k) * 32 + lane], v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wt, v[e], acc[k][e]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kRegRows; ++j) {
+    if (mid + j >= hi) break;
+    const float wt = weight(mid + j);
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      float v[8];
+      unpack_bf16x8(q[j][k], v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wt, v[e], acc[k][e]);
+    }
+  }
+  __syncwarp();  // every lane has read its staged rows: the partial sum may overwrite them
+  float* part = reinterpret_cast<float*>(stage);
+#pragma unroll
+  for (int k = 0; k < KC; ++k) {
+    float* p = part + 8 * (lane + 32 * k);
+    *reinterpret_cast<float4*>(p) = make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]);
+    *reinterpret_cast<float4*>(p + 4) = make_float4(acc[k][4], acc[k][5], acc[k][6], acc[k][7]);
+  }
+  __syncthreads();  // partial sums in place; every read of the old state is done
+  if (warp == 0) {
+    constexpr int kWarpFloats = kStagedRows * KC * 32 * 4;
+    const float* parts = reinterpret_cast<const float*>(rows_sh);
+#pragma unroll
+    for (int k = 0; k < KC; ++k) {
+      const int d = 8 * (lane + 32 * k);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float4 t = *reinterpret_cast<const float4*>(parts + d + 4 * h);
+        for (int ww = 1; ww < kWarps; ++ww) {
+          const float4 u = *reinterpret_cast<const float4*>(parts + ww * kWarpFloats + d + 4 * h);
+          t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+        }
+        acc[k][4 * h] = t.x; acc[k][4 * h + 1] = t.y; acc[k][4 * h + 2] = t.z; acc[k][4 * h + 3] = t.w;
+      }
+    }
+    finish_entry<KC>(a, i, t0, lane, nch, acc, rc, rs, slot);
+  }
+  if (i == cu[b]) copy_state<KC, 2>(a, b, s, end, warp * rpw, (warp + 1) * rpw, lane, nch);
+}
 
 // ---------------------------------------------------------------- variants
 // c128a with per-channel gates: one block per entry. Token k of the entry's span (k = t - start, start =
@@ -823,12 +1102,38 @@ cudaError_t launch_variant_kc(const CompressArgs& a, int max_groups, int window_
 template <int KC>
 cudaError_t launch_kc(const CompressArgs& a, int max_groups, int window_blocks, int per_seq,
                       cudaStream_t stream) {
-  const bool block_group = a.ratio > 32;
-  const int entry_blocks = block_group ? max_groups : (max_groups + kWarps - 1) / kWarps;
-  const dim3 grid(window_blocks + entry_blocks), block(kWarps * 32);
-  if (block_group)
-    return launch_pdl(compress_append_kernel<KC, true>, grid, block, 0, stream, a, window_blocks, per_seq);
-  return launch_pdl(compress_append_kernel<KC, false>, grid, block, 0, stream, a, window_blocks, per_seq);
+  if (a.ratio != kGroupRows) {
+    if (a.ratio != kBlockRatio) return cudaErrorInvalidValue;
+    const dim3 grid(window_blocks + max_groups), block(kWarps * 32);
+    // with the static arrays (12 KB) the total passes 48 KB: opt in
+    const size_t smem = (size_t)kWarps * kStagedRows * KC * 32 * sizeof(uint4);
+    cudaError_t e = cudaFuncSetAttribute(compress_group_block_kernel<KC, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(compress_group_block_kernel<KC, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (a.dim == 256 * KC)
+      return launch_pdl(compress_group_block_kernel<KC, true>, grid, block, smem, stream, a, window_blocks,
+                        per_seq);
+    return launch_pdl(compress_group_block_kernel<KC, false>, grid, block, smem, stream, a, window_blocks,
+                      per_seq);
+  }
+  const dim3 grid(window_blocks + (max_groups + kWarps - 1) / kWarps), block(kWarps * 32);
+  const size_t smem = (size_t)kWarps * kGroupRows * KC * 32 * sizeof(uint4);
+  if (smem > 32 * 1024) {  // with the static arrays (12 KB) past 48 KB: opt in
+    cudaError_t e = cudaFuncSetAttribute(compress_group_warp_kernel<KC, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(compress_group_warp_kernel<KC, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  if (a.dim == 256 * KC)
+    return launch_pdl(compress_group_warp_kernel<KC, true>, grid, block, smem, stream, a, window_blocks,
+                      per_seq);
+  return launch_pdl(compress_group_warp_kernel<KC, false>, grid, block, smem, stream, a, window_blocks,
+                    per_seq);
 }
 
 
