@@ -540,7 +540,7 @@ __global__ void __launch_bounds__(kWarps * 32, KC <= 2 ? 4 : 2)
   finish_entry<KC>(a, i, t0, lane, nch, acc, rc, rs, slot);
   // this warp consumed every old state row and gate it read (the sums and
   // the softmax reductions depend on them), so the state may be rewritten
-  if (i == cu[b]) copy_state<KC, 2>(a, b, s, end, 0, r, lane, nch);
+  if (i == cu[b]) copy_state<KC, kGroupRows>(a, b, s, end, 0, r, lane, nch);
 }
 
 // Ratio 128: one block per group; the leading blocks copy window rows. Warp
@@ -723,7 +723,7 @@ __global__ void __launch_bounds__(kWarps * 32, KC <= 2 ? 2 : 1)
     }
     finish_entry<KC>(a, i, t0, lane, nch, acc, rc, rs, slot);
   }
-  if (i == cu[b]) copy_state<KC, 2>(a, b, s, end, warp * rpw, (warp + 1) * rpw, lane, nch);
+  if (i == cu[b]) copy_state<KC, KC <= 2 ? 8 : 4>(a, b, s, end, warp * rpw, (warp + 1) * rpw, lane, nch);
 }
 
 // ---------------------------------------------------------------- variants
