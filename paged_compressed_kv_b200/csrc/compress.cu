@@ -382,7 +382,8 @@ __device__ __forceinline__ bool seq_tables(const CompressArgs& a, int* cu_sh, in
         if (lane == a.batch - 1) meta_sh[a.batch] = make_int2(0, c1);
       }
       if (a.cu_entries) {
-        if (lane <= a.batch) cu_sh[lane] = a.cu_entries[lane];
+        if (lane < a.batch) cu_sh[lane] = a.cu_entries[lane];
+        if (lane == 0) cu_sh[a.batch] = a.cu_entries[a.batch];
       } else {
         int x = n;
 #pragma unroll
@@ -957,43 +958,76 @@ __global__ void __launch_bounds__(kWarps * 32) compress_variant_kernel(CompressA
 }
 
 
-// c4a variants, one warp per entry: the span (4 or 8 tokens) fits in a lane's
-// registers. Per-token gates: the weights once per token (lane t), added in
-// ascending t; per-channel gates: per dim, the maximum over the tokens, then
-// the sums of exp(z - m) and of exp(z - m) * x in ascending t.
-template <int KC>
-__device__ void warp_variant_entry(const CompressArgs& a, int i, int b, const int32_t* cu) {
-  constexpr int kSpan = 8;  // 2r for r = 4
+// c4a variants, one warp per entry. The span's rows (4 tokens, or 8 with the
+// overlapping window) go into the warp's shared memory with cp.async (lane l
+// copies and later reads chunks l, l + 32, ...); with per-token gates the
+// gate, bias and block-table loads and the RoPE cos / sin are issued while the
+// rows are in flight. Per-token gates: the weights once per token (lane t),
+// added in ascending t; per-channel gates: per dim, the maximum over the
+// tokens, then the sums of exp(z - m) and of exp(z - m) * x in ascending t.
+constexpr int kVariantSpan = 2 * kGroupRows;
+
+__host__ __device__ inline size_t variant_warp_smem(int kc, int batch) {
+  const size_t tables = batch + 1 <= kCuSmem ? (size_t)((batch + 4) & ~3) * 4 + (size_t)(batch + 1) * 8 : 0;
+  return (size_t)kWarps * kVariantSpan * kc * 32 * 16 + tables;
+}
+
+template <int KC, bool kFull>
+__device__ void warp_variant_entry(const CompressArgs& a, int i, int b, const int32_t* cu,
+                                   const int2* meta, uint4* stage) {
+  constexpr int r = kGroupRows;
+  constexpr int spb = kLogicalBlock / kGroupRows;
   const int lane = threadIdx.x & 31;
-  const int nch = a.dim >> 3;
-  const int r = a.ratio;
-  const int s = a.seq_start[b];
-  const int end = s + (a.cu_seqlens[b + 1] - a.cu_seqlens[b]);
-  const int t0 = (s / r + (i - cu[b])) * r;
+  const int nch = kFull ? 32 * KC : a.dim >> 3;
+  const int s = meta ? meta[b].x : a.seq_start[b];
+  const int c0 = meta ? meta[b].y : a.cu_seqlens[b];
+  const int end = s + ((meta ? meta[b + 1].y : a.cu_seqlens[b + 1]) - c0);
+  const int g = s / r + (i - cu[b]);
+  const int t0 = g * r;
   const int start = t0 - (a.overlap ? r : 0);
   const int lo = max(0, start), hi = min(t0 + r, end);
   const int np = hi - lo, k0 = lo - start;
   const int old_base = (s / r) * r - (a.overlap ? r : 0);
-  uint4 q[kSpan][KC];
 #pragma unroll
-  for (int j = 0; j < kSpan; ++j) {
+  for (int j = 0; j < kVariantSpan; ++j) {
     if (j < np) {
       const int tt = lo + j;
       const uint16_t* row = tt < s ? a.state_x + ((size_t)b * a.state_rows + (tt - old_base)) * a.dim
-                                   : a.x + (size_t)(a.cu_seqlens[b] + (tt - s)) * a.dim;
-      load_row<KC>(row, lane, nch, q[j]);
+                                   : a.x + (size_t)(c0 + (tt - s)) * a.dim;
+#pragma unroll
+      for (int k = 0; k < KC; ++k)
+        if (kFull || lane + 32 * k < nch) cp_async16(stage + (j * KC + k) * 32 + lane, row + 8 * (lane + 32 * k));
     }
+  }
+  // per-token gates: lane t < np holds token lo + t's logit and bias
+  float gate = 0.f, bias = 0.f;
+  if (a.gate_dim == 1 && lane < np) {
+    const int tt = lo + lane;
+    gate = tt < s ? a.state_gate[(size_t)b * a.state_rows + (tt - old_base)] : a.gate[c0 + (tt - s)];
+    bias = a.pos_bias[k0 + lane];
+  }
+  long long slot = -1;
+  int page = -1;
+  if (a.slot_mapping) slot = a.slot_mapping[i];
+  else if (g / spb < a.main.max_blocks) page = a.main.block_table[(size_t)b * a.main.max_blocks + g / spb];
+  float rc = 1.f, rs = 0.f;
+  if (a.rope.rope_dim) rope_pair_lane(a.rope, lane, (long long)t0, &rc, &rs);
+  if (!a.slot_mapping) {
+    if (g / spb >= a.main.max_blocks) {
+      if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
+    } else if (page < 0 || page >= a.main.num_pages) {
+      if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_PAGE);
+    } else {
+      slot = (long long)page * spb + g % spb;
+    }
+  }
+  if (slot >= (long long)a.main.num_pages * spb) {
+    if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
+    slot = -1;
   }
   float acc[KC][8];
   if (a.gate_dim == 1) {
-    // lane t < np: logit of token lo + t plus its bias; softmax across lanes
-    float z = -INFINITY;
-    if (lane < np) {
-      const int tt = lo + lane;
-      const float g = tt < s ? a.state_gate[(size_t)b * a.state_rows + (tt - old_base)]
-                             : a.gate[a.cu_seqlens[b] + (tt - s)];
-      z = g + a.pos_bias[k0 + lane];
-    }
+    const float z = lane < np ? gate + bias : -INFINITY;
     const float m = warp_max(z);
     const float u = lane < np ? expf(z - m) : 0.f;
     const float sum = warp_sum(u);
@@ -1002,19 +1036,22 @@ __device__ void warp_variant_entry(const CompressArgs& a, int i, int b, const in
     for (int k = 0; k < KC; ++k)
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
+    cp_async_wait_all();
 #pragma unroll
-    for (int j = 0; j < kSpan; ++j) {
+    for (int j = 0; j < kVariantSpan; ++j) {
       const float wt = __shfl_sync(0xffffffffu, w, j);
       if (j >= np) break;
 #pragma unroll
       for (int k = 0; k < KC; ++k) {
+        if (!kFull && lane + 32 * k >= nch) continue;
         float v[8];
-        unpack_bf16x8(q[j][k], v);
+        unpack_bf16x8(stage[(j * KC + k) * 32 + lane], v);
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(wt, v[e], acc[k][e]);
       }
     }
   } else {
+    cp_async_wait_all();
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
       const int c = lane + 32 * k;
@@ -1024,62 +1061,67 @@ __device__ void warp_variant_entry(const CompressArgs& a, int i, int b, const in
         m[e] = -INFINITY;
         su[e] = sv[e] = 0.f;
       }
-      if (c < nch) {
+      if (kFull || c < nch) {
 #pragma unroll
-        for (int j = 0; j < kSpan; ++j) {
+        for (int j = 0; j < kVariantSpan; ++j) {
           if (j >= np) break;
           float z[8];
           gate_chunk(a, b, s, old_base, lo + j, c, z);
-          const float bias = a.pos_bias[k0 + j];
+          const float bj = a.pos_bias[k0 + j];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], z[e] + bias);
+          for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], z[e] + bj);
         }
 #pragma unroll
-        for (int j = 0; j < kSpan; ++j) {
+        for (int j = 0; j < kVariantSpan; ++j) {
           if (j >= np) break;
           float z[8], v[8];
           gate_chunk(a, b, s, old_base, lo + j, c, z);
-          unpack_bf16x8(q[j][k], v);
-          const float bias = a.pos_bias[k0 + j];
+          unpack_bf16x8(stage[(j * KC + k) * 32 + lane], v);
+          const float bj = a.pos_bias[k0 + j];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float u = expf(z[e] + bias - m[e]);
+            const float u = expf(z[e] + bj - m[e]);
             su[e] += u;
             sv[e] = fmaf(u, v[e], sv[e]);
           }
         }
       }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[k][e] = c < nch ? __fdiv_rn(sv[e], su[e]) : 0.f;
+      for (int e = 0; e < 8; ++e) acc[k][e] = (kFull || c < nch) ? __fdiv_rn(sv[e], su[e]) : 0.f;
     }
   }
-  finish_entry<KC>(a, i, b, t0, lane, nch, acc);
+  __syncwarp();  // every lane has read its rows before the stage is reused
+  finish_entry<KC>(a, i, t0, lane, nch, acc, rc, rs, slot);
 }
 
-template <int KC>
-__global__ void __launch_bounds__(kWarps * 32) compress_variant_warp_kernel(CompressArgs a,
-                                                                           int window_blocks,
-                                                                           int window_blocks_per_seq) {
-  __shared__ int cu_sh[kCuSmem];
+template <int KC, bool kFull>
+__global__ void __launch_bounds__(kWarps * 32, KC <= 2 ? 3 : 1)
+    compress_variant_warp_kernel(CompressArgs a, int window_blocks, int window_blocks_per_seq) {
+  extern __shared__ uint4 dyn_sh[];  // [kWarps][kVariantSpan][KC][32], then the tables
+  int* cu_sh = reinterpret_cast<int*>(dyn_sh + kWarps * kVariantSpan * KC * 32);
+  int2* meta_sh = reinterpret_cast<int2*>(cu_sh + ((a.batch + 4) & ~3));
   tc::pdl_wait();  // x, the gates and the state (earlier work in the stream) are complete
   tc::pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nch = a.dim >> 3;
+  const int nch = kFull ? 32 * KC : a.dim >> 3;
   if ((int)blockIdx.x < window_blocks) {
     window_row<KC>(a, blockIdx.x / window_blocks_per_seq,
                    (blockIdx.x % window_blocks_per_seq) * kWarps + warp, lane, nch);
     return;
   }
-  const int32_t* cu = entry_prefix(a, cu_sh);
+  const bool cached = seq_tables<kGroupRows>(a, cu_sh, meta_sh);
+  const int32_t* cu = cached ? cu_sh : a.cu_entries;
+  const int2* meta = cached ? meta_sh : nullptr;
   const int i = (blockIdx.x - window_blocks) * kWarps + warp;
   if (i >= cu[a.batch]) return;  // uniform over the warp
   const int b = seq_of(cu, a.batch, i);
   // the warp of the sequence's first entry also builds the second (both read
   // the old state with the overlapping window) and then rewrites the state
   if (a.overlap && i == cu[b] + 1) return;
-  warp_variant_entry<KC>(a, i, b, cu);
+  uint4* stage = dyn_sh + (size_t)warp * kVariantSpan * KC * 32;
+  warp_variant_entry<KC, kFull>(a, i, b, cu, meta, stage);
   if (i == cu[b]) {
-    if (a.overlap && i + 1 < cu[b + 1]) warp_variant_entry<KC>(a, i + 1, b, cu);
+    if (a.overlap && i + 1 < cu[b + 1]) warp_variant_entry<KC, kFull>(a, i + 1, b, cu, meta, stage);
     variant_state<KC>(a, b);
   }
 }
@@ -1087,10 +1129,21 @@ __global__ void __launch_bounds__(kWarps * 32) compress_variant_warp_kernel(Comp
 template <int KC>
 cudaError_t launch_variant_kc(const CompressArgs& a, int max_groups, int window_blocks, int per_seq,
                               cudaStream_t stream) {
-  if (a.ratio <= kWarps)  // c4a: one warp per entry
-    return launch_pdl(compress_variant_warp_kernel<KC>,
-                      dim3(window_blocks + (max_groups + kWarps - 1) / kWarps), dim3(kWarps * 32), 0,
-                      stream, a, window_blocks, per_seq);
+  if (a.ratio == kGroupRows) {  // c4a: one warp per entry
+    const size_t smem = variant_warp_smem(KC, a.batch);
+    cudaError_t e = cudaFuncSetAttribute(compress_variant_warp_kernel<KC, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(compress_variant_warp_kernel<KC, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(window_blocks + (max_groups + kWarps - 1) / kWarps), block(kWarps * 32);
+    if (a.dim == 256 * KC)
+      return launch_pdl(compress_variant_warp_kernel<KC, true>, grid, block, smem, stream, a, window_blocks,
+                        per_seq);
+    return launch_pdl(compress_variant_warp_kernel<KC, false>, grid, block, smem, stream, a, window_blocks,
+                      per_seq);
+  }
   const size_t smem = (size_t)3 * kWarps * a.dim * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(compress_variant_kernel<KC>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

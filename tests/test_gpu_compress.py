@@ -255,6 +255,22 @@ def test_inline_slot_mapping_equals_explicit_bitwise(ratio):
     assert torch.equal(a.state_x, b.state_x) and torch.equal(a.state_g, b.state_g)
 
 
+@pytest.mark.parametrize("ratio", [4, 128])
+@pytest.mark.parametrize("batch", [31, 32, 33])
+def test_batch_at_the_one_warp_table_limit(ratio, batch):
+    """Batches of 31, 32 and 33 sequences, with the slot mapping passed and
+    without: the kernel's per-call sequence tables are built by one warp up
+    to 32 sequences (the entry total sits one past the last lane) and by the
+    whole block above; every entry, the state and the window match the oracle."""
+    r = synth.rng(470 + batch + ratio)
+    n = [int(v) for v in r.integers(1, 700, batch)]
+    for inline in (False, True):
+        ap = Appender(471 + batch + ratio, n, ratio)
+        while any(d < N for d, N in zip(ap.done, ap.n)):
+            ap.append([int(v) for v in r.integers(0, 400, batch)], inline_slots=inline)
+        check_against_oracle(ap)
+
+
 def test_inline_slot_mapping_arguments():
     """Exactly one of slot_mapping / cu_entries missing is an argument error."""
     from paged_compressed_kv_b200 import v4kv
