@@ -98,25 +98,24 @@ __device__ __forceinline__ void rope_warp(float (&e)[KC][8], int lane, int nch, 
   rope_warp<KC>(e, lane, nch, rp, pos, c0, s0);
 }
 
-// v / scale as far as its e4m3 code is concerned, y = 1 / scale rounded to
-// nearest. The product v * y is within 2 fp32 ulps of v / scale (two
-// roundings of relative size 2^-24 each), and the correctly rounded quotient
-// within half an ulp of it, so both give the same e4m3 code unless v / scale
-// lies near the midpoint between two neighbouring codes. The code of a
-// normal-range value (binades 2^-6 .. 2^8) depends only on the 3 leading
-// mantissa bits and the rounding bit below them, so a midpoint is a pattern of
-// 0x80000 in the 20 low mantissa bits; within 8 ulps of it, and below the
-// normal e4m3 range or for infinities and NaNs, the IEEE quotient is formed
-// instead. The codes are therefore those of float2_to_e4m3x2(v / scale).
-__device__ __forceinline__ float e4m3_quotient(float v, float scale, float y) {
-  const float q = __fmul_rn(v, y);
+// e4m3 codes of v / scale from the product q = v * y, y = 1 / scale rounded to
+// nearest. The product is within 2 fp32 ulps of v / scale (two roundings of
+// relative size 2^-24 each), and the correctly rounded quotient within half an
+// ulp of it, so both give the same e4m3 code unless v / scale lies near the
+// midpoint between two neighbouring codes. The code of a normal-range value
+// (binades 2^-6 .. 2^8) depends only on the 3 leading mantissa bits and the
+// rounding bit below them, so a midpoint is a pattern of 0x80000 in the 20 low
+// mantissa bits. quotient_needs_ieee(q) is true within 8 ulps of such a
+// pattern, below the normal e4m3 range, and for infinities and NaNs: there the
+// IEEE quotient is formed instead, so the codes are those of
+// float2_to_e4m3x2(v / scale).
+__device__ __forceinline__ bool quotient_needs_ieee(float q) {
   const uint32_t u = __float_as_uint(q) & 0x7fffffffu;
   // outside [2^-6, inf): the unsigned difference wraps past the range
   const bool outside = u - 0x3c800000u >= 0x7f800000u - 0x3c800000u;
   // low 20 mantissa bits within 8 of 0x80000
   const bool near_mid = ((u + 8u - 0x80000u) & 0xfffffu) <= 16u;
-  if (outside || near_mid) return __fdiv_rn(v, scale);
-  return q;
+  return outside || near_mid;
 }
 
 // quantise (fp8: absmax over the warp's whole vector) or round (bf16) one
@@ -138,12 +137,25 @@ __device__ __forceinline__ void store_entry_warp(const PoolArgs& pool, long long
 #pragma unroll
     for (int k = 0; k < KC; ++k) {
       const int c = lane + 32 * k;
+      // the products; the IEEE quotient only where one needs it (one vote per
+      // chunk row, so the common case has no per-value branch)
+      float qv[8];
+      bool ieee = false;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        qv[i] = __fmul_rn(e[k][i], y);
+        ieee |= quotient_needs_ieee(qv[i]);
+      }
+      ieee = ieee && c < nch;
+      if (__any_sync(0xffffffffu, ieee) && ieee) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (quotient_needs_ieee(qv[i])) qv[i] = __fdiv_rn(e[k][i], scale);
+      }
       if (c >= nch) continue;
       uint16_t q[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        q[i] = float2_to_e4m3x2(e4m3_quotient(e[k][2 * i], scale, y),
-                                e4m3_quotient(e[k][2 * i + 1], scale, y));
+      for (int i = 0; i < 4; ++i) q[i] = float2_to_e4m3x2(qv[2 * i], qv[2 * i + 1]);
       *reinterpret_cast<uint2*>(base + 8 * c) =
           make_uint2((uint32_t)q[0] | ((uint32_t)q[1] << 16), (uint32_t)q[2] | ((uint32_t)q[3] << 16));
     }
@@ -513,11 +525,15 @@ __global__ void __launch_bounds__(kWarps * 32, KC <= 2 ? 4 : 2)
     if (lane == 0) flag(a.dev_status, V4KV_DEV_BAD_SLOT);
     slot = -1;
   }
-  // 3. the gate softmax over the np present tokens; lane j holds w[j]
+  // 3. the gate softmax over the np present tokens (lanes 0 .. 3, reduced
+  // among themselves); lane j holds w[j]
   const float z = lane < np ? gate + bias : -INFINITY;
-  const float m = warp_max(z);
+  float m = fmaxf(z, __shfl_xor_sync(0xffffffffu, z, 1));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
   const float ez = lane < np ? expf(z - m) : 0.f;
-  const float wl = __fdiv_rn(ez, warp_sum(ez));
+  float sum = ez + __shfl_xor_sync(0xffffffffu, ez, 1);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+  const float wl = lane < np ? __fdiv_rn(ez, sum) : 0.f;
 
   float acc[KC][8];
 #pragma unroll
