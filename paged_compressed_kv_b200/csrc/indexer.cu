@@ -376,12 +376,17 @@ __device__ __forceinline__ unsigned long long comp_key(uint32_t key, int j) {
 
 // bitonic sort of v[0 .. n) (n a power of two) in descending order
 // number of the n keys v[] (distinct) larger than `mine`; every thread reads
-// the same v[j] at a time (shared-memory broadcast)
+// the same keys at a time (shared-memory broadcast), two per 16-byte load, so
+// a warp's scan costs one shared-memory wavefront per two keys. v is 16-byte
+// aligned.
 __device__ __forceinline__ int rank_of(unsigned long long mine, const unsigned long long* v, int n) {
+  const ulonglong2* v2 = reinterpret_cast<const ulonglong2*>(v);
   int r = 0;
   int j = 0;
-  for (; j + 4 <= n; j += 4)
-    r += (v[j] > mine) + (v[j + 1] > mine) + (v[j + 2] > mine) + (v[j + 3] > mine);
+  for (; j + 4 <= n; j += 4) {
+    const ulonglong2 x = v2[j >> 1], y = v2[(j >> 1) + 1];
+    r += (x.x > mine) + (x.y > mine) + (y.x > mine) + (y.y > mine);
+  }
   for (; j < n; ++j) r += v[j] > mine;
   return r;
 }
@@ -449,8 +454,8 @@ __device__ void radix_select_exact(const float* sc, int n, int k, unsigned long 
 __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexArgs a) {
   __shared__ uint32_t hist[kBins];
   __shared__ uint32_t scan_sh[32];
-  __shared__ unsigned long long sel[kMaxK];
-  __shared__ unsigned long long cand[kCandCap];
+  __shared__ __align__(16) unsigned long long sel[kMaxK];
+  __shared__ __align__(16) unsigned long long cand[kCandCap];
   __shared__ float red[32];
   __shared__ float q_f[kIdxMaxDim];
   __shared__ float qs_sh;
@@ -522,6 +527,12 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexArgs 
           if (p < (uint32_t)kCandCap) cand[p] = comp_key(key, j);
         }
       };
+      // a float below f0, the smallest float whose key reaches the threshold
+      // bin, has a key below it (the key is monotone in the float order), so a
+      // load of four such scores needs no per-score work (a NaN fails every
+      // comparison and takes the exact test)
+      const uint32_t k0 = tb << kBinShift;
+      const float f0 = __uint_as_float((k0 & 0x80000000u) ? (k0 & 0x7fffffffu) : ~k0);
       const float4* sc4 = reinterpret_cast<const float4*>(sc);
       const int n4 = (n + 3) / 4;
       for (int q0 = threadIdx.x; q0 < n4; q0 += 4 * blockDim.x) {
@@ -533,6 +544,7 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexArgs 
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
+          if (v[u].x < f0 && v[u].y < f0 && v[u].z < f0 && v[u].w < f0) continue;
           const int j = 4 * (q0 + u * blockDim.x);
           take(v[u].x, j);
           take(v[u].y, j + 1);
@@ -565,10 +577,11 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexArgs 
   const int valid = min(n, k);
   for (int i = threadIdx.x; i < valid; i += blockDim.x) {
     const unsigned long long mine = sel[i];
-    const int r = rank_of(mine, sel, valid);
     const int32_t idx = (int32_t)(0xffffffffu - (uint32_t)(mine & 0xffffffffull));
+    const float raw = a.score_out ? sc[idx] : 0.f;  // requested before the ranking
+    const int r = rank_of(mine, sel, valid);
     a.topk_out[(size_t)b * k + r] = idx;
-    if (a.score_out) a.score_out[(size_t)b * k + r] = __fmul_rn(sc[idx], qs_sh);
+    if (a.score_out) a.score_out[(size_t)b * k + r] = __fmul_rn(raw, qs_sh);
   }
   for (int i = valid + threadIdx.x; i < k; i += blockDim.x) {
     a.topk_out[(size_t)b * k + i] = -1;
