@@ -477,6 +477,20 @@ def test_variants_match_oracle_and_chunking(ratio, opts):
         assert np.array_equal(a.prequant[s].view(np.uint32), b.prequant[s].view(np.uint32))
 
 
+@pytest.mark.parametrize("dim", [200, 1024])
+@pytest.mark.parametrize("opts", [dict(overlap=True), dict(overlap=True, per_channel=True, norm=True)])
+def test_c4a_variants_at_other_widths(dim, opts):
+    """The c4a variant kernel at a ragged width (one partial chunk row per
+    lane) and at 1024 dims (four chunk rows per lane): random chunks against
+    the oracle, reading back the rolling state of the overlapping window."""
+    n = [700, 129, 5, 300]
+    ap = Appender(480 + dim, n, 4, dim=dim, **opts)
+    r = synth.rng(481 + dim)
+    while any(d < N for d, N in zip(ap.done, ap.n)):
+        ap.append([int(r.integers(0, 260)) for _ in n])
+    check_against_oracle(ap)
+
+
 def test_variant_arguments():
     """The overlapping window is c4a's only; odd option values are rejected."""
     from paged_compressed_kv_b200 import v4kv
