@@ -218,6 +218,24 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
 // hit eight different bank groups. Stages of 256 entries (four boxes) rotate
 // through a three-deep ring; every thread scores one entry of each stage with
 // the same ascending-d chain as the generic kernel.
+// L2 policy for data read once: evicted first, so that it does not push out
+// the scores, which the select reads back
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t policy;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+  return policy;
+}
+
+// tc::tma_load_2d with an L2 cache policy
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const void* tmap, int x, int y, uint64_t* bar,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(tc::smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 constexpr int kTmaBox = 64;                    // rows per box
 constexpr int kTmaBatch = 256;                 // entries per stage = threads
 constexpr int kTmaStages = 3;
@@ -272,6 +290,7 @@ __global__ void __launch_bounds__(kTmaBatch) index_score_tma_kernel(const __grid
   }
   __syncthreads();
   const uint32_t stages_s = tc::smem_u32(stages);
+  const uint64_t keys_policy = l2_evict_first_policy();  // keys are read once
   auto issue = [&](int bi) {  // thread 0: the boxes of stage bi
     const int s = bi % kTmaStages;
     uint32_t bytes = 0;
@@ -283,7 +302,8 @@ __global__ void __launch_bounds__(kTmaBatch) index_score_tma_kernel(const __grid
     for (int k = 0; k < kTmaBatch / kTmaBox; ++k) {
       const int g = bi * (kTmaBatch / kTmaBox) + k;
       if (g < ngroups && row0[g] >= 0)
-        tc::tma_load_2d(stages_s + s * kStageBytes + k * kRowsPerBox * 128, &keys, 0, (int)row0[g], &full[s]);
+        tma_load_2d_hint(stages_s + s * kStageBytes + k * kRowsPerBox * 128, &keys, 0, (int)row0[g], &full[s],
+                         keys_policy);
     }
   };
   int issued = 0;  // thread 0: stages issued so far
