@@ -479,7 +479,7 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexArgs 
   __shared__ float red[32];
   __shared__ float q_f[kIdxMaxDim];
   __shared__ float qs_sh;
-  __shared__ uint32_t n_sel_sh, n_cand_sh, bin_sh, above_sh;
+  __shared__ uint32_t n_sel_sh, n_cand_sh, bin_sh, above_sh, n_hit_sh;
   __shared__ uint32_t pick_sh[2];
 
   const int b = blockIdx.x;
@@ -495,6 +495,7 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexArgs 
   if (threadIdx.x == 0) {
     n_sel_sh = 0;
     n_cand_sh = 0;
+    n_hit_sh = 0;
     bin_sh = 0xffffffffu;  // "not found" -> exact path
     above_sh = 0;
   }
@@ -555,27 +556,48 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexArgs 
       const float f0 = __uint_as_float((k0 & 0x80000000u) ? (k0 & 0x7fffffffu) : ~k0);
       const float4* sc4 = reinterpret_cast<const float4*>(sc);
       const int n4 = (n + 3) / 4;
-      for (int q0 = threadIdx.x; q0 < n4; q0 += 4 * blockDim.x) {
+      // pass 1: the float4 loads holding a score at or above the threshold bin
+      // (about one in twenty) are listed in shared memory (`hist`, free until
+      // the exact path), one atomic per warp and round; pass 2 takes their
+      // scores, spread over all threads
+      uint32_t* hitq = hist;
+      const int lane = threadIdx.x & 31;
+      const uint32_t below = (1u << lane) - 1u;
+      for (int q0 = threadIdx.x - lane; q0 < n4; q0 += 4 * blockDim.x) {  // warp-uniform
         float4 v[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int q = q0 + u * blockDim.x;
+          const int q = q0 + lane + u * blockDim.x;
           v[u] = q < n4 ? sc4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          if (v[u].x < f0 && v[u].y < f0 && v[u].z < f0 && v[u].w < f0) continue;
-          const int j = 4 * (q0 + u * blockDim.x);
-          take(v[u].x, j);
-          take(v[u].y, j + 1);
-          take(v[u].z, j + 2);
-          take(v[u].w, j + 3);
+          const int q = q0 + lane + u * blockDim.x;
+          const bool hit = q < n4 && !(v[u].x < f0 && v[u].y < f0 && v[u].z < f0 && v[u].w < f0);
+          const uint32_t m = __ballot_sync(0xffffffffu, hit);
+          if (m == 0u) continue;
+          const int leader = __ffs(m) - 1;
+          uint32_t base = 0;
+          if (lane == leader) base = atomicAdd(&n_hit_sh, (uint32_t)__popc(m));
+          base = __shfl_sync(0xffffffffu, base, leader);
+          const uint32_t pos = base + __popc(m & below);
+          if (hit && pos < (uint32_t)kBins) hitq[pos] = (uint32_t)q;
         }
+      }
+      __syncthreads();
+      const uint32_t nh = min(n_hit_sh, (uint32_t)kBins);  // more: the counts below disagree, exact path
+      for (uint32_t h = threadIdx.x; h < nh; h += blockDim.x) {
+        const int q = (int)hitq[h];
+        const float4 x = sc4[q];
+        take(x.x, 4 * q);
+        take(x.y, 4 * q + 1);
+        take(x.z, 4 * q + 2);
+        take(x.w, 4 * q + 3);
       }
     }
     __syncthreads();
     const uint32_t nc = n_cand_sh;
-    if (tb == 0xffffffffu || nc > (uint32_t)kCandCap || n_sel_sh != above) {
+    if (tb == 0xffffffffu || nc > (uint32_t)kCandCap || n_sel_sh != above || n_hit_sh > (uint32_t)kBins) {
       // too many entries share the threshold bin: exact radix path
       for (int i = threadIdx.x; i < kpow; i += blockDim.x) sel[i] = 0ull;
       __syncthreads();
